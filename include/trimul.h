@@ -1,0 +1,184 @@
+/*
+ * trimul.h -- C ABI of the B200 (sm_100a) triangle multiplicative update.
+ *
+ * The operation (one "layer", one direction) on a pair tensor z [B, N, N, c_z]
+ * with pair mask m [B, N, N]:
+ *
+ *   zhat_ij = LayerNorm_{c_z}(z_ij)
+ *   a_ij    = m_ij * sigmoid(zhat_ij W_ag^T + b_ag) (.) (zhat_ij W_ap^T + b_ap)
+ *   b_ij    = m_ij * sigmoid(zhat_ij W_bg^T + b_bg) (.) (zhat_ij W_bp^T + b_bp)
+ *   outgoing: x_ij = sum_k a_ik (.) b_jk        incoming: x_ij = sum_k a_ki (.) b_kj
+ *   out_ij  = m_ij * sigmoid(zhat_ij W_g^T + b_g) (.) (LayerNorm_{c_h}(x_ij) W_o^T + b_o)
+ *
+ * Sources: "RFProteina architecture" (BioNeMo Inference Runtime documentation),
+ * section "Inside the velocity network" (a pair update applies outgoing, then
+ * incoming triangle multiplication, each as a masked residual), section
+ * "Triangle multiplication on SM90" (the three-kernel chain: K1 input projection
+ * with the input LayerNorm folded into its weights, K2 the contraction compiled
+ * per direction, K3 output gate and projection with both LayerNorms folded) and
+ * section "Dual-GEMM gates" (the one-input gate sigma(x W_g^T + b_g) (.) (x W_p^T + b_p)
+ * that also applies the pair mask and emits its output transposed for the
+ * contraction, and the two-input gate sigma(x0 W_g^T + b_g) (.) (x1 W_p^T + b_p)
+ * with x0 the normalized pair tensor and x1 the contracted hidden tensor).
+ *
+ * Conventions for every entry point:
+ *   - All tensors are device pointers owned by the caller. Nothing here frees them.
+ *   - Pair tensors are contiguous [B, N, N, C], channel fastest (channel-last).
+ *   - Intermediate tensors a, b, x are contiguous [B, c_h, N, N] (channel-major:
+ *     every channel is one N x N matrix), which is the layout the contraction reads.
+ *   - Linear weights are row-major [out, in] with y = x W^T + bias. Bias and
+ *     LayerNorm beta pointers may be NULL (= 0); LayerNorm gamma may be NULL (= 1).
+ *   - `stream` is a cudaStream_t (NULL = legacy default stream). Forward calls
+ *     are asynchronous on it, allocate nothing and never synchronize.
+ *   - There is no fallback: an unsupported shape, dtype or device is an error.
+ *   - Errors are returned as trimul_status_t; tri_mul_last_error() gives a
+ *     human-readable detail for the calling thread.
+ */
+#ifndef TRIMUL_H
+#define TRIMUL_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    TRIMUL_OK = 0,
+    TRIMUL_ERR_INVALID_ARG = 1,        /* NULL pointer, bad size, unknown enum, aliasing */
+    TRIMUL_ERR_UNSUPPORTED_SHAPE = 2,  /* (c_z, c_h) or N outside the compiled set */
+    TRIMUL_ERR_UNSUPPORTED_DEVICE = 3, /* current device is not compute capability 10.0 */
+    TRIMUL_ERR_WORKSPACE = 4,          /* no workspace bound, or bound one too small */
+    TRIMUL_ERR_CUDA = 5,               /* a CUDA runtime / driver call failed */
+    TRIMUL_ERR_DEVICE_TIMEOUT = 6,     /* a kernel gave up on a bounded wait (see below) */
+    TRIMUL_ERR_ALIGNMENT = 7           /* a tensor pointer is not 16-byte aligned */
+} trimul_status_t;
+
+typedef enum { TRIMUL_OUTGOING = 0, TRIMUL_INCOMING = 1 } trimul_direction_t;
+
+typedef enum { TRIMUL_F32 = 0, TRIMUL_BF16 = 1 } trimul_dtype_t;
+
+/* A pair tensor [B, N, N, C], contiguous, channel-last. */
+typedef struct {
+    void *data;
+    int64_t B, N, C;
+    trimul_dtype_t dtype;
+} trimul_pair_t;
+
+/* Layer weights, all device pointers of storage type `dtype`, in this order:
+ *   ln_in_g, ln_in_b [c_z]            input LayerNorm
+ *   w_ag, w_ap, w_bg, w_bp [c_h, c_z]; b_ag, b_ap, b_bg, b_bp [c_h]
+ *   w_g [c_z, c_z], b_g [c_z]         output gate
+ *   ln_out_g, ln_out_b [c_h]          output LayerNorm
+ *   w_o [c_z, c_h], b_o [c_z]         output projection
+ * eps: LayerNorm epsilon for both norms (variance is the biased one, eps inside
+ * the square root). */
+typedef struct {
+    int32_t c_z, c_h;
+    trimul_dtype_t dtype;
+    float eps;
+    const void *ln_in_g, *ln_in_b;
+    const void *w_ag, *b_ag, *w_ap, *b_ap;
+    const void *w_bg, *b_bg, *w_bp, *b_bp;
+    const void *w_g, *b_g;
+    const void *ln_out_g, *ln_out_b;
+    const void *w_o, *b_o;
+} trimul_weights_desc_t;
+
+/* Opaque layer handle: the weights repacked for both compute paths. */
+typedef struct trimul_layer trimul_layer_t;
+
+/* Build a layer handle from weights already on the current device.
+ * The handle holds its own device copy: for the bf16 tensor-core path the input
+ * LayerNorm gamma is folded into W_ag/W_ap/W_bg/W_bp/W_g and the output
+ * LayerNorm gamma into W_o (bf16, [out, in]), with per-row correction vectors
+ * sum_k W'[r, k] and sum_k beta[k] W[r, k] + bias[r] in fp32 (the folding of
+ * "Triangle multiplication on SM90"); for the fp32 path it keeps fp32 copies.
+ * Runs on `stream` and synchronizes it before returning, so the caller may free
+ * the source weights afterwards. Supported (c_z, c_h): any multiple of 32 up to
+ * 512 for the fp32 path; (128, 128) and (384, 128) for the bf16 path (checked
+ * at forward time). */
+trimul_status_t tri_mul_layer_create(const trimul_weights_desc_t *weights, void *stream,
+                                     trimul_layer_t **layer_out);
+
+/* Free the handle and its device memory. NULL is ignored. */
+void tri_mul_layer_destroy(trimul_layer_t *layer);
+
+/* Bytes of workspace tri_mul_forward needs for B x N x N with compute type
+ * `dtype` (the dtype of z): a, b and x, each [B, c_h, N, N] of that type,
+ * 256-byte aligned. Returns 0 for an invalid layer or size. */
+size_t tri_mul_workspace_bytes(const trimul_layer_t *layer, int64_t B, int64_t N,
+                               trimul_dtype_t dtype);
+
+/* Attach caller-owned device workspace to the handle (replaces any earlier one).
+ * The handle does not own it. Two forwards that run concurrently on different
+ * streams must use different handles (or different workspaces). */
+trimul_status_t tri_mul_layer_bind_workspace(trimul_layer_t *layer, void *workspace,
+                                             size_t bytes);
+
+/* One triangle multiplicative update (one direction). Returns the update only;
+ * the residual add z += update is the caller's.
+ *   z    : [B, N, N, c_z], dtype F32 (fp32 SIMT path) or BF16 (tensor-core path)
+ *   mask : [B, N, N] in z's dtype with values 0 or 1, or NULL for all ones
+ *   out  : [B, N, N, c_z]; F32 for the F32 path; F32 or BF16 for the BF16 path
+ *          (must not overlap z or the workspace)
+ * Requirements: N % 8 == 0 and N >= 8 (the pages pad token axes to multiples
+ * of 8); B >= 1; every pointer 16-byte aligned; a workspace of at least
+ * tri_mul_workspace_bytes() bound. The BF16 path needs an sm_100 device. */
+trimul_status_t tri_mul_forward(const trimul_pair_t *z, const void *mask,
+                                const trimul_layer_t *layer, trimul_direction_t direction,
+                                trimul_pair_t *out, void *stream);
+
+/* Step K1 alone ("x_x" input gate): a and b from z, written channel-major
+ * [B, c_h, N, N] in z's dtype. Same requirements as tri_mul_forward. */
+trimul_status_t tri_mul_project(const trimul_pair_t *z, const void *mask,
+                                const trimul_layer_t *layer, void *a_out, void *b_out,
+                                void *stream);
+
+/* Step K2 alone (the contraction): x from a and b, all [B, C, N, N] of `dtype`.
+ *   outgoing: x[b,c,i,j] = sum_k a[b,c,i,k] b[b,c,j,k]
+ *   incoming: x[b,c,i,j] = sum_k a[b,c,k,i] b[b,c,k,j]
+ * BF16: fp32 accumulation, bf16 result, C any positive value. F32: fp32 FMA.
+ * N % 8 == 0. x must not overlap a or b. */
+trimul_status_t tri_mul_contract(const void *a, const void *b, void *x, int64_t B, int64_t C,
+                                 int64_t N, trimul_dtype_t dtype, trimul_direction_t direction,
+                                 void *stream);
+
+/* Step K3 alone ("x0_x1" output gate): out from z, the mask and x [B, c_h, N, N]
+ * (x in z's dtype). Same requirements as tri_mul_forward. */
+trimul_status_t tri_mul_output_gate(const trimul_pair_t *z, const void *mask, const void *x,
+                                    const trimul_layer_t *layer, trimul_pair_t *out,
+                                    void *stream);
+
+/* Optional per-kernel timing: when `events` is non-NULL, every later
+ * tri_mul_forward on this handle records events[0] before K1, events[1] after
+ * K1, events[2] after K2 and events[3] after K3 on its stream. The four values
+ * are cudaEvent_t created by the caller; NULL switches recording off. */
+trimul_status_t tri_mul_layer_set_timing_events(trimul_layer_t *layer, void *const *events);
+
+/* Number of kernels one tri_mul_forward launches (for launch accounting). */
+int tri_mul_kernels_per_forward(void);
+
+/* Synchronize the current device, then read and clear the library's device
+ * error word. Every wait inside the bf16 kernels is bounded (about one second);
+ * a wait that runs out makes its kernel stop early, and this call reports
+ * TRIMUL_ERR_DEVICE_TIMEOUT. Outputs of such a launch are undefined. */
+trimul_status_t tri_mul_check_device_status(void);
+
+/* Static description of a status code. */
+const char *tri_mul_status_string(trimul_status_t status);
+
+/* Detail of the last error raised on the calling thread ("" if none). */
+const char *tri_mul_last_error(void);
+
+/* ABI version of this header (major * 100 + minor). */
+int tri_mul_abi_version(void);
+
+#define TRIMUL_ABI_VERSION 100
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* TRIMUL_H */

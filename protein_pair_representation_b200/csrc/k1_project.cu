@@ -1,0 +1,312 @@
+// k1_project.cu -- K1, the input LayerNorm + gated projection on tensor cores (sm_100a).
+//
+// Computes, for every pair p = (b, i, j) and hidden channel c,
+//   a[b, c, i, j] = m_p * sigmoid(zhat_p . W_ag[c] + b_ag[c]) * (zhat_p . W_ap[c] + b_ap[c])
+// and b likewise, with zhat_p = LayerNorm(z_p) ("RFProteina architecture", section
+// "Dual-GEMM gates": the one-input gate that reads the normalized pair tensor,
+// applies the mask and emits its output transposed for the contraction; section
+// "Triangle multiplication on SM90": K1 with the input LayerNorm folded into its
+// weights).
+//
+// LayerNorm folding: with W' = W * gamma (per input column, rounded to bf16),
+//   zhat . W = rstd_p * (z_p . W' - mean_p * sum_k W'_k) + (sum_k beta_k W_k + bias)
+// so the tensor cores multiply the raw bf16 z tile, and the epilogue applies the
+// per-pair (mean, rstd) and the per-channel (sum W', shift) pair of constants.
+//
+// Tile: 128 consecutive pairs of one batch element (one TMEM lane per pair) times
+// NCOL packed weight rows. Packed row layout inside a group: 32-row blocks, each
+// [16 gate rows, 16 projection rows] for 16 channels, so one 32-column TMEM load
+// gives a thread both factors of 16 outputs. c_z = 128 uses NCOL = 256 (one group
+// per operand); c_z = 384 uses NCOL = 128 (two groups per operand) so that the
+// group's weights stay resident in shared memory. A CTA keeps one group for its
+// whole life (grid is a multiple of the group count).
+//
+// Warps: 0-7 epilogue (two warpgroups, half the columns each), 8-11 LayerNorm
+// statistics (one thread per pair), 12 TMA producer, 13 TMEM allocator + MMA issuer.
+#include "kernels.h"
+#include "sm100.cuh"
+
+namespace trimul {
+
+template <int CZ>
+struct K1Cfg {
+    static constexpr int C_H = kHidden;
+    static constexpr int NCOL = (CZ == 128) ? 256 : 128;
+    static constexpr int KC = CZ / 64;                 // 64-channel chunks of z per tile
+    static constexpr int CPG = NCOL / 2;               // output channels per group
+    static constexpr int G = 4 * C_H / NCOL;           // groups
+    static constexpr int GPO = G / 2;                  // groups per operand
+    static constexpr int NB = 512 / NCOL;              // TMEM accumulator buffers
+    static constexpr int CH_WG = CPG / 2;              // channels per epilogue warpgroup
+    static constexpr int BLK_WG = CH_WG / 16;          // 32-column blocks per warpgroup
+    static constexpr int W_BYTES = NCOL * CZ * 2;
+    static constexpr int CHUNK = 128 * 64 * 2;         // one z chunk: 128 pairs x 64 channels
+    static constexpr int STG_BYTES = CH_WG * 128 * 2;  // per warpgroup: [channels][128 pairs] bf16
+    static constexpr int SNB = 2;                      // stats ring depth
+    static constexpr int FIXED = 1024 + W_BYTES + 2 * STG_BYTES + SNB * 128 * 16 + 1024;
+    static constexpr int S = (232448 - FIXED) / CHUNK > 8 ? 8 : (232448 - FIXED) / CHUNK;
+    static constexpr size_t SMEM = FIXED + (size_t)S * CHUNK;
+    static constexpr int THREADS = 448;
+    static constexpr int TMA_WARP = 12, MMA_WARP = 13;
+};
+
+struct K1Smem {
+    uint64_t wbar;
+    uint64_t full[8], empty[8];
+    uint64_t tfull[4], tempty[4];
+    uint64_t sfull[2], sempty[2];
+    uint64_t drain;
+    uint32_t tmem_base;
+    int abort_flag;
+};
+
+template <int CZ>
+__global__ void __launch_bounds__(448, 1) k1_project_kernel(const __grid_constant__ K1Args p) {
+    using C = K1Cfg<CZ>;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *base = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint8_t *w_s = base;                                   // KC chunks of [NCOL][64] bf16
+    uint8_t *chunks = w_s + C::W_BYTES;                    // S chunks of [128][64] bf16
+    uint8_t *staging = chunks + C::S * C::CHUNK;           // 2 x [CH_WG][128] bf16
+    float4 *stats = reinterpret_cast<float4 *>(staging + 2 * C::STG_BYTES);  // [SNB][128]
+    K1Smem &s = *reinterpret_cast<K1Smem *>(stats + C::SNB * 128);
+
+    const int warp = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31;
+    volatile int *abort_flag = &s.abort_flag;
+
+    const int group = blockIdx.x % C::G;
+    const int cta_in_group = blockIdx.x / C::G;
+    const int ctas_per_group = gridDim.x / C::G;
+    const int num_ptiles = p.B * p.tiles_per_batch;
+    const int operand = group / C::GPO;
+    const int ch0 = (group % C::GPO) * C::CPG;
+
+    if (threadIdx.x == 0) {
+        mbar_init(&s.wbar, 1);
+        for (int i = 0; i < C::S; ++i) {
+            mbar_init(&s.full[i], 1);
+            mbar_init(&s.empty[i], 1 + 4);  // MMA commit + 4 stats warps
+        }
+        for (int i = 0; i < C::NB; ++i) {
+            mbar_init(&s.tfull[i], 1);
+            mbar_init(&s.tempty[i], 8);
+        }
+        for (int i = 0; i < C::SNB; ++i) {
+            mbar_init(&s.sfull[i], 4);
+            mbar_init(&s.sempty[i], 8);
+        }
+        mbar_init(&s.drain, 1);
+        s.abort_flag = 0;
+        fence_mbarrier_init();
+    }
+    if (warp == C::MMA_WARP) {
+        tmem_alloc(&s.tmem_base, 512);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem_base = s.tmem_base;
+
+    if (warp == C::TMA_WARP) {
+        if (lane == 0) {
+            tma_prefetch_desc(&p.tm_z);
+            tma_prefetch_desc(&p.tm_w);
+            // resident weights of this CTA's group
+            mbar_arrive_expect_tx(&s.wbar, C::W_BYTES);
+            for (int kc = 0; kc < C::KC; ++kc)
+                tma_load_2d(w_s + kc * C::NCOL * 128, &p.tm_w, &s.wbar, kc * 64, group * C::NCOL);
+            int stage = 0;
+            uint32_t phase = 0;
+            uint32_t filled = 0;
+            for (int pt = cta_in_group; pt < num_ptiles; pt += ctas_per_group) {
+                const int b = pt / p.tiles_per_batch;
+                const int p0 = (pt - b * p.tiles_per_batch) * 128;
+                for (int kc = 0; kc < C::KC; ++kc) {
+                    if (!mbar_wait(&s.empty[stage], phase ^ 1, abort_flag, kErrTimeoutProducer)) goto producer_abort;
+                    mbar_arrive_expect_tx(&s.full[stage], C::CHUNK);
+                    tma_load_3d(chunks + stage * C::CHUNK, &p.tm_z, &s.full[stage], kc * 64, p0, b);
+                    ++filled;
+                    if (++stage == C::S) { stage = 0; phase ^= 1; }
+                }
+            }
+            goto producer_done;
+        producer_abort:
+            for (uint32_t i = 0; i < (filled < (uint32_t)C::S ? filled : (uint32_t)C::S); ++i) {
+                uint32_t f = filled - 1 - i;
+                mbar_drain(&s.full[f % C::S], (f / C::S) & 1);
+            }
+        producer_done:
+            mbar_drain(&s.wbar, 0);
+        }
+    } else if (warp == C::MMA_WARP) {
+        if (lane == 0) {
+            const uint32_t idesc = idesc_bf16_f32(128, C::NCOL, false, false);
+            bool ok = mbar_wait(&s.wbar, 0, abort_flag, kErrTimeoutMma);
+            int stage = 0;
+            uint32_t phase = 0;
+            int abuf = 0;
+            uint32_t aphase = 0;
+            for (int pt = cta_in_group; ok && pt < num_ptiles; pt += ctas_per_group) {
+                if (!mbar_wait(&s.tempty[abuf], aphase ^ 1, abort_flag, kErrTimeoutMma)) break;
+                tc_fence_after();
+                const uint32_t d_tmem = tmem_base + abuf * C::NCOL;
+                for (int kc = 0; kc < C::KC; ++kc) {
+                    if (!mbar_wait(&s.full[stage], phase, abort_flag, kErrTimeoutMma)) { ok = false; break; }
+                    tc_fence_after();
+                    const uint8_t *za = chunks + stage * C::CHUNK;
+                    const uint8_t *wb = w_s + kc * C::NCOL * 128;
+#pragma unroll
+                    for (int kk = 0; kk < 4; ++kk) {
+                        uint64_t ad = smem_desc_sw128(za + kk * 32, 16, 1024);
+                        uint64_t bd = smem_desc_sw128(wb + kk * 32, 16, 1024);
+                        tc_mma_bf16(d_tmem, ad, bd, idesc, (kc | kk) != 0);
+                    }
+                    tc_commit(&s.empty[stage]);
+                    if (++stage == C::S) { stage = 0; phase ^= 1; }
+                }
+                if (!ok) break;
+                tc_commit(&s.tfull[abuf]);
+                if (++abuf == C::NB) { abuf = 0; aphase ^= 1; }
+            }
+            tc_commit(&s.drain);
+            mbar_drain(&s.drain, 0);
+        }
+    } else if (warp >= 8) {
+        // LayerNorm statistics: thread = pair row of the tile
+        const int row = (warp - 8) * 32 + lane;
+        int stage = 0;
+        uint32_t phase = 0;
+        int sbuf = 0;
+        uint32_t sphase = 0;
+        for (int pt = cta_in_group; pt < num_ptiles; pt += ctas_per_group) {
+            const int b = pt / p.tiles_per_batch;
+            const int p0 = (pt - b * p.tiles_per_batch) * 128;
+            float shift = 0.f, s1 = 0.f, s2 = 0.f;
+            bool ok = true;
+            for (int kc = 0; kc < C::KC; ++kc) {
+                if (!__all_sync(0xffffffffu, mbar_wait(&s.full[stage], phase, abort_flag, kErrTimeoutEpilogue))) { ok = false; break; }
+                const uint8_t *zc = chunks + stage * C::CHUNK;
+#pragma unroll
+                for (int u = 0; u < 8; ++u) {
+                    uint4 w = *reinterpret_cast<const uint4 *>(zc + sw128_offset(row, u));
+                    float v[8] = {bf16_lo(w.x), bf16_hi(w.x), bf16_lo(w.y), bf16_hi(w.y),
+                                  bf16_lo(w.z), bf16_hi(w.z), bf16_lo(w.w), bf16_hi(w.w)};
+                    if (kc == 0 && u == 0) shift = v[0];
+#pragma unroll
+                    for (int e = 0; e < 8; ++e) {
+                        float d = v[e] - shift;
+                        s1 += d;
+                        s2 = fmaf(d, d, s2);
+                    }
+                }
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&s.empty[stage]);
+                if (++stage == C::S) { stage = 0; phase ^= 1; }
+            }
+            if (!ok) break;
+            const float inv_n = 1.0f / (float)CZ;
+            const float dm = s1 * inv_n;
+            const float var = fmaxf(s2 * inv_n - dm * dm, 0.f);
+            const float mean = shift + dm;
+            const float rstd = rsqrtf(var + p.eps);
+            const long long pi = (long long)p0 + row;
+            float m = 1.f;
+            if (p.mask) m = (pi < p.NN) ? __uint_as_float((uint32_t)p.mask[(long long)b * p.NN + pi] << 16) : 0.f;
+            if (!__all_sync(0xffffffffu, mbar_wait(&s.sempty[sbuf], sphase ^ 1, abort_flag, kErrTimeoutEpilogue))) break;
+            stats[sbuf * 128 + row] = make_float4(mean, rstd, m, 0.f);
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&s.sfull[sbuf]);
+            if (++sbuf == C::SNB) { sbuf = 0; sphase ^= 1; }
+        }
+    } else {
+        // epilogue: warpgroup wg handles channels [ch0 + wg*CH_WG, +CH_WG)
+        const int wg = warp >> 2;
+        const int q = warp & 3;
+        const int row = q * 32 + lane;
+        uint16_t *stg = reinterpret_cast<uint16_t *>(staging + wg * C::STG_BYTES);
+        const bool leader = (threadIdx.x & 127) == 0;
+        const CUtensorMap *tm_out = operand == 0 ? &p.tm_a : &p.tm_b;
+        const float4 *vec = p.vec + operand * C::C_H + ch0 + wg * C::CH_WG;
+        int abuf = 0;
+        uint32_t aphase = 0;
+        int sbuf = 0;
+        uint32_t sphase = 0;
+        for (int pt = cta_in_group; pt < num_ptiles; pt += ctas_per_group) {
+            const int b = pt / p.tiles_per_batch;
+            const int p0 = (pt - b * p.tiles_per_batch) * 128;
+            if (!group_all(mbar_wait(&s.sfull[sbuf], sphase, abort_flag, kErrTimeoutEpilogue), 1 + wg, 128)) break;
+            const float4 st = stats[sbuf * 128 + row];
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&s.sempty[sbuf]);
+            if (++sbuf == C::SNB) { sbuf = 0; sphase ^= 1; }
+            const float mean = st.x, rstd = st.y, m = st.z;
+
+            if (!group_all(mbar_wait(&s.tfull[abuf], aphase, abort_flag, kErrTimeoutEpilogue), 1 + wg, 128)) break;
+            tc_fence_after();
+            if (leader) tma_store_wait_read<0>();
+            named_bar_sync(1 + wg, 128);
+#pragma unroll 1
+            for (int blk = 0; blk < C::BLK_WG; ++blk) {
+                float v[32];
+                tmem_ld32(tmem_base + abuf * C::NCOL + ((uint32_t)(q * 32) << 16) + (wg * C::BLK_WG + blk) * 32, v);
+                tc_wait_ld();
+#pragma unroll
+                for (int e = 0; e < 16; ++e) {
+                    const float4 cv = __ldg(&vec[blk * 16 + e]);
+                    const float g = fmaf(rstd, fmaf(-mean, cv.x, v[e]), cv.y);
+                    const float pr = fmaf(rstd, fmaf(-mean, cv.z, v[16 + e]), cv.w);
+                    const float out = sigmoid_tanh(g) * pr * m;
+                    stg[(blk * 16 + e) * 128 + row] = __bfloat16_as_ushort(__float2bfloat16_rn(out));
+                }
+            }
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&s.tempty[abuf]);
+            if (++abuf == C::NB) { abuf = 0; aphase ^= 1; }
+            fence_proxy_async_smem();
+            named_bar_sync(1 + wg, 128);
+            if (leader) {
+                tma_store_3d(tm_out, stg, p0, ch0 + wg * C::CH_WG, b);
+                tma_store_commit();
+            }
+        }
+        if (leader) tma_store_wait_all<0>();
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    if (warp == C::MMA_WARP) {
+        tc_fence_after();
+        tmem_dealloc(tmem_base, 512);
+    }
+}
+
+int k1_ncol(int c_z) { return c_z == 128 ? K1Cfg<128>::NCOL : K1Cfg<384>::NCOL; }
+int k1_groups(int c_z) { return c_z == 128 ? K1Cfg<128>::G : K1Cfg<384>::G; }
+int k1_channels_per_warpgroup(int c_z) { return c_z == 128 ? K1Cfg<128>::CH_WG : K1Cfg<384>::CH_WG; }
+size_t k1_smem_bytes(int c_z) { return c_z == 128 ? K1Cfg<128>::SMEM : K1Cfg<384>::SMEM; }
+
+template <int CZ>
+static cudaError_t k1_launch_t(const K1Args &args, int grid, cudaStream_t stream) {
+    static int configured_device = -1;
+    int dev = 0;
+    cudaGetDevice(&dev);
+    if (configured_device != dev) {
+        cudaError_t e = cudaFuncSetAttribute(k1_project_kernel<CZ>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                             (int)K1Cfg<CZ>::SMEM);
+        if (e != cudaSuccess) return e;
+        configured_device = dev;
+    }
+    k1_project_kernel<CZ><<<grid, K1Cfg<CZ>::THREADS, K1Cfg<CZ>::SMEM, stream>>>(args);
+    return cudaGetLastError();
+}
+
+cudaError_t k1_launch(int c_z, const K1Args &args, int grid, cudaStream_t stream) {
+    if (c_z == 128) return k1_launch_t<128>(args, grid, stream);
+    if (c_z == 384) return k1_launch_t<384>(args, grid, stream);
+    return cudaErrorInvalidValue;
+}
+
+}  // namespace trimul

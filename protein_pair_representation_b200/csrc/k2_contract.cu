@@ -1,0 +1,243 @@
+// k2_contract.cu -- K2, the triangle contraction on tensor cores (sm_100a).
+//
+// For every (batch, channel) c the contraction is one N x N x N matrix product
+// ("RFProteina architecture", section "Triangle multiplication on SM90": K2 runs
+// the contraction itself, one direction at a time):
+//   outgoing  X_c = A_c B_c^T   (x_ij = sum_k a_ik b_jk; both operands K-major)
+//   incoming  X_c = A_c^T B_c   (x_ij = sum_k a_ki b_kj; both operands MN-major)
+// a, b, x are [B*c_h][N][N] bf16. The two directions differ only in the TMA boxes
+// and in the major-ness bits of the shared-memory descriptors.
+//
+// Persistent kernel, one CTA per SM, 128 x 256 output tiles, 64-deep k chunks:
+//   warp 8      TMA producer (one elected lane) filling a 4-stage ring
+//   warp 9      TMEM allocator and MMA issuer (tcgen05.mma, fp32 accumulators in
+//               two 256-column TMEM buffers so the epilogue of tile t overlaps
+//               the MMAs of tile t+1)
+//   warps 0-7   epilogue: two warpgroups, each drains 128 of the 256 columns
+//               (tcgen05.ld), rounds to bf16, stages through 128B-swizzled shared
+//               memory and writes with TMA stores.
+#include "kernels.h"
+#include "sm100.cuh"
+
+namespace trimul {
+
+namespace k2 {
+constexpr int BM = 128, BN = 256, BK = 64;
+constexpr int STAGES = 4;
+constexpr int A_BYTES = BM * BK * 2;               // 16 KB
+constexpr int B_BYTES = BN * BK * 2;               // 32 KB
+constexpr int STAGE_BYTES = A_BYTES + B_BYTES;     // 48 KB
+constexpr int STG_BYTES = BM * 64 * 2;             // 16 KB: 128 rows x 64 bf16
+constexpr int EPI_WARPS = 8;
+constexpr int TMA_WARP = 8, MMA_WARP = 9;
+constexpr int THREADS = 320;
+constexpr int TMEM_COLS = 512;
+
+struct Smem {
+    uint64_t full[STAGES], empty[STAGES];
+    uint64_t tfull[2], tempty[2];
+    uint64_t drain;
+    uint32_t tmem_base;
+    int abort_flag;
+};
+constexpr size_t SMEM_BYTES = 1024 /*align*/ + STAGES * STAGE_BYTES + 2 * STG_BYTES + 1024;
+}  // namespace k2
+
+__global__ void __launch_bounds__(k2::THREADS, 1) k2_contract_kernel(const __grid_constant__ K2Args p) {
+    using namespace k2;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *base = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint8_t *stages = base;
+    uint8_t *staging = base + STAGES * STAGE_BYTES;
+    Smem &s = *reinterpret_cast<Smem *>(staging + 2 * STG_BYTES);
+
+    const int warp = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31;
+    volatile int *abort_flag = &s.abort_flag;
+
+    if (threadIdx.x == 0) {
+        for (int i = 0; i < STAGES; ++i) {
+            mbar_init(&s.full[i], 1);
+            mbar_init(&s.empty[i], 1);
+        }
+        for (int i = 0; i < 2; ++i) {
+            mbar_init(&s.tfull[i], 1);
+            mbar_init(&s.tempty[i], EPI_WARPS);
+        }
+        mbar_init(&s.drain, 1);
+        s.abort_flag = 0;
+        fence_mbarrier_init();
+    }
+    if (warp == TMA_WARP && lane == 0) {
+        tma_prefetch_desc(&p.tm_a);
+        tma_prefetch_desc(&p.tm_b);
+        tma_prefetch_desc(&p.tm_x);
+    }
+    if (warp == MMA_WARP) {
+        tmem_alloc(&s.tmem_base, TMEM_COLS);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem_base = s.tmem_base;
+
+    const int tiles_per_channel = p.m_tiles * p.n_tiles;
+    const int num_tiles = p.BC * tiles_per_channel;
+
+    if (warp == TMA_WARP) {
+        if (lane == 0) {
+            int stage = 0;
+            uint32_t phase = 0;
+            uint32_t filled = 0;  // number of stage fills issued (for the abort drain)
+            for (int t = blockIdx.x; t < num_tiles; t += gridDim.x) {
+                const int bc = t / tiles_per_channel;
+                const int r = t - bc * tiles_per_channel;
+                const int m0 = (r / p.n_tiles) * BM;
+                const int n0 = (r % p.n_tiles) * BN;
+                for (int kc = 0; kc < p.k_chunks; ++kc) {
+                    if (!mbar_wait(&s.empty[stage], phase ^ 1, abort_flag, kErrTimeoutProducer)) goto producer_abort;
+                    uint8_t *sa = stages + stage * STAGE_BYTES;
+                    uint8_t *sb = sa + A_BYTES;
+                    mbar_arrive_expect_tx(&s.full[stage], STAGE_BYTES);
+                    const int k0 = kc * BK;
+                    if (!p.incoming) {
+                        tma_load_3d(sa, &p.tm_a, &s.full[stage], k0, m0, bc);
+                        tma_load_3d(sb, &p.tm_b, &s.full[stage], k0, n0, bc);
+                    } else {
+#pragma unroll
+                        for (int h = 0; h < BM / 64; ++h)
+                            tma_load_3d(sa + h * 8192, &p.tm_a, &s.full[stage], m0 + 64 * h, k0, bc);
+#pragma unroll
+                        for (int h = 0; h < BN / 64; ++h)
+                            tma_load_3d(sb + h * 8192, &p.tm_b, &s.full[stage], n0 + 64 * h, k0, bc);
+                    }
+                    ++filled;
+                    if (++stage == STAGES) { stage = 0; phase ^= 1; }
+                }
+            }
+            goto producer_done;
+        producer_abort:
+            // let the copies already issued land before the CTA exits
+            for (uint32_t i = 0; i < (filled < (uint32_t)STAGES ? filled : (uint32_t)STAGES); ++i) {
+                uint32_t f = filled - 1 - i;
+                mbar_drain(&s.full[f % STAGES], (f / STAGES) & 1);
+            }
+        producer_done:;
+        }
+    } else if (warp == MMA_WARP) {
+        if (lane == 0) {
+            const uint32_t idesc = idesc_bf16_f32(BM, BN, p.incoming, p.incoming);
+            int stage = 0;
+            uint32_t phase = 0;
+            int abuf = 0;
+            uint32_t aphase = 0;
+            for (int t = blockIdx.x; t < num_tiles; t += gridDim.x) {
+                if (!mbar_wait(&s.tempty[abuf], aphase ^ 1, abort_flag, kErrTimeoutMma)) break;
+                tc_fence_after();
+                const uint32_t d_tmem = tmem_base + abuf * BN;
+                bool ok = true;
+                for (int kc = 0; kc < p.k_chunks; ++kc) {
+                    if (!mbar_wait(&s.full[stage], phase, abort_flag, kErrTimeoutMma)) { ok = false; break; }
+                    tc_fence_after();
+                    const uint8_t *sa = stages + stage * STAGE_BYTES;
+                    const uint8_t *sb = sa + A_BYTES;
+#pragma unroll
+                    for (int kk = 0; kk < BK / 16; ++kk) {
+                        uint64_t ad, bd;
+                        if (!p.incoming) {
+                            ad = smem_desc_sw128(sa + kk * 32, 16, 1024);
+                            bd = smem_desc_sw128(sb + kk * 32, 16, 1024);
+                        } else {
+                            ad = smem_desc_sw128(sa + kk * 2048, 8192, 1024);
+                            bd = smem_desc_sw128(sb + kk * 2048, 8192, 1024);
+                        }
+                        tc_mma_bf16(d_tmem, ad, bd, idesc, (kc | kk) != 0);
+                    }
+                    tc_commit(&s.empty[stage]);
+                    if (++stage == STAGES) { stage = 0; phase ^= 1; }
+                }
+                if (!ok) break;
+                tc_commit(&s.tfull[abuf]);
+                if (++abuf == 2) { abuf = 0; aphase ^= 1; }
+            }
+            // all MMAs issued by this thread are complete once this arrives
+            tc_commit(&s.drain);
+            mbar_drain(&s.drain, 0);
+        }
+    } else {
+        // epilogue warpgroups
+        const int wg = warp >> 2;            // 0 or 1: which 128 columns
+        const int q = warp & 3;              // TMEM lane quarter
+        const int row = q * 32 + lane;       // accumulator row = output row within the tile
+        uint8_t *stg = staging + wg * STG_BYTES;
+        const bool leader = (threadIdx.x & 127) == 0;
+        int abuf = 0;
+        uint32_t aphase = 0;
+        for (int t = blockIdx.x; t < num_tiles; t += gridDim.x) {
+            const int bc = t / tiles_per_channel;
+            const int r = t - bc * tiles_per_channel;
+            const int m0 = (r / p.n_tiles) * BM;
+            const int n0 = (r % p.n_tiles) * BN;
+            if (!group_all(mbar_wait(&s.tfull[abuf], aphase, abort_flag, kErrTimeoutEpilogue), 1 + wg, 128)) break;
+            tc_fence_after();
+#pragma unroll 1
+            for (int sub = 0; sub < 2; ++sub) {
+                if (leader) tma_store_wait_read<0>();
+                named_bar_sync(1 + wg, 128);
+#pragma unroll
+                for (int half = 0; half < 2; ++half) {
+                    const int col = wg * 128 + sub * 64 + half * 32;
+                    float v[32];
+                    tmem_ld32(tmem_base + abuf * BN + ((uint32_t)(q * 32) << 16) + col, v);
+                    tc_wait_ld();
+#pragma unroll
+                    for (int u = 0; u < 4; ++u) {
+                        uint4 w;
+                        w.x = pack_bf16x2(v[8 * u + 0], v[8 * u + 1]);
+                        w.y = pack_bf16x2(v[8 * u + 2], v[8 * u + 3]);
+                        w.z = pack_bf16x2(v[8 * u + 4], v[8 * u + 5]);
+                        w.w = pack_bf16x2(v[8 * u + 6], v[8 * u + 7]);
+                        *reinterpret_cast<uint4 *>(stg + sw128_offset(row, half * 4 + u)) = w;
+                    }
+                }
+                fence_proxy_async_smem();
+                named_bar_sync(1 + wg, 128);
+                if (leader) {
+                    tma_store_3d(&p.tm_x, stg, n0 + wg * 128 + sub * 64, m0, bc);
+                    tma_store_commit();
+                }
+            }
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&s.tempty[abuf]);
+            if (++abuf == 2) { abuf = 0; aphase ^= 1; }
+        }
+        if (leader) tma_store_wait_all<0>();
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    if (warp == MMA_WARP) {
+        tc_fence_after();
+        tmem_dealloc(tmem_base, TMEM_COLS);
+    }
+}
+
+size_t k2_smem_bytes() { return k2::SMEM_BYTES; }
+
+cudaError_t k2_launch(const K2Args &args, int grid, cudaStream_t stream) {
+    static int configured_device = -1;
+    int dev = 0;
+    cudaGetDevice(&dev);
+    if (configured_device != dev) {
+        cudaError_t e = cudaFuncSetAttribute(k2_contract_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                             (int)k2::SMEM_BYTES);
+        if (e != cudaSuccess) return e;
+        configured_device = dev;
+    }
+    k2_contract_kernel<<<grid, k2::THREADS, k2::SMEM_BYTES, stream>>>(args);
+    return cudaGetLastError();
+}
+
+}  // namespace trimul

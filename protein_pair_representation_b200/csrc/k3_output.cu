@@ -1,0 +1,374 @@
+// k3_output.cu -- K3, the output LayerNorm + gated output projection on tensor cores.
+//
+// For every pair p and output channel n:
+//   out[p, n] = m_p * sigmoid(zhat_p . W_g[n] + b_g[n]) * (LN(x_p) . W_o[n] + b_o[n])
+// with zhat_p = LayerNorm_{c_z}(z_p) and LN(x_p) the LayerNorm over the c_h channels of
+// the contracted x ("RFProteina architecture", section "Dual-GEMM gates": the two-input
+// gate with x0 the normalized input pair tensor and x1 the contracted hidden tensor;
+// section "Triangle multiplication on SM90": K3 with both LayerNorms folded into its
+// weights). Both norms are folded as in K1:
+//   x . W_o' -> rstd_x (acc1 - mean_x sum W_o') + shift_o, with W_o' = W_o * gamma_out
+//   z . W_g' -> rstd_z (acc2 - mean_z sum W_g') + shift_g, with W_g' = W_g * gamma_in
+//
+// Tile: 128 consecutive pairs (one TMEM lane each) times 128 output channels. x arrives
+// channel-major ([c_h][pairs], pairs contiguous) and is the MN-major A operand of the
+// first GEMM; z is channel-last and the K-major A operand of the second. c_z = 384 uses
+// three column groups (a CTA keeps one group) so each group's weights stay resident.
+//
+// Warps: 0-7 epilogue (two warpgroups, 64 output channels each), 8-11 LayerNorm
+// statistics of x and z (one thread per pair), 12 TMA producer, 13 TMEM + MMA.
+#include "kernels.h"
+#include "sm100.cuh"
+
+namespace trimul {
+
+template <int CZ, bool OUT_F32>
+struct K3Cfg {
+    static constexpr int C_H = kHidden;
+    static constexpr int NCOL = 128;                 // output channels per group
+    static constexpr int G = CZ / NCOL;
+    static constexpr int XC = C_H / 64;              // x chunks per tile (64 channels each)
+    static constexpr int ZC = CZ / 64;               // z chunks per tile
+    static constexpr int CPT = XC + ZC;              // chunks per tile
+    static constexpr int WO_BYTES = NCOL * C_H * 2;
+    static constexpr int WG_BYTES = NCOL * CZ * 2;
+    static constexpr int CHUNK = 128 * 64 * 2;
+    static constexpr int STG_BYTES = 128 * 128;      // per warpgroup: 128 rows x 128 bytes
+    static constexpr int COLS_PER_STORE = OUT_F32 ? 32 : 64;
+    static constexpr int SNB = 2;
+    static constexpr int FIXED = 1024 + WO_BYTES + WG_BYTES + 2 * STG_BYTES + SNB * 128 * 32 + 1024;
+    static constexpr int S = (232448 - FIXED) / CHUNK > 8 ? 8 : (232448 - FIXED) / CHUNK;
+    static constexpr size_t SMEM = FIXED + (size_t)S * CHUNK;
+    static constexpr int THREADS = 448;
+    static constexpr int TMA_WARP = 12, MMA_WARP = 13;
+};
+
+struct K3Smem {
+    uint64_t wbar;
+    uint64_t full[8], empty[8];
+    uint64_t tfull[2], tempty[2];
+    uint64_t sfull[2], sempty[2];
+    uint64_t drain;
+    uint32_t tmem_base;
+    int abort_flag;
+};
+
+struct K3Stats {
+    float mean_z, rstd_z, mean_x, rstd_x, mask, pad0, pad1, pad2;
+};
+
+template <int CZ, bool OUT_F32>
+__global__ void __launch_bounds__(448, 1) k3_output_kernel(const __grid_constant__ K3Args p) {
+    using C = K3Cfg<CZ, OUT_F32>;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *base = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint8_t *wo_s = base;                              // XC chunks of [128 rows][64] bf16
+    uint8_t *wg_s = wo_s + C::WO_BYTES;                // ZC chunks of [128 rows][64] bf16
+    uint8_t *chunks = wg_s + C::WG_BYTES;              // S chunks
+    uint8_t *staging = chunks + C::S * C::CHUNK;       // 2 x 16 KB
+    K3Stats *stats = reinterpret_cast<K3Stats *>(staging + 2 * C::STG_BYTES);
+    K3Smem &s = *reinterpret_cast<K3Smem *>(stats + C::SNB * 128);
+
+    const int warp = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31;
+    volatile int *abort_flag = &s.abort_flag;
+
+    const int group = blockIdx.x % C::G;
+    const int cta_in_group = blockIdx.x / C::G;
+    const int ctas_per_group = gridDim.x / C::G;
+    const int num_ptiles = p.B * p.tiles_per_batch;
+    const int n0 = group * C::NCOL;
+
+    if (threadIdx.x == 0) {
+        mbar_init(&s.wbar, 1);
+        for (int i = 0; i < C::S; ++i) {
+            mbar_init(&s.full[i], 1);
+            mbar_init(&s.empty[i], 1 + 4);
+        }
+        for (int i = 0; i < 2; ++i) {
+            mbar_init(&s.tfull[i], 1);
+            mbar_init(&s.tempty[i], 8);
+        }
+        for (int i = 0; i < C::SNB; ++i) {
+            mbar_init(&s.sfull[i], 4);
+            mbar_init(&s.sempty[i], 8);
+        }
+        mbar_init(&s.drain, 1);
+        s.abort_flag = 0;
+        fence_mbarrier_init();
+    }
+    if (warp == C::MMA_WARP) {
+        tmem_alloc(&s.tmem_base, 512);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem_base = s.tmem_base;
+
+    if (warp == C::TMA_WARP) {
+        if (lane == 0) {
+            tma_prefetch_desc(&p.tm_x);
+            tma_prefetch_desc(&p.tm_z);
+            mbar_arrive_expect_tx(&s.wbar, C::WO_BYTES + C::WG_BYTES);
+            for (int c = 0; c < C::XC; ++c)
+                tma_load_2d(wo_s + c * C::NCOL * 128, &p.tm_wo, &s.wbar, c * 64, n0);
+            for (int c = 0; c < C::ZC; ++c)
+                tma_load_2d(wg_s + c * C::NCOL * 128, &p.tm_wg, &s.wbar, c * 64, n0);
+            int stage = 0;
+            uint32_t phase = 0;
+            uint32_t filled = 0;
+            for (int pt = cta_in_group; pt < num_ptiles; pt += ctas_per_group) {
+                const int b = pt / p.tiles_per_batch;
+                const int p0 = (pt - b * p.tiles_per_batch) * 128;
+                for (int c = 0; c < C::CPT; ++c) {
+                    if (!mbar_wait(&s.empty[stage], phase ^ 1, abort_flag, kErrTimeoutProducer)) goto producer_abort;
+                    uint8_t *dst = chunks + stage * C::CHUNK;
+                    mbar_arrive_expect_tx(&s.full[stage], C::CHUNK);
+                    if (c < C::XC) {
+                        // x: K = channels c*64..+63 (rows), M = pairs (two 64-pair MN blocks)
+                        tma_load_3d(dst, &p.tm_x, &s.full[stage], p0, c * 64, b);
+                        tma_load_3d(dst + 8192, &p.tm_x, &s.full[stage], p0 + 64, c * 64, b);
+                    } else {
+                        tma_load_3d(dst, &p.tm_z, &s.full[stage], (c - C::XC) * 64, p0, b);
+                    }
+                    ++filled;
+                    if (++stage == C::S) { stage = 0; phase ^= 1; }
+                }
+            }
+            goto producer_done;
+        producer_abort:
+            for (uint32_t i = 0; i < (filled < (uint32_t)C::S ? filled : (uint32_t)C::S); ++i) {
+                uint32_t f = filled - 1 - i;
+                mbar_drain(&s.full[f % C::S], (f / C::S) & 1);
+            }
+        producer_done:
+            mbar_drain(&s.wbar, 0);
+        }
+    } else if (warp == C::MMA_WARP) {
+        if (lane == 0) {
+            const uint32_t idesc_x = idesc_bf16_f32(128, C::NCOL, true, false);
+            const uint32_t idesc_z = idesc_bf16_f32(128, C::NCOL, false, false);
+            bool ok = mbar_wait(&s.wbar, 0, abort_flag, kErrTimeoutMma);
+            int stage = 0;
+            uint32_t phase = 0;
+            int abuf = 0;
+            uint32_t aphase = 0;
+            for (int pt = cta_in_group; ok && pt < num_ptiles; pt += ctas_per_group) {
+                if (!mbar_wait(&s.tempty[abuf], aphase ^ 1, abort_flag, kErrTimeoutMma)) break;
+                tc_fence_after();
+                const uint32_t d1 = tmem_base + abuf * 256;     // x . W_o'
+                const uint32_t d2 = d1 + 128;                   // z . W_g'
+                for (int c = 0; c < C::CPT; ++c) {
+                    if (!mbar_wait(&s.full[stage], phase, abort_flag, kErrTimeoutMma)) { ok = false; break; }
+                    tc_fence_after();
+                    const uint8_t *ch = chunks + stage * C::CHUNK;
+                    if (c < C::XC) {
+                        const uint8_t *wb = wo_s + c * C::NCOL * 128;
+#pragma unroll
+                        for (int kk = 0; kk < 4; ++kk) {
+                            uint64_t ad = smem_desc_sw128(ch + kk * 2048, 8192, 1024);
+                            uint64_t bd = smem_desc_sw128(wb + kk * 32, 16, 1024);
+                            tc_mma_bf16(d1, ad, bd, idesc_x, (c | kk) != 0);
+                        }
+                    } else {
+                        const int zc = c - C::XC;
+                        const uint8_t *wb = wg_s + zc * C::NCOL * 128;
+#pragma unroll
+                        for (int kk = 0; kk < 4; ++kk) {
+                            uint64_t ad = smem_desc_sw128(ch + kk * 32, 16, 1024);
+                            uint64_t bd = smem_desc_sw128(wb + kk * 32, 16, 1024);
+                            tc_mma_bf16(d2, ad, bd, idesc_z, (zc | kk) != 0);
+                        }
+                    }
+                    tc_commit(&s.empty[stage]);
+                    if (++stage == C::S) { stage = 0; phase ^= 1; }
+                }
+                if (!ok) break;
+                tc_commit(&s.tfull[abuf]);
+                if (++abuf == 2) { abuf = 0; aphase ^= 1; }
+            }
+            tc_commit(&s.drain);
+            mbar_drain(&s.drain, 0);
+        }
+    } else if (warp >= 8) {
+        // statistics of x (over c_h) and z (over c_z) for pair `row`
+        const int row = (warp - 8) * 32 + lane;
+        const int mblk = row >> 6;         // which 64-pair MN block of an x chunk
+        const int r64 = row & 63;
+        int stage = 0;
+        uint32_t phase = 0;
+        int sbuf = 0;
+        uint32_t sphase = 0;
+        for (int pt = cta_in_group; pt < num_ptiles; pt += ctas_per_group) {
+            const int b = pt / p.tiles_per_batch;
+            const int p0 = (pt - b * p.tiles_per_batch) * 128;
+            float xs = 0.f, x1 = 0.f, x2 = 0.f;
+            float zs = 0.f, z1 = 0.f, z2 = 0.f;
+            bool ok = true;
+            for (int c = 0; c < C::CPT; ++c) {
+                if (!__all_sync(0xffffffffu, mbar_wait(&s.full[stage], phase, abort_flag, kErrTimeoutEpilogue))) { ok = false; break; }
+                const uint8_t *ch = chunks + stage * C::CHUNK;
+                if (c < C::XC) {
+                    // MN-major: K row kr holds 64 pairs; this pair's element sits in 16-byte
+                    // unit (r64 / 8) of that row, swizzled with the row index.
+                    const uint8_t *blk = ch + mblk * 8192;
+#pragma unroll 8
+                    for (int kr = 0; kr < 64; ++kr) {
+                        const uint16_t bits = *reinterpret_cast<const uint16_t *>(
+                            blk + sw128_offset(kr, r64 >> 3) + (r64 & 7) * 2);
+                        const float v = __uint_as_float((uint32_t)bits << 16);
+                        if (c == 0 && kr == 0) xs = v;
+                        const float d = v - xs;
+                        x1 += d;
+                        x2 = fmaf(d, d, x2);
+                    }
+                } else {
+#pragma unroll
+                    for (int u = 0; u < 8; ++u) {
+                        uint4 w = *reinterpret_cast<const uint4 *>(ch + sw128_offset(row, u));
+                        float v[8] = {bf16_lo(w.x), bf16_hi(w.x), bf16_lo(w.y), bf16_hi(w.y),
+                                      bf16_lo(w.z), bf16_hi(w.z), bf16_lo(w.w), bf16_hi(w.w)};
+                        if (c == C::XC && u == 0) zs = v[0];
+#pragma unroll
+                        for (int e = 0; e < 8; ++e) {
+                            const float d = v[e] - zs;
+                            z1 += d;
+                            z2 = fmaf(d, d, z2);
+                        }
+                    }
+                }
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&s.empty[stage]);
+                if (++stage == C::S) { stage = 0; phase ^= 1; }
+            }
+            if (!ok) break;
+            const float inv_h = 1.0f / (float)C::C_H, inv_z = 1.0f / (float)CZ;
+            const float dx = x1 * inv_h, dz = z1 * inv_z;
+            K3Stats st;
+            st.mean_x = xs + dx;
+            st.rstd_x = rsqrtf(fmaxf(x2 * inv_h - dx * dx, 0.f) + p.eps);
+            st.mean_z = zs + dz;
+            st.rstd_z = rsqrtf(fmaxf(z2 * inv_z - dz * dz, 0.f) + p.eps);
+            const long long pi = (long long)p0 + row;
+            st.mask = 1.f;
+            if (p.mask) st.mask = (pi < p.NN) ? __uint_as_float((uint32_t)p.mask[(long long)b * p.NN + pi] << 16) : 0.f;
+            st.pad0 = st.pad1 = st.pad2 = 0.f;
+            if (!__all_sync(0xffffffffu, mbar_wait(&s.sempty[sbuf], sphase ^ 1, abort_flag, kErrTimeoutEpilogue))) break;
+            stats[sbuf * 128 + row] = st;
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&s.sfull[sbuf]);
+            if (++sbuf == C::SNB) { sbuf = 0; sphase ^= 1; }
+        }
+    } else {
+        // epilogue: warpgroup wg handles output channels n0 + wg*64 .. +63
+        const int wg = warp >> 2;
+        const int q = warp & 3;
+        const int row = q * 32 + lane;
+        uint8_t *stg = staging + wg * C::STG_BYTES;
+        const bool leader = (threadIdx.x & 127) == 0;
+        const float4 *vec = p.vec + n0 + wg * 64;
+        int abuf = 0;
+        uint32_t aphase = 0;
+        int sbuf = 0;
+        uint32_t sphase = 0;
+        for (int pt = cta_in_group; pt < num_ptiles; pt += ctas_per_group) {
+            const int b = pt / p.tiles_per_batch;
+            const int p0 = (pt - b * p.tiles_per_batch) * 128;
+            if (!group_all(mbar_wait(&s.sfull[sbuf], sphase, abort_flag, kErrTimeoutEpilogue), 1 + wg, 128)) break;
+            const K3Stats st = stats[sbuf * 128 + row];
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&s.sempty[sbuf]);
+            if (++sbuf == C::SNB) { sbuf = 0; sphase ^= 1; }
+
+            if (!group_all(mbar_wait(&s.tfull[abuf], aphase, abort_flag, kErrTimeoutEpilogue), 1 + wg, 128)) break;
+            tc_fence_after();
+            const uint32_t t1 = tmem_base + abuf * 256 + ((uint32_t)(q * 32) << 16) + wg * 64;
+            const uint32_t t2 = t1 + 128;
+#pragma unroll 1
+            for (int sc = 0; sc < 64 / C::COLS_PER_STORE; ++sc) {
+                if (leader) tma_store_wait_read<0>();
+                named_bar_sync(1 + wg, 128);
+#pragma unroll 1
+                for (int h = 0; h < C::COLS_PER_STORE / 32; ++h) {
+                    const int col = sc * C::COLS_PER_STORE + h * 32;   // within this warpgroup's 64
+                    float o[32], g[32];
+                    tmem_ld32(t1 + col, o);
+                    tmem_ld32(t2 + col, g);
+                    tc_wait_ld();
+#pragma unroll
+                    for (int e = 0; e < 32; ++e) {
+                        const float4 cv = __ldg(&vec[col + e]);
+                        const float ov = fmaf(st.rstd_x, fmaf(-st.mean_x, cv.x, o[e]), cv.y);
+                        const float gv = fmaf(st.rstd_z, fmaf(-st.mean_z, cv.z, g[e]), cv.w);
+                        o[e] = st.mask * sigmoid_exp(gv) * ov;
+                    }
+                    if (OUT_F32) {
+#pragma unroll
+                        for (int u = 0; u < 8; ++u)
+                            *reinterpret_cast<float4 *>(stg + sw128_offset(row, u)) =
+                                make_float4(o[4 * u], o[4 * u + 1], o[4 * u + 2], o[4 * u + 3]);
+                    } else {
+#pragma unroll
+                        for (int u = 0; u < 4; ++u) {
+                            uint4 w;
+                            w.x = pack_bf16x2(o[8 * u + 0], o[8 * u + 1]);
+                            w.y = pack_bf16x2(o[8 * u + 2], o[8 * u + 3]);
+                            w.z = pack_bf16x2(o[8 * u + 4], o[8 * u + 5]);
+                            w.w = pack_bf16x2(o[8 * u + 6], o[8 * u + 7]);
+                            *reinterpret_cast<uint4 *>(stg + sw128_offset(row, h * 4 + u)) = w;
+                        }
+                    }
+                }
+                fence_proxy_async_smem();
+                named_bar_sync(1 + wg, 128);
+                if (leader) {
+                    tma_store_3d(&p.tm_out, stg, n0 + wg * 64 + sc * C::COLS_PER_STORE, p0, b);
+                    tma_store_commit();
+                }
+            }
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&s.tempty[abuf]);
+            if (++abuf == 2) { abuf = 0; aphase ^= 1; }
+        }
+        if (leader) tma_store_wait_all<0>();
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    if (warp == C::MMA_WARP) {
+        tc_fence_after();
+        tmem_dealloc(tmem_base, 512);
+    }
+}
+
+int k3_groups(int c_z) { return c_z / 128; }
+
+size_t k3_smem_bytes(int c_z, bool out_f32) {
+    if (c_z == 128) return out_f32 ? K3Cfg<128, true>::SMEM : K3Cfg<128, false>::SMEM;
+    return out_f32 ? K3Cfg<384, true>::SMEM : K3Cfg<384, false>::SMEM;
+}
+
+template <int CZ, bool F32>
+static cudaError_t k3_launch_t(const K3Args &args, int grid, cudaStream_t stream) {
+    static int configured_device = -1;
+    int dev = 0;
+    cudaGetDevice(&dev);
+    if (configured_device != dev) {
+        cudaError_t e = cudaFuncSetAttribute(k3_output_kernel<CZ, F32>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                             (int)K3Cfg<CZ, F32>::SMEM);
+        if (e != cudaSuccess) return e;
+        configured_device = dev;
+    }
+    k3_output_kernel<CZ, F32><<<grid, K3Cfg<CZ, F32>::THREADS, K3Cfg<CZ, F32>::SMEM, stream>>>(args);
+    return cudaGetLastError();
+}
+
+cudaError_t k3_launch(int c_z, bool out_f32, const K3Args &args, int grid, cudaStream_t stream) {
+    if (c_z == 128) return out_f32 ? k3_launch_t<128, true>(args, grid, stream) : k3_launch_t<128, false>(args, grid, stream);
+    if (c_z == 384) return out_f32 ? k3_launch_t<384, true>(args, grid, stream) : k3_launch_t<384, false>(args, grid, stream);
+    return cudaErrorInvalidValue;
+}
+
+}  // namespace trimul

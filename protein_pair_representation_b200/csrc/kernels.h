@@ -1,0 +1,105 @@
+// kernels.h -- launch interface between the host-side C ABI and the CUDA kernels.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace trimul {
+
+constexpr int kHidden = 128;  // c_h of the tensor-core path
+
+// ---- bf16 tensor-core path ---------------------------------------------------------
+
+struct K1Args {
+    CUtensorMap tm_z;      // z [B][N*N][c_z] bf16, box {64, 128, 1}, 128B swizzle
+    CUtensorMap tm_w;      // packed weights [4*c_h][c_z] bf16, box {64, NCOL}, 128B swizzle
+    CUtensorMap tm_a;      // a [B][c_h][N*N] bf16, box {128, channels per warpgroup, 1}
+    CUtensorMap tm_b;      // b, same as tm_a
+    const uint16_t *mask;  // [B][N*N] bf16 bits, or nullptr
+    const float4 *vec;     // [2][c_h] {sum W'_gate, shift_gate, sum W'_proj, shift_proj}
+    int B, N;
+    long long NN;
+    int tiles_per_batch;   // ceil(NN / 128)
+    float eps;
+};
+
+struct K2Args {
+    CUtensorMap tm_a, tm_b, tm_x;
+    int BC, N;
+    int m_tiles, n_tiles, k_chunks;
+    bool incoming;
+};
+
+struct K3Args {
+    CUtensorMap tm_x;      // x [B][c_h][N*N] bf16, box {64, 64, 1}, 128B swizzle (MN-major A)
+    CUtensorMap tm_z;      // z [B][N*N][c_z] bf16, box {64, 128, 1}, 128B swizzle
+    CUtensorMap tm_wo;     // folded W_o [c_z][c_h] bf16, box {64, 128}
+    CUtensorMap tm_wg;     // folded W_g [c_z][c_z] bf16, box {64, 128}
+    CUtensorMap tm_out;    // out [B][N*N][c_z] f32 (box {32,128,1}) or bf16 (box {64,128,1})
+    const uint16_t *mask;
+    const float4 *vec;     // [c_z] {sum W_o', shift_o, sum W_g', shift_g}
+    int B, N;
+    long long NN;
+    int tiles_per_batch;
+    float eps;
+};
+
+// Kernel resource queries (dynamic shared memory bytes) and launches.
+size_t k1_smem_bytes(int c_z);
+int k1_groups(int c_z);
+int k1_ncol(int c_z);
+int k1_channels_per_warpgroup(int c_z);
+cudaError_t k1_launch(int c_z, const K1Args &args, int grid, cudaStream_t stream);
+
+size_t k2_smem_bytes();
+cudaError_t k2_launch(const K2Args &args, int grid, cudaStream_t stream);
+
+size_t k3_smem_bytes(int c_z, bool out_f32);
+int k3_groups(int c_z);
+cudaError_t k3_launch(int c_z, bool out_f32, const K3Args &args, int grid, cudaStream_t stream);
+
+// ---- weight folding (layer creation) -----------------------------------------------
+
+struct FoldArgs {
+    const void *w;        // source [R][K]
+    const void *gamma;    // [K] or nullptr (= 1)
+    const void *beta;     // [K] or nullptr (= 0)
+    const void *bias;     // [R] or nullptr (= 0)
+    int src_bf16;         // storage type of w / gamma / beta / bias
+    int R, K;
+    uint16_t *dst;        // bf16 rows [*, K]
+    int row_mode;         // 0: dst row = r; 1: K1 interleaved layout (see k1 packing)
+    int operand;          // row_mode 1: 0 = a, 1 = b
+    int kind;             // row_mode 1: 0 = gate, 1 = projection
+    int ncol, cpg, gpo;   // row_mode 1: group width, channels per group, groups per operand
+    float *sum_out;       // element r * stride: sum_k bf16(W[r,k] * gamma[k])
+    float *shift_out;     // element r * stride: sum_k beta[k] W[r,k] + bias[r]
+    int out_stride;       // in floats
+};
+cudaError_t fold_launch(const FoldArgs &a, cudaStream_t stream);
+
+// Convert n values (bf16 or f32) to f32; optional transpose of an [R][K] matrix.
+cudaError_t to_f32_launch(const void *src, int src_bf16, float *dst, int R, int K, int transpose,
+                          cudaStream_t stream);
+
+// ---- fp32 SIMT path ----------------------------------------------------------------
+
+struct F32Weights {
+    const float *ln_in_g, *ln_in_b;
+    const float *w_ag, *b_ag, *w_ap, *b_ap, *w_bg, *b_bg, *w_bp, *b_bp;
+    const float *w_gT, *b_g;      // W_g transposed: [c_z (in)][c_z (out)]
+    const float *ln_out_g, *ln_out_b;
+    const float *w_oT, *b_o;      // W_o transposed: [c_h (in)][c_z (out)]
+};
+
+cudaError_t f32_project_launch(const float *z, const float *mask, const F32Weights &w, int c_z,
+                               int c_h, int B, int N, float eps, float *a, float *b,
+                               cudaStream_t stream);
+cudaError_t f32_contract_launch(const float *a, const float *b, float *x, int BC, int N,
+                                bool incoming, cudaStream_t stream);
+cudaError_t f32_output_launch(const float *z, const float *mask, const float *x,
+                              const F32Weights &w, int c_z, int c_h, int B, int N, float eps,
+                              float *out, cudaStream_t stream);
+
+}  // namespace trimul

@@ -1,0 +1,599 @@
+// trimul_api.cu -- host side of the C ABI declared in include/trimul.h.
+//
+// Validates every call, owns the repacked layer weights, encodes the TMA tensor maps
+// (driver entry point cuTensorMapEncodeTiled) and launches the three kernels of one
+// update: K1 projection, K2 contraction, K3 output gate. There is no CPU or library
+// fallback: anything outside the compiled set is reported as an error.
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <mutex>
+#include <stdarg.h>
+#include <stdio.h>
+#include <string.h>
+
+#include "kernels.h"
+#include "sm100.cuh"
+#include "trimul.h"
+
+namespace trimul {
+__device__ unsigned int g_device_error = 0;
+}
+
+using namespace trimul;
+
+struct trimul_layer {
+    int c_z, c_h;
+    float eps;
+    bool has_bf16;               // tensor-core packing present
+    void *mem;                   // single device allocation holding everything below
+    // bf16 path
+    uint16_t *k1_w;              // [4*c_h][c_z] packed, folded
+    float4 *k1_vec;              // [2][c_h]
+    uint16_t *k3_wo;             // [c_z][c_h] folded
+    uint16_t *k3_wg;             // [c_z][c_z] folded
+    float4 *k3_vec;              // [c_z]
+    // fp32 path
+    F32Weights f32;
+    // workspace
+    void *ws;
+    size_t ws_bytes;
+    cudaEvent_t events[4];
+    bool timing;
+};
+
+// ------------------------------------------------------------------ error plumbing
+
+static thread_local char g_last_error[512];
+
+static trimul_status_t fail(trimul_status_t st, const char *fmt, ...) {
+    va_list ap;
+    va_start(ap, fmt);
+    vsnprintf(g_last_error, sizeof(g_last_error), fmt, ap);
+    va_end(ap);
+    return st;
+}
+
+static trimul_status_t cuda_fail(cudaError_t e, const char *what) {
+    return fail(TRIMUL_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e));
+}
+
+#define TRY_CUDA(expr, what)                      \
+    do {                                          \
+        cudaError_t _e = (expr);                  \
+        if (_e != cudaSuccess) return cuda_fail(_e, what); \
+    } while (0)
+
+// ------------------------------------------------------------------ device info
+
+struct DeviceInfo {
+    bool known;
+    int major, minor, sms;
+};
+static DeviceInfo g_dev[64];
+static std::mutex g_dev_mu;
+
+static trimul_status_t device_info(DeviceInfo *out) {
+    int dev = 0;
+    TRY_CUDA(cudaGetDevice(&dev), "cudaGetDevice");
+    if (dev < 0 || dev >= 64) return fail(TRIMUL_ERR_UNSUPPORTED_DEVICE, "device index %d", dev);
+    std::lock_guard<std::mutex> lk(g_dev_mu);
+    if (!g_dev[dev].known) {
+        DeviceInfo d{};
+        TRY_CUDA(cudaDeviceGetAttribute(&d.major, cudaDevAttrComputeCapabilityMajor, dev), "attr major");
+        TRY_CUDA(cudaDeviceGetAttribute(&d.minor, cudaDevAttrComputeCapabilityMinor, dev), "attr minor");
+        TRY_CUDA(cudaDeviceGetAttribute(&d.sms, cudaDevAttrMultiProcessorCount, dev), "attr SMs");
+        d.known = true;
+        g_dev[dev] = d;
+    }
+    *out = g_dev[dev];
+    return TRIMUL_OK;
+}
+
+static trimul_status_t require_sm100(DeviceInfo *d) {
+    trimul_status_t st = device_info(d);
+    if (st != TRIMUL_OK) return st;
+    if (!(d->major == 10 && d->minor == 0))
+        return fail(TRIMUL_ERR_UNSUPPORTED_DEVICE, "bf16 path needs compute capability 10.0, device is %d.%d", d->major,
+                    d->minor);
+    return TRIMUL_OK;
+}
+
+// ------------------------------------------------------------------ tensor maps
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *, const cuuint64_t *,
+                                  const cuuint64_t *, const cuuint32_t *, const cuuint32_t *, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+static EncodeTiledFn encode_fn() {
+    static EncodeTiledFn fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void *p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<EncodeTiledFn>(p);
+    });
+    return fn;
+}
+
+// dims / box listed innermost first; strides are the byte strides of dims 1..rank-1.
+static trimul_status_t make_map(CUtensorMap *m, CUtensorMapDataType dt, int rank, const void *ptr,
+                                const uint64_t *dims, const uint64_t *strides, const uint32_t *box,
+                                CUtensorMapSwizzle sw, const char *what) {
+    EncodeTiledFn fn = encode_fn();
+    if (!fn) return fail(TRIMUL_ERR_CUDA, "cuTensorMapEncodeTiled entry point unavailable");
+    cuuint64_t gd[5], gs[4];
+    cuuint32_t bx[5], es[5];
+    for (int i = 0; i < rank; ++i) {
+        gd[i] = dims[i];
+        bx[i] = box[i];
+        es[i] = 1;
+    }
+    for (int i = 0; i < rank - 1; ++i) gs[i] = strides[i];
+    CUresult r = fn(m, dt, (cuuint32_t)rank, const_cast<void *>(ptr), gd, gs, bx, es, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                    sw, CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS) return fail(TRIMUL_ERR_CUDA, "cuTensorMapEncodeTiled(%s) failed: %d", what, (int)r);
+    return TRIMUL_OK;
+}
+
+#define TRY(expr)                                 \
+    do {                                          \
+        trimul_status_t _s = (expr);              \
+        if (_s != TRIMUL_OK) return _s;           \
+    } while (0)
+
+// ------------------------------------------------------------------ validation helpers
+
+static bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+static size_t dtype_size(trimul_dtype_t t) { return t == TRIMUL_BF16 ? 2 : 4; }
+
+static bool overlap(const void *a, size_t na, const void *b, size_t nb) {
+    uintptr_t x = reinterpret_cast<uintptr_t>(a), y = reinterpret_cast<uintptr_t>(b);
+    return na && nb && x < y + nb && y < x + na;
+}
+
+static trimul_status_t check_pair(const trimul_pair_t *t, const char *name) {
+    if (!t || !t->data) return fail(TRIMUL_ERR_INVALID_ARG, "%s: NULL tensor", name);
+    if (t->dtype != TRIMUL_F32 && t->dtype != TRIMUL_BF16) return fail(TRIMUL_ERR_INVALID_ARG, "%s: unknown dtype", name);
+    if (t->B < 1 || t->N < 1 || t->C < 1) return fail(TRIMUL_ERR_INVALID_ARG, "%s: sizes must be positive", name);
+    if (!aligned16(t->data)) return fail(TRIMUL_ERR_ALIGNMENT, "%s: pointer not 16-byte aligned", name);
+    return TRIMUL_OK;
+}
+
+static size_t pair_bytes(const trimul_pair_t *t) {
+    return (size_t)t->B * t->N * t->N * t->C * dtype_size(t->dtype);
+}
+
+static trimul_status_t check_problem(const trimul_pair_t *z, const void *mask, const trimul_layer_t *L) {
+    if (!L) return fail(TRIMUL_ERR_INVALID_ARG, "layer is NULL");
+    TRY(check_pair(z, "z"));
+    if (z->C != L->c_z) return fail(TRIMUL_ERR_INVALID_ARG, "z has %lld channels, layer expects c_z=%d", (long long)z->C, L->c_z);
+    if (z->N < 8 || z->N % 8 != 0) return fail(TRIMUL_ERR_UNSUPPORTED_SHAPE, "N=%lld must be a positive multiple of 8", (long long)z->N);
+    if (z->N > 16384) return fail(TRIMUL_ERR_UNSUPPORTED_SHAPE, "N=%lld exceeds 16384", (long long)z->N);
+    if (mask && !aligned16(mask)) return fail(TRIMUL_ERR_ALIGNMENT, "mask pointer not 16-byte aligned");
+    if (z->dtype == TRIMUL_BF16) {
+        if (!L->has_bf16) return fail(TRIMUL_ERR_UNSUPPORTED_SHAPE, "bf16 path supports (c_z, c_h) = (128,128) or (384,128); layer is (%d,%d)", L->c_z, L->c_h);
+        if ((long long)z->B * z->N * z->N / 128 > (1LL << 30)) return fail(TRIMUL_ERR_UNSUPPORTED_SHAPE, "problem too large");
+    }
+    return TRIMUL_OK;
+}
+
+// ------------------------------------------------------------------ layer
+
+extern "C" trimul_status_t tri_mul_layer_create(const trimul_weights_desc_t *w, void *stream, trimul_layer_t **out) {
+    if (!w || !out) return fail(TRIMUL_ERR_INVALID_ARG, "NULL argument");
+    *out = nullptr;
+    if (w->dtype != TRIMUL_F32 && w->dtype != TRIMUL_BF16) return fail(TRIMUL_ERR_INVALID_ARG, "unknown weight dtype");
+    if (w->c_z < 32 || w->c_h < 32 || w->c_z % 32 || w->c_h % 32 || w->c_z > 512 || w->c_h > 512)
+        return fail(TRIMUL_ERR_UNSUPPORTED_SHAPE, "c_z and c_h must be multiples of 32 in [32, 512]");
+    if (!(w->eps > 0.f)) return fail(TRIMUL_ERR_INVALID_ARG, "eps must be positive");
+    if (!w->w_ag || !w->w_ap || !w->w_bg || !w->w_bp || !w->w_g || !w->w_o)
+        return fail(TRIMUL_ERR_INVALID_ARG, "projection weights may not be NULL");
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    const int cz = w->c_z, ch = w->c_h;
+    const int src_bf16 = w->dtype == TRIMUL_BF16;
+
+    trimul_layer *L = new trimul_layer();
+    memset(L, 0, sizeof(*L));
+    L->c_z = cz;
+    L->c_h = ch;
+    L->eps = w->eps;
+    L->has_bf16 = (ch == kHidden) && (cz == 128 || cz == 384);
+
+    // carve one allocation
+    size_t off = 0;
+    auto take = [&](size_t bytes) { size_t o = off; off = (off + bytes + 255) & ~size_t(255); return o; };
+    size_t o_k1w = 0, o_k1v = 0, o_k3o = 0, o_k3g = 0, o_k3v = 0;
+    if (L->has_bf16) {
+        o_k1w = take((size_t)4 * ch * cz * 2);
+        o_k1v = take((size_t)2 * ch * sizeof(float4));
+        o_k3o = take((size_t)cz * ch * 2);
+        o_k3g = take((size_t)cz * cz * 2);
+        o_k3v = take((size_t)cz * sizeof(float4));
+    }
+    const size_t o_lig = take(cz * 4), o_lib = take(cz * 4);
+    const size_t o_wag = take((size_t)ch * cz * 4), o_wap = take((size_t)ch * cz * 4);
+    const size_t o_wbg = take((size_t)ch * cz * 4), o_wbp = take((size_t)ch * cz * 4);
+    const size_t o_bag = take(ch * 4), o_bap = take(ch * 4), o_bbg = take(ch * 4), o_bbp = take(ch * 4);
+    const size_t o_wgT = take((size_t)cz * cz * 4), o_bg = take(cz * 4);
+    const size_t o_log = take(ch * 4), o_lob = take(ch * 4);
+    const size_t o_woT = take((size_t)ch * cz * 4), o_bo = take(cz * 4);
+    cudaError_t e = cudaMalloc(&L->mem, off);
+    if (e != cudaSuccess) {
+        delete L;
+        return cuda_fail(e, "cudaMalloc(layer)");
+    }
+    uint8_t *m = reinterpret_cast<uint8_t *>(L->mem);
+
+    auto conv = [&](const void *src, size_t o, int R, int K, int tr, const float **dst) -> cudaError_t {
+        if (!src) { *dst = nullptr; return cudaSuccess; }
+        *dst = reinterpret_cast<float *>(m + o);
+        return to_f32_launch(src, src_bf16, reinterpret_cast<float *>(m + o), R, K, tr, st);
+    };
+    cudaError_t ce = cudaSuccess;
+#define CONV(src, o, R, K, tr, dst) if (ce == cudaSuccess) ce = conv(src, o, R, K, tr, dst)
+    CONV(w->ln_in_g, o_lig, 1, cz, 0, &L->f32.ln_in_g);
+    CONV(w->ln_in_b, o_lib, 1, cz, 0, &L->f32.ln_in_b);
+    CONV(w->w_ag, o_wag, ch, cz, 0, &L->f32.w_ag);
+    CONV(w->w_ap, o_wap, ch, cz, 0, &L->f32.w_ap);
+    CONV(w->w_bg, o_wbg, ch, cz, 0, &L->f32.w_bg);
+    CONV(w->w_bp, o_wbp, ch, cz, 0, &L->f32.w_bp);
+    CONV(w->b_ag, o_bag, 1, ch, 0, &L->f32.b_ag);
+    CONV(w->b_ap, o_bap, 1, ch, 0, &L->f32.b_ap);
+    CONV(w->b_bg, o_bbg, 1, ch, 0, &L->f32.b_bg);
+    CONV(w->b_bp, o_bbp, 1, ch, 0, &L->f32.b_bp);
+    CONV(w->w_g, o_wgT, cz, cz, 1, &L->f32.w_gT);
+    CONV(w->b_g, o_bg, 1, cz, 0, &L->f32.b_g);
+    CONV(w->ln_out_g, o_log, 1, ch, 0, &L->f32.ln_out_g);
+    CONV(w->ln_out_b, o_lob, 1, ch, 0, &L->f32.ln_out_b);
+    CONV(w->w_o, o_woT, cz, ch, 1, &L->f32.w_oT);
+    CONV(w->b_o, o_bo, 1, cz, 0, &L->f32.b_o);
+#undef CONV
+
+    if (ce == cudaSuccess && L->has_bf16) {
+        L->k1_w = reinterpret_cast<uint16_t *>(m + o_k1w);
+        L->k1_vec = reinterpret_cast<float4 *>(m + o_k1v);
+        L->k3_wo = reinterpret_cast<uint16_t *>(m + o_k3o);
+        L->k3_wg = reinterpret_cast<uint16_t *>(m + o_k3g);
+        L->k3_vec = reinterpret_cast<float4 *>(m + o_k3v);
+        const int ncol = k1_ncol(cz);
+        const void *srcs[2][2] = {{w->w_ag, w->w_ap}, {w->w_bg, w->w_bp}};
+        const void *biases[2][2] = {{w->b_ag, w->b_ap}, {w->b_bg, w->b_bp}};
+        float *vecf = reinterpret_cast<float *>(L->k1_vec);
+        for (int o = 0; o < 2 && ce == cudaSuccess; ++o)
+            for (int kind = 0; kind < 2 && ce == cudaSuccess; ++kind) {
+                FoldArgs fa{};
+                fa.w = srcs[o][kind];
+                fa.gamma = w->ln_in_g;
+                fa.beta = w->ln_in_b;
+                fa.bias = biases[o][kind];
+                fa.src_bf16 = src_bf16;
+                fa.R = ch;
+                fa.K = cz;
+                fa.dst = L->k1_w;
+                fa.row_mode = 1;
+                fa.operand = o;
+                fa.kind = kind;
+                fa.ncol = ncol;
+                fa.cpg = ncol / 2;
+                fa.gpo = k1_groups(cz) / 2;
+                fa.sum_out = vecf + (size_t)o * ch * 4 + kind * 2;
+                fa.shift_out = vecf + (size_t)o * ch * 4 + kind * 2 + 1;
+                fa.out_stride = 4;
+                ce = fold_launch(fa, st);
+            }
+        float *v3 = reinterpret_cast<float *>(L->k3_vec);
+        if (ce == cudaSuccess) {
+            FoldArgs fa{};
+            fa.w = w->w_o; fa.gamma = w->ln_out_g; fa.beta = w->ln_out_b; fa.bias = w->b_o;
+            fa.src_bf16 = src_bf16; fa.R = cz; fa.K = ch; fa.dst = L->k3_wo; fa.row_mode = 0;
+            fa.sum_out = v3 + 0; fa.shift_out = v3 + 1; fa.out_stride = 4;
+            ce = fold_launch(fa, st);
+        }
+        if (ce == cudaSuccess) {
+            FoldArgs fa{};
+            fa.w = w->w_g; fa.gamma = w->ln_in_g; fa.beta = w->ln_in_b; fa.bias = w->b_g;
+            fa.src_bf16 = src_bf16; fa.R = cz; fa.K = cz; fa.dst = L->k3_wg; fa.row_mode = 0;
+            fa.sum_out = v3 + 2; fa.shift_out = v3 + 3; fa.out_stride = 4;
+            ce = fold_launch(fa, st);
+        }
+    }
+    if (ce == cudaSuccess) ce = cudaStreamSynchronize(st);
+    if (ce != cudaSuccess) {
+        cudaFree(L->mem);
+        delete L;
+        return cuda_fail(ce, "layer packing");
+    }
+    *out = L;
+    return TRIMUL_OK;
+}
+
+extern "C" void tri_mul_layer_destroy(trimul_layer_t *L) {
+    if (!L) return;
+    if (L->mem) cudaFree(L->mem);
+    delete L;
+}
+
+static size_t ws_plane_bytes(int64_t B, int64_t N, int c_h, trimul_dtype_t dt) {
+    return (((size_t)B * c_h * N * N * dtype_size(dt)) + 255) & ~size_t(255);
+}
+
+extern "C" size_t tri_mul_workspace_bytes(const trimul_layer_t *L, int64_t B, int64_t N, trimul_dtype_t dt) {
+    if (!L || B < 1 || N < 1 || (dt != TRIMUL_F32 && dt != TRIMUL_BF16)) return 0;
+    return 3 * ws_plane_bytes(B, N, L->c_h, dt);
+}
+
+extern "C" trimul_status_t tri_mul_layer_bind_workspace(trimul_layer_t *L, void *ws, size_t bytes) {
+    if (!L) return fail(TRIMUL_ERR_INVALID_ARG, "layer is NULL");
+    if (ws && !aligned16(ws)) return fail(TRIMUL_ERR_ALIGNMENT, "workspace not 16-byte aligned");
+    L->ws = ws;
+    L->ws_bytes = ws ? bytes : 0;
+    return TRIMUL_OK;
+}
+
+extern "C" trimul_status_t tri_mul_layer_set_timing_events(trimul_layer_t *L, void *const *events) {
+    if (!L) return fail(TRIMUL_ERR_INVALID_ARG, "layer is NULL");
+    if (!events) {
+        L->timing = false;
+        return TRIMUL_OK;
+    }
+    for (int i = 0; i < 4; ++i) {
+        if (!events[i]) return fail(TRIMUL_ERR_INVALID_ARG, "timing event %d is NULL", i);
+        L->events[i] = reinterpret_cast<cudaEvent_t>(events[i]);
+    }
+    L->timing = true;
+    return TRIMUL_OK;
+}
+
+extern "C" int tri_mul_kernels_per_forward(void) { return 3; }
+
+// ------------------------------------------------------------------ kernel drivers
+
+static int grid_for(int sms, long long work_units, int multiple) {
+    long long g = work_units < sms ? work_units : sms;
+    g = (g / multiple) * multiple;
+    if (g < multiple) g = multiple;
+    return (int)g;
+}
+
+static trimul_status_t run_project_bf16(const trimul_layer_t *L, const void *z, const void *mask, void *a, void *b,
+                                        int B, int N, cudaStream_t st) {
+    DeviceInfo d;
+    TRY(require_sm100(&d));
+    const uint64_t NN = (uint64_t)N * N;
+    const int cz = L->c_z, ch = L->c_h;
+    K1Args p{};
+    {
+        uint64_t dims[3] = {(uint64_t)cz, NN, (uint64_t)B};
+        uint64_t strides[2] = {(uint64_t)cz * 2, NN * cz * 2};
+        uint32_t box[3] = {64, 128, 1};
+        TRY(make_map(&p.tm_z, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, z, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_128B, "K1 z"));
+    }
+    {
+        uint64_t dims[2] = {(uint64_t)cz, (uint64_t)4 * ch};
+        uint64_t strides[1] = {(uint64_t)cz * 2};
+        uint32_t box[2] = {64, (uint32_t)k1_ncol(cz)};
+        TRY(make_map(&p.tm_w, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, L->k1_w, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_128B, "K1 w"));
+    }
+    {
+        uint64_t dims[3] = {NN, (uint64_t)ch, (uint64_t)B};
+        uint64_t strides[2] = {NN * 2, (uint64_t)ch * NN * 2};
+        uint32_t box[3] = {128, (uint32_t)k1_channels_per_warpgroup(cz), 1};
+        TRY(make_map(&p.tm_a, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, a, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_NONE, "K1 a"));
+        TRY(make_map(&p.tm_b, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, b, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_NONE, "K1 b"));
+    }
+    p.mask = reinterpret_cast<const uint16_t *>(mask);
+    p.vec = L->k1_vec;
+    p.B = B;
+    p.N = N;
+    p.NN = (long long)NN;
+    p.tiles_per_batch = (int)((NN + 127) / 128);
+    p.eps = L->eps;
+    const int G = k1_groups(cz);
+    const int grid = grid_for(d.sms, (long long)G * B * p.tiles_per_batch, G);
+    TRY_CUDA(k1_launch(cz, p, grid, st), "K1 launch");
+    return TRIMUL_OK;
+}
+
+static trimul_status_t run_contract_bf16(const void *a, const void *b, void *x, int64_t BC, int N, bool incoming,
+                                         cudaStream_t st) {
+    DeviceInfo d;
+    TRY(require_sm100(&d));
+    K2Args p{};
+    uint64_t dims[3] = {(uint64_t)N, (uint64_t)N, (uint64_t)BC};
+    uint64_t strides[2] = {(uint64_t)N * 2, (uint64_t)N * N * 2};
+    if (!incoming) {
+        uint32_t boxa[3] = {64, 128, 1}, boxb[3] = {64, 256, 1};
+        TRY(make_map(&p.tm_a, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, a, dims, strides, boxa, CU_TENSOR_MAP_SWIZZLE_128B, "K2 a"));
+        TRY(make_map(&p.tm_b, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, b, dims, strides, boxb, CU_TENSOR_MAP_SWIZZLE_128B, "K2 b"));
+    } else {
+        uint32_t box[3] = {64, 64, 1};
+        TRY(make_map(&p.tm_a, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, a, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_128B, "K2 a"));
+        TRY(make_map(&p.tm_b, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, b, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_128B, "K2 b"));
+    }
+    {
+        uint32_t box[3] = {64, 128, 1};
+        TRY(make_map(&p.tm_x, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, x, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_128B, "K2 x"));
+    }
+    p.BC = (int)BC;
+    p.N = N;
+    p.m_tiles = (N + 127) / 128;
+    p.n_tiles = (N + 255) / 256;
+    p.k_chunks = (N + 63) / 64;
+    p.incoming = incoming;
+    const long long tiles = (long long)BC * p.m_tiles * p.n_tiles;
+    const int grid = grid_for(d.sms, tiles, 1);
+    TRY_CUDA(k2_launch(p, grid, st), "K2 launch");
+    return TRIMUL_OK;
+}
+
+static trimul_status_t run_output_bf16(const trimul_layer_t *L, const void *z, const void *mask, const void *x,
+                                       void *out, bool out_f32, int B, int N, cudaStream_t st) {
+    DeviceInfo d;
+    TRY(require_sm100(&d));
+    const uint64_t NN = (uint64_t)N * N;
+    const int cz = L->c_z, ch = L->c_h;
+    K3Args p{};
+    {
+        uint64_t dims[3] = {NN, (uint64_t)ch, (uint64_t)B};
+        uint64_t strides[2] = {NN * 2, (uint64_t)ch * NN * 2};
+        uint32_t box[3] = {64, 64, 1};
+        TRY(make_map(&p.tm_x, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, x, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_128B, "K3 x"));
+    }
+    {
+        uint64_t dims[3] = {(uint64_t)cz, NN, (uint64_t)B};
+        uint64_t strides[2] = {(uint64_t)cz * 2, NN * cz * 2};
+        uint32_t box[3] = {64, 128, 1};
+        TRY(make_map(&p.tm_z, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, z, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_128B, "K3 z"));
+    }
+    {
+        uint64_t dims[2] = {(uint64_t)ch, (uint64_t)cz};
+        uint64_t strides[1] = {(uint64_t)ch * 2};
+        uint32_t box[2] = {64, 128};
+        TRY(make_map(&p.tm_wo, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, L->k3_wo, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_128B, "K3 wo"));
+    }
+    {
+        uint64_t dims[2] = {(uint64_t)cz, (uint64_t)cz};
+        uint64_t strides[1] = {(uint64_t)cz * 2};
+        uint32_t box[2] = {64, 128};
+        TRY(make_map(&p.tm_wg, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, L->k3_wg, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_128B, "K3 wg"));
+    }
+    {
+        const uint64_t es = out_f32 ? 4 : 2;
+        uint64_t dims[3] = {(uint64_t)cz, NN, (uint64_t)B};
+        uint64_t strides[2] = {(uint64_t)cz * es, NN * cz * es};
+        uint32_t box[3] = {out_f32 ? 32u : 64u, 128, 1};
+        TRY(make_map(&p.tm_out, out_f32 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, out, dims,
+                     strides, box, CU_TENSOR_MAP_SWIZZLE_128B, "K3 out"));
+    }
+    p.mask = reinterpret_cast<const uint16_t *>(mask);
+    p.vec = L->k3_vec;
+    p.B = B;
+    p.N = N;
+    p.NN = (long long)NN;
+    p.tiles_per_batch = (int)((NN + 127) / 128);
+    p.eps = L->eps;
+    const int G = k3_groups(cz);
+    const int grid = grid_for(d.sms, (long long)G * B * p.tiles_per_batch, G);
+    TRY_CUDA(k3_launch(cz, out_f32, p, grid, st), "K3 launch");
+    return TRIMUL_OK;
+}
+
+// ------------------------------------------------------------------ public entry points
+
+extern "C" trimul_status_t tri_mul_project(const trimul_pair_t *z, const void *mask, const trimul_layer_t *L, void *a_out,
+                                           void *b_out, void *stream) {
+    TRY(check_problem(z, mask, L));
+    if (!a_out || !b_out) return fail(TRIMUL_ERR_INVALID_ARG, "a_out / b_out NULL");
+    if (!aligned16(a_out) || !aligned16(b_out)) return fail(TRIMUL_ERR_ALIGNMENT, "a_out / b_out not 16-byte aligned");
+    const size_t plane = (size_t)z->B * L->c_h * z->N * z->N * dtype_size(z->dtype);
+    if (overlap(a_out, plane, b_out, plane) || overlap(a_out, plane, z->data, pair_bytes(z)) ||
+        overlap(b_out, plane, z->data, pair_bytes(z)))
+        return fail(TRIMUL_ERR_INVALID_ARG, "a_out, b_out and z overlap");
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    if (z->dtype == TRIMUL_BF16)
+        return run_project_bf16(L, z->data, mask, a_out, b_out, (int)z->B, (int)z->N, st);
+    TRY_CUDA(f32_project_launch(reinterpret_cast<const float *>(z->data), reinterpret_cast<const float *>(mask), L->f32,
+                                L->c_z, L->c_h, (int)z->B, (int)z->N, L->eps, reinterpret_cast<float *>(a_out),
+                                reinterpret_cast<float *>(b_out), st),
+             "fp32 projection launch");
+    return TRIMUL_OK;
+}
+
+extern "C" trimul_status_t tri_mul_contract(const void *a, const void *b, void *x, int64_t B, int64_t C, int64_t N,
+                                            trimul_dtype_t dtype, trimul_direction_t dir, void *stream) {
+    if (!a || !b || !x) return fail(TRIMUL_ERR_INVALID_ARG, "NULL tensor");
+    if (dtype != TRIMUL_F32 && dtype != TRIMUL_BF16) return fail(TRIMUL_ERR_INVALID_ARG, "unknown dtype");
+    if (dir != TRIMUL_OUTGOING && dir != TRIMUL_INCOMING) return fail(TRIMUL_ERR_INVALID_ARG, "unknown direction");
+    if (B < 1 || C < 1) return fail(TRIMUL_ERR_INVALID_ARG, "B and C must be positive");
+    if (N < 8 || N % 8 || N > 16384) return fail(TRIMUL_ERR_UNSUPPORTED_SHAPE, "N=%lld must be a multiple of 8 in [8, 16384]", (long long)N);
+    if (B * C > 65535) return fail(TRIMUL_ERR_UNSUPPORTED_SHAPE, "B*C=%lld exceeds 65535", (long long)(B * C));
+    if (!aligned16(a) || !aligned16(b) || !aligned16(x)) return fail(TRIMUL_ERR_ALIGNMENT, "pointer not 16-byte aligned");
+    const size_t bytes = (size_t)B * C * N * N * dtype_size(dtype);
+    if (overlap(x, bytes, a, bytes) || overlap(x, bytes, b, bytes)) return fail(TRIMUL_ERR_INVALID_ARG, "x overlaps a or b");
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    if (dtype == TRIMUL_BF16) return run_contract_bf16(a, b, x, B * C, (int)N, dir == TRIMUL_INCOMING, st);
+    TRY_CUDA(f32_contract_launch(reinterpret_cast<const float *>(a), reinterpret_cast<const float *>(b),
+                                 reinterpret_cast<float *>(x), (int)(B * C), (int)N, dir == TRIMUL_INCOMING, st),
+             "fp32 contraction launch");
+    return TRIMUL_OK;
+}
+
+extern "C" trimul_status_t tri_mul_output_gate(const trimul_pair_t *z, const void *mask, const void *x,
+                                               const trimul_layer_t *L, trimul_pair_t *out, void *stream) {
+    TRY(check_problem(z, mask, L));
+    TRY(check_pair(out, "out"));
+    if (!x) return fail(TRIMUL_ERR_INVALID_ARG, "x is NULL");
+    if (!aligned16(x)) return fail(TRIMUL_ERR_ALIGNMENT, "x not 16-byte aligned");
+    if (out->B != z->B || out->N != z->N || out->C != z->C) return fail(TRIMUL_ERR_INVALID_ARG, "out shape differs from z");
+    if (z->dtype == TRIMUL_F32 && out->dtype != TRIMUL_F32) return fail(TRIMUL_ERR_INVALID_ARG, "fp32 path writes fp32 out");
+    if (overlap(out->data, pair_bytes(out), z->data, pair_bytes(z))) return fail(TRIMUL_ERR_INVALID_ARG, "out overlaps z");
+    const size_t xbytes = (size_t)z->B * L->c_h * z->N * z->N * dtype_size(z->dtype);
+    if (overlap(out->data, pair_bytes(out), x, xbytes)) return fail(TRIMUL_ERR_INVALID_ARG, "out overlaps x");
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    if (z->dtype == TRIMUL_BF16)
+        return run_output_bf16(L, z->data, mask, x, out->data, out->dtype == TRIMUL_F32, (int)z->B, (int)z->N, st);
+    TRY_CUDA(f32_output_launch(reinterpret_cast<const float *>(z->data), reinterpret_cast<const float *>(mask),
+                               reinterpret_cast<const float *>(x), L->f32, L->c_z, L->c_h, (int)z->B, (int)z->N, L->eps,
+                               reinterpret_cast<float *>(out->data), st),
+             "fp32 output launch");
+    return TRIMUL_OK;
+}
+
+extern "C" trimul_status_t tri_mul_forward(const trimul_pair_t *z, const void *mask, const trimul_layer_t *L,
+                                           trimul_direction_t dir, trimul_pair_t *out, void *stream) {
+    TRY(check_problem(z, mask, L));
+    TRY(check_pair(out, "out"));
+    if (dir != TRIMUL_OUTGOING && dir != TRIMUL_INCOMING) return fail(TRIMUL_ERR_INVALID_ARG, "unknown direction");
+    if (out->B != z->B || out->N != z->N || out->C != z->C) return fail(TRIMUL_ERR_INVALID_ARG, "out shape differs from z");
+    if (z->dtype == TRIMUL_F32 && out->dtype != TRIMUL_F32) return fail(TRIMUL_ERR_INVALID_ARG, "fp32 path writes fp32 out");
+    const size_t plane = ws_plane_bytes(z->B, z->N, L->c_h, z->dtype);
+    if (!L->ws || L->ws_bytes < 3 * plane)
+        return fail(TRIMUL_ERR_WORKSPACE, "workspace of %zu bytes needed, %zu bound", 3 * plane, L->ws_bytes);
+    if (overlap(out->data, pair_bytes(out), z->data, pair_bytes(z))) return fail(TRIMUL_ERR_INVALID_ARG, "out overlaps z");
+    if (overlap(out->data, pair_bytes(out), L->ws, 3 * plane) || overlap(z->data, pair_bytes(z), L->ws, 3 * plane))
+        return fail(TRIMUL_ERR_INVALID_ARG, "z or out overlaps the workspace");
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    uint8_t *ws = reinterpret_cast<uint8_t *>(L->ws);
+    void *a = ws, *b = ws + plane, *x = ws + 2 * plane;
+    if (L->timing) TRY_CUDA(cudaEventRecord(L->events[0], st), "event record");
+    TRY(tri_mul_project(z, mask, L, a, b, stream));
+    if (L->timing) TRY_CUDA(cudaEventRecord(L->events[1], st), "event record");
+    TRY(tri_mul_contract(a, b, x, z->B, L->c_h, z->N, z->dtype, dir, stream));
+    if (L->timing) TRY_CUDA(cudaEventRecord(L->events[2], st), "event record");
+    TRY(tri_mul_output_gate(z, mask, x, L, out, stream));
+    if (L->timing) TRY_CUDA(cudaEventRecord(L->events[3], st), "event record");
+    return TRIMUL_OK;
+}
+
+extern "C" trimul_status_t tri_mul_check_device_status(void) {
+    TRY_CUDA(cudaDeviceSynchronize(), "cudaDeviceSynchronize");
+    unsigned int v = 0, zero = 0;
+    TRY_CUDA(cudaMemcpyFromSymbol(&v, g_device_error, sizeof(v)), "read device error word");
+    if (v) {
+        TRY_CUDA(cudaMemcpyToSymbol(g_device_error, &zero, sizeof(zero)), "clear device error word");
+        return fail(TRIMUL_ERR_DEVICE_TIMEOUT, "a kernel gave up on a bounded wait (code 0x%x)", v);
+    }
+    return TRIMUL_OK;
+}
+
+extern "C" const char *tri_mul_status_string(trimul_status_t s) {
+    switch (s) {
+        case TRIMUL_OK: return "ok";
+        case TRIMUL_ERR_INVALID_ARG: return "invalid argument";
+        case TRIMUL_ERR_UNSUPPORTED_SHAPE: return "unsupported shape";
+        case TRIMUL_ERR_UNSUPPORTED_DEVICE: return "unsupported device";
+        case TRIMUL_ERR_WORKSPACE: return "workspace missing or too small";
+        case TRIMUL_ERR_CUDA: return "CUDA error";
+        case TRIMUL_ERR_DEVICE_TIMEOUT: return "device wait timed out";
+        case TRIMUL_ERR_ALIGNMENT: return "pointer not 16-byte aligned";
+    }
+    return "unknown status";
+}
+
+extern "C" const char *tri_mul_last_error(void) { return g_last_error; }
+
+extern "C" int tri_mul_abi_version(void) { return TRIMUL_ABI_VERSION; }

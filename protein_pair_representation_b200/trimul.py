@@ -1,0 +1,261 @@
+"""Python binding of the C ABI in include/trimul.h (argument marshalling only).
+
+Every step of the update runs in the CUDA library; this module only turns torch
+tensors into pointers and sizes, allocates the workspace through torch (the
+caller's allocator) and turns status codes into exceptions. If the library is
+missing the calls raise; there is no other implementation to fall back to.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import threading
+
+import torch
+
+from . import build as _build
+
+OUTGOING = 0
+INCOMING = 1
+F32 = 0
+BF16 = 1
+_DIRS = {"outgoing": OUTGOING, "incoming": INCOMING, OUTGOING: OUTGOING, INCOMING: INCOMING}
+
+WEIGHT_ORDER = (
+    "ln_in_g", "ln_in_b", "w_ag", "b_ag", "w_ap", "b_ap", "w_bg", "b_bg",
+    "w_bp", "b_bp", "w_g", "b_g", "ln_out_g", "ln_out_b", "w_o", "b_o",
+)
+
+STATUS_NAMES = {
+    0: "TRIMUL_OK", 1: "TRIMUL_ERR_INVALID_ARG", 2: "TRIMUL_ERR_UNSUPPORTED_SHAPE",
+    3: "TRIMUL_ERR_UNSUPPORTED_DEVICE", 4: "TRIMUL_ERR_WORKSPACE", 5: "TRIMUL_ERR_CUDA",
+    6: "TRIMUL_ERR_DEVICE_TIMEOUT", 7: "TRIMUL_ERR_ALIGNMENT",
+}
+
+
+class TriMulError(RuntimeError):
+    def __init__(self, status: int, detail: str):
+        super().__init__(f"{STATUS_NAMES.get(status, status)}: {detail}")
+        self.status = status
+        self.detail = detail
+
+
+class _Pair(ctypes.Structure):
+    _fields_ = [("data", ctypes.c_void_p), ("B", ctypes.c_int64), ("N", ctypes.c_int64),
+                ("C", ctypes.c_int64), ("dtype", ctypes.c_int)]
+
+
+class _WeightsDesc(ctypes.Structure):
+    _fields_ = [("c_z", ctypes.c_int32), ("c_h", ctypes.c_int32), ("dtype", ctypes.c_int),
+                ("eps", ctypes.c_float)] + [(n, ctypes.c_void_p) for n in WEIGHT_ORDER]
+
+
+_lib = None
+_lib_lock = threading.Lock()
+
+
+def library_path() -> str:
+    return _build.LIB_PATH
+
+
+def load_library():
+    """Load libtrimul.so (built in-tree by protein_pair_representation_b200.build)."""
+    global _lib
+    with _lib_lock:
+        if _lib is not None:
+            return _lib
+        path = _build.LIB_PATH
+        if not os.path.exists(path):
+            raise RuntimeError(f"CUDA library not built: {path} is missing "
+                               "(run python -m protein_pair_representation_b200.build)")
+        lib = ctypes.CDLL(path)
+        vp, i64, st = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int
+        P = ctypes.POINTER
+        lib.tri_mul_layer_create.argtypes = [P(_WeightsDesc), vp, P(vp)]
+        lib.tri_mul_layer_destroy.argtypes = [vp]
+        lib.tri_mul_layer_destroy.restype = None
+        lib.tri_mul_workspace_bytes.argtypes = [vp, i64, i64, st]
+        lib.tri_mul_workspace_bytes.restype = ctypes.c_size_t
+        lib.tri_mul_layer_bind_workspace.argtypes = [vp, vp, ctypes.c_size_t]
+        lib.tri_mul_forward.argtypes = [P(_Pair), vp, vp, st, P(_Pair), vp]
+        lib.tri_mul_project.argtypes = [P(_Pair), vp, vp, vp, vp, vp]
+        lib.tri_mul_contract.argtypes = [vp, vp, vp, i64, i64, i64, st, st, vp]
+        lib.tri_mul_output_gate.argtypes = [P(_Pair), vp, vp, vp, P(_Pair), vp]
+        lib.tri_mul_layer_set_timing_events.argtypes = [vp, P(vp)]
+        lib.tri_mul_kernels_per_forward.argtypes = []
+        lib.tri_mul_check_device_status.argtypes = []
+        lib.tri_mul_status_string.argtypes = [st]
+        lib.tri_mul_status_string.restype = ctypes.c_char_p
+        lib.tri_mul_last_error.argtypes = []
+        lib.tri_mul_last_error.restype = ctypes.c_char_p
+        lib.tri_mul_abi_version.argtypes = []
+        for name in ("tri_mul_layer_create", "tri_mul_layer_bind_workspace", "tri_mul_forward",
+                     "tri_mul_project", "tri_mul_contract", "tri_mul_output_gate",
+                     "tri_mul_layer_set_timing_events", "tri_mul_check_device_status"):
+            getattr(lib, name).restype = ctypes.c_int
+        _lib = lib
+        return lib
+
+
+def _check(status: int):
+    if status != 0:
+        lib = load_library()
+        raise TriMulError(status, lib.tri_mul_last_error().decode(errors="replace"))
+
+
+def _dtype_code(dt: torch.dtype) -> int:
+    if dt == torch.float32:
+        return F32
+    if dt == torch.bfloat16:
+        return BF16
+    raise TypeError(f"unsupported dtype {dt}")
+
+
+def _stream_ptr(stream) -> ctypes.c_void_p:
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream)
+
+
+def _pair(t: torch.Tensor) -> _Pair:
+    if t.dim() != 4 or t.shape[1] != t.shape[2]:
+        raise ValueError(f"pair tensor must be [B, N, N, C], got {tuple(t.shape)}")
+    if not t.is_contiguous():
+        raise ValueError("pair tensor must be contiguous")
+    return _Pair(t.data_ptr(), t.shape[0], t.shape[1], t.shape[3], _dtype_code(t.dtype))
+
+
+def _mask_ptr(mask, z):
+    if mask is None:
+        return None
+    if mask.dtype != z.dtype or tuple(mask.shape) != tuple(z.shape[:3]) or not mask.is_contiguous():
+        raise ValueError("mask must be a contiguous [B, N, N] tensor in z's dtype")
+    return mask.data_ptr()
+
+
+class TriMulLayer:
+    """A triangle multiplicative update layer (weights repacked on the device).
+
+    weights: dict name -> CUDA tensor (all float32 or all bfloat16), names as in
+    WEIGHT_ORDER; biases and LayerNorm parameters may be missing (None).
+    """
+
+    def __init__(self, weights: dict, eps: float = 1e-5, stream=None):
+        self._lib = load_library()
+        w_ag = weights["w_ag"]
+        c_h, c_z = w_ag.shape
+        dt = w_ag.dtype
+        self._keep = []
+        desc = _WeightsDesc()
+        desc.c_z, desc.c_h, desc.dtype, desc.eps = c_z, c_h, _dtype_code(dt), eps
+        for n in WEIGHT_ORDER:
+            t = weights.get(n)
+            if t is None:
+                setattr(desc, n, None)
+                continue
+            if t.dtype != dt or not t.is_cuda:
+                raise ValueError(f"weight {n} must be a CUDA tensor of dtype {dt}")
+            t = t.contiguous()
+            self._keep.append(t)
+            setattr(desc, n, t.data_ptr())
+        handle = ctypes.c_void_p()
+        _check(self._lib.tri_mul_layer_create(ctypes.byref(desc), _stream_ptr(stream), ctypes.byref(handle)))
+        self._keep = []
+        self.handle = handle
+        self.c_z, self.c_h, self.eps = c_z, c_h, eps
+        self.device = w_ag.device
+        self._ws = None
+        self._events = None
+
+    def close(self):
+        if getattr(self, "handle", None):
+            self._lib.tri_mul_layer_destroy(self.handle)
+            self.handle = None
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
+
+    def workspace_bytes(self, B: int, N: int, dtype: torch.dtype) -> int:
+        return int(self._lib.tri_mul_workspace_bytes(self.handle, B, N, _dtype_code(dtype)))
+
+    def bind_workspace(self, buf: torch.Tensor | None):
+        """Attach a caller-allocated uint8 CUDA buffer (or None) as the workspace."""
+        self._ws = buf
+        ptr = None if buf is None else buf.data_ptr()
+        nbytes = 0 if buf is None else buf.numel() * buf.element_size()
+        _check(self._lib.tri_mul_layer_bind_workspace(self.handle, ptr, nbytes))
+
+    def ensure_workspace(self, B: int, N: int, dtype: torch.dtype):
+        need = self.workspace_bytes(B, N, dtype)
+        if self._ws is None or self._ws.numel() < need:
+            self.bind_workspace(torch.empty(need, dtype=torch.uint8, device=self.device))
+
+    def set_timing_events(self, events):
+        """events: four torch.cuda.Event(enable_timing=True) or None."""
+        self._events = events
+        if events is None:
+            _check(self._lib.tri_mul_layer_set_timing_events(self.handle, None))
+            return
+        arr = (ctypes.c_void_p * 4)(*[e.cuda_event for e in events])
+        _check(self._lib.tri_mul_layer_set_timing_events(self.handle, arr))
+
+    def forward(self, z: torch.Tensor, mask: torch.Tensor | None = None, direction="outgoing",
+                out: torch.Tensor | None = None, out_dtype: torch.dtype | None = None, stream=None):
+        B, N = z.shape[0], z.shape[1]
+        self.ensure_workspace(B, N, z.dtype)
+        if out is None:
+            out = torch.empty(z.shape, dtype=out_dtype or torch.float32, device=z.device)
+        zp, op = _pair(z), _pair(out)
+        _check(self._lib.tri_mul_forward(ctypes.byref(zp), _mask_ptr(mask, z), self.handle,
+                                         _DIRS[direction], ctypes.byref(op), _stream_ptr(stream)))
+        return out
+
+    __call__ = forward
+
+    def project(self, z: torch.Tensor, mask: torch.Tensor | None = None, stream=None):
+        """K1 alone: a, b as [B, c_h, N, N] in z's dtype."""
+        B, N = z.shape[0], z.shape[1]
+        a = torch.empty((B, self.c_h, N, N), dtype=z.dtype, device=z.device)
+        b = torch.empty_like(a)
+        zp = _pair(z)
+        _check(self._lib.tri_mul_project(ctypes.byref(zp), _mask_ptr(mask, z), self.handle,
+                                         a.data_ptr(), b.data_ptr(), _stream_ptr(stream)))
+        return a, b
+
+    def output_gate(self, z: torch.Tensor, x: torch.Tensor, mask: torch.Tensor | None = None,
+                    out: torch.Tensor | None = None, out_dtype: torch.dtype | None = None, stream=None):
+        """K3 alone: out from z and x [B, c_h, N, N] (x in z's dtype)."""
+        if x.dtype != z.dtype or not x.is_contiguous() or tuple(x.shape) != (z.shape[0], self.c_h, z.shape[1], z.shape[2]):
+            raise ValueError("x must be a contiguous [B, c_h, N, N] tensor in z's dtype")
+        if out is None:
+            out = torch.empty(z.shape, dtype=out_dtype or torch.float32, device=z.device)
+        zp, op = _pair(z), _pair(out)
+        _check(self._lib.tri_mul_output_gate(ctypes.byref(zp), _mask_ptr(mask, z), x.data_ptr(), self.handle,
+                                             ctypes.byref(op), _stream_ptr(stream)))
+        return out
+
+
+def contract(a: torch.Tensor, b: torch.Tensor, direction="outgoing", out: torch.Tensor | None = None, stream=None):
+    """K2 alone on [B, C, N, N] tensors (float32 or bfloat16)."""
+    lib = load_library()
+    if a.shape != b.shape or a.dim() != 4 or a.shape[2] != a.shape[3] or a.dtype != b.dtype:
+        raise ValueError("a and b must be [B, C, N, N] of one dtype")
+    if not (a.is_contiguous() and b.is_contiguous()):
+        raise ValueError("a and b must be contiguous")
+    if out is None:
+        out = torch.empty_like(a)
+    B, C, N, _ = a.shape
+    _check(lib.tri_mul_contract(a.data_ptr(), b.data_ptr(), out.data_ptr(), B, C, N, _dtype_code(a.dtype),
+                                _DIRS[direction], _stream_ptr(stream)))
+    return out
+
+
+def check_device_status():
+    _check(load_library().tri_mul_check_device_status())
+
+
+def kernels_per_forward() -> int:
+    return int(load_library().tri_mul_kernels_per_forward())

@@ -1,0 +1,86 @@
+"""The C-ABI library builds, loads and exports what include/trimul.h declares (no GPU needed).
+
+Only calls that are answered on the host before any CUDA work are made here: status
+strings, version queries and argument validation that must fail before a launch.
+"""
+import ctypes
+import os
+import re
+
+import pytest
+
+from protein_pair_representation_b200 import build
+from protein_pair_representation_b200 import trimul as tm
+
+HEADER = os.path.join(build.ROOT, "include", "trimul.h")
+
+
+@pytest.fixture(scope="module")
+def lib():
+    build.build_library()
+    return tm.load_library()
+
+
+def declared_functions():
+    with open(HEADER) as f:
+        src = f.read()
+    return sorted(set(re.findall(r"\b(tri_mul_\w+)\s*\(", src)))
+
+
+def test_header_declares_the_entry_points():
+    names = declared_functions()
+    for must in ("tri_mul_forward", "tri_mul_layer_create", "tri_mul_layer_destroy", "tri_mul_project",
+                 "tri_mul_contract", "tri_mul_output_gate", "tri_mul_workspace_bytes",
+                 "tri_mul_layer_bind_workspace", "tri_mul_check_device_status"):
+        assert must in names
+
+
+def test_every_declared_symbol_is_exported(lib):
+    missing = [n for n in declared_functions() if not hasattr(lib, n)]
+    assert not missing, f"not exported: {missing}"
+
+
+def test_library_is_built_for_sm100a(lib):
+    # the fatbin must carry sm_100a code: cuobjdump is not used; nvcc's -gencode list is the record
+    assert "arch=compute_100a,code=sm_100a" in build.NVCC_FLAGS
+
+
+def test_status_strings_and_versions(lib):
+    for code in range(8):
+        assert lib.tri_mul_status_string(code)
+    assert lib.tri_mul_status_string(99) == b"unknown status"
+    assert lib.tri_mul_abi_version() == 100
+    assert lib.tri_mul_kernels_per_forward() == 3
+
+
+def test_null_arguments_are_rejected_on_the_host(lib):
+    handle = ctypes.c_void_p()
+    assert lib.tri_mul_layer_create(None, None, ctypes.byref(handle)) == 1
+    z = tm._Pair(0, 1, 8, 128, tm.BF16)
+    out = tm._Pair(0, 1, 8, 128, tm.F32)
+    assert lib.tri_mul_forward(ctypes.byref(z), None, None, 0, ctypes.byref(out), None) == 1
+    assert b"layer is NULL" in lib.tri_mul_last_error()
+
+
+def test_contract_validation_happens_before_any_launch(lib):
+    fake = ctypes.c_void_p(1 << 20)  # never dereferenced: validation fails first
+    # N not a multiple of 8
+    assert lib.tri_mul_contract(fake, fake, fake, 1, 4, 12, tm.BF16, 0, None) == 2
+    # unknown direction
+    assert lib.tri_mul_contract(fake, fake, fake, 1, 4, 16, tm.BF16, 7, None) == 1
+    # misaligned pointer
+    bad = ctypes.c_void_p((1 << 20) + 8)
+    assert lib.tri_mul_contract(bad, fake, ctypes.c_void_p(1 << 24), 1, 4, 16, tm.BF16, 0, None) == 7
+    # x overlapping a
+    assert lib.tri_mul_contract(fake, ctypes.c_void_p(1 << 24), fake, 1, 4, 16, tm.BF16, 0, None) == 1
+    # too many channels for the grid
+    assert lib.tri_mul_contract(fake, ctypes.c_void_p(1 << 30), ctypes.c_void_p(1 << 34), 1, 70000, 16, tm.F32, 0, None) == 2
+
+
+def test_layer_create_rejects_bad_widths_before_allocating(lib):
+    desc = tm._WeightsDesc()
+    desc.c_z, desc.c_h, desc.dtype, desc.eps = 100, 128, tm.BF16, 1e-5
+    handle = ctypes.c_void_p()
+    assert lib.tri_mul_layer_create(ctypes.byref(desc), None, ctypes.byref(handle)) == 2
+    desc.c_z, desc.eps = 128, 0.0
+    assert lib.tri_mul_layer_create(ctypes.byref(desc), None, ctypes.byref(handle)) == 1
