@@ -26,6 +26,11 @@
  *   - Pair tensors are contiguous [B, N, N, C], channel fastest (channel-last).
  *   - Intermediate tensors a, b, x are contiguous [B, c_h, N, N] (channel-major:
  *     every channel is one N x N matrix), which is the layout the contraction reads.
+ *     For a BF16 z they are stored as F16 (IEEE half: same 2 bytes and tensor-core
+ *     rate as bf16, 3 more mantissa bits); x is stored pre-multiplied by the power of
+ *     two tri_mul_contract_scale(N) (about 1/sqrt(N)) to stay far inside the F16
+ *     range, and the output LayerNorm is evaluated with eps * scale^2, which is the
+ *     same function of the unscaled x. For an F32 z they are F32 with scale 1.
  *   - Linear weights are row-major [out, in] with y = x W^T + bias. Bias and
  *     LayerNorm beta pointers may be NULL (= 0); LayerNorm gamma may be NULL (= 1).
  *   - `stream` is a cudaStream_t (NULL = legacy default stream). Forward calls
@@ -52,12 +57,17 @@ typedef enum {
     TRIMUL_ERR_WORKSPACE = 4,          /* no workspace bound, or bound one too small */
     TRIMUL_ERR_CUDA = 5,               /* a CUDA runtime / driver call failed */
     TRIMUL_ERR_DEVICE_TIMEOUT = 6,     /* a kernel gave up on a bounded wait (see below) */
-    TRIMUL_ERR_ALIGNMENT = 7           /* a tensor pointer is not 16-byte aligned */
+    TRIMUL_ERR_ALIGNMENT = 7,          /* a tensor pointer is not 16-byte aligned */
+    TRIMUL_ERR_RANGE = 8               /* a non-finite or out-of-range (|v| > 65504) fp16
+                                          intermediate was seen (reported by
+                                          tri_mul_check_device_status) */
 } trimul_status_t;
 
 typedef enum { TRIMUL_OUTGOING = 0, TRIMUL_INCOMING = 1 } trimul_direction_t;
 
-typedef enum { TRIMUL_F32 = 0, TRIMUL_BF16 = 1 } trimul_dtype_t;
+/* F32: IEEE binary32. BF16: bfloat16. F16: IEEE binary16 (the intermediate type of
+ * the tensor-core path). */
+typedef enum { TRIMUL_F32 = 0, TRIMUL_BF16 = 1, TRIMUL_F16 = 2 } trimul_dtype_t;
 
 /* A pair tensor [B, N, N, C], contiguous, channel-last. */
 typedef struct {
@@ -90,11 +100,12 @@ typedef struct {
 typedef struct trimul_layer trimul_layer_t;
 
 /* Build a layer handle from weights already on the current device.
- * The handle holds its own device copy: for the bf16 tensor-core path the input
- * LayerNorm gamma is folded into W_ag/W_ap/W_bg/W_bp/W_g and the output
- * LayerNorm gamma into W_o (bf16, [out, in]), with per-row correction vectors
- * sum_k W'[r, k] and sum_k beta[k] W[r, k] + bias[r] in fp32 (the folding of
- * "Triangle multiplication on SM90"); for the fp32 path it keeps fp32 copies.
+ * The handle holds its own device copy: for the tensor-core path the input
+ * LayerNorm gamma is folded into W_ag/W_ap/W_bg/W_bp/W_g (bf16, the type of z)
+ * and the output LayerNorm gamma into W_o (F16, the type of x), all [out, in],
+ * with per-row correction vectors sum_k W'[r, k] and sum_k beta[k] W[r, k] + bias[r]
+ * in fp32 (the folding of "Triangle multiplication on SM90"); for the fp32 path it
+ * keeps fp32 copies.
  * Runs on `stream` and synchronizes it before returning, so the caller may free
  * the source weights afterwards. Supported (c_z, c_h): any multiple of 32 up to
  * 512 for the fp32 path; (128, 128) and (384, 128) for the bf16 path (checked
@@ -105,9 +116,9 @@ trimul_status_t tri_mul_layer_create(const trimul_weights_desc_t *weights, void 
 /* Free the handle and its device memory. NULL is ignored. */
 void tri_mul_layer_destroy(trimul_layer_t *layer);
 
-/* Bytes of workspace tri_mul_forward needs for B x N x N with compute type
- * `dtype` (the dtype of z): a, b and x, each [B, c_h, N, N] of that type,
- * 256-byte aligned. Returns 0 for an invalid layer or size. */
+/* Bytes of workspace tri_mul_forward needs for B x N x N with z of type `dtype`:
+ * a, b and x, each [B, c_h, N, N] of the intermediate type (F16 for a BF16 z,
+ * F32 for an F32 z), 256-byte aligned. Returns 0 for an invalid layer or size. */
 size_t tri_mul_workspace_bytes(const trimul_layer_t *layer, int64_t B, int64_t N,
                                trimul_dtype_t dtype);
 
@@ -131,25 +142,34 @@ trimul_status_t tri_mul_forward(const trimul_pair_t *z, const void *mask,
                                 trimul_pair_t *out, void *stream);
 
 /* Step K1 alone ("x_x" input gate): a and b from z, written channel-major
- * [B, c_h, N, N] in z's dtype. Same requirements as tri_mul_forward. */
+ * [B, c_h, N, N] in the intermediate type (F16 for a BF16 z, F32 for an F32 z).
+ * Same requirements as tri_mul_forward. */
 trimul_status_t tri_mul_project(const trimul_pair_t *z, const void *mask,
                                 const trimul_layer_t *layer, void *a_out, void *b_out,
                                 void *stream);
 
 /* Step K2 alone (the contraction): x from a and b, all [B, C, N, N] of `dtype`.
- *   outgoing: x[b,c,i,j] = sum_k a[b,c,i,k] b[b,c,j,k]
- *   incoming: x[b,c,i,j] = sum_k a[b,c,k,i] b[b,c,k,j]
- * BF16: fp32 accumulation, bf16 result, C any positive value. F32: fp32 FMA.
- * N % 8 == 0. x must not overlap a or b. */
+ *   outgoing: x[b,c,i,j] = x_scale * sum_k a[b,c,i,k] b[b,c,j,k]
+ *   incoming: x[b,c,i,j] = x_scale * sum_k a[b,c,k,i] b[b,c,k,j]
+ * F16 / BF16: tensor cores, fp32 accumulation, result rounded to `dtype` after the
+ * scaling (sm_100 only). F32: fp32 FMA on CUDA cores. N % 8 == 0, 8 <= N <= 16384,
+ * B * C <= 65535. x must not overlap a or b. Use a power of two for x_scale to keep
+ * the scaling exact. */
 trimul_status_t tri_mul_contract(const void *a, const void *b, void *x, int64_t B, int64_t C,
                                  int64_t N, trimul_dtype_t dtype, trimul_direction_t direction,
-                                 void *stream);
+                                 float x_scale, void *stream);
+
+/* The power of two tri_mul_forward multiplies x by on the tensor-core path:
+ * 2^-ceil(log2(N) / 2). Returns 0 for N < 1. */
+float tri_mul_contract_scale(int64_t N);
 
 /* Step K3 alone ("x0_x1" output gate): out from z, the mask and x [B, c_h, N, N]
- * (x in z's dtype). Same requirements as tri_mul_forward. */
+ * in the intermediate type, where x holds x_scale times the contraction (x_scale > 0;
+ * the output LayerNorm then uses eps * x_scale^2). Same requirements as
+ * tri_mul_forward. */
 trimul_status_t tri_mul_output_gate(const trimul_pair_t *z, const void *mask, const void *x,
-                                    const trimul_layer_t *layer, trimul_pair_t *out,
-                                    void *stream);
+                                    float x_scale, const trimul_layer_t *layer,
+                                    trimul_pair_t *out, void *stream);
 
 /* Optional per-kernel timing: when `events` is non-NULL, every later
  * tri_mul_forward on this handle records events[0] before K1, events[1] after
@@ -161,9 +181,11 @@ trimul_status_t tri_mul_layer_set_timing_events(trimul_layer_t *layer, void *con
 int tri_mul_kernels_per_forward(void);
 
 /* Synchronize the current device, then read and clear the library's device
- * error word. Every wait inside the bf16 kernels is bounded (about one second);
- * a wait that runs out makes its kernel stop early, and this call reports
- * TRIMUL_ERR_DEVICE_TIMEOUT. Outputs of such a launch are undefined. */
+ * error word. Every wait inside the tensor-core kernels is bounded (about one
+ * second); a wait that runs out makes its kernel stop early, and this call reports
+ * TRIMUL_ERR_DEVICE_TIMEOUT. K3 also flags a non-finite x (an F16 intermediate that
+ * overflowed, or a non-finite input) as TRIMUL_ERR_RANGE. Outputs of such a launch
+ * are undefined. */
 trimul_status_t tri_mul_check_device_status(void);
 
 /* Static description of a status code. */

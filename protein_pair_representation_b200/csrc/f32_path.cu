@@ -85,7 +85,7 @@ __global__ void __launch_bounds__(f32::THREADS) f32_project_kernel(const float *
 }
 
 __global__ void __launch_bounds__(256) f32_contract_kernel(const float *a, const float *b, float *x, int N,
-                                                           int incoming) {
+                                                           int incoming, float x_scale) {
     __shared__ float As[16][64 + 4];
     __shared__ float Bs[16][64 + 4];
     const int c = blockIdx.z;
@@ -125,13 +125,13 @@ __global__ void __launch_bounds__(256) f32_contract_kernel(const float *a, const
     for (int u = 0; u < 4; ++u)
         for (int v = 0; v < 4; ++v) {
             const int i = i0 + ty * 4 + u, j = j0 + tx * 4 + v;
-            if (i < N && j < N) x[c * plane + (long long)i * N + j] = acc[u][v];
+            if (i < N && j < N) x[c * plane + (long long)i * N + j] = acc[u][v] * x_scale;
         }
 }
 
 __global__ void __launch_bounds__(f32::THREADS) f32_output_kernel(const float *z, const float *mask, const float *x,
                                                                   F32Weights w, int c_z, int c_h, long long NN,
-                                                                  float eps, float *out) {
+                                                                  float eps, float eps_x, float *out) {
     using namespace f32;
     extern __shared__ float sm[];
     const int ldz = c_z + 1, ldx = c_h + 1;
@@ -148,7 +148,7 @@ __global__ void __launch_bounds__(f32::THREADS) f32_output_kernel(const float *z
     }
     __syncthreads();
     layernorm_rows(zs, TP, c_z, ldz, w.ln_in_g, w.ln_in_b, eps);
-    layernorm_rows(xs, TP, c_h, ldx, w.ln_out_g, w.ln_out_b, eps);
+    layernorm_rows(xs, TP, c_h, ldx, w.ln_out_g, w.ln_out_b, eps_x);
     __syncthreads();
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -189,14 +189,14 @@ cudaError_t f32_project_launch(const float *z, const float *mask, const F32Weigh
 }
 
 cudaError_t f32_contract_launch(const float *a, const float *b, float *x, int BC, int N, bool incoming,
-                                cudaStream_t stream) {
+                                float x_scale, cudaStream_t stream) {
     dim3 grid((N + 63) / 64, (N + 63) / 64, BC);
-    f32_contract_kernel<<<grid, 256, 0, stream>>>(a, b, x, N, incoming ? 1 : 0);
+    f32_contract_kernel<<<grid, 256, 0, stream>>>(a, b, x, N, incoming ? 1 : 0, x_scale);
     return cudaGetLastError();
 }
 
 cudaError_t f32_output_launch(const float *z, const float *mask, const float *x, const F32Weights &w, int c_z,
-                              int c_h, int B, int N, float eps, float *out, cudaStream_t stream) {
+                              int c_h, int B, int N, float eps, float eps_x, float *out, cudaStream_t stream) {
     const long long NN = (long long)N * N;
     const size_t smem = (size_t)f32::TP * ((c_z + 1) + (c_h + 1)) * sizeof(float);
     if (smem > 48 * 1024) {
@@ -204,7 +204,7 @@ cudaError_t f32_output_launch(const float *z, const float *mask, const float *x,
         if (e != cudaSuccess) return e;
     }
     const long long blocks = (long long)B * (NN / f32::TP);
-    f32_output_kernel<<<(unsigned)blocks, f32::THREADS, smem, stream>>>(z, mask, x, w, c_z, c_h, NN, eps, out);
+    f32_output_kernel<<<(unsigned)blocks, f32::THREADS, smem, stream>>>(z, mask, x, w, c_z, c_h, NN, eps, eps_x, out);
     return cudaGetLastError();
 }
 

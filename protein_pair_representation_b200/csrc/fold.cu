@@ -32,9 +32,17 @@ __global__ void fold_kernel(FoldArgs a) {
         const float w = load_as_f32(a.w, r * a.K + k, a.src_bf16);
         const float g = a.gamma ? load_as_f32(a.gamma, k, a.src_bf16) : 1.0f;
         const float bt = a.beta ? load_as_f32(a.beta, k, a.src_bf16) : 0.0f;
-        const __nv_bfloat16 wf = __float2bfloat16_rn(w * g);
-        a.dst[(size_t)dst_row * a.K + k] = __bfloat16_as_ushort(wf);
-        sum_w += (double)__bfloat162float(wf);
+        float wq;
+        if (a.dst_f16) {
+            const __half h = __float2half_rn(w * g);
+            a.dst[(size_t)dst_row * a.K + k] = __half_as_ushort(h);
+            wq = __half2float(h);
+        } else {
+            const __nv_bfloat16 h = __float2bfloat16_rn(w * g);
+            a.dst[(size_t)dst_row * a.K + k] = __bfloat16_as_ushort(h);
+            wq = __bfloat162float(h);
+        }
+        sum_w += (double)wq;
         shift += (double)bt * (double)w;
     }
     __shared__ double red[2][32];

@@ -2,7 +2,7 @@
 //
 // Computes, for every pair p = (b, i, j) and hidden channel c,
 //   a[b, c, i, j] = m_p * sigmoid(zhat_p . W_ag[c] + b_ag[c]) * (zhat_p . W_ap[c] + b_ap[c])
-// and b likewise, with zhat_p = LayerNorm(z_p) ("RFProteina architecture", section
+// and b likewise (stored as fp16), with zhat_p = LayerNorm(z_p) ("RFProteina architecture", section
 // "Dual-GEMM gates": the one-input gate that reads the normalized pair tensor,
 // applies the mask and emits its output transposed for the contraction; section
 // "Triangle multiplication on SM90": K1 with the input LayerNorm folded into its
@@ -142,7 +142,7 @@ __global__ void __launch_bounds__(448, 1) k1_project_kernel(const __grid_constan
         }
     } else if (warp == C::MMA_WARP) {
         if (lane == 0) {
-            const uint32_t idesc = idesc_bf16_f32(128, C::NCOL, false, false);
+            const uint32_t idesc = idesc_f32acc(128, C::NCOL, false, false, false);
             bool ok = mbar_wait(&s.wbar, 0, abort_flag, kErrTimeoutMma);
             int stage = 0;
             uint32_t phase = 0;
@@ -258,7 +258,7 @@ __global__ void __launch_bounds__(448, 1) k1_project_kernel(const __grid_constan
                     const float g = fmaf(rstd, fmaf(-mean, cv.x, v[e]), cv.y);
                     const float pr = fmaf(rstd, fmaf(-mean, cv.z, v[16 + e]), cv.w);
                     const float out = sigmoid_tanh(g) * pr * m;
-                    stg[(blk * 16 + e) * 128 + row] = __bfloat16_as_ushort(__float2bfloat16_rn(out));
+                    stg[(blk * 16 + e) * 128 + row] = __half_as_ushort(__float2half_rn(out));
                 }
             }
             tc_fence_before();

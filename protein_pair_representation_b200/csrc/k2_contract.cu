@@ -5,8 +5,10 @@
 // the contraction itself, one direction at a time):
 //   outgoing  X_c = A_c B_c^T   (x_ij = sum_k a_ik b_jk; both operands K-major)
 //   incoming  X_c = A_c^T B_c   (x_ij = sum_k a_ki b_kj; both operands MN-major)
-// a, b, x are [B*c_h][N][N] bf16. The two directions differ only in the TMA boxes
-// and in the major-ness bits of the shared-memory descriptors.
+// a, b, x are [B*c_h][N][N] of one 16-bit type (fp16 on the update path, bf16 also
+// supported), with fp32 accumulation and an optional power-of-two scale applied to
+// the result before rounding. The two directions differ only in the TMA boxes and
+// in the major-ness bits of the shared-memory descriptors.
 //
 // Persistent kernel, one CTA per SM, 128 x 256 output tiles, 64-deep k chunks:
 //   warp 8      TMA producer (one elected lane) filling a 4-stage ring
@@ -14,7 +16,7 @@
 //               two 256-column TMEM buffers so the epilogue of tile t overlaps
 //               the MMAs of tile t+1)
 //   warps 0-7   epilogue: two warpgroups, each drains 128 of the 256 columns
-//               (tcgen05.ld), rounds to bf16, stages through 128B-swizzled shared
+//               (tcgen05.ld), scales, rounds to 16 bits, stages through 128B-swizzled shared
 //               memory and writes with TMA stores.
 #include "kernels.h"
 #include "sm100.cuh"
@@ -127,7 +129,7 @@ __global__ void __launch_bounds__(k2::THREADS, 1) k2_contract_kernel(const __gri
         }
     } else if (warp == MMA_WARP) {
         if (lane == 0) {
-            const uint32_t idesc = idesc_bf16_f32(BM, BN, p.incoming, p.incoming);
+            const uint32_t idesc = idesc_f32acc(BM, BN, p.incoming, p.incoming, p.f16);
             int stage = 0;
             uint32_t phase = 0;
             int abuf = 0;
@@ -192,12 +194,21 @@ __global__ void __launch_bounds__(k2::THREADS, 1) k2_contract_kernel(const __gri
                     tmem_ld32(tmem_base + abuf * BN + ((uint32_t)(q * 32) << 16) + col, v);
                     tc_wait_ld();
 #pragma unroll
+                    for (int e = 0; e < 32; ++e) v[e] *= p.x_scale;
+#pragma unroll
                     for (int u = 0; u < 4; ++u) {
                         uint4 w;
-                        w.x = pack_bf16x2(v[8 * u + 0], v[8 * u + 1]);
-                        w.y = pack_bf16x2(v[8 * u + 2], v[8 * u + 3]);
-                        w.z = pack_bf16x2(v[8 * u + 4], v[8 * u + 5]);
-                        w.w = pack_bf16x2(v[8 * u + 6], v[8 * u + 7]);
+                        if (p.f16) {
+                            w.x = pack_f16x2(v[8 * u + 0], v[8 * u + 1]);
+                            w.y = pack_f16x2(v[8 * u + 2], v[8 * u + 3]);
+                            w.z = pack_f16x2(v[8 * u + 4], v[8 * u + 5]);
+                            w.w = pack_f16x2(v[8 * u + 6], v[8 * u + 7]);
+                        } else {
+                            w.x = pack_bf16x2(v[8 * u + 0], v[8 * u + 1]);
+                            w.y = pack_bf16x2(v[8 * u + 2], v[8 * u + 3]);
+                            w.z = pack_bf16x2(v[8 * u + 4], v[8 * u + 5]);
+                            w.w = pack_bf16x2(v[8 * u + 6], v[8 * u + 7]);
+                        }
                         *reinterpret_cast<uint4 *>(stg + sw128_offset(row, half * 4 + u)) = w;
                     }
                 }

@@ -14,7 +14,7 @@ constexpr int kHidden = 128;  // c_h of the tensor-core path
 struct K1Args {
     CUtensorMap tm_z;      // z [B][N*N][c_z] bf16, box {64, 128, 1}, 128B swizzle
     CUtensorMap tm_w;      // packed weights [4*c_h][c_z] bf16, box {64, NCOL}, 128B swizzle
-    CUtensorMap tm_a;      // a [B][c_h][N*N] bf16, box {128, channels per warpgroup, 1}
+    CUtensorMap tm_a;      // a [B][c_h][N*N] f16, box {128, channels per warpgroup, 1}
     CUtensorMap tm_b;      // b, same as tm_a
     const uint16_t *mask;  // [B][N*N] bf16 bits, or nullptr
     const float4 *vec;     // [2][c_h] {sum W'_gate, shift_gate, sum W'_proj, shift_proj}
@@ -29,12 +29,14 @@ struct K2Args {
     int BC, N;
     int m_tiles, n_tiles, k_chunks;
     bool incoming;
+    bool f16;              // operands and result in fp16 (else bf16)
+    float x_scale;         // result = x_scale * sum_k ...
 };
 
 struct K3Args {
-    CUtensorMap tm_x;      // x [B][c_h][N*N] bf16, box {64, 64, 1}, 128B swizzle (MN-major A)
+    CUtensorMap tm_x;      // x [B][c_h][N*N] f16, box {64, 64, 1}, 128B swizzle (MN-major A)
     CUtensorMap tm_z;      // z [B][N*N][c_z] bf16, box {64, 128, 1}, 128B swizzle
-    CUtensorMap tm_wo;     // folded W_o [c_z][c_h] bf16, box {64, 128}
+    CUtensorMap tm_wo;     // folded W_o [c_z][c_h] f16, box {64, 128}
     CUtensorMap tm_wg;     // folded W_g [c_z][c_z] bf16, box {64, 128}
     CUtensorMap tm_out;    // out [B][N*N][c_z] f32 (box {32,128,1}) or bf16 (box {64,128,1})
     const uint16_t *mask;
@@ -42,7 +44,8 @@ struct K3Args {
     int B, N;
     long long NN;
     int tiles_per_batch;
-    float eps;
+    float eps;             // input LayerNorm
+    float eps_x;           // output LayerNorm on the stored (scaled) x: eps * x_scale^2
 };
 
 // Kernel resource queries (dynamic shared memory bytes) and launches.
@@ -68,7 +71,8 @@ struct FoldArgs {
     const void *bias;     // [R] or nullptr (= 0)
     int src_bf16;         // storage type of w / gamma / beta / bias
     int R, K;
-    uint16_t *dst;        // bf16 rows [*, K]
+    uint16_t *dst;        // bf16 (or f16 when dst_f16) rows [*, K]
+    int dst_f16;
     int row_mode;         // 0: dst row = r; 1: K1 interleaved layout (see k1 packing)
     int operand;          // row_mode 1: 0 = a, 1 = b
     int kind;             // row_mode 1: 0 = gate, 1 = projection
@@ -97,9 +101,9 @@ cudaError_t f32_project_launch(const float *z, const float *mask, const F32Weigh
                                int c_h, int B, int N, float eps, float *a, float *b,
                                cudaStream_t stream);
 cudaError_t f32_contract_launch(const float *a, const float *b, float *x, int BC, int N,
-                                bool incoming, cudaStream_t stream);
+                                bool incoming, float x_scale, cudaStream_t stream);
 cudaError_t f32_output_launch(const float *z, const float *mask, const float *x,
                               const F32Weights &w, int c_z, int c_h, int B, int N, float eps,
-                              float *out, cudaStream_t stream);
+                              float eps_x, float *out, cudaStream_t stream);
 
 }  // namespace trimul

@@ -5,6 +5,7 @@
 
 #include <cuda.h>
 #include <cuda_bf16.h>
+#include <cuda_fp16.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
 
@@ -18,6 +19,7 @@ enum : unsigned int {
     kErrTimeoutMma = 1u << 1,
     kErrTimeoutEpilogue = 1u << 2,
     kErrTimeoutDrain = 1u << 3,
+    kErrRange = 1u << 4,            // a non-finite fp16 intermediate
 };
 
 // About one second at the B200 boost clock.
@@ -251,12 +253,13 @@ __device__ __forceinline__ uint64_t smem_desc_sw128(const void *smem_ptr, uint32
     return d;
 }
 
-// Instruction descriptor: kind::f16 with bf16 A/B, fp32 D, dense.
-__host__ __device__ constexpr uint32_t idesc_bf16_f32(int M, int N, bool a_mn_major,
-                                                      bool b_mn_major) {
+// Instruction descriptor: kind::f16, fp32 D, dense; A and B both f16 (f16 = true) or
+// both bf16 (the two operands of one MMA always share their type).
+__host__ __device__ constexpr uint32_t idesc_f32acc(int M, int N, bool a_mn_major, bool b_mn_major,
+                                                    bool f16) {
     return (1u << 4)                              // D format: f32
-           | (1u << 7)                            // A format: bf16
-           | (1u << 10)                           // B format: bf16
+           | ((f16 ? 0u : 1u) << 7)               // A format: f16 = 0, bf16 = 1
+           | ((f16 ? 0u : 1u) << 10)              // B format: f16 = 0, bf16 = 1
            | ((a_mn_major ? 1u : 0u) << 15)       // A major-ness
            | ((b_mn_major ? 1u : 0u) << 16)       // B major-ness
            | ((uint32_t)(N >> 3) << 17)           // N / 8
@@ -277,6 +280,11 @@ __device__ __forceinline__ float sigmoid_exp(float v) { return __fdividef(1.0f, 
 
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
     __nv_bfloat162 h = __floats2bfloat162_rn(lo, hi);
+    return *reinterpret_cast<uint32_t *>(&h);
+}
+
+__device__ __forceinline__ uint32_t pack_f16x2(float lo, float hi) {
+    __half2 h = __floats2half2_rn(lo, hi);
     return *reinterpret_cast<uint32_t *>(&h);
 }
 

@@ -148,7 +148,7 @@ static trimul_status_t make_map(CUtensorMap *m, CUtensorMapDataType dt, int rank
 
 static bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
-static size_t dtype_size(trimul_dtype_t t) { return t == TRIMUL_BF16 ? 2 : 4; }
+static size_t dtype_size(trimul_dtype_t t) { return t == TRIMUL_F32 ? 4 : 2; }
 
 static bool overlap(const void *a, size_t na, const void *b, size_t nb) {
     uintptr_t x = reinterpret_cast<uintptr_t>(a), y = reinterpret_cast<uintptr_t>(b);
@@ -289,7 +289,7 @@ extern "C" trimul_status_t tri_mul_layer_create(const trimul_weights_desc_t *w, 
         if (ce == cudaSuccess) {
             FoldArgs fa{};
             fa.w = w->w_o; fa.gamma = w->ln_out_g; fa.beta = w->ln_out_b; fa.bias = w->b_o;
-            fa.src_bf16 = src_bf16; fa.R = cz; fa.K = ch; fa.dst = L->k3_wo; fa.row_mode = 0;
+            fa.src_bf16 = src_bf16; fa.R = cz; fa.K = ch; fa.dst = L->k3_wo; fa.dst_f16 = 1; fa.row_mode = 0;
             fa.sum_out = v3 + 0; fa.shift_out = v3 + 1; fa.out_stride = 4;
             ce = fold_launch(fa, st);
         }
@@ -382,8 +382,8 @@ static trimul_status_t run_project_bf16(const trimul_layer_t *L, const void *z, 
         uint64_t dims[3] = {NN, (uint64_t)ch, (uint64_t)B};
         uint64_t strides[2] = {NN * 2, (uint64_t)ch * NN * 2};
         uint32_t box[3] = {128, (uint32_t)k1_channels_per_warpgroup(cz), 1};
-        TRY(make_map(&p.tm_a, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, a, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_NONE, "K1 a"));
-        TRY(make_map(&p.tm_b, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, b, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_NONE, "K1 b"));
+        TRY(make_map(&p.tm_a, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 3, a, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_NONE, "K1 a"));
+        TRY(make_map(&p.tm_b, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 3, b, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_NONE, "K1 b"));
     }
     p.mask = reinterpret_cast<const uint16_t *>(mask);
     p.vec = L->k1_vec;
@@ -398,26 +398,29 @@ static trimul_status_t run_project_bf16(const trimul_layer_t *L, const void *z, 
     return TRIMUL_OK;
 }
 
-static trimul_status_t run_contract_bf16(const void *a, const void *b, void *x, int64_t BC, int N, bool incoming,
-                                         cudaStream_t st) {
+static trimul_status_t run_contract_tc(const void *a, const void *b, void *x, int64_t BC, int N, bool incoming,
+                                       bool f16, float x_scale, cudaStream_t st) {
     DeviceInfo d;
     TRY(require_sm100(&d));
     K2Args p{};
+    const CUtensorMapDataType dt = f16 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
     uint64_t dims[3] = {(uint64_t)N, (uint64_t)N, (uint64_t)BC};
     uint64_t strides[2] = {(uint64_t)N * 2, (uint64_t)N * N * 2};
     if (!incoming) {
         uint32_t boxa[3] = {64, 128, 1}, boxb[3] = {64, 256, 1};
-        TRY(make_map(&p.tm_a, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, a, dims, strides, boxa, CU_TENSOR_MAP_SWIZZLE_128B, "K2 a"));
-        TRY(make_map(&p.tm_b, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, b, dims, strides, boxb, CU_TENSOR_MAP_SWIZZLE_128B, "K2 b"));
+        TRY(make_map(&p.tm_a, dt, 3, a, dims, strides, boxa, CU_TENSOR_MAP_SWIZZLE_128B, "K2 a"));
+        TRY(make_map(&p.tm_b, dt, 3, b, dims, strides, boxb, CU_TENSOR_MAP_SWIZZLE_128B, "K2 b"));
     } else {
         uint32_t box[3] = {64, 64, 1};
-        TRY(make_map(&p.tm_a, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, a, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_128B, "K2 a"));
-        TRY(make_map(&p.tm_b, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, b, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_128B, "K2 b"));
+        TRY(make_map(&p.tm_a, dt, 3, a, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_128B, "K2 a"));
+        TRY(make_map(&p.tm_b, dt, 3, b, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_128B, "K2 b"));
     }
     {
         uint32_t box[3] = {64, 128, 1};
-        TRY(make_map(&p.tm_x, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, x, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_128B, "K2 x"));
+        TRY(make_map(&p.tm_x, dt, 3, x, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_128B, "K2 x"));
     }
+    p.f16 = f16;
+    p.x_scale = x_scale;
     p.BC = (int)BC;
     p.N = N;
     p.m_tiles = (N + 127) / 128;
@@ -431,7 +434,7 @@ static trimul_status_t run_contract_bf16(const void *a, const void *b, void *x, 
 }
 
 static trimul_status_t run_output_bf16(const trimul_layer_t *L, const void *z, const void *mask, const void *x,
-                                       void *out, bool out_f32, int B, int N, cudaStream_t st) {
+                                       float x_scale, void *out, bool out_f32, int B, int N, cudaStream_t st) {
     DeviceInfo d;
     TRY(require_sm100(&d));
     const uint64_t NN = (uint64_t)N * N;
@@ -441,7 +444,7 @@ static trimul_status_t run_output_bf16(const trimul_layer_t *L, const void *z, c
         uint64_t dims[3] = {NN, (uint64_t)ch, (uint64_t)B};
         uint64_t strides[2] = {NN * 2, (uint64_t)ch * NN * 2};
         uint32_t box[3] = {64, 64, 1};
-        TRY(make_map(&p.tm_x, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, x, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_128B, "K3 x"));
+        TRY(make_map(&p.tm_x, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 3, x, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_128B, "K3 x"));
     }
     {
         uint64_t dims[3] = {(uint64_t)cz, NN, (uint64_t)B};
@@ -453,7 +456,7 @@ static trimul_status_t run_output_bf16(const trimul_layer_t *L, const void *z, c
         uint64_t dims[2] = {(uint64_t)ch, (uint64_t)cz};
         uint64_t strides[1] = {(uint64_t)ch * 2};
         uint32_t box[2] = {64, 128};
-        TRY(make_map(&p.tm_wo, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, L->k3_wo, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_128B, "K3 wo"));
+        TRY(make_map(&p.tm_wo, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, L->k3_wo, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_128B, "K3 wo"));
     }
     {
         uint64_t dims[2] = {(uint64_t)cz, (uint64_t)cz};
@@ -476,6 +479,7 @@ static trimul_status_t run_output_bf16(const trimul_layer_t *L, const void *z, c
     p.NN = (long long)NN;
     p.tiles_per_batch = (int)((NN + 127) / 128);
     p.eps = L->eps;
+    p.eps_x = L->eps * x_scale * x_scale;
     const int G = k3_groups(cz);
     const int grid = grid_for(d.sms, (long long)G * B * p.tiles_per_batch, G);
     TRY_CUDA(k3_launch(cz, out_f32, p, grid, st), "K3 launch");
@@ -503,10 +507,18 @@ extern "C" trimul_status_t tri_mul_project(const trimul_pair_t *z, const void *m
     return TRIMUL_OK;
 }
 
+extern "C" float tri_mul_contract_scale(int64_t N) {
+    if (N < 1) return 0.f;
+    int lg = 0;
+    while ((int64_t(1) << lg) < N) ++lg;       // ceil(log2 N)
+    return ldexpf(1.0f, -((lg + 1) / 2));       // 2^-ceil(log2(N) / 2)
+}
+
 extern "C" trimul_status_t tri_mul_contract(const void *a, const void *b, void *x, int64_t B, int64_t C, int64_t N,
-                                            trimul_dtype_t dtype, trimul_direction_t dir, void *stream) {
+                                            trimul_dtype_t dtype, trimul_direction_t dir, float x_scale, void *stream) {
     if (!a || !b || !x) return fail(TRIMUL_ERR_INVALID_ARG, "NULL tensor");
-    if (dtype != TRIMUL_F32 && dtype != TRIMUL_BF16) return fail(TRIMUL_ERR_INVALID_ARG, "unknown dtype");
+    if (dtype != TRIMUL_F32 && dtype != TRIMUL_BF16 && dtype != TRIMUL_F16) return fail(TRIMUL_ERR_INVALID_ARG, "unknown dtype");
+    if (!(x_scale > 0.f) || !(x_scale < 3.0e38f)) return fail(TRIMUL_ERR_INVALID_ARG, "x_scale must be positive and finite");
     if (dir != TRIMUL_OUTGOING && dir != TRIMUL_INCOMING) return fail(TRIMUL_ERR_INVALID_ARG, "unknown direction");
     if (B < 1 || C < 1) return fail(TRIMUL_ERR_INVALID_ARG, "B and C must be positive");
     if (N < 8 || N % 8 || N > 16384) return fail(TRIMUL_ERR_UNSUPPORTED_SHAPE, "N=%lld must be a multiple of 8 in [8, 16384]", (long long)N);
@@ -515,16 +527,18 @@ extern "C" trimul_status_t tri_mul_contract(const void *a, const void *b, void *
     const size_t bytes = (size_t)B * C * N * N * dtype_size(dtype);
     if (overlap(x, bytes, a, bytes) || overlap(x, bytes, b, bytes)) return fail(TRIMUL_ERR_INVALID_ARG, "x overlaps a or b");
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
-    if (dtype == TRIMUL_BF16) return run_contract_bf16(a, b, x, B * C, (int)N, dir == TRIMUL_INCOMING, st);
+    if (dtype != TRIMUL_F32)
+        return run_contract_tc(a, b, x, B * C, (int)N, dir == TRIMUL_INCOMING, dtype == TRIMUL_F16, x_scale, st);
     TRY_CUDA(f32_contract_launch(reinterpret_cast<const float *>(a), reinterpret_cast<const float *>(b),
-                                 reinterpret_cast<float *>(x), (int)(B * C), (int)N, dir == TRIMUL_INCOMING, st),
+                                 reinterpret_cast<float *>(x), (int)(B * C), (int)N, dir == TRIMUL_INCOMING, x_scale, st),
              "fp32 contraction launch");
     return TRIMUL_OK;
 }
 
-extern "C" trimul_status_t tri_mul_output_gate(const trimul_pair_t *z, const void *mask, const void *x,
+extern "C" trimul_status_t tri_mul_output_gate(const trimul_pair_t *z, const void *mask, const void *x, float x_scale,
                                                const trimul_layer_t *L, trimul_pair_t *out, void *stream) {
     TRY(check_problem(z, mask, L));
+    if (!(x_scale > 0.f) || !(x_scale < 3.0e38f)) return fail(TRIMUL_ERR_INVALID_ARG, "x_scale must be positive and finite");
     TRY(check_pair(out, "out"));
     if (!x) return fail(TRIMUL_ERR_INVALID_ARG, "x is NULL");
     if (!aligned16(x)) return fail(TRIMUL_ERR_ALIGNMENT, "x not 16-byte aligned");
@@ -535,10 +549,10 @@ extern "C" trimul_status_t tri_mul_output_gate(const trimul_pair_t *z, const voi
     if (overlap(out->data, pair_bytes(out), x, xbytes)) return fail(TRIMUL_ERR_INVALID_ARG, "out overlaps x");
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
     if (z->dtype == TRIMUL_BF16)
-        return run_output_bf16(L, z->data, mask, x, out->data, out->dtype == TRIMUL_F32, (int)z->B, (int)z->N, st);
+        return run_output_bf16(L, z->data, mask, x, x_scale, out->data, out->dtype == TRIMUL_F32, (int)z->B, (int)z->N, st);
     TRY_CUDA(f32_output_launch(reinterpret_cast<const float *>(z->data), reinterpret_cast<const float *>(mask),
                                reinterpret_cast<const float *>(x), L->f32, L->c_z, L->c_h, (int)z->B, (int)z->N, L->eps,
-                               reinterpret_cast<float *>(out->data), st),
+                               L->eps * x_scale * x_scale, reinterpret_cast<float *>(out->data), st),
              "fp32 output launch");
     return TRIMUL_OK;
 }
@@ -562,9 +576,11 @@ extern "C" trimul_status_t tri_mul_forward(const trimul_pair_t *z, const void *m
     if (L->timing) TRY_CUDA(cudaEventRecord(L->events[0], st), "event record");
     TRY(tri_mul_project(z, mask, L, a, b, stream));
     if (L->timing) TRY_CUDA(cudaEventRecord(L->events[1], st), "event record");
-    TRY(tri_mul_contract(a, b, x, z->B, L->c_h, z->N, z->dtype, dir, stream));
+    const bool tc = z->dtype == TRIMUL_BF16;
+    const float x_scale = tc ? tri_mul_contract_scale(z->N) : 1.0f;
+    TRY(tri_mul_contract(a, b, x, z->B, L->c_h, z->N, tc ? TRIMUL_F16 : TRIMUL_F32, dir, x_scale, stream));
     if (L->timing) TRY_CUDA(cudaEventRecord(L->events[2], st), "event record");
-    TRY(tri_mul_output_gate(z, mask, x, L, out, stream));
+    TRY(tri_mul_output_gate(z, mask, x, x_scale, L, out, stream));
     if (L->timing) TRY_CUDA(cudaEventRecord(L->events[3], st), "event record");
     return TRIMUL_OK;
 }
@@ -575,6 +591,8 @@ extern "C" trimul_status_t tri_mul_check_device_status(void) {
     TRY_CUDA(cudaMemcpyFromSymbol(&v, g_device_error, sizeof(v)), "read device error word");
     if (v) {
         TRY_CUDA(cudaMemcpyToSymbol(g_device_error, &zero, sizeof(zero)), "clear device error word");
+        if (v == (unsigned int)kErrRange)
+            return fail(TRIMUL_ERR_RANGE, "a non-finite fp16 intermediate (x) was seen (code 0x%x)", v);
         return fail(TRIMUL_ERR_DEVICE_TIMEOUT, "a kernel gave up on a bounded wait (code 0x%x)", v);
     }
     return TRIMUL_OK;
@@ -590,6 +608,7 @@ extern "C" const char *tri_mul_status_string(trimul_status_t s) {
         case TRIMUL_ERR_CUDA: return "CUDA error";
         case TRIMUL_ERR_DEVICE_TIMEOUT: return "device wait timed out";
         case TRIMUL_ERR_ALIGNMENT: return "pointer not 16-byte aligned";
+        case TRIMUL_ERR_RANGE: return "intermediate out of fp16 range";
     }
     return "unknown status";
 }

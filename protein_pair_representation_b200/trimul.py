@@ -19,6 +19,7 @@ OUTGOING = 0
 INCOMING = 1
 F32 = 0
 BF16 = 1
+F16 = 2
 _DIRS = {"outgoing": OUTGOING, "incoming": INCOMING, OUTGOING: OUTGOING, INCOMING: INCOMING}
 
 WEIGHT_ORDER = (
@@ -29,7 +30,7 @@ WEIGHT_ORDER = (
 STATUS_NAMES = {
     0: "TRIMUL_OK", 1: "TRIMUL_ERR_INVALID_ARG", 2: "TRIMUL_ERR_UNSUPPORTED_SHAPE",
     3: "TRIMUL_ERR_UNSUPPORTED_DEVICE", 4: "TRIMUL_ERR_WORKSPACE", 5: "TRIMUL_ERR_CUDA",
-    6: "TRIMUL_ERR_DEVICE_TIMEOUT", 7: "TRIMUL_ERR_ALIGNMENT",
+    6: "TRIMUL_ERR_DEVICE_TIMEOUT", 7: "TRIMUL_ERR_ALIGNMENT", 8: "TRIMUL_ERR_RANGE",
 }
 
 
@@ -79,8 +80,10 @@ def load_library():
         lib.tri_mul_layer_bind_workspace.argtypes = [vp, vp, ctypes.c_size_t]
         lib.tri_mul_forward.argtypes = [P(_Pair), vp, vp, st, P(_Pair), vp]
         lib.tri_mul_project.argtypes = [P(_Pair), vp, vp, vp, vp, vp]
-        lib.tri_mul_contract.argtypes = [vp, vp, vp, i64, i64, i64, st, st, vp]
-        lib.tri_mul_output_gate.argtypes = [P(_Pair), vp, vp, vp, P(_Pair), vp]
+        lib.tri_mul_contract.argtypes = [vp, vp, vp, i64, i64, i64, st, st, ctypes.c_float, vp]
+        lib.tri_mul_contract_scale.argtypes = [i64]
+        lib.tri_mul_contract_scale.restype = ctypes.c_float
+        lib.tri_mul_output_gate.argtypes = [P(_Pair), vp, vp, ctypes.c_float, vp, P(_Pair), vp]
         lib.tri_mul_layer_set_timing_events.argtypes = [vp, P(vp)]
         lib.tri_mul_kernels_per_forward.argtypes = []
         lib.tri_mul_check_device_status.argtypes = []
@@ -108,7 +111,19 @@ def _dtype_code(dt: torch.dtype) -> int:
         return F32
     if dt == torch.bfloat16:
         return BF16
+    if dt == torch.float16:
+        return F16
     raise TypeError(f"unsupported dtype {dt}")
+
+
+def intermediate_dtype(z_dtype: torch.dtype) -> torch.dtype:
+    """Storage type of a, b and x: float16 for a bfloat16 z, float32 for a float32 z."""
+    return torch.float16 if z_dtype == torch.bfloat16 else torch.float32
+
+
+def contract_scale(N: int) -> float:
+    """The power of two tri_mul_forward stores x multiplied by on the tensor-core path."""
+    return float(load_library().tri_mul_contract_scale(N))
 
 
 def _stream_ptr(stream) -> ctypes.c_void_p:
@@ -216,9 +231,9 @@ class TriMulLayer:
     __call__ = forward
 
     def project(self, z: torch.Tensor, mask: torch.Tensor | None = None, stream=None):
-        """K1 alone: a, b as [B, c_h, N, N] in z's dtype."""
+        """K1 alone: a, b as [B, c_h, N, N] in the intermediate dtype."""
         B, N = z.shape[0], z.shape[1]
-        a = torch.empty((B, self.c_h, N, N), dtype=z.dtype, device=z.device)
+        a = torch.empty((B, self.c_h, N, N), dtype=intermediate_dtype(z.dtype), device=z.device)
         b = torch.empty_like(a)
         zp = _pair(z)
         _check(self._lib.tri_mul_project(ctypes.byref(zp), _mask_ptr(mask, z), self.handle,
@@ -226,20 +241,23 @@ class TriMulLayer:
         return a, b
 
     def output_gate(self, z: torch.Tensor, x: torch.Tensor, mask: torch.Tensor | None = None,
-                    out: torch.Tensor | None = None, out_dtype: torch.dtype | None = None, stream=None):
-        """K3 alone: out from z and x [B, c_h, N, N] (x in z's dtype)."""
-        if x.dtype != z.dtype or not x.is_contiguous() or tuple(x.shape) != (z.shape[0], self.c_h, z.shape[1], z.shape[2]):
-            raise ValueError("x must be a contiguous [B, c_h, N, N] tensor in z's dtype")
+                    out: torch.Tensor | None = None, out_dtype: torch.dtype | None = None, x_scale: float = 1.0,
+                    stream=None):
+        """K3 alone: out from z and x [B, c_h, N, N] (intermediate dtype, holding x_scale * x)."""
+        if (x.dtype != intermediate_dtype(z.dtype) or not x.is_contiguous()
+                or tuple(x.shape) != (z.shape[0], self.c_h, z.shape[1], z.shape[2])):
+            raise ValueError("x must be a contiguous [B, c_h, N, N] tensor in the intermediate dtype")
         if out is None:
             out = torch.empty(z.shape, dtype=out_dtype or torch.float32, device=z.device)
         zp, op = _pair(z), _pair(out)
-        _check(self._lib.tri_mul_output_gate(ctypes.byref(zp), _mask_ptr(mask, z), x.data_ptr(), self.handle,
-                                             ctypes.byref(op), _stream_ptr(stream)))
+        _check(self._lib.tri_mul_output_gate(ctypes.byref(zp), _mask_ptr(mask, z), x.data_ptr(), x_scale,
+                                             self.handle, ctypes.byref(op), _stream_ptr(stream)))
         return out
 
 
-def contract(a: torch.Tensor, b: torch.Tensor, direction="outgoing", out: torch.Tensor | None = None, stream=None):
-    """K2 alone on [B, C, N, N] tensors (float32 or bfloat16)."""
+def contract(a: torch.Tensor, b: torch.Tensor, direction="outgoing", out: torch.Tensor | None = None,
+             x_scale: float = 1.0, stream=None):
+    """K2 alone on [B, C, N, N] tensors (float16 / bfloat16 on tensor cores, float32 on CUDA cores)."""
     lib = load_library()
     if a.shape != b.shape or a.dim() != 4 or a.shape[2] != a.shape[3] or a.dtype != b.dtype:
         raise ValueError("a and b must be [B, C, N, N] of one dtype")
@@ -249,7 +267,7 @@ def contract(a: torch.Tensor, b: torch.Tensor, direction="outgoing", out: torch.
         out = torch.empty_like(a)
     B, C, N, _ = a.shape
     _check(lib.tri_mul_contract(a.data_ptr(), b.data_ptr(), out.data_ptr(), B, C, N, _dtype_code(a.dtype),
-                                _DIRS[direction], _stream_ptr(stream)))
+                                _DIRS[direction], x_scale, _stream_ptr(stream)))
     return out
 
 

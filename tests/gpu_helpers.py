@@ -5,6 +5,7 @@ import numpy as np
 import torch
 
 BF16_REL = 2.0 ** -8   # one bf16 ulp relative to the value (round-to-nearest is half of it)
+F16_REL = 2.0 ** -10   # one fp16 ulp relative to the value
 
 
 def torch_dtype(kind: str):
@@ -41,12 +42,13 @@ def assert_close_rms(got, ref, tol, what=""):
     return ratio
 
 
-def assert_close_bf16(got, ref, rms_tol, what=""):
-    """Elementwise |got - ref| <= one bf16 ulp of |ref| + rms_tol * RMS(ref) (bf16-stored results)."""
+def assert_close_ulp(got, ref, rms_tol, rel=BF16_REL, what=""):
+    """Elementwise |got - ref| <= rel * |ref| + rms_tol * RMS(ref) (results stored in a 16-bit type;
+    rel is one ulp of that type relative to the value)."""
     got = np.asarray(got, dtype=np.float64)
     ref = np.asarray(ref, dtype=np.float64)
     assert np.all(np.isfinite(got)), f"{what}: non-finite values"
-    bound = BF16_REL * np.abs(ref) + rms_tol * rms(ref)
+    bound = rel * np.abs(ref) + rms_tol * rms(ref)
     bad = np.abs(got - ref) > bound
     if bad.any():
         i = np.unravel_index(np.argmax(np.abs(got - ref) - bound), ref.shape)
@@ -56,3 +58,11 @@ def assert_close_bf16(got, ref, rms_tol, what=""):
 def to_pair_major(t: torch.Tensor) -> np.ndarray:
     """[B, C, N, N] device tensor -> [B, N, N, C] float64 numpy."""
     return t.float().permute(0, 2, 3, 1).contiguous().cpu().numpy().astype(np.float64)
+
+
+def assert_close_bf16(got, ref, rms_tol, what=""):
+    assert_close_ulp(got, ref, rms_tol, BF16_REL, what)
+
+
+def assert_close_f16(got, ref, rms_tol, what=""):
+    assert_close_ulp(got, ref, rms_tol, F16_REL, what)

@@ -46,7 +46,7 @@ def test_library_is_built_for_sm100a(lib):
 
 
 def test_status_strings_and_versions(lib):
-    for code in range(8):
+    for code in range(9):
         assert lib.tri_mul_status_string(code)
     assert lib.tri_mul_status_string(99) == b"unknown status"
     assert lib.tri_mul_abi_version() == 100
@@ -65,16 +65,29 @@ def test_null_arguments_are_rejected_on_the_host(lib):
 def test_contract_validation_happens_before_any_launch(lib):
     fake = ctypes.c_void_p(1 << 20)  # never dereferenced: validation fails first
     # N not a multiple of 8
-    assert lib.tri_mul_contract(fake, fake, fake, 1, 4, 12, tm.BF16, 0, None) == 2
+    assert lib.tri_mul_contract(fake, fake, fake, 1, 4, 12, tm.F16, 0, 1.0, None) == 2
     # unknown direction
-    assert lib.tri_mul_contract(fake, fake, fake, 1, 4, 16, tm.BF16, 7, None) == 1
+    assert lib.tri_mul_contract(fake, fake, fake, 1, 4, 16, tm.F16, 7, 1.0, None) == 1
     # misaligned pointer
     bad = ctypes.c_void_p((1 << 20) + 8)
-    assert lib.tri_mul_contract(bad, fake, ctypes.c_void_p(1 << 24), 1, 4, 16, tm.BF16, 0, None) == 7
+    assert lib.tri_mul_contract(bad, fake, ctypes.c_void_p(1 << 24), 1, 4, 16, tm.F16, 0, 1.0, None) == 7
     # x overlapping a
-    assert lib.tri_mul_contract(fake, ctypes.c_void_p(1 << 24), fake, 1, 4, 16, tm.BF16, 0, None) == 1
+    assert lib.tri_mul_contract(fake, ctypes.c_void_p(1 << 24), fake, 1, 4, 16, tm.BF16, 0, 1.0, None) == 1
     # too many channels for the grid
-    assert lib.tri_mul_contract(fake, ctypes.c_void_p(1 << 30), ctypes.c_void_p(1 << 34), 1, 70000, 16, tm.F32, 0, None) == 2
+    assert lib.tri_mul_contract(fake, ctypes.c_void_p(1 << 30), ctypes.c_void_p(1 << 34), 1, 70000, 16, tm.F32, 0,
+                                1.0, None) == 2
+    # scale must be positive
+    assert lib.tri_mul_contract(fake, ctypes.c_void_p(1 << 30), ctypes.c_void_p(1 << 34), 1, 4, 16, tm.F16, 0,
+                                0.0, None) == 1
+
+
+def test_contract_scale_is_a_power_of_two_near_inverse_sqrt_n(lib):
+    import math
+    for N, expect in ((1, 1.0), (8, 0.25), (64, 0.125), (256, 1 / 16), (512, 1 / 32), (2048, 1 / 64)):
+        s = lib.tri_mul_contract_scale(N)
+        assert s == expect, (N, s)
+        assert math.log2(s) == int(math.log2(s))
+    assert lib.tri_mul_contract_scale(0) == 0.0
 
 
 def test_layer_create_rejects_bad_widths_before_allocating(lib):
@@ -84,3 +97,14 @@ def test_layer_create_rejects_bad_widths_before_allocating(lib):
     assert lib.tri_mul_layer_create(ctypes.byref(desc), None, ctypes.byref(handle)) == 2
     desc.c_z, desc.eps = 128, 0.0
     assert lib.tri_mul_layer_create(ctypes.byref(desc), None, ctypes.byref(handle)) == 1
+
+
+@pytest.mark.skipif(__import__("torch").cuda.is_available(), reason="would launch on fake pointers")
+def test_adjacent_f16_planes_pass_validation(lib):
+    """Planes placed back to back (2 bytes per element for F16) do not count as overlapping:
+    validation passes and the call only fails later, at the CUDA device query, on a GPU-less host."""
+    B, C, N = 1, 4, 16
+    plane = B * C * N * N * 2
+    a, b, x = ctypes.c_void_p(1 << 20), ctypes.c_void_p((1 << 20) + plane), ctypes.c_void_p((1 << 20) + 2 * plane)
+    st = lib.tri_mul_contract(a, b, x, B, C, N, tm.F16, 0, 1.0, None)
+    assert st in (3, 5), lib.tri_mul_last_error()

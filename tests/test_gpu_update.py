@@ -128,8 +128,9 @@ def test_stage_entry_points_compose_to_forward():
     for d in ("outgoing", "incoming"):
         full = layer.forward(z, m, d)
         a, b = layer.project(z, m)
-        x = tm.contract(a, b, d)
-        staged = layer.output_gate(z, x, m)
+        scale = tm.contract_scale(z.shape[1])
+        x = tm.contract(a, b, d, x_scale=scale)
+        staged = layer.output_gate(z, x, m, x_scale=scale)
         torch.cuda.synchronize()
         assert torch.equal(full, staged)
 
