@@ -171,6 +171,28 @@ trimul_status_t tri_mul_output_gate(const trimul_pair_t *z, const void *mask, co
                                     float x_scale, const trimul_layer_t *layer,
                                     trimul_pair_t *out, void *stream);
 
+/* tri_mul_forward for callers that cannot allocate device memory (for example a plug-in
+ * inside a framework that owns the allocator and gives it no way to ask for memory, or
+ * a path that must not risk an allocation failing or stalling mid-work). Same arguments,
+ * kernels and results as tri_mul_forward, but a, b and x live in a fixed array built
+ * into the library (TRIMUL_NOALLOC_SCRATCH_BYTES of device memory on every GPU that
+ * loads it, held until the process exits) instead of a bound workspace; the layer's
+ * workspace and timing events are not used. It allocates nothing.
+ *   - Problems whose a, b and x need more than TRIMUL_NOALLOC_SCRATCH_BYTES (that is,
+ *     tri_mul_workspace_bytes() > TRIMUL_NOALLOC_SCRATCH_BYTES; for a BF16 z with
+ *     c_h = 128 the limit is B * N * N <= 65536, e.g. N = 256 at B = 1) are rejected
+ *     with TRIMUL_ERR_WORKSPACE.
+ *   - The first call on each device looks up the array's device address (once, with
+ *     that device current); make that first call before any stream capture.
+ *   - All calls share the one array and it keeps the last call's contents (nothing in
+ *     it needs to start at zero). Calls that overlap on the GPU (different streams
+ *     without ordering between them, or concurrent host threads) race on it: order them.
+ * This entry point is an engineering addition with no counterpart in the pages. */
+#define TRIMUL_NOALLOC_SCRATCH_BYTES (48u * 1024u * 1024u)
+trimul_status_t tri_mul_forward_noalloc(const trimul_pair_t *z, const void *mask,
+                                        const trimul_layer_t *layer, trimul_direction_t direction,
+                                        trimul_pair_t *out, void *stream);
+
 /* Optional per-kernel timing: when `events` is non-NULL, every later
  * tri_mul_forward on this handle records events[0] before K1, events[1] after
  * K1, events[2] after K2 and events[3] after K3 on its stream. The four values

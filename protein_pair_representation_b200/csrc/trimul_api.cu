@@ -54,6 +54,11 @@ static trimul_status_t fail(trimul_status_t st, const char *fmt, ...) {
     return st;
 }
 
+namespace trimul {
+// Lets other translation units of the library set the calling thread's error detail.
+trimul_status_t set_last_error(trimul_status_t st, const char *msg) { return fail(st, "%s", msg); }
+}  // namespace trimul
+
 static trimul_status_t cuda_fail(cudaError_t e, const char *what) {
     return fail(TRIMUL_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e));
 }
