@@ -26,6 +26,9 @@ __global__ void fold_kernel(FoldArgs a) {
         const int g = a.operand * a.gpo + r / a.cpg;
         const int rr = r % a.cpg;
         dst_row = g * a.ncol + (rr / 16) * 32 + a.kind * 16 + (rr % 16);
+    } else if (a.row_mode == 2) {
+        // one block of rows per operand: [gate rows of all channels, projection rows of all channels]
+        dst_row = a.operand * 2 * a.R + a.kind * a.R + r;
     }
     double sum_w = 0.0, shift = 0.0;
     for (int k = tid; k < a.K; k += blockDim.x) {

@@ -13,13 +13,13 @@
 // so the tensor cores multiply the raw bf16 z tile, and the epilogue applies the
 // per-pair (mean, rstd) and the per-channel (sum W', shift) pair of constants.
 //
-// Tile: 128 consecutive pairs of one batch element (one TMEM lane per pair) times
-// NCOL packed weight rows. Packed row layout inside a group: 32-row blocks, each
-// [16 gate rows, 16 projection rows] for 16 channels, so one 32-column TMEM load
-// gives a thread both factors of 16 outputs. c_z = 128 uses NCOL = 256 (one group
-// per operand); c_z = 384 uses NCOL = 128 (two groups per operand) so that the
-// group's weights stay resident in shared memory. A CTA keeps one group for its
-// whole life (grid is a multiple of the group count).
+// Two kernels. c_z = 128 (k1_project_cm_kernel, further below) puts one hidden channel
+// on each TMEM lane. c_z = 384 (k1_project_kernel) puts one pair on each TMEM lane:
+// 128 consecutive pairs of one batch element times NCOL = 128 packed weight rows, laid
+// out in 32-row blocks of [16 gate rows, 16 projection rows] for 16 channels so one
+// 32-column TMEM load gives a thread both factors of 16 outputs, with four column groups
+// (two per operand) so each group's weights stay resident in shared memory. A CTA keeps
+// one group for its whole life (the grid is a multiple of the group count).
 //
 // Warps: 0-7 epilogue (two warpgroups, half the columns each), 8-11 LayerNorm
 // statistics (one thread per pair), 12 TMA producer, 13 TMEM allocator + MMA issuer.
@@ -283,10 +283,281 @@ __global__ void __launch_bounds__(448, 1) k1_project_kernel(const __grid_constan
     }
 }
 
-int k1_ncol(int c_z) { return c_z == 128 ? K1Cfg<128>::NCOL : K1Cfg<384>::NCOL; }
-int k1_groups(int c_z) { return c_z == 128 ? K1Cfg<128>::G : K1Cfg<384>::G; }
-int k1_channels_per_warpgroup(int c_z) { return c_z == 128 ? K1Cfg<128>::CH_WG : K1Cfg<384>::CH_WG; }
-size_t k1_smem_bytes(int c_z) { return c_z == 128 ? K1Cfg<128>::SMEM : K1Cfg<384>::SMEM; }
+// ------------------------------------------------------------------------------------------
+// K1 for c_z = 128: accumulators with one TMEM lane per hidden channel.
+//
+// D_gate[c, p] = W'_gate[c] . z_p and D_proj[c, p] = W'_proj[c] . z_p for the 128 channels
+// of one operand (a or b) and 128 pairs: A = folded weights [128 channels x c_z], B = the z
+// tile [128 pairs x c_z], both K-major. A thread of the epilogue owns one channel for the
+// whole kernel, so that channel's four folding constants stay in registers; the per-pair
+// LayerNorm statistics are read from shared memory (broadcast, four pairs per load); and
+// consecutive pairs of one channel are consecutive columns, which pack directly into
+// 16-byte rows of the channel-major output tile.
+// Warps: 0-7 epilogue (warpgroup 0: pairs 0-63 of the tile, warpgroup 1: pairs 64-127),
+// 8-11 LayerNorm statistics, 12 TMA producer, 13 TMEM allocator + MMA issuer.
+struct K1CmCfg {
+    static constexpr int CZ = 128, C_H = kHidden, KC = CZ / 64;
+    static constexpr int G = 2;                               // one group per operand
+    static constexpr int W_CHUNK = 2 * C_H * 64 * 2;          // [gate 128 rows, proj 128 rows] x 64 k
+    static constexpr int W_BYTES = KC * W_CHUNK;              // 64 KB
+    static constexpr int CHUNK = 128 * 64 * 2;                // z chunk: 128 pairs x 64 channels
+    static constexpr int STG_BYTES = C_H * 64 * 2;            // per warpgroup: [128 ch][64 pairs] f16
+    static constexpr int SNB = 2;
+    static constexpr int STATS_BYTES = SNB * 3 * 128 * 4;     // mean, rstd, mask per pair
+    static constexpr int FIXED = 1024 + W_BYTES + 2 * STG_BYTES + STATS_BYTES + 1024;
+    static constexpr int S = (232448 - FIXED) / CHUNK > 8 ? 8 : (232448 - FIXED) / CHUNK;
+    static constexpr size_t SMEM = FIXED + (size_t)S * CHUNK;
+    static constexpr int THREADS = 448;
+    static constexpr int TMA_WARP = 12, MMA_WARP = 13;
+};
+
+__global__ void __launch_bounds__(448, 1) k1_project_cm_kernel(const __grid_constant__ K1Args p) {
+    using C = K1CmCfg;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *base = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint8_t *w_s = base;                                  // KC chunks of [256 rows][64] bf16
+    uint8_t *chunks = w_s + C::W_BYTES;                   // S chunks of [128 pairs][64] bf16
+    uint8_t *staging = chunks + C::S * C::CHUNK;          // 2 x [128 ch][64 pairs] f16, 128B swizzle
+    float *st_mean = reinterpret_cast<float *>(staging + 2 * C::STG_BYTES);  // [SNB][128]
+    float *st_rstd = st_mean + C::SNB * 128;
+    float *st_mask = st_rstd + C::SNB * 128;
+    K1Smem &s = *reinterpret_cast<K1Smem *>(st_mask + C::SNB * 128);
+
+    const int warp = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31;
+    volatile int *abort_flag = &s.abort_flag;
+
+    const int operand = blockIdx.x % C::G;
+    const int cta_in_group = blockIdx.x / C::G;
+    const int ctas_per_group = gridDim.x / C::G;
+    const int num_ptiles = p.B * p.tiles_per_batch;
+
+    if (threadIdx.x == 0) {
+        mbar_init(&s.wbar, 1);
+        for (int i = 0; i < C::S; ++i) {
+            mbar_init(&s.full[i], 1);
+            mbar_init(&s.empty[i], 1 + 4);  // MMA commit + 4 stats warps
+        }
+        for (int i = 0; i < 2; ++i) {
+            mbar_init(&s.tfull[i], 1);
+            mbar_init(&s.tempty[i], 8);
+        }
+        for (int i = 0; i < C::SNB; ++i) {
+            mbar_init(&s.sfull[i], 4);
+            mbar_init(&s.sempty[i], 8);
+        }
+        mbar_init(&s.drain, 1);
+        s.abort_flag = 0;
+        fence_mbarrier_init();
+    }
+    if (warp == C::MMA_WARP) {
+        tmem_alloc(&s.tmem_base, 512);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem_base = s.tmem_base;
+
+    if (warp == C::TMA_WARP) {
+        if (lane == 0) {
+            tma_prefetch_desc(&p.tm_z);
+            tma_prefetch_desc(&p.tm_w);
+            mbar_arrive_expect_tx(&s.wbar, C::W_BYTES);
+            for (int kc = 0; kc < C::KC; ++kc)
+                tma_load_2d(w_s + kc * C::W_CHUNK, &p.tm_w, &s.wbar, kc * 64, operand * 2 * C::C_H);
+            int stage = 0;
+            uint32_t phase = 0;
+            uint32_t filled = 0;
+            for (int pt = cta_in_group; pt < num_ptiles; pt += ctas_per_group) {
+                const int b = pt / p.tiles_per_batch;
+                const int p0 = (pt - b * p.tiles_per_batch) * 128;
+                for (int kc = 0; kc < C::KC; ++kc) {
+                    if (!mbar_wait(&s.empty[stage], phase ^ 1, abort_flag, kErrTimeoutProducer)) goto producer_abort;
+                    mbar_arrive_expect_tx(&s.full[stage], C::CHUNK);
+                    tma_load_3d(chunks + stage * C::CHUNK, &p.tm_z, &s.full[stage], kc * 64, p0, b);
+                    ++filled;
+                    if (++stage == C::S) { stage = 0; phase ^= 1; }
+                }
+            }
+            goto producer_done;
+        producer_abort:
+            for (uint32_t i = 0; i < (filled < (uint32_t)C::S ? filled : (uint32_t)C::S); ++i) {
+                uint32_t f = filled - 1 - i;
+                mbar_drain(&s.full[f % C::S], (f / C::S) & 1);
+            }
+        producer_done:
+            mbar_drain(&s.wbar, 0);
+        }
+    } else if (warp == C::MMA_WARP) {
+        if (lane == 0) {
+            const uint32_t idesc = idesc_f32acc(128, 128, false, false, false);
+            bool ok = mbar_wait(&s.wbar, 0, abort_flag, kErrTimeoutMma);
+            int stage = 0;
+            uint32_t phase = 0;
+            int abuf = 0;
+            uint32_t aphase = 0;
+            for (int pt = cta_in_group; ok && pt < num_ptiles; pt += ctas_per_group) {
+                if (!mbar_wait(&s.tempty[abuf], aphase ^ 1, abort_flag, kErrTimeoutMma)) break;
+                tc_fence_after();
+                const uint32_t d_gate = tmem_base + abuf * 256;
+                const uint32_t d_proj = d_gate + 128;
+                for (int kc = 0; kc < C::KC; ++kc) {
+                    if (!mbar_wait(&s.full[stage], phase, abort_flag, kErrTimeoutMma)) { ok = false; break; }
+                    tc_fence_after();
+                    const uint8_t *zc = chunks + stage * C::CHUNK;
+                    const uint8_t *wg = w_s + kc * C::W_CHUNK;
+#pragma unroll
+                    for (int kk = 0; kk < 4; ++kk) {
+                        const uint64_t bd = smem_desc_sw128(zc + kk * 32, 16, 1024);
+                        const uint64_t ag = smem_desc_sw128(wg + kk * 32, 16, 1024);
+                        const uint64_t ap = smem_desc_sw128(wg + C::C_H * 128 + kk * 32, 16, 1024);
+                        tc_mma_bf16(d_gate, ag, bd, idesc, (kc | kk) != 0);
+                        tc_mma_bf16(d_proj, ap, bd, idesc, (kc | kk) != 0);
+                    }
+                    tc_commit(&s.empty[stage]);
+                    if (++stage == C::S) { stage = 0; phase ^= 1; }
+                }
+                if (!ok) break;
+                tc_commit(&s.tfull[abuf]);
+                if (++abuf == 2) { abuf = 0; aphase ^= 1; }
+            }
+            tc_commit(&s.drain);
+            mbar_drain(&s.drain, 0);
+        }
+    } else if (warp >= 8) {
+        // LayerNorm statistics: thread = pair row of the tile
+        const int row = (warp - 8) * 32 + lane;
+        int stage = 0;
+        uint32_t phase = 0;
+        int sbuf = 0;
+        uint32_t sphase = 0;
+        for (int pt = cta_in_group; pt < num_ptiles; pt += ctas_per_group) {
+            const int b = pt / p.tiles_per_batch;
+            const int p0 = (pt - b * p.tiles_per_batch) * 128;
+            const long long pi = (long long)p0 + row;
+            float m = 1.f;   // issued first so that its latency overlaps the chunk reads
+            if (p.mask) m = (pi < p.NN) ? __uint_as_float((uint32_t)p.mask[(long long)b * p.NN + pi] << 16) : 0.f;
+            float shift = 0.f, s1 = 0.f, s2 = 0.f;
+            bool ok = true;
+            for (int kc = 0; kc < C::KC; ++kc) {
+                if (!__all_sync(0xffffffffu, mbar_wait(&s.full[stage], phase, abort_flag, kErrTimeoutEpilogue))) { ok = false; break; }
+                const uint8_t *zc = chunks + stage * C::CHUNK;
+#pragma unroll
+                for (int u = 0; u < 8; ++u) {
+                    uint4 w = *reinterpret_cast<const uint4 *>(zc + sw128_offset(row, u));
+                    float v[8] = {bf16_lo(w.x), bf16_hi(w.x), bf16_lo(w.y), bf16_hi(w.y),
+                                  bf16_lo(w.z), bf16_hi(w.z), bf16_lo(w.w), bf16_hi(w.w)};
+                    if (kc == 0 && u == 0) shift = v[0];
+#pragma unroll
+                    for (int e = 0; e < 8; ++e) {
+                        float d = v[e] - shift;
+                        s1 += d;
+                        s2 = fmaf(d, d, s2);
+                    }
+                }
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&s.empty[stage]);
+                if (++stage == C::S) { stage = 0; phase ^= 1; }
+            }
+            if (!ok) break;
+            const float inv_n = 1.0f / (float)C::CZ;
+            const float dm = s1 * inv_n;
+            const float var = fmaxf(s2 * inv_n - dm * dm, 0.f);
+            if (!__all_sync(0xffffffffu, mbar_wait(&s.sempty[sbuf], sphase ^ 1, abort_flag, kErrTimeoutEpilogue))) break;
+            st_mean[sbuf * 128 + row] = shift + dm;
+            st_rstd[sbuf * 128 + row] = rsqrtf(var + p.eps);
+            st_mask[sbuf * 128 + row] = m;
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&s.sfull[sbuf]);
+            if (++sbuf == C::SNB) { sbuf = 0; sphase ^= 1; }
+        }
+    } else {
+        // epilogue: thread = hidden channel c of this CTA's operand; warpgroup wg = pair half
+        const int wg = warp >> 2;
+        const int q = warp & 3;
+        const int c = q * 32 + lane;
+        uint8_t *stg = staging + wg * C::STG_BYTES;
+        const bool leader = (threadIdx.x & 127) == 0;
+        const CUtensorMap *tm_out = operand == 0 ? &p.tm_a : &p.tm_b;
+        const float4 cv = p.vec[operand * C::C_H + c];   // {sum W'_gate, shift_gate, sum W'_proj, shift_proj}
+        const uint32_t lane_off = (uint32_t)(q * 32) << 16;
+        int abuf = 0;
+        uint32_t aphase = 0;
+        int sbuf = 0;
+        uint32_t sphase = 0;
+        for (int pt = cta_in_group; pt < num_ptiles; pt += ctas_per_group) {
+            const int b = pt / p.tiles_per_batch;
+            const int p0 = (pt - b * p.tiles_per_batch) * 128;
+            if (!group_all(mbar_wait(&s.sfull[sbuf], sphase, abort_flag, kErrTimeoutEpilogue), 1 + wg, 128)) break;
+            if (!group_all(mbar_wait(&s.tfull[abuf], aphase, abort_flag, kErrTimeoutEpilogue), 1 + wg, 128)) break;
+            tc_fence_after();
+            if (leader) tma_store_wait_read<0>();
+            named_bar_sync(1 + wg, 128);
+            const float *smean = st_mean + sbuf * 128, *srstd = st_rstd + sbuf * 128, *smask = st_mask + sbuf * 128;
+#pragma unroll 1
+            for (int blk = 0; blk < 2; ++blk) {
+                const int col = wg * 64 + blk * 32;          // first pair of this 32-pair block
+                float g[32], pr[32];
+                tmem_ld32(tmem_base + abuf * 256 + lane_off + col, g);
+                tmem_ld32(tmem_base + abuf * 256 + 128 + lane_off + col, pr);
+                tc_wait_ld();
+#pragma unroll
+                for (int j = 0; j < 32; j += 4) {
+                    const float4 mu = *reinterpret_cast<const float4 *>(smean + col + j);
+                    const float4 rs = *reinterpret_cast<const float4 *>(srstd + col + j);
+                    const float4 mk = *reinterpret_cast<const float4 *>(smask + col + j);
+                    const float mus[4] = {mu.x, mu.y, mu.z, mu.w};
+                    const float rss[4] = {rs.x, rs.y, rs.z, rs.w};
+                    const float mks[4] = {mk.x, mk.y, mk.z, mk.w};
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        const float gv = fmaf(rss[e], fmaf(-mus[e], cv.x, g[j + e]), cv.y);
+                        const float pv = fmaf(rss[e], fmaf(-mus[e], cv.z, pr[j + e]), cv.w);
+                        g[j + e] = sigmoid_tanh(gv) * pv * mks[e];
+                    }
+                }
+#pragma unroll
+                for (int u = 0; u < 4; ++u) {
+                    uint4 w;
+                    w.x = pack_f16x2(g[8 * u + 0], g[8 * u + 1]);
+                    w.y = pack_f16x2(g[8 * u + 2], g[8 * u + 3]);
+                    w.z = pack_f16x2(g[8 * u + 4], g[8 * u + 5]);
+                    w.w = pack_f16x2(g[8 * u + 6], g[8 * u + 7]);
+                    *reinterpret_cast<uint4 *>(stg + sw128_offset(c, blk * 4 + u)) = w;
+                }
+            }
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) {
+                mbar_arrive(&s.tempty[abuf]);
+                mbar_arrive(&s.sempty[sbuf]);
+            }
+            if (++abuf == 2) { abuf = 0; aphase ^= 1; }
+            if (++sbuf == C::SNB) { sbuf = 0; sphase ^= 1; }
+            fence_proxy_async_smem();
+            named_bar_sync(1 + wg, 128);
+            if (leader) {
+                tma_store_3d(tm_out, stg, p0 + 64 * wg, 0, b);
+                tma_store_commit();
+            }
+        }
+        if (leader) tma_store_wait_all<0>();
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    if (warp == C::MMA_WARP) {
+        tc_fence_after();
+        tmem_dealloc(tmem_base, 512);
+    }
+}
+
+int k1_ncol(int c_z) { return c_z == 128 ? 2 * K1CmCfg::C_H : K1Cfg<384>::NCOL; }
+int k1_groups(int c_z) { return c_z == 128 ? K1CmCfg::G : K1Cfg<384>::G; }
+int k1_channels_per_warpgroup(int c_z) { return c_z == 128 ? K1CmCfg::C_H : K1Cfg<384>::CH_WG; }
+int k1_row_mode(int c_z) { return c_z == 128 ? 2 : 1; }
+size_t k1_smem_bytes(int c_z) { return c_z == 128 ? K1CmCfg::SMEM : K1Cfg<384>::SMEM; }
 
 template <int CZ>
 static cudaError_t k1_launch_t(const K1Args &args, int grid, cudaStream_t stream) {
@@ -303,8 +574,22 @@ static cudaError_t k1_launch_t(const K1Args &args, int grid, cudaStream_t stream
     return cudaGetLastError();
 }
 
+static cudaError_t k1_launch_cm(const K1Args &args, int grid, cudaStream_t stream) {
+    static int configured_device = -1;
+    int dev = 0;
+    cudaGetDevice(&dev);
+    if (configured_device != dev) {
+        cudaError_t e = cudaFuncSetAttribute(k1_project_cm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                             (int)K1CmCfg::SMEM);
+        if (e != cudaSuccess) return e;
+        configured_device = dev;
+    }
+    k1_project_cm_kernel<<<grid, K1CmCfg::THREADS, K1CmCfg::SMEM, stream>>>(args);
+    return cudaGetLastError();
+}
+
 cudaError_t k1_launch(int c_z, const K1Args &args, int grid, cudaStream_t stream) {
-    if (c_z == 128) return k1_launch_t<128>(args, grid, stream);
+    if (c_z == 128) return k1_launch_cm(args, grid, stream);
     if (c_z == 384) return k1_launch_t<384>(args, grid, stream);
     return cudaErrorInvalidValue;
 }

@@ -36,7 +36,8 @@ struct K3Cfg {
     static constexpr int STG_BYTES = 128 * 128;      // per warpgroup: 128 rows x 128 bytes
     static constexpr int COLS_PER_STORE = OUT_F32 ? 32 : 64;
     static constexpr int SNB = 2;
-    static constexpr int FIXED = 1024 + WO_BYTES + WG_BYTES + 2 * STG_BYTES + SNB * 128 * 32 + 1024;
+    static constexpr int VEC_BYTES = NCOL * 16;          // folding constants of this group's columns
+    static constexpr int FIXED = 1024 + WO_BYTES + WG_BYTES + 2 * STG_BYTES + SNB * 128 * 32 + VEC_BYTES + 1024;
     static constexpr int S = (232448 - FIXED) / CHUNK > 8 ? 8 : (232448 - FIXED) / CHUNK;
     static constexpr size_t SMEM = FIXED + (size_t)S * CHUNK;
     static constexpr int THREADS = 448;
@@ -67,7 +68,8 @@ __global__ void __launch_bounds__(448, 1) k3_output_kernel(const __grid_constant
     uint8_t *chunks = wg_s + C::WG_BYTES;              // S chunks
     uint8_t *staging = chunks + C::S * C::CHUNK;       // 2 x 16 KB
     K3Stats *stats = reinterpret_cast<K3Stats *>(staging + 2 * C::STG_BYTES);
-    K3Smem &s = *reinterpret_cast<K3Smem *>(stats + C::SNB * 128);
+    float4 *vec_s = reinterpret_cast<float4 *>(stats + C::SNB * 128);   // [NCOL]
+    K3Smem &s = *reinterpret_cast<K3Smem *>(vec_s + C::NCOL);
 
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
@@ -97,6 +99,7 @@ __global__ void __launch_bounds__(448, 1) k3_output_kernel(const __grid_constant
         s.abort_flag = 0;
         fence_mbarrier_init();
     }
+    if (threadIdx.x < C::NCOL) vec_s[threadIdx.x] = p.vec[n0 + threadIdx.x];
     if (warp == C::MMA_WARP) {
         tmem_alloc(&s.tmem_base, 512);
         tmem_relinquish();
@@ -269,7 +272,7 @@ __global__ void __launch_bounds__(448, 1) k3_output_kernel(const __grid_constant
         const int row = q * 32 + lane;
         uint8_t *stg = staging + wg * C::STG_BYTES;
         const bool leader = (threadIdx.x & 127) == 0;
-        const float4 *vec = p.vec + n0 + wg * 64;
+        const float4 *vec = vec_s + wg * 64;
         int abuf = 0;
         uint32_t aphase = 0;
         int sbuf = 0;
@@ -300,7 +303,7 @@ __global__ void __launch_bounds__(448, 1) k3_output_kernel(const __grid_constant
                     tc_wait_ld();
 #pragma unroll
                     for (int e = 0; e < 32; ++e) {
-                        const float4 cv = __ldg(&vec[col + e]);
+                        const float4 cv = vec[col + e];
                         const float ov = fmaf(st.rstd_x, fmaf(-st.mean_x, cv.x, o[e]), cv.y);
                         const float gv = fmaf(st.rstd_z, fmaf(-st.mean_z, cv.z, g[e]), cv.w);
                         o[e] = st.mask * sigmoid_exp(gv) * ov;

@@ -14,7 +14,8 @@ constexpr int kHidden = 128;  // c_h of the tensor-core path
 struct K1Args {
     CUtensorMap tm_z;      // z [B][N*N][c_z] bf16, box {64, 128, 1}, 128B swizzle
     CUtensorMap tm_w;      // packed weights [4*c_h][c_z] bf16, box {64, NCOL}, 128B swizzle
-    CUtensorMap tm_a;      // a [B][c_h][N*N] f16, box {128, channels per warpgroup, 1}
+    CUtensorMap tm_a;      // a [B][c_h][N*N] f16; c_z = 128: box {64, 128, 1} 128B swizzle,
+                           // c_z = 384: box {128, channels per warpgroup, 1} no swizzle
     CUtensorMap tm_b;      // b, same as tm_a
     const uint16_t *mask;  // [B][N*N] bf16 bits, or nullptr
     const float4 *vec;     // [2][c_h] {sum W'_gate, shift_gate, sum W'_proj, shift_proj}
@@ -54,6 +55,7 @@ int k1_groups(int c_z);
 int k1_ncol(int c_z);
 int k1_channels_per_warpgroup(int c_z);
 cudaError_t k1_launch(int c_z, const K1Args &args, int grid, cudaStream_t stream);
+int k1_row_mode(int c_z);
 
 size_t k2_smem_bytes();
 cudaError_t k2_launch(const K2Args &args, int grid, cudaStream_t stream);
@@ -73,7 +75,7 @@ struct FoldArgs {
     int R, K;
     uint16_t *dst;        // bf16 (or f16 when dst_f16) rows [*, K]
     int dst_f16;
-    int row_mode;         // 0: dst row = r; 1: K1 interleaved layout (see k1 packing)
+    int row_mode;         // 0: dst row = r; 1: K1 interleaved layout (c_z = 384); 2: K1 blocked layout (c_z = 128)
     int operand;          // row_mode 1: 0 = a, 1 = b
     int kind;             // row_mode 1: 0 = gate, 1 = projection
     int ncol, cpg, gpo;   // row_mode 1: group width, channels per group, groups per operand

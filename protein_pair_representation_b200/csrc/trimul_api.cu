@@ -279,7 +279,7 @@ extern "C" trimul_status_t tri_mul_layer_create(const trimul_weights_desc_t *w, 
                 fa.R = ch;
                 fa.K = cz;
                 fa.dst = L->k1_w;
-                fa.row_mode = 1;
+                fa.row_mode = k1_row_mode(cz);
                 fa.operand = o;
                 fa.kind = kind;
                 fa.ncol = ncol;
@@ -386,9 +386,13 @@ static trimul_status_t run_project_bf16(const trimul_layer_t *L, const void *z, 
     {
         uint64_t dims[3] = {NN, (uint64_t)ch, (uint64_t)B};
         uint64_t strides[2] = {NN * 2, (uint64_t)ch * NN * 2};
-        uint32_t box[3] = {128, (uint32_t)k1_channels_per_warpgroup(cz), 1};
-        TRY(make_map(&p.tm_a, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 3, a, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_NONE, "K1 a"));
-        TRY(make_map(&p.tm_b, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 3, b, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_NONE, "K1 b"));
+        // c_z = 128: channel-lane kernel stores [128 channels][64 pairs] tiles through a 128B swizzle;
+        // c_z = 384: pair-lane kernel stores [channels][128 pairs] rows without swizzle
+        const bool cm = k1_row_mode(cz) == 2;
+        uint32_t box[3] = {cm ? 64u : 128u, (uint32_t)k1_channels_per_warpgroup(cz), 1};
+        const CUtensorMapSwizzle sw = cm ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE;
+        TRY(make_map(&p.tm_a, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 3, a, dims, strides, box, sw, "K1 a"));
+        TRY(make_map(&p.tm_b, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 3, b, dims, strides, box, sw, "K1 b"));
     }
     p.mask = reinterpret_cast<const uint16_t *>(mask);
     p.vec = L->k1_vec;
