@@ -154,6 +154,22 @@ class ClockSampler:
                 "reasons": sorted(reasons), "samples": len(sm)}
 
 
+def max_over_ranks(value_ms, dist=None, device=None):
+    """The largest of every rank's elapsed time (the job's time); identity on one rank."""
+    if dist is None:
+        return float(value_ms)
+    import torch
+    t = torch.tensor([float(value_ms)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_ms_per_layer(max_elapsed_ms, steps, n_dirs, world):
+    """Whole-job milliseconds per layer: every rank ran `steps` steps of `n_dirs` layers in
+    `max_elapsed_ms` (the slowest rank), so the job processed steps * n_dirs * world layers."""
+    return max_elapsed_ms / (steps * n_dirs * world)
+
+
 def dist_setup(gpus):
     rank = int(os.environ.get("RANK", "0"))
     world = int(os.environ.get("WORLD_SIZE", "1"))
@@ -286,11 +302,7 @@ def run_ours(args):
     sync_all()
     clock_info = clocks.stop()
     tm.check_device_status()
-    elapsed = t0.elapsed_time(t1)
-    if dist is not None:
-        t = torch.tensor([elapsed], device=dev, dtype=torch.float64)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        elapsed = float(t.item())
+    elapsed = max_over_ranks(t0.elapsed_time(t1), dist, dev)
     kernel_ms = {k: statistics.mean(ev[d][i].elapsed_time(ev[d][i + 1]) for ev in kev for d in range(len(dirs)))
                  for i, k in enumerate(KERNEL_NAMES)}
 
@@ -317,12 +329,8 @@ def run_ours(args):
             e2e_step()
         e1.record()
         sync_all()
-        e_el = e0.elapsed_time(e1)
-        if dist is not None:
-            t = torch.tensor([e_el], device=dev, dtype=torch.float64)
-            dist.all_reduce(t, op=dist.ReduceOp.MAX)
-            e_el = float(t.item())
-        e2e = {"value": e_el / (args.steps * len(dirs) * world), "unit": "ms/layer",
+        e_el = max_over_ranks(e0.elapsed_time(e1), dist, dev)
+        e2e = {"value": job_ms_per_layer(e_el, args.steps, len(dirs), world), "unit": "ms/layer",
                "h2d_bytes_per_step": z_host.numel() * 2 + m_host.numel() * 2,
                "d2h_bytes_per_step": sum(o.numel() * o.element_size() for o in out_host)}
 
@@ -342,7 +350,7 @@ def run_ours(args):
     peaks = measured_peaks()
     out_bytes = 4 if out_dt == torch.float32 else 2
     flops, nbytes = layer_work(inp.B, inp.N, inp.c_z, inp.c_h, out_bytes)
-    layer_ms = elapsed / (args.steps * len(dirs) * world)
+    layer_ms = job_ms_per_layer(elapsed, args.steps, len(dirs), world)
     layer_ms_single = elapsed / (args.steps * len(dirs))
     kernels = {}
     for k in KERNEL_NAMES:

@@ -210,6 +210,14 @@ int tri_mul_kernels_per_forward(void);
  * are undefined. */
 trimul_status_t tri_mul_check_device_status(void);
 
+/* Failure-path self-test: launches one kernel on `stream` that waits, with the same
+ * bounded wait the tensor-core kernels use, on a barrier nothing will complete. The
+ * wait gives up after about one second and records the timeout in the device error
+ * word; a following tri_mul_check_device_status() must return
+ * TRIMUL_ERR_DEVICE_TIMEOUT, and the device stays usable. No fault, trap or hang is
+ * involved. sm_100 only. */
+trimul_status_t tri_mul_selftest_bounded_wait(void *stream);
+
 /* Static description of a status code. */
 const char *tri_mul_status_string(trimul_status_t status);
 

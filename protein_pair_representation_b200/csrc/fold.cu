@@ -36,12 +36,13 @@ __global__ void fold_kernel(FoldArgs a) {
         const float g = a.gamma ? load_as_f32(a.gamma, k, a.src_bf16) : 1.0f;
         const float bt = a.beta ? load_as_f32(a.beta, k, a.src_bf16) : 0.0f;
         float wq;
+        const float sc = a.scale == 0.f ? 1.f : a.scale;
         if (a.dst_f16) {
-            const __half h = __float2half_rn(w * g);
+            const __half h = __float2half_rn(w * g * sc);
             a.dst[(size_t)dst_row * a.K + k] = __half_as_ushort(h);
             wq = __half2float(h);
         } else {
-            const __nv_bfloat16 h = __float2bfloat16_rn(w * g);
+            const __nv_bfloat16 h = __float2bfloat16_rn(w * g * sc);
             a.dst[(size_t)dst_row * a.K + k] = __bfloat16_as_ushort(h);
             wq = __bfloat162float(h);
         }
@@ -65,8 +66,9 @@ __global__ void fold_kernel(FoldArgs a) {
             s1 += red[1][w];
         }
         const double bias = a.bias ? (double)load_as_f32(a.bias, r, a.src_bf16) : 0.0;
-        a.sum_out[(size_t)r * a.out_stride] = (float)s0;
-        a.shift_out[(size_t)r * a.out_stride] = (float)(s1 + bias);
+        const double sc = a.scale == 0.f ? 1.0 : (double)a.scale;
+        a.sum_out[(size_t)r * a.out_stride] = (float)s0;          // already the sum of the scaled row
+        a.shift_out[(size_t)r * a.out_stride] = (float)((s1 + bias) * sc);
     }
 }
 

@@ -54,7 +54,7 @@ struct K1Smem {
     uint64_t wbar;
     uint64_t full[8], empty[8];
     uint64_t tfull[4], tempty[4];
-    uint64_t sfull[2], sempty[2];
+    uint64_t sfull[4], sempty[4];
     uint64_t drain;
     uint32_t tmem_base;
     int abort_flag;
@@ -293,25 +293,40 @@ __global__ void __launch_bounds__(448, 1) k1_project_kernel(const __grid_constan
 // LayerNorm statistics are read from shared memory (broadcast, four pairs per load); and
 // consecutive pairs of one channel are consecutive columns, which pack directly into
 // 16-byte rows of the channel-major output tile.
-// Warps: 0-7 epilogue (warpgroup 0: pairs 0-63 of the tile, warpgroup 1: pairs 64-127),
-// 8-11 LayerNorm statistics, 12 TMA producer, 13 TMEM allocator + MMA issuer.
+// The gate is evaluated in f16x2 (tanh.approx.f16x2 on g/2, the gate rows being folded
+// with an extra factor 1/2), as are the products with the projection and the mask.
+// Warps: 0-15 epilogue (warpgroup w: pairs [32w, 32w+32) of the tile), 16-19 LayerNorm
+// statistics, 20 TMA producer, 21 TMEM allocator + MMA issuer.
 struct K1CmCfg {
     static constexpr int CZ = 128, C_H = kHidden, KC = CZ / 64;
     static constexpr int G = 2;                               // one group per operand
     static constexpr int W_CHUNK = 2 * C_H * 64 * 2;          // [gate 128 rows, proj 128 rows] x 64 k
     static constexpr int W_BYTES = KC * W_CHUNK;              // 64 KB
     static constexpr int CHUNK = 128 * 64 * 2;                // z chunk: 128 pairs x 64 channels
-    static constexpr int STG_BYTES = C_H * 64 * 2;            // per warpgroup: [128 ch][64 pairs] f16
+    static constexpr int STG_BYTES = C_H * 64 * 2;            // per pair half: [128 ch][64 pairs] f16
     static constexpr int SNB = 2;
-    static constexpr int STATS_BYTES = SNB * 3 * 128 * 4;     // mean, rstd, mask per pair
+    static constexpr int STATS_BYTES = SNB * 128 * (4 + 4 + 2);   // mean, rstd (f32), mask (f16) per pair
     static constexpr int FIXED = 1024 + W_BYTES + 2 * STG_BYTES + STATS_BYTES + 1024;
     static constexpr int S = (232448 - FIXED) / CHUNK > 8 ? 8 : (232448 - FIXED) / CHUNK;
     static constexpr size_t SMEM = FIXED + (size_t)S * CHUNK;
-    static constexpr int THREADS = 448;
-    static constexpr int TMA_WARP = 12, MMA_WARP = 13;
+    static constexpr int EPI_WARPS = 16;                      // four warpgroups, 32 pairs each
+    static constexpr int STATS_WARP0 = 16, STATS_WARPS = 4;
+    static constexpr int TMA_WARP = 20, MMA_WARP = 21;
+    static constexpr int THREADS = 22 * 32;
 };
 
-__global__ void __launch_bounds__(448, 1) k1_project_cm_kernel(const __grid_constant__ K1Args p) {
+__device__ __forceinline__ uint32_t h2_as_u32(__half2 h) { return *reinterpret_cast<uint32_t *>(&h); }
+__device__ __forceinline__ __half2 u32_as_h2(uint32_t u) { return *reinterpret_cast<__half2 *>(&u); }
+
+// 0.5 + 0.5 tanh(x) on two halves at once (x = g / 2: the gate rows are pre-scaled by 1/2).
+__device__ __forceinline__ __half2 sigmoid_of_half_arg_h2(__half2 x) {
+    uint32_t t;
+    asm("tanh.approx.f16x2 %0, %1;" : "=r"(t) : "r"(h2_as_u32(x)));
+    const __half2 half = __float2half2_rn(0.5f);
+    return __hfma2(u32_as_h2(t), half, half);
+}
+
+__global__ void __launch_bounds__(K1CmCfg::THREADS, 1) k1_project_cm_kernel(const __grid_constant__ K1Args p) {
     using C = K1CmCfg;
     extern __shared__ uint8_t smem_raw[];
     uint8_t *base = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -320,7 +335,7 @@ __global__ void __launch_bounds__(448, 1) k1_project_cm_kernel(const __grid_cons
     uint8_t *staging = chunks + C::S * C::CHUNK;          // 2 x [128 ch][64 pairs] f16, 128B swizzle
     float *st_mean = reinterpret_cast<float *>(staging + 2 * C::STG_BYTES);  // [SNB][128]
     float *st_rstd = st_mean + C::SNB * 128;
-    float *st_mask = st_rstd + C::SNB * 128;
+    __half *st_mask = reinterpret_cast<__half *>(st_rstd + C::SNB * 128);    // [SNB][128]
     K1Smem &s = *reinterpret_cast<K1Smem *>(st_mask + C::SNB * 128);
 
     const int warp = threadIdx.x >> 5;
@@ -336,15 +351,15 @@ __global__ void __launch_bounds__(448, 1) k1_project_cm_kernel(const __grid_cons
         mbar_init(&s.wbar, 1);
         for (int i = 0; i < C::S; ++i) {
             mbar_init(&s.full[i], 1);
-            mbar_init(&s.empty[i], 1 + 4);  // MMA commit + 4 stats warps
+            mbar_init(&s.empty[i], 1 + C::STATS_WARPS);  // MMA commit + stats warps
         }
         for (int i = 0; i < 2; ++i) {
             mbar_init(&s.tfull[i], 1);
-            mbar_init(&s.tempty[i], 8);
+            mbar_init(&s.tempty[i], C::EPI_WARPS);
         }
         for (int i = 0; i < C::SNB; ++i) {
-            mbar_init(&s.sfull[i], 4);
-            mbar_init(&s.sempty[i], 8);
+            mbar_init(&s.sfull[i], C::STATS_WARPS);
+            mbar_init(&s.sempty[i], C::EPI_WARPS);
         }
         mbar_init(&s.drain, 1);
         s.abort_flag = 0;
@@ -425,9 +440,9 @@ __global__ void __launch_bounds__(448, 1) k1_project_cm_kernel(const __grid_cons
             tc_commit(&s.drain);
             mbar_drain(&s.drain, 0);
         }
-    } else if (warp >= 8) {
+    } else if (warp >= C::STATS_WARP0) {
         // LayerNorm statistics: thread = pair row of the tile
-        const int row = (warp - 8) * 32 + lane;
+        const int row = (warp - C::STATS_WARP0) * 32 + lane;
         int stage = 0;
         uint32_t phase = 0;
         int sbuf = 0;
@@ -436,8 +451,8 @@ __global__ void __launch_bounds__(448, 1) k1_project_cm_kernel(const __grid_cons
             const int b = pt / p.tiles_per_batch;
             const int p0 = (pt - b * p.tiles_per_batch) * 128;
             const long long pi = (long long)p0 + row;
-            float m = 1.f;   // issued first so that its latency overlaps the chunk reads
-            if (p.mask) m = (pi < p.NN) ? __uint_as_float((uint32_t)p.mask[(long long)b * p.NN + pi] << 16) : 0.f;
+            uint16_t mbits = 0x3F80u;   // bf16 1.0; the load is issued first so its latency overlaps
+            if (p.mask) mbits = (pi < p.NN) ? p.mask[(long long)b * p.NN + pi] : (uint16_t)0;
             float shift = 0.f, s1 = 0.f, s2 = 0.f;
             bool ok = true;
             for (int kc = 0; kc < C::KC; ++kc) {
@@ -467,20 +482,27 @@ __global__ void __launch_bounds__(448, 1) k1_project_cm_kernel(const __grid_cons
             if (!__all_sync(0xffffffffu, mbar_wait(&s.sempty[sbuf], sphase ^ 1, abort_flag, kErrTimeoutEpilogue))) break;
             st_mean[sbuf * 128 + row] = shift + dm;
             st_rstd[sbuf * 128 + row] = rsqrtf(var + p.eps);
-            st_mask[sbuf * 128 + row] = m;
+            st_mask[sbuf * 128 + row] = __float2half_rn(__uint_as_float((uint32_t)mbits << 16));
             __syncwarp();
             if (lane == 0) mbar_arrive(&s.sfull[sbuf]);
             if (++sbuf == C::SNB) { sbuf = 0; sphase ^= 1; }
         }
     } else {
-        // epilogue: thread = hidden channel c of this CTA's operand; warpgroup wg = pair half
+        // epilogue: thread = hidden channel c of this CTA's operand; warpgroup wg owns the
+        // 32 pairs [32 wg, 32 wg + 32) of the tile; warpgroups 2h and 2h+1 share the staging
+        // buffer and the TMA store of pair half h.
         const int wg = warp >> 2;
+        const int half = wg >> 1;
+        const int sub = wg & 1;
         const int q = warp & 3;
         const int c = q * 32 + lane;
-        uint8_t *stg = staging + wg * C::STG_BYTES;
-        const bool leader = (threadIdx.x & 127) == 0;
+        const int col = 32 * wg;
+        uint8_t *stg = staging + half * C::STG_BYTES;
+        const bool leader = (threadIdx.x & 255) == 0;
+        const uint32_t bar_id = 1 + half;
         const CUtensorMap *tm_out = operand == 0 ? &p.tm_a : &p.tm_b;
-        const float4 cv = p.vec[operand * C::C_H + c];   // {sum W'_gate, shift_gate, sum W'_proj, shift_proj}
+        // {sum W'_gate, shift_gate, sum W'_proj, shift_proj}; the gate entries are for g / 2
+        const float4 cv = p.vec[operand * C::C_H + c];
         const uint32_t lane_off = (uint32_t)(q * 32) << 16;
         int abuf = 0;
         uint32_t aphase = 0;
@@ -489,43 +511,45 @@ __global__ void __launch_bounds__(448, 1) k1_project_cm_kernel(const __grid_cons
         for (int pt = cta_in_group; pt < num_ptiles; pt += ctas_per_group) {
             const int b = pt / p.tiles_per_batch;
             const int p0 = (pt - b * p.tiles_per_batch) * 128;
-            if (!group_all(mbar_wait(&s.sfull[sbuf], sphase, abort_flag, kErrTimeoutEpilogue), 1 + wg, 128)) break;
-            if (!group_all(mbar_wait(&s.tfull[abuf], aphase, abort_flag, kErrTimeoutEpilogue), 1 + wg, 128)) break;
+            if (!group_all(mbar_wait(&s.sfull[sbuf], sphase, abort_flag, kErrTimeoutEpilogue), bar_id, 256)) break;
+            if (!group_all(mbar_wait(&s.tfull[abuf], aphase, abort_flag, kErrTimeoutEpilogue), bar_id, 256)) break;
             tc_fence_after();
             if (leader) tma_store_wait_read<0>();
-            named_bar_sync(1 + wg, 128);
-            const float *smean = st_mean + sbuf * 128, *srstd = st_rstd + sbuf * 128, *smask = st_mask + sbuf * 128;
+            named_bar_sync(bar_id, 256);
+            const float *smean = st_mean + sbuf * 128 + col, *srstd = st_rstd + sbuf * 128 + col;
+            const __half *smask = st_mask + sbuf * 128 + col;
 #pragma unroll 1
-            for (int blk = 0; blk < 2; ++blk) {
-                const int col = wg * 64 + blk * 32;          // first pair of this 32-pair block
-                float g[32], pr[32];
-                tmem_ld32(tmem_base + abuf * 256 + lane_off + col, g);
-                tmem_ld32(tmem_base + abuf * 256 + 128 + lane_off + col, pr);
+            for (int hh = 0; hh < 2; ++hh) {          // two halves of 16 pairs
+                float g[16], pr[16];
+                tmem_ld16(tmem_base + abuf * 256 + lane_off + col + 16 * hh, g);
+                tmem_ld16(tmem_base + abuf * 256 + 128 + lane_off + col + 16 * hh, pr);
                 tc_wait_ld();
+                uint32_t outw[8];
 #pragma unroll
-                for (int j = 0; j < 32; j += 4) {
-                    const float4 mu = *reinterpret_cast<const float4 *>(smean + col + j);
-                    const float4 rs = *reinterpret_cast<const float4 *>(srstd + col + j);
-                    const float4 mk = *reinterpret_cast<const float4 *>(smask + col + j);
+                for (int j = 0; j < 16; j += 4) {
+                    const float4 mu = *reinterpret_cast<const float4 *>(smean + 16 * hh + j);
+                    const float4 rs = *reinterpret_cast<const float4 *>(srstd + 16 * hh + j);
+                    const uint2 mk = *reinterpret_cast<const uint2 *>(smask + 16 * hh + j);
                     const float mus[4] = {mu.x, mu.y, mu.z, mu.w};
                     const float rss[4] = {rs.x, rs.y, rs.z, rs.w};
-                    const float mks[4] = {mk.x, mk.y, mk.z, mk.w};
+                    float gv[4], pv[4];
 #pragma unroll
                     for (int e = 0; e < 4; ++e) {
-                        const float gv = fmaf(rss[e], fmaf(-mus[e], cv.x, g[j + e]), cv.y);
-                        const float pv = fmaf(rss[e], fmaf(-mus[e], cv.z, pr[j + e]), cv.w);
-                        g[j + e] = sigmoid_tanh(gv) * pv * mks[e];
+                        gv[e] = fmaf(rss[e], fmaf(-mus[e], cv.x, g[j + e]), cv.y);
+                        pv[e] = fmaf(rss[e], fmaf(-mus[e], cv.z, pr[j + e]), cv.w);
+                    }
+#pragma unroll
+                    for (int h = 0; h < 2; ++h) {
+                        const __half2 sg = sigmoid_of_half_arg_h2(__floats2half2_rn(gv[2 * h], gv[2 * h + 1]));
+                        const __half2 ph = __floats2half2_rn(pv[2 * h], pv[2 * h + 1]);
+                        const __half2 mh = u32_as_h2(h == 0 ? mk.x : mk.y);
+                        outw[j / 2 + h] = h2_as_u32(__hmul2(__hmul2(sg, ph), mh));
                     }
                 }
 #pragma unroll
-                for (int u = 0; u < 4; ++u) {
-                    uint4 w;
-                    w.x = pack_f16x2(g[8 * u + 0], g[8 * u + 1]);
-                    w.y = pack_f16x2(g[8 * u + 2], g[8 * u + 3]);
-                    w.z = pack_f16x2(g[8 * u + 4], g[8 * u + 5]);
-                    w.w = pack_f16x2(g[8 * u + 6], g[8 * u + 7]);
-                    *reinterpret_cast<uint4 *>(stg + sw128_offset(c, blk * 4 + u)) = w;
-                }
+                for (int u = 0; u < 2; ++u)
+                    *reinterpret_cast<uint4 *>(stg + sw128_offset(c, sub * 4 + 2 * hh + u)) =
+                        make_uint4(outw[4 * u], outw[4 * u + 1], outw[4 * u + 2], outw[4 * u + 3]);
             }
             tc_fence_before();
             __syncwarp();
@@ -536,9 +560,9 @@ __global__ void __launch_bounds__(448, 1) k1_project_cm_kernel(const __grid_cons
             if (++abuf == 2) { abuf = 0; aphase ^= 1; }
             if (++sbuf == C::SNB) { sbuf = 0; sphase ^= 1; }
             fence_proxy_async_smem();
-            named_bar_sync(1 + wg, 128);
+            named_bar_sync(bar_id, 256);
             if (leader) {
-                tma_store_3d(tm_out, stg, p0 + 64 * wg, 0, b);
+                tma_store_3d(tm_out, stg, p0 + 64 * half, 0, b);
                 tma_store_commit();
             }
         }

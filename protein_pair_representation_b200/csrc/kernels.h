@@ -79,6 +79,7 @@ struct FoldArgs {
     int operand;          // row_mode 1: 0 = a, 1 = b
     int kind;             // row_mode 1: 0 = gate, 1 = projection
     int ncol, cpg, gpo;   // row_mode 1: group width, channels per group, groups per operand
+    float scale;          // multiplies the folded row, its sum and its shift (1 = none; powers of two are exact)
     float *sum_out;       // element r * stride: sum_k bf16(W[r,k] * gamma[k])
     float *shift_out;     // element r * stride: sum_k beta[k] W[r,k] + bias[r]
     int out_stride;       // in floats

@@ -280,6 +280,9 @@ extern "C" trimul_status_t tri_mul_layer_create(const trimul_weights_desc_t *w, 
                 fa.K = cz;
                 fa.dst = L->k1_w;
                 fa.row_mode = k1_row_mode(cz);
+                // the c_z = 128 kernel evaluates sigmoid(g) as 0.5 + 0.5 tanh(g / 2) and takes
+                // the gate rows pre-scaled by 1/2 (exact in bf16)
+                fa.scale = (fa.row_mode == 2 && kind == 0) ? 0.5f : 1.0f;
                 fa.operand = o;
                 fa.kind = kind;
                 fa.ncol = ncol;
@@ -591,6 +594,30 @@ extern "C" trimul_status_t tri_mul_forward(const trimul_pair_t *z, const void *m
     if (L->timing) TRY_CUDA(cudaEventRecord(L->events[2], st), "event record");
     TRY(tri_mul_output_gate(z, mask, x, x_scale, L, out, stream));
     if (L->timing) TRY_CUDA(cudaEventRecord(L->events[3], st), "event record");
+    return TRIMUL_OK;
+}
+
+// One CTA waits, with the kernels' bounded wait, on an mbarrier that nothing arrives at:
+// the wait gives up after its limit (about one second), raises the abort flag and the device
+// error word, and the kernel exits normally.
+__global__ void selftest_bounded_wait_kernel() {
+    __shared__ uint64_t bar;
+    __shared__ int abort_flag;
+    if (threadIdx.x == 0) {
+        mbar_init(&bar, 1);
+        abort_flag = 0;
+        fence_mbarrier_init();
+    }
+    __syncthreads();
+    if (threadIdx.x == 0) (void)mbar_wait(&bar, 0, &abort_flag, kErrTimeoutEpilogue);
+    __syncthreads();
+}
+
+extern "C" trimul_status_t tri_mul_selftest_bounded_wait(void *stream) {
+    DeviceInfo d;
+    TRY(require_sm100(&d));
+    selftest_bounded_wait_kernel<<<1, 32, 0, reinterpret_cast<cudaStream_t>(stream)>>>();
+    TRY_CUDA(cudaGetLastError(), "self-test launch");
     return TRIMUL_OK;
 }
 

@@ -9,7 +9,7 @@ import torch
 
 import oracle
 import trimul_inputs as ti
-from gpu_helpers import assert_close_bf16, assert_close_f16, assert_close_rms, to_pair_major, upload
+from gpu_helpers import F16_REL, assert_close_bf16, assert_close_f16, assert_close_rms, assert_close_ulp, to_pair_major, upload
 from protein_pair_representation_b200 import trimul as tm
 
 pytestmark = pytest.mark.gpu
@@ -86,8 +86,10 @@ def test_project_bf16(c_z, affine, B, N, mask):
     # random gamma: W * gamma is rounded to bf16 (up to 2^-9 per weight), which the
     # end-to-end tolerance absorbs; checked here at that tolerance.
     tol = 2e-2 if affine else 2e-3
-    assert_close_f16(to_pair_major(a), ra, tol, what=f"K1 a c_z={c_z} N={N}")
-    assert_close_f16(to_pair_major(b), rb, tol, what=f"K1 b c_z={c_z} N={N}")
+    # c_z = 128 evaluates sigmoid(g) * p * m in f16x2: up to ~3 half-precision roundings
+    rel = (4 if c_z == 128 else 1) * F16_REL
+    assert_close_ulp(to_pair_major(a), ra, tol, rel, what=f"K1 a c_z={c_z} N={N}")
+    assert_close_ulp(to_pair_major(b), rb, tol, rel, what=f"K1 b c_z={c_z} N={N}")
     tm.check_device_status()
 
 
