@@ -108,6 +108,8 @@ __global__ void __launch_bounds__(448, 1) k1_project_kernel(const __grid_constan
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem_base = s.tmem_base;
+    pdl_launch_dependents();
+    if (warp != C::TMA_WARP) pdl_wait();       // the producer waits after its weight loads
 
     if (warp == C::TMA_WARP) {
         if (lane == 0) {
@@ -117,6 +119,7 @@ __global__ void __launch_bounds__(448, 1) k1_project_kernel(const __grid_constan
             mbar_arrive_expect_tx(&s.wbar, C::W_BYTES);
             for (int kc = 0; kc < C::KC; ++kc)
                 tma_load_2d(w_s + kc * C::NCOL * 128, &p.tm_w, &s.wbar, kc * 64, group * C::NCOL);
+            pdl_wait();
             int stage = 0;
             uint32_t phase = 0;
             uint32_t filled = 0;
@@ -373,6 +376,8 @@ __global__ void __launch_bounds__(K1CmCfg::THREADS, 1) k1_project_cm_kernel(cons
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem_base = s.tmem_base;
+    pdl_launch_dependents();
+    if (warp != C::TMA_WARP) pdl_wait();       // the producer waits after its weight loads
 
     if (warp == C::TMA_WARP) {
         if (lane == 0) {
@@ -381,6 +386,7 @@ __global__ void __launch_bounds__(K1CmCfg::THREADS, 1) k1_project_cm_kernel(cons
             mbar_arrive_expect_tx(&s.wbar, C::W_BYTES);
             for (int kc = 0; kc < C::KC; ++kc)
                 tma_load_2d(w_s + kc * C::W_CHUNK, &p.tm_w, &s.wbar, kc * 64, operand * 2 * C::C_H);
+            pdl_wait();
             int stage = 0;
             uint32_t phase = 0;
             uint32_t filled = 0;
@@ -594,8 +600,7 @@ static cudaError_t k1_launch_t(const K1Args &args, int grid, cudaStream_t stream
         if (e != cudaSuccess) return e;
         configured_device = dev;
     }
-    k1_project_kernel<CZ><<<grid, K1Cfg<CZ>::THREADS, K1Cfg<CZ>::SMEM, stream>>>(args);
-    return cudaGetLastError();
+    return launch_pdl(k1_project_kernel<CZ>, grid, K1Cfg<CZ>::THREADS, K1Cfg<CZ>::SMEM, stream, args);
 }
 
 static cudaError_t k1_launch_cm(const K1Args &args, int grid, cudaStream_t stream) {
@@ -608,8 +613,7 @@ static cudaError_t k1_launch_cm(const K1Args &args, int grid, cudaStream_t strea
         if (e != cudaSuccess) return e;
         configured_device = dev;
     }
-    k1_project_cm_kernel<<<grid, K1CmCfg::THREADS, K1CmCfg::SMEM, stream>>>(args);
-    return cudaGetLastError();
+    return launch_pdl(k1_project_cm_kernel, grid, K1CmCfg::THREADS, K1CmCfg::SMEM, stream, args);
 }
 
 cudaError_t k1_launch(int c_z, const K1Args &args, int grid, cudaStream_t stream) {

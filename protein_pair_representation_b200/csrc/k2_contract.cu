@@ -83,6 +83,8 @@ __global__ void __launch_bounds__(k2::THREADS, 1) k2_contract_kernel(const __gri
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem_base = s.tmem_base;
+    pdl_launch_dependents();
+    pdl_wait();
 
     const int tiles_per_channel = p.m_tiles * p.n_tiles;
     const int num_tiles = p.BC * tiles_per_channel;
@@ -247,8 +249,7 @@ cudaError_t k2_launch(const K2Args &args, int grid, cudaStream_t stream) {
         if (e != cudaSuccess) return e;
         configured_device = dev;
     }
-    k2_contract_kernel<<<grid, k2::THREADS, k2::SMEM_BYTES, stream>>>(args);
-    return cudaGetLastError();
+    return launch_pdl(k2_contract_kernel, grid, k2::THREADS, k2::SMEM_BYTES, stream, args);
 }
 
 }  // namespace trimul

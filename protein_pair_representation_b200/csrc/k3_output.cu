@@ -108,6 +108,8 @@ __global__ void __launch_bounds__(448, 1) k3_output_kernel(const __grid_constant
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem_base = s.tmem_base;
+    pdl_launch_dependents();
+    if (warp != C::TMA_WARP) pdl_wait();       // the producer waits after its weight loads
 
     if (warp == C::TMA_WARP) {
         if (lane == 0) {
@@ -118,6 +120,7 @@ __global__ void __launch_bounds__(448, 1) k3_output_kernel(const __grid_constant
                 tma_load_2d(wo_s + c * C::NCOL * 128, &p.tm_wo, &s.wbar, c * 64, n0);
             for (int c = 0; c < C::ZC; ++c)
                 tma_load_2d(wg_s + c * C::NCOL * 128, &p.tm_wg, &s.wbar, c * 64, n0);
+            pdl_wait();
             int stage = 0;
             uint32_t phase = 0;
             uint32_t filled = 0;
@@ -366,8 +369,7 @@ static cudaError_t k3_launch_t(const K3Args &args, int grid, cudaStream_t stream
         if (e != cudaSuccess) return e;
         configured_device = dev;
     }
-    k3_output_kernel<CZ, F32><<<grid, K3Cfg<CZ, F32>::THREADS, K3Cfg<CZ, F32>::SMEM, stream>>>(args);
-    return cudaGetLastError();
+    return launch_pdl(k3_output_kernel<CZ, F32>, grid, K3Cfg<CZ, F32>::THREADS, K3Cfg<CZ, F32>::SMEM, stream, args);
 }
 
 cudaError_t k3_launch(int c_z, bool out_f32, const K3Args &args, int grid, cudaStream_t stream) {

@@ -49,6 +49,25 @@ struct K3Args {
     float eps_x;           // output LayerNorm on the stored (scaled) x: eps * x_scale^2
 };
 
+// Launch with programmatic stream serialization: the kernel may begin while the previous
+// kernel of the stream finishes; every kernel launched this way calls pdl_wait() before it
+// touches memory the previous kernel may write or read.
+template <typename Kernel, typename Args>
+inline cudaError_t launch_pdl(Kernel kernel, int grid, int block, size_t smem, cudaStream_t stream,
+                              const Args &args) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)grid);
+    cfg.blockDim = dim3((unsigned)block);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kernel, args);
+}
+
 // Kernel resource queries (dynamic shared memory bytes) and launches.
 size_t k1_smem_bytes(int c_z);
 int k1_groups(int c_z);

@@ -112,6 +112,17 @@ __device__ __forceinline__ void mbar_drain(uint64_t *bar, uint32_t parity) {
     }
 }
 
+// ------------------------------------------------------------------ programmatic dependent launch
+
+// Lets the next kernel in the stream start its prologue on SMs this grid leaves free.
+__device__ __forceinline__ void pdl_launch_dependents() {
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
+// Waits until the previous kernel in the stream has completed and its memory operations
+// are visible (returns at once for a launch without the programmatic-serialization attribute).
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+
 // ------------------------------------------------------------------ named barriers
 
 __device__ __forceinline__ void named_bar_sync(uint32_t id, uint32_t nthreads) {
