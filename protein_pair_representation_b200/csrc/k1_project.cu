@@ -186,22 +186,27 @@ __global__ void __launch_bounds__(448, 1) k1_project_kernel(const __grid_constan
         for (int pt = cta_in_group; pt < num_ptiles; pt += ctas_per_group) {
             const int b = pt / p.tiles_per_batch;
             const int p0 = (pt - b * p.tiles_per_batch) * 128;
-            float shift = 0.f, s1 = 0.f, s2 = 0.f;
+            // shifted sums in packed pairs: s1 = sum(v - shift), s2 = sum((v - shift)^2), with
+            // the row's first entry as the shift
+            float shift = 0.f;
+            float2 nsh = make_float2(0.f, 0.f), s1 = make_float2(0.f, 0.f), s2 = make_float2(0.f, 0.f);
             bool ok = true;
             for (int kc = 0; kc < C::KC; ++kc) {
                 if (!__all_sync(0xffffffffu, mbar_wait(&s.full[stage], phase, abort_flag, kErrTimeoutEpilogue))) { ok = false; break; }
                 const uint8_t *zc = chunks + stage * C::CHUNK;
 #pragma unroll
                 for (int u = 0; u < 8; ++u) {
-                    uint4 w = *reinterpret_cast<const uint4 *>(zc + sw128_offset(row, u));
-                    float v[8] = {bf16_lo(w.x), bf16_hi(w.x), bf16_lo(w.y), bf16_hi(w.y),
-                                  bf16_lo(w.z), bf16_hi(w.z), bf16_lo(w.w), bf16_hi(w.w)};
-                    if (kc == 0 && u == 0) shift = v[0];
+                    const uint4 w = *reinterpret_cast<const uint4 *>(zc + sw128_offset(row, u));
+                    const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
+                    if (kc == 0 && u == 0) {
+                        shift = bf16_lo(w.x);
+                        nsh = make_float2(-shift, -shift);
+                    }
 #pragma unroll
-                    for (int e = 0; e < 8; ++e) {
-                        float d = v[e] - shift;
-                        s1 += d;
-                        s2 = fmaf(d, d, s2);
+                    for (int e = 0; e < 4; ++e) {
+                        const float2 d = f2_add(make_float2(bf16_lo(ws[e]), bf16_hi(ws[e])), nsh);
+                        s1 = f2_add(s1, d);
+                        s2 = f2_fma(d, d, s2);
                     }
                 }
                 __syncwarp();
@@ -210,8 +215,8 @@ __global__ void __launch_bounds__(448, 1) k1_project_kernel(const __grid_constan
             }
             if (!ok) break;
             const float inv_n = 1.0f / (float)CZ;
-            const float dm = s1 * inv_n;
-            const float var = fmaxf(s2 * inv_n - dm * dm, 0.f);
+            const float dm = (s1.x + s1.y) * inv_n;
+            const float var = fmaxf((s2.x + s2.y) * inv_n - dm * dm, 0.f);
             const float mean = shift + dm;
             const float rstd = rsqrtf(var + p.eps);
             const long long pi = (long long)p0 + row;
@@ -321,12 +326,11 @@ struct K1CmCfg {
 __device__ __forceinline__ uint32_t h2_as_u32(__half2 h) { return *reinterpret_cast<uint32_t *>(&h); }
 __device__ __forceinline__ __half2 u32_as_h2(uint32_t u) { return *reinterpret_cast<__half2 *>(&u); }
 
-// 0.5 + 0.5 tanh(x) on two halves at once (x = g / 2: the gate rows are pre-scaled by 1/2).
-__device__ __forceinline__ __half2 sigmoid_of_half_arg_h2(__half2 x) {
+// tanh of two halves at once (hardware approximation).
+__device__ __forceinline__ __half2 tanh_h2(__half2 x) {
     uint32_t t;
     asm("tanh.approx.f16x2 %0, %1;" : "=r"(t) : "r"(h2_as_u32(x)));
-    const __half2 half = __float2half2_rn(0.5f);
-    return __hfma2(u32_as_h2(t), half, half);
+    return u32_as_h2(t);
 }
 
 __global__ void __launch_bounds__(K1CmCfg::THREADS, 1) k1_project_cm_kernel(const __grid_constant__ K1Args p) {
@@ -336,10 +340,10 @@ __global__ void __launch_bounds__(K1CmCfg::THREADS, 1) k1_project_cm_kernel(cons
     uint8_t *w_s = base;                                  // KC chunks of [256 rows][64] bf16
     uint8_t *chunks = w_s + C::W_BYTES;                   // S chunks of [128 pairs][64] bf16
     uint8_t *staging = chunks + C::S * C::CHUNK;          // 2 x [128 ch][64 pairs] f16, 128B swizzle
-    float *st_mean = reinterpret_cast<float *>(staging + 2 * C::STG_BYTES);  // [SNB][128]
-    float *st_rstd = st_mean + C::SNB * 128;
-    __half *st_mask = reinterpret_cast<__half *>(st_rstd + C::SNB * 128);    // [SNB][128]
-    K1Smem &s = *reinterpret_cast<K1Smem *>(st_mask + C::SNB * 128);
+    float *st_nmean = reinterpret_cast<float *>(staging + 2 * C::STG_BYTES);  // [SNB][128] -mean
+    float *st_rstd = st_nmean + C::SNB * 128;
+    __half *st_hmask = reinterpret_cast<__half *>(st_rstd + C::SNB * 128);    // [SNB][128] mask / 2
+    K1Smem &s = *reinterpret_cast<K1Smem *>(st_hmask + C::SNB * 128);
 
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
@@ -459,22 +463,27 @@ __global__ void __launch_bounds__(K1CmCfg::THREADS, 1) k1_project_cm_kernel(cons
             const long long pi = (long long)p0 + row;
             uint16_t mbits = 0x3F80u;   // bf16 1.0; the load is issued first so its latency overlaps
             if (p.mask) mbits = (pi < p.NN) ? p.mask[(long long)b * p.NN + pi] : (uint16_t)0;
-            float shift = 0.f, s1 = 0.f, s2 = 0.f;
+            // shifted sums in packed pairs: s1 = sum(v - shift), s2 = sum((v - shift)^2), with
+            // the row's first entry as the shift
+            float shift = 0.f;
+            float2 nsh = make_float2(0.f, 0.f), s1 = make_float2(0.f, 0.f), s2 = make_float2(0.f, 0.f);
             bool ok = true;
             for (int kc = 0; kc < C::KC; ++kc) {
                 if (!__all_sync(0xffffffffu, mbar_wait(&s.full[stage], phase, abort_flag, kErrTimeoutEpilogue))) { ok = false; break; }
                 const uint8_t *zc = chunks + stage * C::CHUNK;
 #pragma unroll
                 for (int u = 0; u < 8; ++u) {
-                    uint4 w = *reinterpret_cast<const uint4 *>(zc + sw128_offset(row, u));
-                    float v[8] = {bf16_lo(w.x), bf16_hi(w.x), bf16_lo(w.y), bf16_hi(w.y),
-                                  bf16_lo(w.z), bf16_hi(w.z), bf16_lo(w.w), bf16_hi(w.w)};
-                    if (kc == 0 && u == 0) shift = v[0];
+                    const uint4 w = *reinterpret_cast<const uint4 *>(zc + sw128_offset(row, u));
+                    const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
+                    if (kc == 0 && u == 0) {
+                        shift = bf16_lo(w.x);
+                        nsh = make_float2(-shift, -shift);
+                    }
 #pragma unroll
-                    for (int e = 0; e < 8; ++e) {
-                        float d = v[e] - shift;
-                        s1 += d;
-                        s2 = fmaf(d, d, s2);
+                    for (int e = 0; e < 4; ++e) {
+                        const float2 d = f2_add(make_float2(bf16_lo(ws[e]), bf16_hi(ws[e])), nsh);
+                        s1 = f2_add(s1, d);
+                        s2 = f2_fma(d, d, s2);
                     }
                 }
                 __syncwarp();
@@ -483,12 +492,12 @@ __global__ void __launch_bounds__(K1CmCfg::THREADS, 1) k1_project_cm_kernel(cons
             }
             if (!ok) break;
             const float inv_n = 1.0f / (float)C::CZ;
-            const float dm = s1 * inv_n;
-            const float var = fmaxf(s2 * inv_n - dm * dm, 0.f);
+            const float dm = (s1.x + s1.y) * inv_n;
+            const float var = fmaxf((s2.x + s2.y) * inv_n - dm * dm, 0.f);
             if (!__all_sync(0xffffffffu, mbar_wait(&s.sempty[sbuf], sphase ^ 1, abort_flag, kErrTimeoutEpilogue))) break;
-            st_mean[sbuf * 128 + row] = shift + dm;
+            st_nmean[sbuf * 128 + row] = -(shift + dm);
             st_rstd[sbuf * 128 + row] = rsqrtf(var + p.eps);
-            st_mask[sbuf * 128 + row] = __float2half_rn(__uint_as_float((uint32_t)mbits << 16));
+            st_hmask[sbuf * 128 + row] = __float2half_rn(0.5f * __uint_as_float((uint32_t)mbits << 16));
             __syncwarp();
             if (lane == 0) mbar_arrive(&s.sfull[sbuf]);
             if (++sbuf == C::SNB) { sbuf = 0; sphase ^= 1; }
@@ -509,6 +518,8 @@ __global__ void __launch_bounds__(K1CmCfg::THREADS, 1) k1_project_cm_kernel(cons
         const CUtensorMap *tm_out = operand == 0 ? &p.tm_a : &p.tm_b;
         // {sum W'_gate, shift_gate, sum W'_proj, shift_proj}; the gate entries are for g / 2
         const float4 cv = p.vec[operand * C::C_H + c];
+        const float2 cg_sum = make_float2(cv.x, cv.x), cg_shift = make_float2(cv.y, cv.y);
+        const float2 cp_sum = make_float2(cv.z, cv.z), cp_shift = make_float2(cv.w, cv.w);
         const uint32_t lane_off = (uint32_t)(q * 32) << 16;
         int abuf = 0;
         uint32_t aphase = 0;
@@ -522,8 +533,8 @@ __global__ void __launch_bounds__(K1CmCfg::THREADS, 1) k1_project_cm_kernel(cons
             tc_fence_after();
             if (leader) tma_store_wait_read<0>();
             named_bar_sync(bar_id, 256);
-            const float *smean = st_mean + sbuf * 128 + col, *srstd = st_rstd + sbuf * 128 + col;
-            const __half *smask = st_mask + sbuf * 128 + col;
+            const float *snmean = st_nmean + sbuf * 128 + col, *srstd = st_rstd + sbuf * 128 + col;
+            const __half *shmask = st_hmask + sbuf * 128 + col;
 #pragma unroll 1
             for (int hh = 0; hh < 2; ++hh) {          // two halves of 16 pairs
                 float g[16], pr[16];
@@ -533,23 +544,20 @@ __global__ void __launch_bounds__(K1CmCfg::THREADS, 1) k1_project_cm_kernel(cons
                 uint32_t outw[8];
 #pragma unroll
                 for (int j = 0; j < 16; j += 4) {
-                    const float4 mu = *reinterpret_cast<const float4 *>(smean + 16 * hh + j);
+                    const float4 nm = *reinterpret_cast<const float4 *>(snmean + 16 * hh + j);
                     const float4 rs = *reinterpret_cast<const float4 *>(srstd + 16 * hh + j);
-                    const uint2 mk = *reinterpret_cast<const uint2 *>(smask + 16 * hh + j);
-                    const float mus[4] = {mu.x, mu.y, mu.z, mu.w};
-                    const float rss[4] = {rs.x, rs.y, rs.z, rs.w};
-                    float gv[4], pv[4];
-#pragma unroll
-                    for (int e = 0; e < 4; ++e) {
-                        gv[e] = fmaf(rss[e], fmaf(-mus[e], cv.x, g[j + e]), cv.y);
-                        pv[e] = fmaf(rss[e], fmaf(-mus[e], cv.z, pr[j + e]), cv.w);
-                    }
+                    const uint2 mk = *reinterpret_cast<const uint2 *>(shmask + 16 * hh + j);
 #pragma unroll
                     for (int h = 0; h < 2; ++h) {
-                        const __half2 sg = sigmoid_of_half_arg_h2(__floats2half2_rn(gv[2 * h], gv[2 * h + 1]));
-                        const __half2 ph = __floats2half2_rn(pv[2 * h], pv[2 * h + 1]);
-                        const __half2 mh = u32_as_h2(h == 0 ? mk.x : mk.y);
-                        outw[j / 2 + h] = h2_as_u32(__hmul2(__hmul2(sg, ph), mh));
+                        // two consecutive pairs of this channel in one packed lane pair
+                        const float2 nm2 = h == 0 ? make_float2(nm.x, nm.y) : make_float2(nm.z, nm.w);
+                        const float2 rs2 = h == 0 ? make_float2(rs.x, rs.y) : make_float2(rs.z, rs.w);
+                        const float2 gv = f2_fma(rs2, f2_fma(nm2, cg_sum, make_float2(g[j + 2 * h], g[j + 2 * h + 1])), cg_shift);
+                        const float2 pv = f2_fma(rs2, f2_fma(nm2, cp_sum, make_float2(pr[j + 2 * h], pr[j + 2 * h + 1])), cp_shift);
+                        // mask * sigmoid(2 x) = (mask / 2) tanh(x) + mask / 2, x being the halved gate
+                        const __half2 hm = u32_as_h2(h == 0 ? mk.x : mk.y);
+                        const __half2 gm = __hfma2(tanh_h2(__floats2half2_rn(gv.x, gv.y)), hm, hm);
+                        outw[j / 2 + h] = h2_as_u32(__hmul2(gm, __floats2half2_rn(pv.x, pv.y)));
                     }
                 }
 #pragma unroll

@@ -54,8 +54,10 @@ struct K3Smem {
     int abort_flag;
 };
 
+// Per-pair values the epilogue needs, in the form it uses them: negated means, the x rstd,
+// half the z rstd (the gate is evaluated as tanh of half its argument) and half the mask.
 struct K3Stats {
-    float mean_z, rstd_z, mean_x, rstd_x, mask, pad0, pad1, pad2;
+    float nmean_z, hrstd_z, nmean_x, rstd_x, hmask, pad0, pad1, pad2;
 };
 
 template <int CZ, bool OUT_F32>
@@ -68,8 +70,10 @@ __global__ void __launch_bounds__(448, 1) k3_output_kernel(const __grid_constant
     uint8_t *chunks = wg_s + C::WG_BYTES;              // S chunks
     uint8_t *staging = chunks + C::S * C::CHUNK;       // 2 x 16 KB
     K3Stats *stats = reinterpret_cast<K3Stats *>(staging + 2 * C::STG_BYTES);
-    float4 *vec_s = reinterpret_cast<float4 *>(stats + C::SNB * 128);   // [NCOL]
-    K3Smem &s = *reinterpret_cast<K3Smem *>(vec_s + C::NCOL);
+    // folding constants of this group's columns, one array each: sum W_o', shift_o,
+    // sum W_g', shift_g / 2
+    float *vec_s = reinterpret_cast<float *>(stats + C::SNB * 128);   // [4][NCOL]
+    K3Smem &s = *reinterpret_cast<K3Smem *>(vec_s + 4 * C::NCOL);
 
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
@@ -99,7 +103,13 @@ __global__ void __launch_bounds__(448, 1) k3_output_kernel(const __grid_constant
         s.abort_flag = 0;
         fence_mbarrier_init();
     }
-    if (threadIdx.x < C::NCOL) vec_s[threadIdx.x] = p.vec[n0 + threadIdx.x];
+    if (threadIdx.x < C::NCOL) {
+        const float4 v = p.vec[n0 + threadIdx.x];
+        vec_s[threadIdx.x] = v.x;
+        vec_s[C::NCOL + threadIdx.x] = v.y;
+        vec_s[2 * C::NCOL + threadIdx.x] = v.z;
+        vec_s[3 * C::NCOL + threadIdx.x] = 0.5f * v.w;
+    }
     if (warp == C::MMA_WARP) {
         tmem_alloc(&s.tmem_base, 512);
         tmem_relinquish();
@@ -209,8 +219,11 @@ __global__ void __launch_bounds__(448, 1) k3_output_kernel(const __grid_constant
         for (int pt = cta_in_group; pt < num_ptiles; pt += ctas_per_group) {
             const int b = pt / p.tiles_per_batch;
             const int p0 = (pt - b * p.tiles_per_batch) * 128;
-            float xs = 0.f, x1 = 0.f, x2 = 0.f, xabs = 0.f;
-            float zs = 0.f, z1 = 0.f, z2 = 0.f;
+            // shifted sums in packed pairs (shift = the first entry of each norm's row)
+            float xs = 0.f, zs = 0.f;
+            float2 nxs = make_float2(0.f, 0.f), nzs = make_float2(0.f, 0.f);
+            float2 x1 = make_float2(0.f, 0.f), x2 = make_float2(0.f, 0.f);
+            float2 z1 = make_float2(0.f, 0.f), z2 = make_float2(0.f, 0.f);
             bool ok = true;
             for (int c = 0; c < C::CPT; ++c) {
                 if (!__all_sync(0xffffffffu, mbar_wait(&s.full[stage], phase, abort_flag, kErrTimeoutEpilogue))) { ok = false; break; }
@@ -220,28 +233,33 @@ __global__ void __launch_bounds__(448, 1) k3_output_kernel(const __grid_constant
                     // unit (r64 / 8) of that row, swizzled with the row index.
                     const uint8_t *blk = ch + mblk * 8192;
 #pragma unroll 8
-                    for (int kr = 0; kr < 64; ++kr) {
-                        const uint16_t bits = *reinterpret_cast<const uint16_t *>(
-                            blk + sw128_offset(kr, r64 >> 3) + (r64 & 7) * 2);
-                        const float v = __half2float(__ushort_as_half(bits));
-                        xabs = fmaxf(xabs, fabsf(v));
-                        if (c == 0 && kr == 0) xs = v;
-                        const float d = v - xs;
-                        x1 += d;
-                        x2 = fmaf(d, d, x2);
+                    for (int kr = 0; kr < 64; kr += 2) {
+                        const float v0 = __half2float(__ushort_as_half(*reinterpret_cast<const uint16_t *>(
+                            blk + sw128_offset(kr, r64 >> 3) + (r64 & 7) * 2)));
+                        const float v1 = __half2float(__ushort_as_half(*reinterpret_cast<const uint16_t *>(
+                            blk + sw128_offset(kr + 1, r64 >> 3) + (r64 & 7) * 2)));
+                        if (c == 0 && kr == 0) {
+                            xs = v0;
+                            nxs = make_float2(-v0, -v0);
+                        }
+                        const float2 d = f2_add(make_float2(v0, v1), nxs);
+                        x1 = f2_add(x1, d);
+                        x2 = f2_fma(d, d, x2);
                     }
                 } else {
 #pragma unroll
                     for (int u = 0; u < 8; ++u) {
-                        uint4 w = *reinterpret_cast<const uint4 *>(ch + sw128_offset(row, u));
-                        float v[8] = {bf16_lo(w.x), bf16_hi(w.x), bf16_lo(w.y), bf16_hi(w.y),
-                                      bf16_lo(w.z), bf16_hi(w.z), bf16_lo(w.w), bf16_hi(w.w)};
-                        if (c == C::XC && u == 0) zs = v[0];
+                        const uint4 w = *reinterpret_cast<const uint4 *>(ch + sw128_offset(row, u));
+                        const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
+                        if (c == C::XC && u == 0) {
+                            zs = bf16_lo(w.x);
+                            nzs = make_float2(-zs, -zs);
+                        }
 #pragma unroll
-                        for (int e = 0; e < 8; ++e) {
-                            const float d = v[e] - zs;
-                            z1 += d;
-                            z2 = fmaf(d, d, z2);
+                        for (int e = 0; e < 4; ++e) {
+                            const float2 d = f2_add(make_float2(bf16_lo(ws[e]), bf16_hi(ws[e])), nzs);
+                            z1 = f2_add(z1, d);
+                            z2 = f2_fma(d, d, z2);
                         }
                     }
                 }
@@ -251,16 +269,20 @@ __global__ void __launch_bounds__(448, 1) k3_output_kernel(const __grid_constant
             }
             if (!ok) break;
             const float inv_h = 1.0f / (float)C::C_H, inv_z = 1.0f / (float)CZ;
-            const float dx = x1 * inv_h, dz = z1 * inv_z;
+            const float sx1 = x1.x + x1.y, sx2 = x2.x + x2.y;
+            const float sz1 = z1.x + z1.y, sz2 = z2.x + z2.y;
+            const float dx = sx1 * inv_h, dz = sz1 * inv_z;
             K3Stats st;
-            st.mean_x = xs + dx;
-            st.rstd_x = rsqrtf(fmaxf(x2 * inv_h - dx * dx, 0.f) + p.eps_x);
-            if (!(xabs <= 65504.f)) atomicOr(&g_device_error, (unsigned int)kErrRange);  // inf or NaN in x
-            st.mean_z = zs + dz;
-            st.rstd_z = rsqrtf(fmaxf(z2 * inv_z - dz * dz, 0.f) + p.eps);
+            st.nmean_x = -(xs + dx);
+            st.rstd_x = rsqrtf(fmaxf(sx2 * inv_h - dx * dx, 0.f) + p.eps_x);
+            // an inf or NaN anywhere in this pair's x makes the shifted square sum inf or NaN
+            if (!(fabsf(sx2) <= 3.0e38f)) atomicOr(&g_device_error, (unsigned int)kErrRange);
+            st.nmean_z = -(zs + dz);
+            st.hrstd_z = 0.5f * rsqrtf(fmaxf(sz2 * inv_z - dz * dz, 0.f) + p.eps);
             const long long pi = (long long)p0 + row;
-            st.mask = 1.f;
-            if (p.mask) st.mask = (pi < p.NN) ? __uint_as_float((uint32_t)p.mask[(long long)b * p.NN + pi] << 16) : 0.f;
+            float m = 1.f;
+            if (p.mask) m = (pi < p.NN) ? __uint_as_float((uint32_t)p.mask[(long long)b * p.NN + pi] << 16) : 0.f;
+            st.hmask = 0.5f * m;
             st.pad0 = st.pad1 = st.pad2 = 0.f;
             if (!__all_sync(0xffffffffu, mbar_wait(&s.sempty[sbuf], sphase ^ 1, abort_flag, kErrTimeoutEpilogue))) break;
             stats[sbuf * 128 + row] = st;
@@ -275,7 +297,8 @@ __global__ void __launch_bounds__(448, 1) k3_output_kernel(const __grid_constant
         const int row = q * 32 + lane;
         uint8_t *stg = staging + wg * C::STG_BYTES;
         const bool leader = (threadIdx.x & 127) == 0;
-        const float4 *vec = vec_s + wg * 64;
+        const float *v_sum_o = vec_s + wg * 64, *v_shift_o = v_sum_o + C::NCOL;
+        const float *v_sum_g = v_sum_o + 2 * C::NCOL, *v_hshift_g = v_sum_o + 3 * C::NCOL;
         int abuf = 0;
         uint32_t aphase = 0;
         int sbuf = 0;
@@ -285,6 +308,9 @@ __global__ void __launch_bounds__(448, 1) k3_output_kernel(const __grid_constant
             const int p0 = (pt - b * p.tiles_per_batch) * 128;
             if (!group_all(mbar_wait(&s.sfull[sbuf], sphase, abort_flag, kErrTimeoutEpilogue), 1 + wg, 128)) break;
             const K3Stats st = stats[sbuf * 128 + row];
+            const float2 nmx = make_float2(st.nmean_x, st.nmean_x), rx = make_float2(st.rstd_x, st.rstd_x);
+            const float2 nmz = make_float2(st.nmean_z, st.nmean_z), hrz = make_float2(st.hrstd_z, st.hrstd_z);
+            const float2 hm = make_float2(st.hmask, st.hmask);
             __syncwarp();
             if (lane == 0) mbar_arrive(&s.sempty[sbuf]);
             if (++sbuf == C::SNB) { sbuf = 0; sphase ^= 1; }
@@ -305,11 +331,27 @@ __global__ void __launch_bounds__(448, 1) k3_output_kernel(const __grid_constant
                     tmem_ld32(t2 + col, g);
                     tc_wait_ld();
 #pragma unroll
-                    for (int e = 0; e < 32; ++e) {
-                        const float4 cv = vec[col + e];
-                        const float ov = fmaf(st.rstd_x, fmaf(-st.mean_x, cv.x, o[e]), cv.y);
-                        const float gv = fmaf(st.rstd_z, fmaf(-st.mean_z, cv.z, g[e]), cv.w);
-                        o[e] = st.mask * sigmoid_exp(gv) * ov;
+                    for (int e = 0; e < 32; e += 4) {
+                        const float4 so = *reinterpret_cast<const float4 *>(v_sum_o + col + e);
+                        const float4 ho = *reinterpret_cast<const float4 *>(v_shift_o + col + e);
+                        const float4 sg = *reinterpret_cast<const float4 *>(v_sum_g + col + e);
+                        const float4 hg = *reinterpret_cast<const float4 *>(v_hshift_g + col + e);
+#pragma unroll
+                        for (int k = 0; k < 2; ++k) {
+                            // output channels e + 2k and e + 2k + 1 of this pair, packed
+                            const float2 so2 = k == 0 ? make_float2(so.x, so.y) : make_float2(so.z, so.w);
+                            const float2 ho2 = k == 0 ? make_float2(ho.x, ho.y) : make_float2(ho.z, ho.w);
+                            const float2 sg2 = k == 0 ? make_float2(sg.x, sg.y) : make_float2(sg.z, sg.w);
+                            const float2 hg2 = k == 0 ? make_float2(hg.x, hg.y) : make_float2(hg.z, hg.w);
+                            const int i = e + 2 * k;
+                            const float2 ov = f2_fma(rx, f2_fma(nmx, so2, make_float2(o[i], o[i + 1])), ho2);
+                            // half the gate argument; mask * sigmoid(2 y) = (mask / 2) tanh(y) + mask / 2
+                            const float2 gh = f2_fma(hrz, f2_fma(nmz, sg2, make_float2(g[i], g[i + 1])), hg2);
+                            const float2 gm = f2_fma(hm, make_float2(tanh_approx(gh.x), tanh_approx(gh.y)), hm);
+                            const float2 r = f2_mul(gm, ov);
+                            o[i] = r.x;
+                            o[i + 1] = r.y;
+                        }
                     }
                     if (OUT_F32) {
 #pragma unroll
