@@ -311,10 +311,11 @@ struct K1CmCfg {
     static constexpr int W_CHUNK = 2 * C_H * 64 * 2;          // [gate 128 rows, proj 128 rows] x 64 k
     static constexpr int W_BYTES = KC * W_CHUNK;              // 64 KB
     static constexpr int CHUNK = 128 * 64 * 2;                // z chunk: 128 pairs x 64 channels
-    static constexpr int STG_BYTES = C_H * 64 * 2;            // per pair half: [128 ch][64 pairs] f16
+    static constexpr int WARP_STG = 32 * 32 * 2;              // per epilogue warp: [32 ch][32 pairs] f16
+    static constexpr int STG_TOTAL = 16 * WARP_STG;           // 32 KB for the 16 epilogue warps
     static constexpr int SNB = 2;
     static constexpr int STATS_BYTES = SNB * 128 * (4 + 4 + 2);   // mean, rstd (f32), mask (f16) per pair
-    static constexpr int FIXED = 1024 + W_BYTES + 2 * STG_BYTES + STATS_BYTES + 1024;
+    static constexpr int FIXED = 1024 + W_BYTES + STG_TOTAL + STATS_BYTES + 1024;
     static constexpr int S = (232448 - FIXED) / CHUNK > 8 ? 8 : (232448 - FIXED) / CHUNK;
     static constexpr size_t SMEM = FIXED + (size_t)S * CHUNK;
     static constexpr int EPI_WARPS = 16;                      // four warpgroups, 32 pairs each
@@ -339,8 +340,8 @@ __global__ void __launch_bounds__(K1CmCfg::THREADS, 1) k1_project_cm_kernel(cons
     uint8_t *base = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint8_t *w_s = base;                                  // KC chunks of [256 rows][64] bf16
     uint8_t *chunks = w_s + C::W_BYTES;                   // S chunks of [128 pairs][64] bf16
-    uint8_t *staging = chunks + C::S * C::CHUNK;          // 2 x [128 ch][64 pairs] f16, 128B swizzle
-    float *st_nmean = reinterpret_cast<float *>(staging + 2 * C::STG_BYTES);  // [SNB][128] -mean
+    uint8_t *staging = chunks + C::S * C::CHUNK;          // 16 x [32 ch][32 pairs] f16, 64B swizzle
+    float *st_nmean = reinterpret_cast<float *>(staging + C::STG_TOTAL);     // [SNB][128] -mean
     float *st_rstd = st_nmean + C::SNB * 128;
     __half *st_hmask = reinterpret_cast<__half *>(st_rstd + C::SNB * 128);    // [SNB][128] mask / 2
     K1Smem &s = *reinterpret_cast<K1Smem *>(st_hmask + C::SNB * 128);
@@ -504,17 +505,14 @@ __global__ void __launch_bounds__(K1CmCfg::THREADS, 1) k1_project_cm_kernel(cons
         }
     } else {
         // epilogue: thread = hidden channel c of this CTA's operand; warpgroup wg owns the
-        // 32 pairs [32 wg, 32 wg + 32) of the tile; warpgroups 2h and 2h+1 share the staging
-        // buffer and the TMA store of pair half h.
+        // 32 pairs [32 wg, 32 wg + 32) of the tile. Every warp runs on its own: it waits on the
+        // barriers itself, stages its [32 channels][32 pairs] block in its own 2 KB of shared
+        // memory (64-byte rows, 64-byte swizzle) and issues that block's TMA store.
         const int wg = warp >> 2;
-        const int half = wg >> 1;
-        const int sub = wg & 1;
         const int q = warp & 3;
         const int c = q * 32 + lane;
         const int col = 32 * wg;
-        uint8_t *stg = staging + half * C::STG_BYTES;
-        const bool leader = (threadIdx.x & 255) == 0;
-        const uint32_t bar_id = 1 + half;
+        uint8_t *stg = staging + warp * C::WARP_STG;
         const CUtensorMap *tm_out = operand == 0 ? &p.tm_a : &p.tm_b;
         // {sum W'_gate, shift_gate, sum W'_proj, shift_proj}; the gate entries are for g / 2
         const float4 cv = p.vec[operand * C::C_H + c];
@@ -528,11 +526,12 @@ __global__ void __launch_bounds__(K1CmCfg::THREADS, 1) k1_project_cm_kernel(cons
         for (int pt = cta_in_group; pt < num_ptiles; pt += ctas_per_group) {
             const int b = pt / p.tiles_per_batch;
             const int p0 = (pt - b * p.tiles_per_batch) * 128;
-            if (!group_all(mbar_wait(&s.sfull[sbuf], sphase, abort_flag, kErrTimeoutEpilogue), bar_id, 256)) break;
-            if (!group_all(mbar_wait(&s.tfull[abuf], aphase, abort_flag, kErrTimeoutEpilogue), bar_id, 256)) break;
+            if (!__all_sync(0xffffffffu, mbar_wait(&s.sfull[sbuf], sphase, abort_flag, kErrTimeoutEpilogue) &&
+                                             mbar_wait(&s.tfull[abuf], aphase, abort_flag, kErrTimeoutEpilogue)))
+                break;
             tc_fence_after();
-            if (leader) tma_store_wait_read<0>();
-            named_bar_sync(bar_id, 256);
+            if (lane == 0) tma_store_wait_read<0>();   // this warp's previous store has read its block
+            __syncwarp();
             const float *snmean = st_nmean + sbuf * 128 + col, *srstd = st_rstd + sbuf * 128 + col;
             const __half *shmask = st_hmask + sbuf * 128 + col;
 #pragma unroll 1
@@ -562,25 +561,24 @@ __global__ void __launch_bounds__(K1CmCfg::THREADS, 1) k1_project_cm_kernel(cons
                 }
 #pragma unroll
                 for (int u = 0; u < 2; ++u)
-                    *reinterpret_cast<uint4 *>(stg + sw128_offset(c, sub * 4 + 2 * hh + u)) =
+                    *reinterpret_cast<uint4 *>(stg + sw64_offset(lane, 2 * hh + u)) =
                         make_uint4(outw[4 * u], outw[4 * u + 1], outw[4 * u + 2], outw[4 * u + 3]);
             }
             tc_fence_before();
+            fence_proxy_async_smem();
             __syncwarp();
             if (lane == 0) {
                 mbar_arrive(&s.tempty[abuf]);
                 mbar_arrive(&s.sempty[sbuf]);
+                if (p0 + col < p.NN) {                  // blocks wholly past the last pair are not stored
+                    tma_store_3d(tm_out, stg, p0 + col, q * 32, b);
+                    tma_store_commit();
+                }
             }
             if (++abuf == 2) { abuf = 0; aphase ^= 1; }
             if (++sbuf == C::SNB) { sbuf = 0; sphase ^= 1; }
-            fence_proxy_async_smem();
-            named_bar_sync(bar_id, 256);
-            if (leader) {
-                tma_store_3d(tm_out, stg, p0 + 64 * half, 0, b);
-                tma_store_commit();
-            }
         }
-        if (leader) tma_store_wait_all<0>();
+        if (lane == 0) tma_store_wait_all<0>();
     }
 
     tc_fence_before();

@@ -16,7 +16,7 @@
 // three column groups (a CTA keeps one group) so each group's weights stay resident.
 //
 // Warps: 0-7 epilogue (two warpgroups, 64 output channels each), 8-11 LayerNorm
-// statistics of x and z (one thread per pair), 12 TMA producer, 13 TMEM + MMA.
+// statistics of x and 12-15 of z (one thread per pair each), 16 TMA producer, 17 TMEM + MMA.
 #include "kernels.h"
 #include "sm100.cuh"
 
@@ -40,8 +40,9 @@ struct K3Cfg {
     static constexpr int FIXED = 1024 + WO_BYTES + WG_BYTES + 2 * STG_BYTES + SNB * 128 * 32 + VEC_BYTES + 1024;
     static constexpr int S = (232448 - FIXED) / CHUNK > 8 ? 8 : (232448 - FIXED) / CHUNK;
     static constexpr size_t SMEM = FIXED + (size_t)S * CHUNK;
-    static constexpr int THREADS = 448;
-    static constexpr int TMA_WARP = 12, MMA_WARP = 13;
+    static constexpr int THREADS = 576;
+    static constexpr int STATS_WARP0 = 8;
+    static constexpr int TMA_WARP = 16, MMA_WARP = 17;
 };
 
 struct K3Smem {
@@ -61,7 +62,7 @@ struct K3Stats {
 };
 
 template <int CZ, bool OUT_F32>
-__global__ void __launch_bounds__(448, 1) k3_output_kernel(const __grid_constant__ K3Args p) {
+__global__ void __launch_bounds__(576, 1) k3_output_kernel(const __grid_constant__ K3Args p) {
     using C = K3Cfg<CZ, OUT_F32>;
     extern __shared__ uint8_t smem_raw[];
     uint8_t *base = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -89,14 +90,14 @@ __global__ void __launch_bounds__(448, 1) k3_output_kernel(const __grid_constant
         mbar_init(&s.wbar, 1);
         for (int i = 0; i < C::S; ++i) {
             mbar_init(&s.full[i], 1);
-            mbar_init(&s.empty[i], 1 + 4);
+            mbar_init(&s.empty[i], 1 + 8);  // MMA commit + both statistics roles
         }
         for (int i = 0; i < 2; ++i) {
             mbar_init(&s.tfull[i], 1);
             mbar_init(&s.tempty[i], 8);
         }
         for (int i = 0; i < C::SNB; ++i) {
-            mbar_init(&s.sfull[i], 4);
+            mbar_init(&s.sfull[i], 8);     // x and z statistics warps
             mbar_init(&s.sempty[i], 8);
         }
         mbar_init(&s.drain, 1);
@@ -142,9 +143,9 @@ __global__ void __launch_bounds__(448, 1) k3_output_kernel(const __grid_constant
                     uint8_t *dst = chunks + stage * C::CHUNK;
                     mbar_arrive_expect_tx(&s.full[stage], C::CHUNK);
                     if (c < C::XC) {
-                        // x: K = channels c*64..+63 (rows), M = pairs (two 64-pair MN blocks)
-                        tma_load_3d(dst, &p.tm_x, &s.full[stage], p0, c * 64, b);
-                        tma_load_3d(dst + 8192, &p.tm_x, &s.full[stage], p0 + 64, c * 64, b);
+                        // x: K = channels c*64..+63 (rows), M = pairs: both 64-pair MN blocks
+                        // ([block][channel][64 pairs]) in one copy
+                        tma_load_4d(dst, &p.tm_x, &s.full[stage], 0, c * 64, p0 / 64, b);
                     } else {
                         tma_load_3d(dst, &p.tm_z, &s.full[stage], (c - C::XC) * 64, p0, b);
                     }
@@ -207,9 +208,14 @@ __global__ void __launch_bounds__(448, 1) k3_output_kernel(const __grid_constant
             tc_commit(&s.drain);
             mbar_drain(&s.drain, 0);
         }
-    } else if (warp >= 8) {
-        // statistics of x (over c_h) and z (over c_z) for pair `row`
-        const int row = (warp - 8) * 32 + lane;
+    } else if (warp >= C::STATS_WARP0) {
+        // LayerNorm statistics, one thread per pair `row`: warps 8-11 take x over c_h (from the
+        // x chunks), warps 12-15 z over c_z (from the z chunks). Both roles wait for and release
+        // every chunk in order (releasing the other role's chunks at once): a role that skipped
+        // chunks could run more than a ring ahead of the producer and then match the parity of
+        // an older phase of a stage's barrier.
+        const bool xrole = warp < C::STATS_WARP0 + 4;
+        const int row = ((warp - C::STATS_WARP0) & 3) * 32 + lane;
         const int mblk = row >> 6;         // which 64-pair MN block of an x chunk
         const int r64 = row & 63;
         int stage = 0;
@@ -219,47 +225,50 @@ __global__ void __launch_bounds__(448, 1) k3_output_kernel(const __grid_constant
         for (int pt = cta_in_group; pt < num_ptiles; pt += ctas_per_group) {
             const int b = pt / p.tiles_per_batch;
             const int p0 = (pt - b * p.tiles_per_batch) * 128;
-            // shifted sums in packed pairs (shift = the first entry of each norm's row)
-            float xs = 0.f, zs = 0.f;
-            float2 nxs = make_float2(0.f, 0.f), nzs = make_float2(0.f, 0.f);
-            float2 x1 = make_float2(0.f, 0.f), x2 = make_float2(0.f, 0.f);
-            float2 z1 = make_float2(0.f, 0.f), z2 = make_float2(0.f, 0.f);
+            const long long pi = (long long)p0 + row;
+            uint16_t mbits = 0x3F80u;      // bf16 1.0; issued first so its latency overlaps the sums
+            if (!xrole && p.mask) mbits = (pi < p.NN) ? p.mask[(long long)b * p.NN + pi] : (uint16_t)0;
+            // shifted sums in packed pairs (shift = the first entry of the row)
+            float sh = 0.f;
+            float2 nsh = make_float2(0.f, 0.f), s1 = make_float2(0.f, 0.f), s2 = make_float2(0.f, 0.f);
             bool ok = true;
             for (int c = 0; c < C::CPT; ++c) {
                 if (!__all_sync(0xffffffffu, mbar_wait(&s.full[stage], phase, abort_flag, kErrTimeoutEpilogue))) { ok = false; break; }
-                const uint8_t *ch = chunks + stage * C::CHUNK;
-                if (c < C::XC) {
-                    // MN-major: K row kr holds 64 pairs; this pair's element sits in 16-byte
-                    // unit (r64 / 8) of that row, swizzled with the row index.
-                    const uint8_t *blk = ch + mblk * 8192;
+                if (xrole == (c < C::XC)) {
+                    const uint8_t *ch = chunks + stage * C::CHUNK;
+                    if (xrole) {
+                        // MN-major: K row kr holds 64 pairs; this pair's element sits in 16-byte
+                        // unit (r64 / 8) of that row, swizzled with the row index.
+                        const uint8_t *blk = ch + mblk * 8192;
 #pragma unroll 8
-                    for (int kr = 0; kr < 64; kr += 2) {
-                        const float v0 = __half2float(__ushort_as_half(*reinterpret_cast<const uint16_t *>(
-                            blk + sw128_offset(kr, r64 >> 3) + (r64 & 7) * 2)));
-                        const float v1 = __half2float(__ushort_as_half(*reinterpret_cast<const uint16_t *>(
-                            blk + sw128_offset(kr + 1, r64 >> 3) + (r64 & 7) * 2)));
-                        if (c == 0 && kr == 0) {
-                            xs = v0;
-                            nxs = make_float2(-v0, -v0);
+                        for (int kr = 0; kr < 64; kr += 2) {
+                            const float v0 = __half2float(__ushort_as_half(*reinterpret_cast<const uint16_t *>(
+                                blk + sw128_offset(kr, r64 >> 3) + (r64 & 7) * 2)));
+                            const float v1 = __half2float(__ushort_as_half(*reinterpret_cast<const uint16_t *>(
+                                blk + sw128_offset(kr + 1, r64 >> 3) + (r64 & 7) * 2)));
+                            if (c == 0 && kr == 0) {
+                                sh = v0;
+                                nsh = make_float2(-v0, -v0);
+                            }
+                            const float2 d = f2_add(make_float2(v0, v1), nsh);
+                            s1 = f2_add(s1, d);
+                            s2 = f2_fma(d, d, s2);
                         }
-                        const float2 d = f2_add(make_float2(v0, v1), nxs);
-                        x1 = f2_add(x1, d);
-                        x2 = f2_fma(d, d, x2);
-                    }
-                } else {
+                    } else {
 #pragma unroll
-                    for (int u = 0; u < 8; ++u) {
-                        const uint4 w = *reinterpret_cast<const uint4 *>(ch + sw128_offset(row, u));
-                        const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
-                        if (c == C::XC && u == 0) {
-                            zs = bf16_lo(w.x);
-                            nzs = make_float2(-zs, -zs);
-                        }
+                        for (int u = 0; u < 8; ++u) {
+                            const uint4 w = *reinterpret_cast<const uint4 *>(ch + sw128_offset(row, u));
+                            const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
+                            if (c == C::XC && u == 0) {
+                                sh = bf16_lo(w.x);
+                                nsh = make_float2(-sh, -sh);
+                            }
 #pragma unroll
-                        for (int e = 0; e < 4; ++e) {
-                            const float2 d = f2_add(make_float2(bf16_lo(ws[e]), bf16_hi(ws[e])), nzs);
-                            z1 = f2_add(z1, d);
-                            z2 = f2_fma(d, d, z2);
+                            for (int e = 0; e < 4; ++e) {
+                                const float2 d = f2_add(make_float2(bf16_lo(ws[e]), bf16_hi(ws[e])), nsh);
+                                s1 = f2_add(s1, d);
+                                s2 = f2_fma(d, d, s2);
+                            }
                         }
                     }
                 }
@@ -268,35 +277,36 @@ __global__ void __launch_bounds__(448, 1) k3_output_kernel(const __grid_constant
                 if (++stage == C::S) { stage = 0; phase ^= 1; }
             }
             if (!ok) break;
-            const float inv_h = 1.0f / (float)C::C_H, inv_z = 1.0f / (float)CZ;
-            const float sx1 = x1.x + x1.y, sx2 = x2.x + x2.y;
-            const float sz1 = z1.x + z1.y, sz2 = z2.x + z2.y;
-            const float dx = sx1 * inv_h, dz = sz1 * inv_z;
-            K3Stats st;
-            st.nmean_x = -(xs + dx);
-            st.rstd_x = rsqrtf(fmaxf(sx2 * inv_h - dx * dx, 0.f) + p.eps_x);
+            const float t1 = s1.x + s1.y, t2 = s2.x + s2.y;
+            const float inv_n = 1.0f / (float)(xrole ? C::C_H : CZ);
+            const float dm = t1 * inv_n;
+            const float rs = rsqrtf(fmaxf(t2 * inv_n - dm * dm, 0.f) + (xrole ? p.eps_x : p.eps));
             // an inf or NaN anywhere in this pair's x makes the shifted square sum inf or NaN
-            if (!(fabsf(sx2) <= 3.0e38f)) atomicOr(&g_device_error, (unsigned int)kErrRange);
-            st.nmean_z = -(zs + dz);
-            st.hrstd_z = 0.5f * rsqrtf(fmaxf(sz2 * inv_z - dz * dz, 0.f) + p.eps);
-            const long long pi = (long long)p0 + row;
-            float m = 1.f;
-            if (p.mask) m = (pi < p.NN) ? __uint_as_float((uint32_t)p.mask[(long long)b * p.NN + pi] << 16) : 0.f;
-            st.hmask = 0.5f * m;
-            st.pad0 = st.pad1 = st.pad2 = 0.f;
+            if (xrole && !(fabsf(t2) <= 3.0e38f)) atomicOr(&g_device_error, (unsigned int)kErrRange);
             if (!__all_sync(0xffffffffu, mbar_wait(&s.sempty[sbuf], sphase ^ 1, abort_flag, kErrTimeoutEpilogue))) break;
-            stats[sbuf * 128 + row] = st;
+            K3Stats &st = stats[sbuf * 128 + row];
+            if (xrole) {
+                st.nmean_x = -(sh + dm);
+                st.rstd_x = rs;
+            } else {
+                st.nmean_z = -(sh + dm);
+                st.hrstd_z = 0.5f * rs;
+                st.hmask = 0.5f * __uint_as_float((uint32_t)mbits << 16);
+            }
             __syncwarp();
             if (lane == 0) mbar_arrive(&s.sfull[sbuf]);
             if (++sbuf == C::SNB) { sbuf = 0; sphase ^= 1; }
         }
     } else {
-        // epilogue: warpgroup wg handles output channels n0 + wg*64 .. +63
+        // epilogue: warpgroup wg handles output channels n0 + wg*64 .. +63; warp q of it the
+        // pairs [32q, 32q + 32) of the tile. Every warp runs on its own: it waits on the
+        // barriers itself, stages its 32 pair rows in its own 4 KB of the warpgroup's staging
+        // buffer and issues the TMA store of that block.
         const int wg = warp >> 2;
         const int q = warp & 3;
         const int row = q * 32 + lane;
-        uint8_t *stg = staging + wg * C::STG_BYTES;
-        const bool leader = (threadIdx.x & 127) == 0;
+        uint8_t *stg = staging + wg * C::STG_BYTES;   // rows [32q, 32q + 32) belong to this warp
+        uint8_t *wstg = stg + q * 32 * 128;
         const float *v_sum_o = vec_s + wg * 64, *v_shift_o = v_sum_o + C::NCOL;
         const float *v_sum_g = v_sum_o + 2 * C::NCOL, *v_hshift_g = v_sum_o + 3 * C::NCOL;
         int abuf = 0;
@@ -306,7 +316,7 @@ __global__ void __launch_bounds__(448, 1) k3_output_kernel(const __grid_constant
         for (int pt = cta_in_group; pt < num_ptiles; pt += ctas_per_group) {
             const int b = pt / p.tiles_per_batch;
             const int p0 = (pt - b * p.tiles_per_batch) * 128;
-            if (!group_all(mbar_wait(&s.sfull[sbuf], sphase, abort_flag, kErrTimeoutEpilogue), 1 + wg, 128)) break;
+            if (!__all_sync(0xffffffffu, mbar_wait(&s.sfull[sbuf], sphase, abort_flag, kErrTimeoutEpilogue))) break;
             const K3Stats st = stats[sbuf * 128 + row];
             const float2 nmx = make_float2(st.nmean_x, st.nmean_x), rx = make_float2(st.rstd_x, st.rstd_x);
             const float2 nmz = make_float2(st.nmean_z, st.nmean_z), hrz = make_float2(st.hrstd_z, st.hrstd_z);
@@ -315,23 +325,23 @@ __global__ void __launch_bounds__(448, 1) k3_output_kernel(const __grid_constant
             if (lane == 0) mbar_arrive(&s.sempty[sbuf]);
             if (++sbuf == C::SNB) { sbuf = 0; sphase ^= 1; }
 
-            if (!group_all(mbar_wait(&s.tfull[abuf], aphase, abort_flag, kErrTimeoutEpilogue), 1 + wg, 128)) break;
+            if (!__all_sync(0xffffffffu, mbar_wait(&s.tfull[abuf], aphase, abort_flag, kErrTimeoutEpilogue))) break;
             tc_fence_after();
             const uint32_t t1 = tmem_base + abuf * 256 + ((uint32_t)(q * 32) << 16) + wg * 64;
             const uint32_t t2 = t1 + 128;
 #pragma unroll 1
             for (int sc = 0; sc < 64 / C::COLS_PER_STORE; ++sc) {
-                if (leader) tma_store_wait_read<0>();
-                named_bar_sync(1 + wg, 128);
+                if (lane == 0) tma_store_wait_read<0>();   // this warp's previous store has read its rows
+                __syncwarp();
 #pragma unroll 1
-                for (int h = 0; h < C::COLS_PER_STORE / 32; ++h) {
-                    const int col = sc * C::COLS_PER_STORE + h * 32;   // within this warpgroup's 64
-                    float o[32], g[32];
-                    tmem_ld32(t1 + col, o);
-                    tmem_ld32(t2 + col, g);
+                for (int h = 0; h < C::COLS_PER_STORE / 16; ++h) {
+                    const int col = sc * C::COLS_PER_STORE + h * 16;   // within this warpgroup's 64
+                    float o[16], g[16];
+                    tmem_ld16(t1 + col, o);
+                    tmem_ld16(t2 + col, g);
                     tc_wait_ld();
 #pragma unroll
-                    for (int e = 0; e < 32; e += 4) {
+                    for (int e = 0; e < 16; e += 4) {
                         const float4 so = *reinterpret_cast<const float4 *>(v_sum_o + col + e);
                         const float4 ho = *reinterpret_cast<const float4 *>(v_shift_o + col + e);
                         const float4 sg = *reinterpret_cast<const float4 *>(v_sum_g + col + e);
@@ -355,25 +365,25 @@ __global__ void __launch_bounds__(448, 1) k3_output_kernel(const __grid_constant
                     }
                     if (OUT_F32) {
 #pragma unroll
-                        for (int u = 0; u < 8; ++u)
-                            *reinterpret_cast<float4 *>(stg + sw128_offset(row, u)) =
+                        for (int u = 0; u < 4; ++u)
+                            *reinterpret_cast<float4 *>(stg + sw128_offset(row, h * 4 + u)) =
                                 make_float4(o[4 * u], o[4 * u + 1], o[4 * u + 2], o[4 * u + 3]);
                     } else {
 #pragma unroll
-                        for (int u = 0; u < 4; ++u) {
+                        for (int u = 0; u < 2; ++u) {
                             uint4 w;
                             w.x = pack_bf16x2(o[8 * u + 0], o[8 * u + 1]);
                             w.y = pack_bf16x2(o[8 * u + 2], o[8 * u + 3]);
                             w.z = pack_bf16x2(o[8 * u + 4], o[8 * u + 5]);
                             w.w = pack_bf16x2(o[8 * u + 6], o[8 * u + 7]);
-                            *reinterpret_cast<uint4 *>(stg + sw128_offset(row, h * 4 + u)) = w;
+                            *reinterpret_cast<uint4 *>(stg + sw128_offset(row, h * 2 + u)) = w;
                         }
                     }
                 }
                 fence_proxy_async_smem();
-                named_bar_sync(1 + wg, 128);
-                if (leader) {
-                    tma_store_3d(&p.tm_out, stg, n0 + wg * 64 + sc * C::COLS_PER_STORE, p0, b);
+                __syncwarp();
+                if (lane == 0 && p0 + q * 32 < p.NN) {   // blocks wholly past the last pair are not stored
+                    tma_store_3d(&p.tm_out, wstg, n0 + wg * 64 + sc * C::COLS_PER_STORE, p0 + q * 32, b);
                     tma_store_commit();
                 }
             }
@@ -382,7 +392,7 @@ __global__ void __launch_bounds__(448, 1) k3_output_kernel(const __grid_constant
             if (lane == 0) mbar_arrive(&s.tempty[abuf]);
             if (++abuf == 2) { abuf = 0; aphase ^= 1; }
         }
-        if (leader) tma_store_wait_all<0>();
+        if (lane == 0) tma_store_wait_all<0>();
     }
 
     tc_fence_before();

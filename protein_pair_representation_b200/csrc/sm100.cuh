@@ -168,6 +168,15 @@ __device__ __forceinline__ void tma_load_3d(void *dst, const CUtensorMap *map, u
         : "memory");
 }
 
+__device__ __forceinline__ void tma_load_4d(void *dst, const CUtensorMap *map, uint64_t *bar,
+                                            int32_t c0, int32_t c1, int32_t c2, int32_t c3) {
+    asm volatile(
+        "cp.async.bulk.tensor.4d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
+        " [%0], [%1, {%3, %4, %5, %6}], [%2];" ::"r"(smem_u32(dst)),
+        "l"(reinterpret_cast<uint64_t>(map)), "r"(smem_u32(bar)), "r"(c0), "r"(c1), "r"(c2), "r"(c3)
+        : "memory");
+}
+
 __device__ __forceinline__ void tma_store_3d(const CUtensorMap *map, const void *src, int32_t c0,
                                              int32_t c1, int32_t c2) {
     asm volatile(
@@ -374,6 +383,12 @@ __device__ __forceinline__ float bf16_hi(uint32_t w) { return __uint_as_float(w 
 // Byte offset of 16-byte unit `u` of row `r` in a 128-byte-swizzled tile (rows of 128 B).
 __device__ __forceinline__ uint32_t sw128_offset(uint32_t r, uint32_t u) {
     return r * 128u + ((u ^ (r & 7u)) << 4);
+}
+
+// Byte offset of 16-byte unit `u` (0..3) of row `r` in a 64-byte-swizzled tile (rows of 64 B;
+// address bits 4-5 are XORed with bits 7-8, so the pattern repeats every 512 bytes).
+__device__ __forceinline__ uint32_t sw64_offset(uint32_t r, uint32_t u) {
+    return r * 64u + ((u ^ ((r >> 1) & 3u)) << 4);
 }
 
 }  // namespace trimul

@@ -389,11 +389,12 @@ static trimul_status_t run_project_bf16(const trimul_layer_t *L, const void *z, 
     {
         uint64_t dims[3] = {NN, (uint64_t)ch, (uint64_t)B};
         uint64_t strides[2] = {NN * 2, (uint64_t)ch * NN * 2};
-        // c_z = 128: channel-lane kernel stores [128 channels][64 pairs] tiles through a 128B swizzle;
-        // c_z = 384: pair-lane kernel stores [channels][128 pairs] rows without swizzle
+        // c_z = 128: each warp of the channel-lane kernel stores a [32 channels][32 pairs] block
+        // through a 64B swizzle; c_z = 384: pair-lane kernel stores [channels][128 pairs] rows
+        // without swizzle
         const bool cm = k1_row_mode(cz) == 2;
-        uint32_t box[3] = {cm ? 64u : 128u, (uint32_t)k1_channels_per_warpgroup(cz), 1};
-        const CUtensorMapSwizzle sw = cm ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE;
+        uint32_t box[3] = {cm ? 32u : 128u, cm ? 32u : (uint32_t)k1_channels_per_warpgroup(cz), 1};
+        const CUtensorMapSwizzle sw = cm ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_NONE;
         TRY(make_map(&p.tm_a, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 3, a, dims, strides, box, sw, "K1 a"));
         TRY(make_map(&p.tm_b, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 3, b, dims, strides, box, sw, "K1 b"));
     }
@@ -453,10 +454,12 @@ static trimul_status_t run_output_bf16(const trimul_layer_t *L, const void *z, c
     const int cz = L->c_z, ch = L->c_h;
     K3Args p{};
     {
-        uint64_t dims[3] = {NN, (uint64_t)ch, (uint64_t)B};
-        uint64_t strides[2] = {NN * 2, (uint64_t)ch * NN * 2};
-        uint32_t box[3] = {64, 64, 1};
-        TRY(make_map(&p.tm_x, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 3, x, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_128B, "K3 x"));
+        // x [B][c_h][N*N] viewed as [B][N*N/64 blocks][c_h][64 pairs], so that one copy brings
+        // the two 64-pair MN blocks of a 128-pair tile for 64 channels (N*N is a multiple of 64)
+        uint64_t dims[4] = {64, (uint64_t)ch, NN / 64, (uint64_t)B};
+        uint64_t strides[3] = {NN * 2, 128, (uint64_t)ch * NN * 2};
+        uint32_t box[4] = {64, 64, 2, 1};
+        TRY(make_map(&p.tm_x, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 4, x, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_128B, "K3 x"));
     }
     {
         uint64_t dims[3] = {(uint64_t)cz, NN, (uint64_t)B};
@@ -480,7 +483,7 @@ static trimul_status_t run_output_bf16(const trimul_layer_t *L, const void *z, c
         const uint64_t es = out_f32 ? 4 : 2;
         uint64_t dims[3] = {(uint64_t)cz, NN, (uint64_t)B};
         uint64_t strides[2] = {(uint64_t)cz * es, NN * cz * es};
-        uint32_t box[3] = {out_f32 ? 32u : 64u, 128, 1};
+        uint32_t box[3] = {out_f32 ? 32u : 64u, 32, 1};   // one warp's 32 pair rows
         TRY(make_map(&p.tm_out, out_f32 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, out, dims,
                      strides, box, CU_TENSOR_MAP_SWIZZLE_128B, "K3 out"));
     }
