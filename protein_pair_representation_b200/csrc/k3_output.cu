@@ -37,7 +37,8 @@ struct K3Cfg {
     static constexpr int COLS_PER_STORE = OUT_F32 ? 32 : 64;
     static constexpr int SNB = 2;
     static constexpr int VEC_BYTES = NCOL * 16;          // folding constants of this group's columns
-    static constexpr int FIXED = 1024 + WO_BYTES + WG_BYTES + 2 * STG_BYTES + SNB * 128 * 32 + VEC_BYTES + 1024;
+    static constexpr int XPART_BYTES = 4 * 128 * 8;      // x partial sums: [4 warps][128 pairs] float2
+    static constexpr int FIXED = 1024 + WO_BYTES + WG_BYTES + 2 * STG_BYTES + SNB * 128 * 32 + VEC_BYTES + XPART_BYTES + 1024;
     static constexpr int S = (232448 - FIXED) / CHUNK > 8 ? 8 : (232448 - FIXED) / CHUNK;
     static constexpr size_t SMEM = FIXED + (size_t)S * CHUNK;
     static constexpr int THREADS = 576;
@@ -74,7 +75,8 @@ __global__ void __launch_bounds__(576, 1) k3_output_kernel(const __grid_constant
     // folding constants of this group's columns, one array each: sum W_o', shift_o,
     // sum W_g', shift_g / 2
     float *vec_s = reinterpret_cast<float *>(stats + C::SNB * 128);   // [4][NCOL]
-    K3Smem &s = *reinterpret_cast<K3Smem *>(vec_s + 4 * C::NCOL);
+    float2 *xpart = reinterpret_cast<float2 *>(vec_s + 4 * C::NCOL);  // [4][128]
+    K3Smem &s = *reinterpret_cast<K3Smem *>(xpart + 4 * 128);
 
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
@@ -232,49 +234,94 @@ __global__ void __launch_bounds__(576, 1) k3_output_kernel(const __grid_constant
             float sh = 0.f;
             float2 nsh = make_float2(0.f, 0.f), s1 = make_float2(0.f, 0.f), s2 = make_float2(0.f, 0.f);
             bool ok = true;
+            // x role: thread (octet o, group gq) sums the 8 pairs [8o, 8o + 8) over the channels
+            // gq, gq + 8, ... of each x chunk from 16-byte rows; the partial sums of the 8 groups
+            // of an octet are combined after the chunks (shuffle, then shared memory)
+            const int xo = row & 15, xg = row >> 4;
+            const uint8_t *xblk_off = nullptr;
+            float2 a1[4], a2[4], xnsh[4];
+#pragma unroll
+            for (int k = 0; k < 4; ++k) a1[k] = a2[k] = xnsh[k] = make_float2(0.f, 0.f);
             for (int c = 0; c < C::CPT; ++c) {
-                if (!__all_sync(0xffffffffu, mbar_wait(&s.full[stage], phase, abort_flag, kErrTimeoutEpilogue))) { ok = false; break; }
-                if (xrole == (c < C::XC)) {
-                    const uint8_t *ch = chunks + stage * C::CHUNK;
-                    if (xrole) {
-                        // MN-major: K row kr holds 64 pairs; this pair's element sits in 16-byte
-                        // unit (r64 / 8) of that row, swizzled with the row index.
-                        const uint8_t *blk = ch + mblk * 8192;
-#pragma unroll 8
-                        for (int kr = 0; kr < 64; kr += 2) {
-                            const float v0 = __half2float(__ushort_as_half(*reinterpret_cast<const uint16_t *>(
-                                blk + sw128_offset(kr, r64 >> 3) + (r64 & 7) * 2)));
-                            const float v1 = __half2float(__ushort_as_half(*reinterpret_cast<const uint16_t *>(
-                                blk + sw128_offset(kr + 1, r64 >> 3) + (r64 & 7) * 2)));
-                            if (c == 0 && kr == 0) {
-                                sh = v0;
-                                nsh = make_float2(-v0, -v0);
-                            }
-                            const float2 d = f2_add(make_float2(v0, v1), nsh);
+                const bool arrived = mbar_wait(&s.full[stage], phase, abort_flag, kErrTimeoutEpilogue);
+                if (xrole ? !group_all(arrived, 1, 128) : !__all_sync(0xffffffffu, arrived)) { ok = false; break; }
+                const uint8_t *ch = chunks + stage * C::CHUNK;
+                if (xrole && c < C::XC) {
+                    // MN-major: K row kr holds 64 pairs per block; 16-byte unit (xo % 8) of a row
+                    // of block xo / 8 holds pairs [8o, 8o + 8), swizzled with the row index
+                    xblk_off = ch + (xo >> 3) * 8192;
+                    if (c == 0) {
+                        const uint4 w0 = *reinterpret_cast<const uint4 *>(xblk_off + sw128_offset(0, xo & 7));
+                        const uint32_t h0[4] = {w0.x, w0.y, w0.z, w0.w};
+#pragma unroll
+                        for (int k = 0; k < 4; ++k) {
+                            const float2 v = __half22float2(*reinterpret_cast<const __half2 *>(&h0[k]));
+                            xnsh[k] = make_float2(-v.x, -v.y);
+                        }
+                        // this thread's own pair (`row`) shift, for the final mean
+                        sh = __half2float(__ushort_as_half(*reinterpret_cast<const uint16_t *>(
+                            ch + mblk * 8192 + sw128_offset(0, r64 >> 3) + (r64 & 7) * 2)));
+                    }
+#pragma unroll
+                    for (int j = 0; j < 8; ++j) {
+                        const uint4 w = *reinterpret_cast<const uint4 *>(xblk_off + sw128_offset(xg + 8 * j, xo & 7));
+                        const uint32_t hw[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+                        for (int k = 0; k < 4; ++k) {
+                            const float2 d = f2_add(__half22float2(*reinterpret_cast<const __half2 *>(&hw[k])), xnsh[k]);
+                            a1[k] = f2_add(a1[k], d);
+                            a2[k] = f2_fma(d, d, a2[k]);
+                        }
+                    }
+                } else if (!xrole && c >= C::XC) {
+#pragma unroll
+                    for (int u = 0; u < 8; ++u) {
+                        const uint4 w = *reinterpret_cast<const uint4 *>(ch + sw128_offset(row, u));
+                        const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
+                        if (c == C::XC && u == 0) {
+                            sh = bf16_lo(w.x);
+                            nsh = make_float2(-sh, -sh);
+                        }
+#pragma unroll
+                        for (int e = 0; e < 4; ++e) {
+                            const float2 d = f2_add(make_float2(bf16_lo(ws[e]), bf16_hi(ws[e])), nsh);
                             s1 = f2_add(s1, d);
                             s2 = f2_fma(d, d, s2);
-                        }
-                    } else {
-#pragma unroll
-                        for (int u = 0; u < 8; ++u) {
-                            const uint4 w = *reinterpret_cast<const uint4 *>(ch + sw128_offset(row, u));
-                            const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
-                            if (c == C::XC && u == 0) {
-                                sh = bf16_lo(w.x);
-                                nsh = make_float2(-sh, -sh);
-                            }
-#pragma unroll
-                            for (int e = 0; e < 4; ++e) {
-                                const float2 d = f2_add(make_float2(bf16_lo(ws[e]), bf16_hi(ws[e])), nsh);
-                                s1 = f2_add(s1, d);
-                                s2 = f2_fma(d, d, s2);
-                            }
                         }
                     }
                 }
                 __syncwarp();
                 if (lane == 0) mbar_arrive(&s.empty[stage]);
                 if (++stage == C::S) { stage = 0; phase ^= 1; }
+            }
+            if (xrole && ok) {
+                // groups 2w and 2w + 1 of an octet sit in lanes o and o + 16 of warp w
+#pragma unroll
+                for (int k = 0; k < 4; ++k) {
+                    a1[k].x += __shfl_xor_sync(0xffffffffu, a1[k].x, 16);
+                    a1[k].y += __shfl_xor_sync(0xffffffffu, a1[k].y, 16);
+                    a2[k].x += __shfl_xor_sync(0xffffffffu, a2[k].x, 16);
+                    a2[k].y += __shfl_xor_sync(0xffffffffu, a2[k].y, 16);
+                }
+                const int xw = warp - C::STATS_WARP0;
+                if (lane < 16) {
+#pragma unroll
+                    for (int k = 0; k < 4; ++k) {
+                        xpart[xw * 128 + 8 * xo + 2 * k] = make_float2(a1[k].x, a2[k].x);
+                        xpart[xw * 128 + 8 * xo + 2 * k + 1] = make_float2(a1[k].y, a2[k].y);
+                    }
+                }
+                named_bar_sync(1, 128);
+                float2 t = xpart[row];
+#pragma unroll
+                for (int w4 = 1; w4 < 4; ++w4) {
+                    const float2 u = xpart[w4 * 128 + row];
+                    t.x += u.x;
+                    t.y += u.y;
+                }
+                s1 = make_float2(t.x, 0.f);
+                s2 = make_float2(t.y, 0.f);
+                named_bar_sync(1, 128);   // every partial is read before the next tile's are written
             }
             if (!ok) break;
             const float t1 = s1.x + s1.y, t2 = s2.x + s2.y;
@@ -283,7 +330,8 @@ __global__ void __launch_bounds__(576, 1) k3_output_kernel(const __grid_constant
             const float rs = rsqrtf(fmaxf(t2 * inv_n - dm * dm, 0.f) + (xrole ? p.eps_x : p.eps));
             // an inf or NaN anywhere in this pair's x makes the shifted square sum inf or NaN
             if (xrole && !(fabsf(t2) <= 3.0e38f)) atomicOr(&g_device_error, (unsigned int)kErrRange);
-            if (!__all_sync(0xffffffffu, mbar_wait(&s.sempty[sbuf], sphase ^ 1, abort_flag, kErrTimeoutEpilogue))) break;
+            const bool freed = mbar_wait(&s.sempty[sbuf], sphase ^ 1, abort_flag, kErrTimeoutEpilogue);
+            if (xrole ? !group_all(freed, 1, 128) : !__all_sync(0xffffffffu, freed)) break;
             K3Stats &st = stats[sbuf * 128 + row];
             if (xrole) {
                 st.nmean_x = -(sh + dm);
@@ -331,17 +379,21 @@ __global__ void __launch_bounds__(576, 1) k3_output_kernel(const __grid_constant
             const uint32_t t2 = t1 + 128;
 #pragma unroll 1
             for (int sc = 0; sc < 64 / C::COLS_PER_STORE; ++sc) {
-                if (lane == 0) tma_store_wait_read<0>();   // this warp's previous store has read its rows
-                __syncwarp();
 #pragma unroll 1
-                for (int h = 0; h < C::COLS_PER_STORE / 16; ++h) {
-                    const int col = sc * C::COLS_PER_STORE + h * 16;   // within this warpgroup's 64
-                    float o[16], g[16];
-                    tmem_ld16(t1 + col, o);
-                    tmem_ld16(t2 + col, g);
+                for (int h = 0; h < C::COLS_PER_STORE / 32; ++h) {
+                    const int col = sc * C::COLS_PER_STORE + h * 32;   // within this warpgroup's 64
+                    float o[32], g[32];
+                    tmem_ld16(t1 + col, *reinterpret_cast<float(*)[16]>(&o[0]));
+                    tmem_ld16(t1 + col + 16, *reinterpret_cast<float(*)[16]>(&o[16]));
+                    tmem_ld16(t2 + col, *reinterpret_cast<float(*)[16]>(&g[0]));
+                    tmem_ld16(t2 + col + 16, *reinterpret_cast<float(*)[16]>(&g[16]));
+                    if (h == 0) {
+                        if (lane == 0) tma_store_wait_read<0>();   // this warp's previous store has read its rows
+                        __syncwarp();
+                    }
                     tc_wait_ld();
 #pragma unroll
-                    for (int e = 0; e < 16; e += 4) {
+                    for (int e = 0; e < 32; e += 4) {
                         const float4 so = *reinterpret_cast<const float4 *>(v_sum_o + col + e);
                         const float4 ho = *reinterpret_cast<const float4 *>(v_shift_o + col + e);
                         const float4 sg = *reinterpret_cast<const float4 *>(v_sum_g + col + e);
@@ -365,18 +417,18 @@ __global__ void __launch_bounds__(576, 1) k3_output_kernel(const __grid_constant
                     }
                     if (OUT_F32) {
 #pragma unroll
-                        for (int u = 0; u < 4; ++u)
-                            *reinterpret_cast<float4 *>(stg + sw128_offset(row, h * 4 + u)) =
+                        for (int u = 0; u < 8; ++u)
+                            *reinterpret_cast<float4 *>(stg + sw128_offset(row, u)) =
                                 make_float4(o[4 * u], o[4 * u + 1], o[4 * u + 2], o[4 * u + 3]);
                     } else {
 #pragma unroll
-                        for (int u = 0; u < 2; ++u) {
+                        for (int u = 0; u < 4; ++u) {
                             uint4 w;
                             w.x = pack_bf16x2(o[8 * u + 0], o[8 * u + 1]);
                             w.y = pack_bf16x2(o[8 * u + 2], o[8 * u + 3]);
                             w.z = pack_bf16x2(o[8 * u + 4], o[8 * u + 5]);
                             w.w = pack_bf16x2(o[8 * u + 6], o[8 * u + 7]);
-                            *reinterpret_cast<uint4 *>(stg + sw128_offset(row, h * 2 + u)) = w;
+                            *reinterpret_cast<uint4 *>(stg + sw128_offset(row, h * 4 + u)) = w;
                         }
                     }
                 }
