@@ -29,6 +29,8 @@ if ROOT not in sys.path:
 
 METRIC = "ms/layer and effective TFLOP/s (fraction of bf16 roofline) for tri-mul at N=512, c_z=128"
 WORKLOAD = "bf16_n512_ragged"
+WORKLOADS = ("bf16_n512_ragged", "bf16_n256_tail10", "bf16_b4_n256_cz384", "bf16_n2048")
+CPU_BASELINE_WORKLOADS = ("bf16_n512_ragged", "bf16_n256_tail10", "bf16_b4_n256_cz384")
 L2_BYTES = 126 * 1024 * 1024
 KERNEL_NAMES = ("k1_project_kernel", "k2_contract_kernel", "k3_output_kernel")
 KERNEL_SOURCES = {"k1_project_kernel": "k1_project.cu", "k2_contract_kernel": "k2_contract.cu",
@@ -42,6 +44,9 @@ def parse_args():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=("ours", "reference"), default="ours")
     ap.add_argument("--out-dtype", choices=("f32", "bf16"), default="f32")
+    ap.add_argument("--workload", choices=WORKLOADS, default=WORKLOAD,
+                    help="the seeded configuration to time (default: the headline N=512 workload; the "
+                         "others are for the per-kernel breakdown at other shapes)")
     ap.add_argument("--no-e2e", action="store_true", help="skip the host-buffer end-to-end leg")
     ap.add_argument("--no-cpu-baseline", action="store_true", help="skip timing the CPU oracle")
     return ap.parse_args()
@@ -196,8 +201,12 @@ def run_reference(args):
     if rank != 0:
         return
     import trimul_inputs as ti
-    inp = ti.make_config(WORKLOAD)
-    dirs = ti.CONFIGS[WORKLOAD]["directions"]
+    if args.workload not in CPU_BASELINE_WORKLOADS:
+        print(json.dumps({"impl": "reference", "unavailable": f"a full fp64 oracle layer of {args.workload} "
+                                                              f"takes hours on the host cores"}), flush=True)
+        return
+    inp = ti.make_config(args.workload)
+    dirs = ti.CONFIGS[args.workload]["directions"]
     import oracle
     for s in range(args.warmup):
         oracle.trimul(inp.z, inp.mask, inp.weights, dirs[s % 2], inp.eps)
@@ -224,9 +233,12 @@ def run_reference(args):
 
 
 def workload_config(inp, compute):
+    lengths = [int(v) for v in inp.lengths]
+    mask = "all-ones mask" if min(lengths) == inp.N else f"ragged mask (L={lengths if inp.B > 1 else lengths[0]})"
     return {"workload": f"triangle multiplicative update, B={inp.B} N={inp.N} c_z={inp.c_z} c_h={inp.c_h}, "
-                        f"bf16 z and weights, ragged mask (L={int(inp.lengths[0])}), outgoing + incoming",
-            "B": inp.B, "N": inp.N, "c_z": inp.c_z, "c_h": inp.c_h, "valid_length": int(inp.lengths[0]),
+                        f"bf16 z and weights, {mask}, outgoing + incoming",
+            "B": inp.B, "N": inp.N, "c_z": inp.c_z, "c_h": inp.c_h,
+            "valid_length": lengths[0] if inp.B == 1 else lengths,
             "directions": ["outgoing", "incoming"], "compute": compute}
 
 
@@ -247,8 +259,8 @@ def run_ours(args):
         import torch.distributed as dist
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
 
-    inp = ti.make_config(WORKLOAD, seed=rank)          # every replica its own seeded problem
-    dirs = ti.CONFIGS[WORKLOAD]["directions"]
+    inp = ti.make_config(args.workload, seed=rank)     # every replica its own seeded problem
+    dirs = ti.CONFIGS[args.workload]["directions"]
     out_dt = torch.float32 if args.out_dtype == "f32" else torch.bfloat16
     z0 = torch.from_numpy(inp.z).to(dev).to(torch.bfloat16)
     m0 = torch.from_numpy(inp.mask).to(dev).to(torch.bfloat16)
@@ -335,7 +347,7 @@ def run_ours(args):
                "d2h_bytes_per_step": sum(o.numel() * o.element_size() for o in out_host)}
 
     cpu = None
-    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+    if rank == 0 and world == 1 and not args.no_cpu_baseline and args.workload in CPU_BASELINE_WORKLOADS:
         ms_cpu, cores = cpu_oracle_layer_ms(inp, dirs)
         cpu = {"value": ms_cpu, "unit": "ms/layer", "cores": cores, "kind": "oracle",
                "sample": f"one full layer per direction ({', '.join(dirs)}) of the same workload, fp64, "

@@ -123,9 +123,10 @@ __global__ void __launch_bounds__(448, 1) k1_project_kernel(const __grid_constan
             int stage = 0;
             uint32_t phase = 0;
             uint32_t filled = 0;
-            for (int pt = cta_in_group; pt < num_ptiles; pt += ctas_per_group) {
-                const int b = pt / p.tiles_per_batch;
-                const int p0 = (pt - b * p.tiles_per_batch) * 128;
+            TileWalk tw(cta_in_group, p.tiles_per_batch);
+            for (int pt = cta_in_group; pt < num_ptiles; pt += ctas_per_group, tw.advance(ctas_per_group, p.tiles_per_batch)) {
+                const int b = tw.b;
+                const int p0 = tw.t * 128;
                 for (int kc = 0; kc < C::KC; ++kc) {
                     if (!mbar_wait(&s.empty[stage], phase ^ 1, abort_flag, kErrTimeoutProducer)) goto producer_abort;
                     mbar_arrive_expect_tx(&s.full[stage], C::CHUNK);
@@ -183,9 +184,10 @@ __global__ void __launch_bounds__(448, 1) k1_project_kernel(const __grid_constan
         uint32_t phase = 0;
         int sbuf = 0;
         uint32_t sphase = 0;
-        for (int pt = cta_in_group; pt < num_ptiles; pt += ctas_per_group) {
-            const int b = pt / p.tiles_per_batch;
-            const int p0 = (pt - b * p.tiles_per_batch) * 128;
+        TileWalk tw(cta_in_group, p.tiles_per_batch);
+        for (int pt = cta_in_group; pt < num_ptiles; pt += ctas_per_group, tw.advance(ctas_per_group, p.tiles_per_batch)) {
+            const int b = tw.b;
+            const int p0 = tw.t * 128;
             // shifted sums in packed pairs: s1 = sum(v - shift), s2 = sum((v - shift)^2), with
             // the row's first entry as the shift
             float shift = 0.f;
@@ -241,9 +243,10 @@ __global__ void __launch_bounds__(448, 1) k1_project_kernel(const __grid_constan
         uint32_t aphase = 0;
         int sbuf = 0;
         uint32_t sphase = 0;
-        for (int pt = cta_in_group; pt < num_ptiles; pt += ctas_per_group) {
-            const int b = pt / p.tiles_per_batch;
-            const int p0 = (pt - b * p.tiles_per_batch) * 128;
+        TileWalk tw(cta_in_group, p.tiles_per_batch);
+        for (int pt = cta_in_group; pt < num_ptiles; pt += ctas_per_group, tw.advance(ctas_per_group, p.tiles_per_batch)) {
+            const int b = tw.b;
+            const int p0 = tw.t * 128;
             if (!group_all(mbar_wait(&s.sfull[sbuf], sphase, abort_flag, kErrTimeoutEpilogue), 1 + wg, 128)) break;
             const float4 st = stats[sbuf * 128 + row];
             __syncwarp();
@@ -395,9 +398,10 @@ __global__ void __launch_bounds__(K1CmCfg::THREADS, 1) k1_project_cm_kernel(cons
             int stage = 0;
             uint32_t phase = 0;
             uint32_t filled = 0;
-            for (int pt = cta_in_group; pt < num_ptiles; pt += ctas_per_group) {
-                const int b = pt / p.tiles_per_batch;
-                const int p0 = (pt - b * p.tiles_per_batch) * 128;
+            TileWalk tw(cta_in_group, p.tiles_per_batch);
+            for (int pt = cta_in_group; pt < num_ptiles; pt += ctas_per_group, tw.advance(ctas_per_group, p.tiles_per_batch)) {
+                const int b = tw.b;
+                const int p0 = tw.t * 128;
                 for (int kc = 0; kc < C::KC; ++kc) {
                     if (!mbar_wait(&s.empty[stage], phase ^ 1, abort_flag, kErrTimeoutProducer)) goto producer_abort;
                     mbar_arrive_expect_tx(&s.full[stage], C::CHUNK);
@@ -458,9 +462,10 @@ __global__ void __launch_bounds__(K1CmCfg::THREADS, 1) k1_project_cm_kernel(cons
         uint32_t phase = 0;
         int sbuf = 0;
         uint32_t sphase = 0;
-        for (int pt = cta_in_group; pt < num_ptiles; pt += ctas_per_group) {
-            const int b = pt / p.tiles_per_batch;
-            const int p0 = (pt - b * p.tiles_per_batch) * 128;
+        TileWalk tw(cta_in_group, p.tiles_per_batch);
+        for (int pt = cta_in_group; pt < num_ptiles; pt += ctas_per_group, tw.advance(ctas_per_group, p.tiles_per_batch)) {
+            const int b = tw.b;
+            const int p0 = tw.t * 128;
             const long long pi = (long long)p0 + row;
             uint16_t mbits = 0x3F80u;   // bf16 1.0; the load is issued first so its latency overlaps
             if (p.mask) mbits = (pi < p.NN) ? p.mask[(long long)b * p.NN + pi] : (uint16_t)0;
@@ -523,9 +528,10 @@ __global__ void __launch_bounds__(K1CmCfg::THREADS, 1) k1_project_cm_kernel(cons
         uint32_t aphase = 0;
         int sbuf = 0;
         uint32_t sphase = 0;
-        for (int pt = cta_in_group; pt < num_ptiles; pt += ctas_per_group) {
-            const int b = pt / p.tiles_per_batch;
-            const int p0 = (pt - b * p.tiles_per_batch) * 128;
+        TileWalk tw(cta_in_group, p.tiles_per_batch);
+        for (int pt = cta_in_group; pt < num_ptiles; pt += ctas_per_group, tw.advance(ctas_per_group, p.tiles_per_batch)) {
+            const int b = tw.b;
+            const int p0 = tw.t * 128;
             if (!__all_sync(0xffffffffu, mbar_wait(&s.sfull[sbuf], sphase, abort_flag, kErrTimeoutEpilogue) &&
                                              mbar_wait(&s.tfull[abuf], aphase, abort_flag, kErrTimeoutEpilogue)))
                 break;

@@ -137,9 +137,10 @@ __global__ void __launch_bounds__(576, 1) k3_output_kernel(const __grid_constant
             int stage = 0;
             uint32_t phase = 0;
             uint32_t filled = 0;
-            for (int pt = cta_in_group; pt < num_ptiles; pt += ctas_per_group) {
-                const int b = pt / p.tiles_per_batch;
-                const int p0 = (pt - b * p.tiles_per_batch) * 128;
+            TileWalk tw(cta_in_group, p.tiles_per_batch);
+            for (int pt = cta_in_group; pt < num_ptiles; pt += ctas_per_group, tw.advance(ctas_per_group, p.tiles_per_batch)) {
+                const int b = tw.b;
+                const int p0 = tw.t * 128;
                 for (int c = 0; c < C::CPT; ++c) {
                     if (!mbar_wait(&s.empty[stage], phase ^ 1, abort_flag, kErrTimeoutProducer)) goto producer_abort;
                     uint8_t *dst = chunks + stage * C::CHUNK;
@@ -224,9 +225,10 @@ __global__ void __launch_bounds__(576, 1) k3_output_kernel(const __grid_constant
         uint32_t phase = 0;
         int sbuf = 0;
         uint32_t sphase = 0;
-        for (int pt = cta_in_group; pt < num_ptiles; pt += ctas_per_group) {
-            const int b = pt / p.tiles_per_batch;
-            const int p0 = (pt - b * p.tiles_per_batch) * 128;
+        TileWalk tw(cta_in_group, p.tiles_per_batch);
+        for (int pt = cta_in_group; pt < num_ptiles; pt += ctas_per_group, tw.advance(ctas_per_group, p.tiles_per_batch)) {
+            const int b = tw.b;
+            const int p0 = tw.t * 128;
             const long long pi = (long long)p0 + row;
             uint16_t mbits = 0x3F80u;      // bf16 1.0; issued first so its latency overlaps the sums
             if (!xrole && p.mask) mbits = (pi < p.NN) ? p.mask[(long long)b * p.NN + pi] : (uint16_t)0;
@@ -361,9 +363,10 @@ __global__ void __launch_bounds__(576, 1) k3_output_kernel(const __grid_constant
         uint32_t aphase = 0;
         int sbuf = 0;
         uint32_t sphase = 0;
-        for (int pt = cta_in_group; pt < num_ptiles; pt += ctas_per_group) {
-            const int b = pt / p.tiles_per_batch;
-            const int p0 = (pt - b * p.tiles_per_batch) * 128;
+        TileWalk tw(cta_in_group, p.tiles_per_batch);
+        for (int pt = cta_in_group; pt < num_ptiles; pt += ctas_per_group, tw.advance(ctas_per_group, p.tiles_per_batch)) {
+            const int b = tw.b;
+            const int p0 = tw.t * 128;
             if (!__all_sync(0xffffffffu, mbar_wait(&s.sfull[sbuf], sphase, abort_flag, kErrTimeoutEpilogue))) break;
             const K3Stats st = stats[sbuf * 128 + row];
             const float2 nmx = make_float2(st.nmean_x, st.nmean_x), rx = make_float2(st.rstd_x, st.rstd_x);

@@ -123,6 +123,23 @@ __device__ __forceinline__ void pdl_launch_dependents() {
 // are visible (returns at once for a launch without the programmatic-serialization attribute).
 __device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
 
+// ------------------------------------------------------------------ persistent tile walk
+
+// Visits the tiles first, first + step, ... of a [batch][tiles_per_batch] grid as (batch b,
+// tile t within the batch) without a division per tile.
+struct TileWalk {
+    int b, t;
+    __device__ __forceinline__ TileWalk(int first, int tiles_per_batch)
+        : b(first / tiles_per_batch), t(first - (first / tiles_per_batch) * tiles_per_batch) {}
+    __device__ __forceinline__ void advance(int step, int tiles_per_batch) {
+        t += step;
+        while (t >= tiles_per_batch) {
+            t -= tiles_per_batch;
+            ++b;
+        }
+    }
+};
+
 // ------------------------------------------------------------------ named barriers
 
 __device__ __forceinline__ void named_bar_sync(uint32_t id, uint32_t nthreads) {
