@@ -306,8 +306,9 @@ __global__ void __launch_bounds__(448, 1) k1_project_kernel(const __grid_constan
 // 16-byte rows of the channel-major output tile.
 // The gate is evaluated in f16x2 (tanh.approx.f16x2 on g/2, the gate rows being folded
 // with an extra factor 1/2), as are the products with the projection and the mask.
-// Warps: 0-15 epilogue (warpgroup w: pairs [32w, 32w+32) of the tile), 16-19 LayerNorm
-// statistics, 20 TMA producer, 21 TMEM allocator + MMA issuer.
+// Warps: 0-15 epilogue (two teams of two warpgroups that take alternate tiles; warpgroup
+// s of a team: pairs [64s, 64s+64) of its tiles), 16-19 LayerNorm statistics, 20 TMA
+// producer, 21 TMEM allocator + MMA issuer.
 struct K1CmCfg {
     static constexpr int CZ = 128, C_H = kHidden, KC = CZ / 64;
     static constexpr int G = 2;                               // one group per operand
@@ -366,11 +367,11 @@ __global__ void __launch_bounds__(K1CmCfg::THREADS, 1) k1_project_cm_kernel(cons
         }
         for (int i = 0; i < 2; ++i) {
             mbar_init(&s.tfull[i], 1);
-            mbar_init(&s.tempty[i], C::EPI_WARPS);
+            mbar_init(&s.tempty[i], C::EPI_WARPS / 2);     // the team that drains buffer i
         }
         for (int i = 0; i < C::SNB; ++i) {
             mbar_init(&s.sfull[i], C::STATS_WARPS);
-            mbar_init(&s.sempty[i], C::EPI_WARPS);
+            mbar_init(&s.sempty[i], C::EPI_WARPS / 2);
         }
         mbar_init(&s.drain, 1);
         s.abort_flag = 0;
@@ -509,80 +510,93 @@ __global__ void __launch_bounds__(K1CmCfg::THREADS, 1) k1_project_cm_kernel(cons
             if (++sbuf == C::SNB) { sbuf = 0; sphase ^= 1; }
         }
     } else {
-        // epilogue: thread = hidden channel c of this CTA's operand; warpgroup wg owns the
-        // 32 pairs [32 wg, 32 wg + 32) of the tile. Every warp runs on its own: it waits on the
-        // barriers itself, stages its [32 channels][32 pairs] block in its own 2 KB of shared
-        // memory (64-byte rows, 64-byte swizzle) and issues that block's TMA store.
+        // epilogue: two teams of eight warps take alternate tiles of this CTA's sequence (team k
+        // drains TMEM buffer k and statistics buffer k), so that one team's waits and TMEM
+        // loads overlap the other team's arithmetic. Thread = hidden channel c; warpgroup s of
+        // a team owns the 64 pairs [64 s, 64 s + 64) of its tiles. Every warp runs on its own:
+        // it waits on the barriers itself and stages each [32 channels][32 pairs] block of its
+        // output in its own 2 KB of shared memory (64-byte rows, 64-byte swizzle) for a TMA
+        // store.
         const int wg = warp >> 2;
+        const int team = wg >> 1;
         const int q = warp & 3;
         const int c = q * 32 + lane;
-        const int col = 32 * wg;
+        const int col0 = 64 * (wg & 1);
         uint8_t *stg = staging + warp * C::WARP_STG;
         const CUtensorMap *tm_out = operand == 0 ? &p.tm_a : &p.tm_b;
         // {sum W'_gate, shift_gate, sum W'_proj, shift_proj}; the gate entries are for g / 2
         const float4 cv = p.vec[operand * C::C_H + c];
         const float2 cg_sum = make_float2(cv.x, cv.x), cg_shift = make_float2(cv.y, cv.y);
         const float2 cp_sum = make_float2(cv.z, cv.z), cp_shift = make_float2(cv.w, cv.w);
-        const uint32_t lane_off = (uint32_t)(q * 32) << 16;
-        int abuf = 0;
-        uint32_t aphase = 0;
-        int sbuf = 0;
-        uint32_t sphase = 0;
-        TileWalk tw(cta_in_group, p.tiles_per_batch);
-        for (int pt = cta_in_group; pt < num_ptiles; pt += ctas_per_group, tw.advance(ctas_per_group, p.tiles_per_batch)) {
+        static_assert(C::SNB == 2, "one statistics buffer per epilogue team");
+        const int abuf = team, sbuf = team;
+        const uint32_t tbase = tmem_base + abuf * 256 + ((uint32_t)(q * 32) << 16);
+        const float *snmean0 = st_nmean + sbuf * 128 + col0, *srstd0 = st_rstd + sbuf * 128 + col0;
+        const __half *shmask0 = st_hmask + sbuf * 128 + col0;
+        uint32_t phase = 0;
+        const int first = cta_in_group + team * ctas_per_group;
+        TileWalk tw(first, p.tiles_per_batch);
+        for (int pt = first; pt < num_ptiles; pt += 2 * ctas_per_group, tw.advance(2 * ctas_per_group, p.tiles_per_batch)) {
             const int b = tw.b;
             const int p0 = tw.t * 128;
-            if (!__all_sync(0xffffffffu, mbar_wait(&s.sfull[sbuf], sphase, abort_flag, kErrTimeoutEpilogue) &&
-                                             mbar_wait(&s.tfull[abuf], aphase, abort_flag, kErrTimeoutEpilogue)))
+            if (!__all_sync(0xffffffffu, mbar_wait(&s.sfull[sbuf], phase, abort_flag, kErrTimeoutEpilogue) &&
+                                             mbar_wait(&s.tfull[abuf], phase, abort_flag, kErrTimeoutEpilogue)))
                 break;
             tc_fence_after();
-            if (lane == 0) tma_store_wait_read<0>();   // this warp's previous store has read its block
-            __syncwarp();
-            const float *snmean = st_nmean + sbuf * 128 + col, *srstd = st_rstd + sbuf * 128 + col;
-            const __half *shmask = st_hmask + sbuf * 128 + col;
 #pragma unroll 1
-            for (int hh = 0; hh < 2; ++hh) {          // two halves of 16 pairs
-                float g[16], pr[16];
-                tmem_ld16(tmem_base + abuf * 256 + lane_off + col + 16 * hh, g);
-                tmem_ld16(tmem_base + abuf * 256 + 128 + lane_off + col + 16 * hh, pr);
-                tc_wait_ld();
-                uint32_t outw[8];
+            for (int blk = 0; blk < 2; ++blk) {         // two store blocks of 32 pairs
+                const int col = col0 + 32 * blk;
+                if (lane == 0) tma_store_wait_read<0>();   // this warp's previous store has read its block
+                __syncwarp();
+#pragma unroll 1
+                for (int hh = 0; hh < 2; ++hh) {      // two halves of 16 pairs
+                    float g[16], pr[16];
+                    tmem_ld16(tbase + col + 16 * hh, g);
+                    tmem_ld16(tbase + 128 + col + 16 * hh, pr);
+                    tc_wait_ld();
+                    if (blk == 1 && hh == 1) {
+                        // the last TMEM load of the tile has landed: hand the buffer back to the
+                        // MMA now, not after this warp's arithmetic and store
+                        tc_fence_before();
+                        __syncwarp();
+                        if (lane == 0) mbar_arrive(&s.tempty[abuf]);
+                    }
+                    const int o = 32 * blk + 16 * hh;
+                    uint32_t outw[8];
 #pragma unroll
-                for (int j = 0; j < 16; j += 4) {
-                    const float4 nm = *reinterpret_cast<const float4 *>(snmean + 16 * hh + j);
-                    const float4 rs = *reinterpret_cast<const float4 *>(srstd + 16 * hh + j);
-                    const uint2 mk = *reinterpret_cast<const uint2 *>(shmask + 16 * hh + j);
+                    for (int j = 0; j < 16; j += 4) {
+                        const float4 nm = *reinterpret_cast<const float4 *>(snmean0 + o + j);
+                        const float4 rs = *reinterpret_cast<const float4 *>(srstd0 + o + j);
+                        const uint2 mk = *reinterpret_cast<const uint2 *>(shmask0 + o + j);
 #pragma unroll
-                    for (int h = 0; h < 2; ++h) {
-                        // two consecutive pairs of this channel in one packed lane pair
-                        const float2 nm2 = h == 0 ? make_float2(nm.x, nm.y) : make_float2(nm.z, nm.w);
-                        const float2 rs2 = h == 0 ? make_float2(rs.x, rs.y) : make_float2(rs.z, rs.w);
-                        const float2 gv = f2_fma(rs2, f2_fma(nm2, cg_sum, make_float2(g[j + 2 * h], g[j + 2 * h + 1])), cg_shift);
-                        const float2 pv = f2_fma(rs2, f2_fma(nm2, cp_sum, make_float2(pr[j + 2 * h], pr[j + 2 * h + 1])), cp_shift);
-                        // mask * sigmoid(2 x) = (mask / 2) tanh(x) + mask / 2, x being the halved gate
-                        const __half2 hm = u32_as_h2(h == 0 ? mk.x : mk.y);
-                        const __half2 gm = __hfma2(tanh_h2(__floats2half2_rn(gv.x, gv.y)), hm, hm);
-                        outw[j / 2 + h] = h2_as_u32(__hmul2(gm, __floats2half2_rn(pv.x, pv.y)));
+                        for (int h = 0; h < 2; ++h) {
+                            // two consecutive pairs of this channel in one packed lane pair
+                            const float2 nm2 = h == 0 ? make_float2(nm.x, nm.y) : make_float2(nm.z, nm.w);
+                            const float2 rs2 = h == 0 ? make_float2(rs.x, rs.y) : make_float2(rs.z, rs.w);
+                            const float2 gv = f2_fma(rs2, f2_fma(nm2, cg_sum, make_float2(g[j + 2 * h], g[j + 2 * h + 1])), cg_shift);
+                            const float2 pv = f2_fma(rs2, f2_fma(nm2, cp_sum, make_float2(pr[j + 2 * h], pr[j + 2 * h + 1])), cp_shift);
+                            // mask * sigmoid(2 x) = (mask / 2) tanh(x) + mask / 2, x being the halved gate
+                            const __half2 hm = u32_as_h2(h == 0 ? mk.x : mk.y);
+                            const __half2 gm = __hfma2(tanh_h2(__floats2half2_rn(gv.x, gv.y)), hm, hm);
+                            outw[j / 2 + h] = h2_as_u32(__hmul2(gm, __floats2half2_rn(pv.x, pv.y)));
+                        }
+                    }
+#pragma unroll
+                    for (int u = 0; u < 2; ++u)
+                        *reinterpret_cast<uint4 *>(stg + sw64_offset(lane, 2 * hh + u)) =
+                            make_uint4(outw[4 * u], outw[4 * u + 1], outw[4 * u + 2], outw[4 * u + 3]);
+                }
+                fence_proxy_async_smem();
+                __syncwarp();
+                if (lane == 0) {
+                    if (blk == 1) mbar_arrive(&s.sempty[sbuf]);   // statistics read in full
+                    if (p0 + col < p.NN) {              // blocks wholly past the last pair are not stored
+                        tma_store_3d(tm_out, stg, p0 + col, q * 32, b);
+                        tma_store_commit();
                     }
                 }
-#pragma unroll
-                for (int u = 0; u < 2; ++u)
-                    *reinterpret_cast<uint4 *>(stg + sw64_offset(lane, 2 * hh + u)) =
-                        make_uint4(outw[4 * u], outw[4 * u + 1], outw[4 * u + 2], outw[4 * u + 3]);
             }
-            tc_fence_before();
-            fence_proxy_async_smem();
-            __syncwarp();
-            if (lane == 0) {
-                mbar_arrive(&s.tempty[abuf]);
-                mbar_arrive(&s.sempty[sbuf]);
-                if (p0 + col < p.NN) {                  // blocks wholly past the last pair are not stored
-                    tma_store_3d(tm_out, stg, p0 + col, q * 32, b);
-                    tma_store_commit();
-                }
-            }
-            if (++abuf == 2) { abuf = 0; aphase ^= 1; }
-            if (++sbuf == C::SNB) { sbuf = 0; sphase ^= 1; }
+            phase ^= 1;
         }
         if (lane == 0) tma_store_wait_all<0>();
     }

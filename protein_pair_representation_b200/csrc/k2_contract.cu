@@ -195,6 +195,13 @@ __global__ void __launch_bounds__(k2::THREADS, 1) k2_contract_kernel(const __gri
                     float v[32];
                     tmem_ld32(tmem_base + abuf * BN + ((uint32_t)(q * 32) << 16) + col, v);
                     tc_wait_ld();
+                    if (sub == 1 && half == 1) {
+                        // the last TMEM load of the tile has landed: hand the buffer back to the
+                        // MMA now, not after the conversion and store
+                        tc_fence_before();
+                        __syncwarp();
+                        if (lane == 0) mbar_arrive(&s.tempty[abuf]);
+                    }
 #pragma unroll
                     for (int e = 0; e < 32; ++e) v[e] *= p.x_scale;
 #pragma unroll
@@ -221,9 +228,6 @@ __global__ void __launch_bounds__(k2::THREADS, 1) k2_contract_kernel(const __gri
                     tma_store_commit();
                 }
             }
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&s.tempty[abuf]);
             if (++abuf == 2) { abuf = 0; aphase ^= 1; }
         }
         if (leader) tma_store_wait_all<0>();

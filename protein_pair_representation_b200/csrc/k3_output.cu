@@ -395,6 +395,13 @@ __global__ void __launch_bounds__(576, 1) k3_output_kernel(const __grid_constant
                         __syncwarp();
                     }
                     tc_wait_ld();
+                    if (sc == 64 / C::COLS_PER_STORE - 1 && h == C::COLS_PER_STORE / 32 - 1) {
+                        // the last TMEM load of the tile has landed: hand the buffer back to the
+                        // MMA now, not after this warp's arithmetic and store
+                        tc_fence_before();
+                        __syncwarp();
+                        if (lane == 0) mbar_arrive(&s.tempty[abuf]);
+                    }
 #pragma unroll
                     for (int e = 0; e < 32; e += 4) {
                         const float4 so = *reinterpret_cast<const float4 *>(v_sum_o + col + e);
@@ -442,9 +449,6 @@ __global__ void __launch_bounds__(576, 1) k3_output_kernel(const __grid_constant
                     tma_store_commit();
                 }
             }
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&s.tempty[abuf]);
             if (++abuf == 2) { abuf = 0; aphase ^= 1; }
         }
         if (lane == 0) tma_store_wait_all<0>();
