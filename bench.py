@@ -49,6 +49,8 @@ def parse_args():
                          "others are for the per-kernel breakdown at other shapes)")
     ap.add_argument("--no-e2e", action="store_true", help="skip the host-buffer end-to-end leg")
     ap.add_argument("--no-cpu-baseline", action="store_true", help="skip timing the CPU oracle")
+    ap.add_argument("--no-pair-update", action="store_true",
+                    help="skip the pair-update leg (outgoing + incoming with residuals, eager and as a CUDA graph)")
     return ap.parse_args()
 
 
@@ -232,6 +234,45 @@ def run_reference(args):
     print(json.dumps(line), flush=True)
 
 
+def pair_update_leg(tm, layer, zs, ms_, n_sets, args, dev):
+    """ms per pair update (outgoing then incoming update, each a masked residual; z_mid and
+    out in bf16) on this rank's workload, launched eagerly and replayed as one CUDA graph per
+    input copy. Inputs cycle through the same L2-defeating copies as the main leg."""
+    import torch
+    try:
+        mids = [torch.empty_like(zs[0]) for _ in range(n_sets)]
+        outs = [torch.empty_like(zs[0]) for _ in range(n_sets)]
+        graphs = [tm.PairUpdateGraph(zs[i], ms_[i], layer, layer) for i in range(n_sets)]
+
+        def eager(s):
+            i = s % n_sets
+            tm.pair_update(zs[i], ms_[i], layer, layer, out=outs[i], z_mid=mids[i])
+
+        def graph(s):
+            graphs[s % n_sets].launch()
+
+        res = {}
+        for name, fn in (("eager_ms", eager), ("graph_ms", graph)):
+            for s in range(max(3, args.warmup)):
+                fn(s)
+            torch.cuda.synchronize()
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record()
+            for s in range(args.steps):
+                fn(s)
+            e1.record()
+            torch.cuda.synchronize()
+            res[name] = e0.elapsed_time(e1) / args.steps
+        tm.check_device_status()
+        for g in graphs:
+            g.close()
+        res.update({"unit": "ms per pair update (two triangle updates with residuals; one layer handle for both)",
+                    "gpu_launches_per_update": 2 * tm.kernels_per_forward()})
+        return res
+    except Exception as exc:       # the headline line must not depend on this leg
+        return {"error": f"{type(exc).__name__}: {exc}"}
+
+
 def workload_config(inp, compute):
     lengths = [int(v) for v in inp.lengths]
     mask = "all-ones mask" if min(lengths) == inp.N else f"ragged mask (L={lengths if inp.B > 1 else lengths[0]})"
@@ -346,6 +387,8 @@ def run_ours(args):
                "h2d_bytes_per_step": z_host.numel() * 2 + m_host.numel() * 2,
                "d2h_bytes_per_step": sum(o.numel() * o.element_size() for o in out_host)}
 
+    pair = None if args.no_pair_update else pair_update_leg(tm, layer, zs, ms_, n_sets, args, dev)
+
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline and args.workload in CPU_BASELINE_WORKLOADS:
         ms_cpu, cores = cpu_oracle_layer_ms(inp, dirs)
@@ -395,7 +438,7 @@ def run_ours(args):
         "vs_baseline": None, "dtype": "bf16", "data": "synthetic", "config": cfg,
         "effective_tflops": sum(flops.values()) / (layer_ms_single * 1e-3) / 1e12 * world,
         "layer_roofline_frac": t_ideal / (layer_ms_single * 1e-3),
-        "roofline": roof, "kernels": kernels, "cpu_baseline": cpu, "e2e": e2e,
+        "roofline": roof, "kernels": kernels, "cpu_baseline": cpu, "e2e": e2e, "pair_update": pair,
         "gpu_launches": args.steps * len(dirs) * tm.kernels_per_forward(), "clocks": clock_info,
     }
     print(json.dumps(line), flush=True)

@@ -193,6 +193,46 @@ trimul_status_t tri_mul_forward_noalloc(const trimul_pair_t *z, const void *mask
                                         const trimul_layer_t *layer, trimul_direction_t direction,
                                         trimul_pair_t *out, void *stream);
 
+/* The masked-residual form of tri_mul_forward: out = z + update, where update is what
+ * tri_mul_forward would write ("RFProteina architecture", section "Two networks around one
+ * state", subsection "Inside the velocity network": each triangle update is applied as a
+ * masked residual; a masked pair keeps its z, its update being 0). The sum is formed in
+ * fp32 from z's stored value and the fp32 update and rounded once to out's type. Same
+ * arguments and requirements as tri_mul_forward. */
+trimul_status_t tri_mul_forward_residual(const trimul_pair_t *z, const void *mask,
+                                         const trimul_layer_t *layer, trimul_direction_t direction,
+                                         trimul_pair_t *out, void *stream);
+
+/* The two triangle updates of one pair update, in order on one stream (same page and
+ * subsection: outgoing, then incoming triangle multiplication, each a masked residual):
+ *   z_mid = z + U_outgoing(z)       with layer_out's weights, stored in z's dtype
+ *   out   = z_mid + U_incoming(z_mid) with layer_in's weights
+ * Each call uses its layer's bound workspace; the same handle may be passed for both (its
+ * workspace is then reused in order). z_mid has z's shape and dtype; out has z's shape and
+ * z's dtype, or F32 on the BF16 path. z, z_mid and out must not overlap one another or
+ * either workspace. Other requirements as tri_mul_forward. */
+trimul_status_t tri_mul_pair_update(const trimul_pair_t *z, const void *mask,
+                                    const trimul_layer_t *layer_out, const trimul_layer_t *layer_in,
+                                    trimul_pair_t *z_mid, trimul_pair_t *out, void *stream);
+
+/* A CUDA graph of one tri_mul_pair_update on fixed buffers ("NVIDIA's BioNeMo Inference
+ * Runtime", section "Three Layers of Acceleration", layer 2: a recorded sequence of GPU
+ * work replayed with little host-side cost per launch). Creation captures the six kernel
+ * launches (with their programmatic-launch edges) on an internal stream and instantiates
+ * the graph; nothing runs. Each tri_mul_graph_launch replays it on `stream`, reading the
+ * current contents of z and mask and writing z_mid and out. The buffers, both layers and
+ * their bound workspaces must stay alive and unchanged in place (contents may change) for
+ * the graph's lifetime; the layers' timing events are not recorded by the graph. */
+typedef struct trimul_graph trimul_graph_t;
+trimul_status_t tri_mul_pair_update_graph_create(const trimul_pair_t *z, const void *mask,
+                                                 const trimul_layer_t *layer_out,
+                                                 const trimul_layer_t *layer_in,
+                                                 trimul_pair_t *z_mid, trimul_pair_t *out,
+                                                 trimul_graph_t **graph_out);
+trimul_status_t tri_mul_graph_launch(const trimul_graph_t *graph, void *stream);
+/* Free the graph. NULL is ignored. */
+void tri_mul_graph_destroy(trimul_graph_t *graph);
+
 /* Optional per-kernel timing: when `events` is non-NULL, every later
  * tri_mul_forward on this handle records events[0] before K1, events[1] after
  * K1, events[2] after K2 and events[3] after K3 on its stream. The four values
@@ -227,7 +267,7 @@ const char *tri_mul_last_error(void);
 /* ABI version of this header (major * 100 + minor). */
 int tri_mul_abi_version(void);
 
-#define TRIMUL_ABI_VERSION 100
+#define TRIMUL_ABI_VERSION 101
 
 #ifdef __cplusplus
 }

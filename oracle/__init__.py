@@ -197,3 +197,16 @@ def trimul_sampled(z, mask, weights, direction, I, J, eps=1e-5, lib=None):
                                      len(J), _ptr(out)), "trimul_sampled")
     del keep
     return out
+
+
+def pair_update(z, mask, weights_out, weights_in, eps=1e-5, lib=None):
+    """One pair update of the triangle stage, in fp64: the outgoing update applied as a
+    masked residual, then the incoming one ("RFProteina architecture", section "Two networks
+    around one state", subsection "Inside the velocity network"):
+        z_mid = z + trimul(z, outgoing; weights_out)
+        out   = z_mid + trimul(z_mid, incoming; weights_in)
+    Returns (z_mid, out). A masked pair keeps its z: its updates are exactly 0."""
+    z = _f64(z)
+    z_mid = z + trimul(z, mask, weights_out, "outgoing", eps, lib=lib)
+    out = z_mid + trimul(z_mid, mask, weights_in, "incoming", eps, lib=lib)
+    return z_mid, out

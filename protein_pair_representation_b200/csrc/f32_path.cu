@@ -131,7 +131,7 @@ __global__ void __launch_bounds__(256) f32_contract_kernel(const float *a, const
 
 __global__ void __launch_bounds__(f32::THREADS) f32_output_kernel(const float *z, const float *mask, const float *x,
                                                                   F32Weights w, int c_z, int c_h, long long NN,
-                                                                  float eps, float eps_x, float *out) {
+                                                                  float eps, float eps_x, int residual, float *out) {
     using namespace f32;
     extern __shared__ float sm[];
     const int ldz = c_z + 1, ldx = c_h + 1;
@@ -170,7 +170,9 @@ __global__ void __launch_bounds__(f32::THREADS) f32_output_kernel(const float *z
         for (int q = 0; q < PPW; ++q) {
             const long long pi = p0 + warp * PPW + q;
             const float m = mask ? mask[(long long)bb * NN + pi] : 1.f;
-            out[((long long)bb * NN + pi) * c_z + n] = m * sigmoid_acc(g[q] + bg) * (o[q] + bo);
+            const long long oi = ((long long)bb * NN + pi) * c_z + n;
+            const float u = m * sigmoid_acc(g[q] + bg) * (o[q] + bo);
+            out[oi] = residual ? __fadd_rn(z[oi], u) : u;   // no FMA contraction: z + (rounded update)
         }
     }
 }
@@ -196,7 +198,8 @@ cudaError_t f32_contract_launch(const float *a, const float *b, float *x, int BC
 }
 
 cudaError_t f32_output_launch(const float *z, const float *mask, const float *x, const F32Weights &w, int c_z,
-                              int c_h, int B, int N, float eps, float eps_x, float *out, cudaStream_t stream) {
+                              int c_h, int B, int N, float eps, float eps_x, bool residual, float *out,
+                              cudaStream_t stream) {
     const long long NN = (long long)N * N;
     const size_t smem = (size_t)f32::TP * ((c_z + 1) + (c_h + 1)) * sizeof(float);
     if (smem > 48 * 1024) {
@@ -204,7 +207,8 @@ cudaError_t f32_output_launch(const float *z, const float *mask, const float *x,
         if (e != cudaSuccess) return e;
     }
     const long long blocks = (long long)B * (NN / f32::TP);
-    f32_output_kernel<<<(unsigned)blocks, f32::THREADS, smem, stream>>>(z, mask, x, w, c_z, c_h, NN, eps, eps_x, out);
+    f32_output_kernel<<<(unsigned)blocks, f32::THREADS, smem, stream>>>(z, mask, x, w, c_z, c_h, NN, eps, eps_x,
+                                                                        residual ? 1 : 0, out);
     return cudaGetLastError();
 }
 

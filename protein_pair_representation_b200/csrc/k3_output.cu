@@ -62,7 +62,7 @@ struct K3Stats {
     float nmean_z, hrstd_z, nmean_x, rstd_x, hmask, pad0, pad1, pad2;
 };
 
-template <int CZ, bool OUT_F32>
+template <int CZ, bool OUT_F32, bool RES>
 __global__ void __launch_bounds__(576, 1) k3_output_kernel(const __grid_constant__ K3Args p) {
     using C = K3Cfg<CZ, OUT_F32>;
     extern __shared__ uint8_t smem_raw[];
@@ -425,6 +425,24 @@ __global__ void __launch_bounds__(576, 1) k3_output_kernel(const __grid_constant
                             o[i + 1] = r.y;
                         }
                     }
+                    if (RES && (long long)p0 + row < p.NN) {
+                        // residual: this pair's z at the block's 32 output channels (from L2: K1
+                        // and this kernel's own z chunk loads have just read it)
+                        const uint4 *zp = reinterpret_cast<const uint4 *>(
+                            p.zres + ((long long)b * p.NN + p0 + row) * CZ + n0 + wg * 64 + col);
+                        uint4 zr[4];
+#pragma unroll
+                        for (int u = 0; u < 4; ++u) zr[u] = zp[u];
+#pragma unroll
+                        for (int u = 0; u < 4; ++u) {
+                            const uint32_t zw[4] = {zr[u].x, zr[u].y, zr[u].z, zr[u].w};
+#pragma unroll
+                            for (int e = 0; e < 4; ++e) {
+                                o[8 * u + 2 * e] += bf16_lo(zw[e]);
+                                o[8 * u + 2 * e + 1] += bf16_hi(zw[e]);
+                            }
+                        }
+                    }
                     if (OUT_F32) {
 #pragma unroll
                         for (int u = 0; u < 8; ++u)
@@ -469,23 +487,30 @@ size_t k3_smem_bytes(int c_z, bool out_f32) {
     return out_f32 ? K3Cfg<384, true>::SMEM : K3Cfg<384, false>::SMEM;
 }
 
-template <int CZ, bool F32>
+template <int CZ, bool F32, bool RES>
 static cudaError_t k3_launch_t(const K3Args &args, int grid, cudaStream_t stream) {
     static int configured_device = -1;
     int dev = 0;
     cudaGetDevice(&dev);
     if (configured_device != dev) {
-        cudaError_t e = cudaFuncSetAttribute(k3_output_kernel<CZ, F32>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+        cudaError_t e = cudaFuncSetAttribute(k3_output_kernel<CZ, F32, RES>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                              (int)K3Cfg<CZ, F32>::SMEM);
         if (e != cudaSuccess) return e;
         configured_device = dev;
     }
-    return launch_pdl(k3_output_kernel<CZ, F32>, grid, K3Cfg<CZ, F32>::THREADS, K3Cfg<CZ, F32>::SMEM, stream, args);
+    return launch_pdl(k3_output_kernel<CZ, F32, RES>, grid, K3Cfg<CZ, F32>::THREADS, K3Cfg<CZ, F32>::SMEM, stream, args);
+}
+
+template <int CZ>
+static cudaError_t k3_launch_cz(bool out_f32, const K3Args &args, int grid, cudaStream_t stream) {
+    if (args.zres)
+        return out_f32 ? k3_launch_t<CZ, true, true>(args, grid, stream) : k3_launch_t<CZ, false, true>(args, grid, stream);
+    return out_f32 ? k3_launch_t<CZ, true, false>(args, grid, stream) : k3_launch_t<CZ, false, false>(args, grid, stream);
 }
 
 cudaError_t k3_launch(int c_z, bool out_f32, const K3Args &args, int grid, cudaStream_t stream) {
-    if (c_z == 128) return out_f32 ? k3_launch_t<128, true>(args, grid, stream) : k3_launch_t<128, false>(args, grid, stream);
-    if (c_z == 384) return out_f32 ? k3_launch_t<384, true>(args, grid, stream) : k3_launch_t<384, false>(args, grid, stream);
+    if (c_z == 128) return k3_launch_cz<128>(out_f32, args, grid, stream);
+    if (c_z == 384) return k3_launch_cz<384>(out_f32, args, grid, stream);
     return cudaErrorInvalidValue;
 }
 

@@ -47,6 +47,7 @@ struct K3Args {
     int tiles_per_batch;
     float eps;             // input LayerNorm
     float eps_x;           // output LayerNorm on the stored (scaled) x: eps * x_scale^2
+    const uint16_t *zres;  // residual: z (bf16, [B][N*N][c_z]) added to the output; null = none
 };
 
 // Launch with programmatic stream serialization: the kernel may begin while the previous
@@ -81,7 +82,7 @@ cudaError_t k2_launch(const K2Args &args, int grid, cudaStream_t stream);
 
 size_t k3_smem_bytes(int c_z, bool out_f32);
 int k3_groups(int c_z);
-cudaError_t k3_launch(int c_z, bool out_f32, const K3Args &args, int grid, cudaStream_t stream);
+cudaError_t k3_launch(int c_z, bool out_f32, const K3Args &args, int grid, cudaStream_t stream);  // residual iff args.zres
 
 // ---- weight folding (layer creation) -----------------------------------------------
 
@@ -126,6 +127,6 @@ cudaError_t f32_contract_launch(const float *a, const float *b, float *x, int BC
                                 bool incoming, float x_scale, cudaStream_t stream);
 cudaError_t f32_output_launch(const float *z, const float *mask, const float *x,
                               const F32Weights &w, int c_z, int c_h, int B, int N, float eps,
-                              float eps_x, float *out, cudaStream_t stream);
+                              float eps_x, bool residual, float *out, cudaStream_t stream);
 
 }  // namespace trimul

@@ -8,6 +8,7 @@
 #include <cuda_runtime.h>
 
 #include <mutex>
+#include <new>
 #include <stdarg.h>
 #include <stdio.h>
 #include <string.h>
@@ -447,7 +448,8 @@ static trimul_status_t run_contract_tc(const void *a, const void *b, void *x, in
 }
 
 static trimul_status_t run_output_bf16(const trimul_layer_t *L, const void *z, const void *mask, const void *x,
-                                       float x_scale, void *out, bool out_f32, int B, int N, cudaStream_t st) {
+                                       float x_scale, void *out, bool out_f32, bool residual, int B, int N,
+                                       cudaStream_t st) {
     DeviceInfo d;
     TRY(require_sm100(&d));
     const uint64_t NN = (uint64_t)N * N;
@@ -495,6 +497,7 @@ static trimul_status_t run_output_bf16(const trimul_layer_t *L, const void *z, c
     p.tiles_per_batch = (int)((NN + 127) / 128);
     p.eps = L->eps;
     p.eps_x = L->eps * x_scale * x_scale;
+    p.zres = residual ? reinterpret_cast<const uint16_t *>(z) : nullptr;
     const int G = k3_groups(cz);
     const int grid = grid_for(d.sms, (long long)G * B * p.tiles_per_batch, G);
     TRY_CUDA(k3_launch(cz, out_f32, p, grid, st), "K3 launch");
@@ -550,8 +553,8 @@ extern "C" trimul_status_t tri_mul_contract(const void *a, const void *b, void *
     return TRIMUL_OK;
 }
 
-extern "C" trimul_status_t tri_mul_output_gate(const trimul_pair_t *z, const void *mask, const void *x, float x_scale,
-                                               const trimul_layer_t *L, trimul_pair_t *out, void *stream) {
+static trimul_status_t output_gate_impl(const trimul_pair_t *z, const void *mask, const void *x, float x_scale,
+                                        const trimul_layer_t *L, trimul_pair_t *out, bool residual, void *stream) {
     TRY(check_problem(z, mask, L));
     if (!(x_scale > 0.f) || !(x_scale < 3.0e38f)) return fail(TRIMUL_ERR_INVALID_ARG, "x_scale must be positive and finite");
     TRY(check_pair(out, "out"));
@@ -564,16 +567,22 @@ extern "C" trimul_status_t tri_mul_output_gate(const trimul_pair_t *z, const voi
     if (overlap(out->data, pair_bytes(out), x, xbytes)) return fail(TRIMUL_ERR_INVALID_ARG, "out overlaps x");
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
     if (z->dtype == TRIMUL_BF16)
-        return run_output_bf16(L, z->data, mask, x, x_scale, out->data, out->dtype == TRIMUL_F32, (int)z->B, (int)z->N, st);
+        return run_output_bf16(L, z->data, mask, x, x_scale, out->data, out->dtype == TRIMUL_F32, residual, (int)z->B,
+                               (int)z->N, st);
     TRY_CUDA(f32_output_launch(reinterpret_cast<const float *>(z->data), reinterpret_cast<const float *>(mask),
                                reinterpret_cast<const float *>(x), L->f32, L->c_z, L->c_h, (int)z->B, (int)z->N, L->eps,
-                               L->eps * x_scale * x_scale, reinterpret_cast<float *>(out->data), st),
+                               L->eps * x_scale * x_scale, residual, reinterpret_cast<float *>(out->data), st),
              "fp32 output launch");
     return TRIMUL_OK;
 }
 
-extern "C" trimul_status_t tri_mul_forward(const trimul_pair_t *z, const void *mask, const trimul_layer_t *L,
-                                           trimul_direction_t dir, trimul_pair_t *out, void *stream) {
+extern "C" trimul_status_t tri_mul_output_gate(const trimul_pair_t *z, const void *mask, const void *x, float x_scale,
+                                               const trimul_layer_t *L, trimul_pair_t *out, void *stream) {
+    return output_gate_impl(z, mask, x, x_scale, L, out, false, stream);
+}
+
+static trimul_status_t forward_impl(const trimul_pair_t *z, const void *mask, const trimul_layer_t *L,
+                                    trimul_direction_t dir, trimul_pair_t *out, bool residual, void *stream) {
     TRY(check_problem(z, mask, L));
     TRY(check_pair(out, "out"));
     if (dir != TRIMUL_OUTGOING && dir != TRIMUL_INCOMING) return fail(TRIMUL_ERR_INVALID_ARG, "unknown direction");
@@ -595,9 +604,104 @@ extern "C" trimul_status_t tri_mul_forward(const trimul_pair_t *z, const void *m
     const float x_scale = tc ? tri_mul_contract_scale(z->N) : 1.0f;
     TRY(tri_mul_contract(a, b, x, z->B, L->c_h, z->N, tc ? TRIMUL_F16 : TRIMUL_F32, dir, x_scale, stream));
     if (L->timing) TRY_CUDA(cudaEventRecord(L->events[2], st), "event record");
-    TRY(tri_mul_output_gate(z, mask, x, x_scale, L, out, stream));
+    TRY(output_gate_impl(z, mask, x, x_scale, L, out, residual, stream));
     if (L->timing) TRY_CUDA(cudaEventRecord(L->events[3], st), "event record");
     return TRIMUL_OK;
+}
+
+extern "C" trimul_status_t tri_mul_forward(const trimul_pair_t *z, const void *mask, const trimul_layer_t *L,
+                                           trimul_direction_t dir, trimul_pair_t *out, void *stream) {
+    return forward_impl(z, mask, L, dir, out, false, stream);
+}
+
+extern "C" trimul_status_t tri_mul_forward_residual(const trimul_pair_t *z, const void *mask, const trimul_layer_t *L,
+                                                    trimul_direction_t dir, trimul_pair_t *out, void *stream) {
+    return forward_impl(z, mask, L, dir, out, true, stream);
+}
+
+// ------------------------------------------------------------------ pair update and its graph
+
+static trimul_status_t check_pair_update(const trimul_pair_t *z, const trimul_layer_t *Lo, const trimul_layer_t *Li,
+                                         const trimul_pair_t *z_mid, const trimul_pair_t *out) {
+    if (!Lo || !Li) return fail(TRIMUL_ERR_INVALID_ARG, "NULL layer");
+    TRY(check_pair(z, "z"));
+    TRY(check_pair(z_mid, "z_mid"));
+    TRY(check_pair(out, "out"));
+    if (z_mid->B != z->B || z_mid->N != z->N || z_mid->C != z->C || z_mid->dtype != z->dtype)
+        return fail(TRIMUL_ERR_INVALID_ARG, "z_mid must have z's shape and dtype");
+    if (overlap(z_mid->data, pair_bytes(z_mid), z->data, pair_bytes(z)) ||
+        overlap(out->data, pair_bytes(out), z_mid->data, pair_bytes(z_mid)))
+        return fail(TRIMUL_ERR_INVALID_ARG, "z, z_mid and out must not overlap");
+    return TRIMUL_OK;
+}
+
+extern "C" trimul_status_t tri_mul_pair_update(const trimul_pair_t *z, const void *mask, const trimul_layer_t *Lo,
+                                               const trimul_layer_t *Li, trimul_pair_t *z_mid, trimul_pair_t *out,
+                                               void *stream) {
+    TRY(check_pair_update(z, Lo, Li, z_mid, out));
+    TRY(forward_impl(z, mask, Lo, TRIMUL_OUTGOING, z_mid, true, stream));
+    return forward_impl(z_mid, mask, Li, TRIMUL_INCOMING, out, true, stream);
+}
+
+struct trimul_graph {
+    cudaGraph_t graph;
+    cudaGraphExec_t exec;
+};
+
+extern "C" trimul_status_t tri_mul_pair_update_graph_create(const trimul_pair_t *z, const void *mask,
+                                                            const trimul_layer_t *Lo, const trimul_layer_t *Li,
+                                                            trimul_pair_t *z_mid, trimul_pair_t *out,
+                                                            trimul_graph_t **graph_out) {
+    if (!graph_out) return fail(TRIMUL_ERR_INVALID_ARG, "graph_out is NULL");
+    *graph_out = nullptr;
+    TRY(check_pair_update(z, Lo, Li, z_mid, out));
+    if (Lo->timing || Li->timing) return fail(TRIMUL_ERR_INVALID_ARG, "switch the layers' timing events off before capture");
+    cudaStream_t cs = nullptr;
+    TRY_CUDA(cudaStreamCreateWithFlags(&cs, cudaStreamNonBlocking), "capture stream");
+    trimul_status_t st = TRIMUL_OK;
+    cudaGraph_t g = nullptr;
+    // relaxed: the first launch of a kernel may still set its shared-memory attribute while
+    // the capture is open (no call made here synchronizes)
+    cudaError_t e = cudaStreamBeginCapture(cs, cudaStreamCaptureModeRelaxed);
+    if (e != cudaSuccess) {
+        st = fail(TRIMUL_ERR_CUDA, "cudaStreamBeginCapture: %s", cudaGetErrorString(e));
+    } else {
+        st = tri_mul_pair_update(z, mask, Lo, Li, z_mid, out, cs);
+        e = cudaStreamEndCapture(cs, &g);             // always end the capture, even after an error
+        if (st == TRIMUL_OK && e != cudaSuccess) st = fail(TRIMUL_ERR_CUDA, "cudaStreamEndCapture: %s", cudaGetErrorString(e));
+    }
+    cudaGraphExec_t ex = nullptr;
+    if (st == TRIMUL_OK) {
+        e = cudaGraphInstantiateWithFlags(&ex, g, 0);
+        if (e != cudaSuccess) st = fail(TRIMUL_ERR_CUDA, "cudaGraphInstantiate: %s", cudaGetErrorString(e));
+    }
+    cudaStreamDestroy(cs);
+    if (st != TRIMUL_OK) {
+        if (ex) cudaGraphExecDestroy(ex);
+        if (g) cudaGraphDestroy(g);
+        return st;
+    }
+    trimul_graph_t *h = new (std::nothrow) trimul_graph_t{g, ex};
+    if (!h) {
+        cudaGraphExecDestroy(ex);
+        cudaGraphDestroy(g);
+        return fail(TRIMUL_ERR_INVALID_ARG, "out of host memory");
+    }
+    *graph_out = h;
+    return TRIMUL_OK;
+}
+
+extern "C" trimul_status_t tri_mul_graph_launch(const trimul_graph_t *graph, void *stream) {
+    if (!graph) return fail(TRIMUL_ERR_INVALID_ARG, "graph is NULL");
+    TRY_CUDA(cudaGraphLaunch(graph->exec, reinterpret_cast<cudaStream_t>(stream)), "graph launch");
+    return TRIMUL_OK;
+}
+
+extern "C" void tri_mul_graph_destroy(trimul_graph_t *graph) {
+    if (!graph) return;
+    cudaGraphExecDestroy(graph->exec);
+    cudaGraphDestroy(graph->graph);
+    delete graph;
 }
 
 // One CTA waits, with the kernels' bounded wait, on an mbarrier that nothing arrives at:

@@ -79,6 +79,12 @@ def load_library():
         lib.tri_mul_workspace_bytes.restype = ctypes.c_size_t
         lib.tri_mul_layer_bind_workspace.argtypes = [vp, vp, ctypes.c_size_t]
         lib.tri_mul_forward.argtypes = [P(_Pair), vp, vp, st, P(_Pair), vp]
+        lib.tri_mul_forward_residual.argtypes = [P(_Pair), vp, vp, st, P(_Pair), vp]
+        lib.tri_mul_pair_update.argtypes = [P(_Pair), vp, vp, vp, P(_Pair), P(_Pair), vp]
+        lib.tri_mul_pair_update_graph_create.argtypes = [P(_Pair), vp, vp, vp, P(_Pair), P(_Pair), P(vp)]
+        lib.tri_mul_graph_launch.argtypes = [vp, vp]
+        lib.tri_mul_graph_destroy.argtypes = [vp]
+        lib.tri_mul_graph_destroy.restype = None
         lib.tri_mul_project.argtypes = [P(_Pair), vp, vp, vp, vp, vp]
         lib.tri_mul_contract.argtypes = [vp, vp, vp, i64, i64, i64, st, st, ctypes.c_float, vp]
         lib.tri_mul_contract_scale.argtypes = [i64]
@@ -93,6 +99,8 @@ def load_library():
         lib.tri_mul_last_error.restype = ctypes.c_char_p
         lib.tri_mul_abi_version.argtypes = []
         for name in ("tri_mul_layer_create", "tri_mul_layer_bind_workspace", "tri_mul_forward",
+                     "tri_mul_forward_residual", "tri_mul_pair_update", "tri_mul_pair_update_graph_create",
+                     "tri_mul_graph_launch",
                      "tri_mul_project", "tri_mul_contract", "tri_mul_output_gate",
                      "tri_mul_layer_set_timing_events", "tri_mul_check_device_status"):
             getattr(lib, name).restype = ctypes.c_int
@@ -218,14 +226,17 @@ class TriMulLayer:
         _check(self._lib.tri_mul_layer_set_timing_events(self.handle, arr))
 
     def forward(self, z: torch.Tensor, mask: torch.Tensor | None = None, direction="outgoing",
-                out: torch.Tensor | None = None, out_dtype: torch.dtype | None = None, stream=None):
+                out: torch.Tensor | None = None, out_dtype: torch.dtype | None = None, stream=None,
+                residual: bool = False):
+        """The update (residual=False) or z + update (residual=True) of one direction."""
         B, N = z.shape[0], z.shape[1]
         self.ensure_workspace(B, N, z.dtype)
         if out is None:
             out = torch.empty(z.shape, dtype=out_dtype or torch.float32, device=z.device)
         zp, op = _pair(z), _pair(out)
-        _check(self._lib.tri_mul_forward(ctypes.byref(zp), _mask_ptr(mask, z), self.handle,
-                                         _DIRS[direction], ctypes.byref(op), _stream_ptr(stream)))
+        fn = self._lib.tri_mul_forward_residual if residual else self._lib.tri_mul_forward
+        _check(fn(ctypes.byref(zp), _mask_ptr(mask, z), self.handle, _DIRS[direction], ctypes.byref(op),
+                  _stream_ptr(stream)))
         return out
 
     __call__ = forward
@@ -269,6 +280,63 @@ def contract(a: torch.Tensor, b: torch.Tensor, direction="outgoing", out: torch.
     _check(lib.tri_mul_contract(a.data_ptr(), b.data_ptr(), out.data_ptr(), B, C, N, _dtype_code(a.dtype),
                                 _DIRS[direction], x_scale, _stream_ptr(stream)))
     return out
+
+
+def pair_update(z: torch.Tensor, mask: torch.Tensor | None, layer_out: TriMulLayer, layer_in: TriMulLayer,
+                out: torch.Tensor | None = None, z_mid: torch.Tensor | None = None, out_dtype: torch.dtype | None = None,
+                stream=None):
+    """One pair update: z_mid = z + U_outgoing(z) (z's dtype), out = z_mid + U_incoming(z_mid)."""
+    B, N = z.shape[0], z.shape[1]
+    layer_out.ensure_workspace(B, N, z.dtype)
+    layer_in.ensure_workspace(B, N, z.dtype)
+    if z_mid is None:
+        z_mid = torch.empty_like(z)
+    if out is None:
+        out = torch.empty(z.shape, dtype=out_dtype or z.dtype, device=z.device)
+    zp, mp, op = _pair(z), _pair(z_mid), _pair(out)
+    _check(load_library().tri_mul_pair_update(ctypes.byref(zp), _mask_ptr(mask, z), layer_out.handle, layer_in.handle,
+                                              ctypes.byref(mp), ctypes.byref(op), _stream_ptr(stream)))
+    return out
+
+
+class PairUpdateGraph:
+    """A CUDA graph of one pair_update on fixed tensors; launch() replays it.
+
+    The tensors and both layers (with their workspaces) must stay alive, in place, for the
+    graph's lifetime; write new inputs into `z` and `mask` between launches.
+    """
+
+    def __init__(self, z: torch.Tensor, mask: torch.Tensor | None, layer_out: TriMulLayer, layer_in: TriMulLayer,
+                 out_dtype: torch.dtype | None = None):
+        self._lib = load_library()
+        B, N = z.shape[0], z.shape[1]
+        layer_out.ensure_workspace(B, N, z.dtype)
+        layer_in.ensure_workspace(B, N, z.dtype)
+        self.z, self.mask, self.layers = z, mask, (layer_out, layer_in)
+        self.z_mid = torch.empty_like(z)
+        self.out = torch.empty(z.shape, dtype=out_dtype or z.dtype, device=z.device)
+        zp, mp, op = _pair(z), _pair(self.z_mid), _pair(self.out)
+        handle = ctypes.c_void_p()
+        torch.cuda.synchronize(z.device)
+        _check(self._lib.tri_mul_pair_update_graph_create(ctypes.byref(zp), _mask_ptr(mask, z), layer_out.handle,
+                                                          layer_in.handle, ctypes.byref(mp), ctypes.byref(op),
+                                                          ctypes.byref(handle)))
+        self.handle = handle
+
+    def launch(self, stream=None) -> torch.Tensor:
+        _check(self._lib.tri_mul_graph_launch(self.handle, _stream_ptr(stream)))
+        return self.out
+
+    def close(self):
+        if getattr(self, "handle", None):
+            self._lib.tri_mul_graph_destroy(self.handle)
+            self.handle = None
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
 
 
 def check_device_status():

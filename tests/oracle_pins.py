@@ -13,7 +13,10 @@ Sources of truth used here:
   * invariants of the definition: incoming = swap(outgoing(swap z)) with the a/b
     projections exchanged, residue-permutation equivariance, masked residues k
     contribute nothing, padding equals truncation, sampled entries equal the
-    full computation, invariance of the output under scaling of the b projection.
+    full computation, invariance of the output under scaling of the b projection,
+  * the pair update (two residual steps): masked pairs keep z bitwise, and with one
+    step's output projection zeroed it reduces to the other step's single update in
+    its own direction.
 """
 from __future__ import annotations
 
@@ -326,10 +329,65 @@ def pin_single_residue_directions_agree(lib):
     assert np.array_equal(o1, o2)
 
 
+# ---------------------------------------------------------------- pair update (two residual steps)
+
+
+def _zero_output_projection(weights):
+    """Weights whose update is exactly 0 everywhere (W_o = 0 and b_o = 0)."""
+    w = {k: (None if v is None else np.array(v, dtype=np.float64, copy=True)) for k, v in weights.items()}
+    w["w_o"][:] = 0.0
+    if w.get("b_o") is not None:
+        w["b_o"][:] = 0.0
+    return w
+
+
+def _two_layers(seed=41):
+    inp = _small(seed=seed)
+    other = _small(seed=seed + 1)          # a second layer: same shapes, other weights
+    return inp, inp.weights, other.weights
+
+
+def pin_pair_update_masked_pairs_keep_z(lib):
+    """Both updates are exactly 0 at a masked pair, so z_mid and out keep z there bitwise."""
+    inp, w1, w2 = _two_layers()
+    z_mid, out = oracle.pair_update(inp.z, inp.mask, w1, w2, inp.eps, lib=lib)
+    masked = inp.mask == 0
+    assert masked.any()
+    z = np.asarray(inp.z, dtype=np.float64)
+    assert np.array_equal(z_mid[masked], z[masked]) and np.array_equal(out[masked], z[masked])
+
+
+def pin_pair_update_first_step_is_outgoing(lib):
+    """With a zero second update the pair update is z + outgoing(z) with the first layer's
+    weights (the incoming update or the other weights give a different result here)."""
+    inp, w1, w2 = _two_layers()
+    _, out = oracle.pair_update(inp.z, inp.mask, w1, _zero_output_projection(w2), inp.eps, lib=lib)
+    z = np.asarray(inp.z, dtype=np.float64)
+    ref = z + oracle.trimul(inp.z, inp.mask, w1, "outgoing", inp.eps, lib=lib)
+    wrong = z + oracle.trimul(inp.z, inp.mask, w1, "incoming", inp.eps, lib=lib)
+    _close(out, ref, what="pair update, step 1")
+    assert np.max(np.abs(out - wrong)) > 1e-6
+
+
+def pin_pair_update_second_step_is_incoming(lib):
+    """With a zero first update the pair update is z + incoming(z) with the second layer's
+    weights."""
+    inp, w1, w2 = _two_layers()
+    z_mid, out = oracle.pair_update(inp.z, inp.mask, _zero_output_projection(w1), w2, inp.eps, lib=lib)
+    z = np.asarray(inp.z, dtype=np.float64)
+    assert np.array_equal(z_mid, z)
+    ref = z + oracle.trimul(inp.z, inp.mask, w2, "incoming", inp.eps, lib=lib)
+    wrong = z + oracle.trimul(inp.z, inp.mask, w2, "outgoing", inp.eps, lib=lib)
+    _close(out, ref, what="pair update, step 2")
+    assert np.max(np.abs(out - wrong)) > 1e-6
+
+
 ALL_PINS = [
     pin_layernorm_library, pin_linear_library, pin_gated_projection_library, pin_contract_library,
     pin_output_gate_library, pin_full_update_library, pin_constant_field_closed_form,
     pin_hand_worked_example, pin_transpose_identity, pin_permutation_equivariance,
     pin_masked_k_contributes_nothing, pin_padding_equals_truncation, pin_sampled_equals_full,
     pin_b_projection_scale_invariance, pin_single_residue_directions_agree,
+    pin_pair_update_masked_pairs_keep_z, pin_pair_update_first_step_is_outgoing,
+    pin_pair_update_second_step_is_incoming,
 ]

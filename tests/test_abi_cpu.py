@@ -49,7 +49,7 @@ def test_status_strings_and_versions(lib):
     for code in range(9):
         assert lib.tri_mul_status_string(code)
     assert lib.tri_mul_status_string(99) == b"unknown status"
-    assert lib.tri_mul_abi_version() == 100
+    assert lib.tri_mul_abi_version() == 101
     assert lib.tri_mul_kernels_per_forward() == 3
 
 
@@ -108,3 +108,16 @@ def test_adjacent_f16_planes_pass_validation(lib):
     a, b, x = ctypes.c_void_p(1 << 20), ctypes.c_void_p((1 << 20) + plane), ctypes.c_void_p((1 << 20) + 2 * plane)
     st = lib.tri_mul_contract(a, b, x, B, C, N, tm.F16, 0, 1.0, None)
     assert st in (3, 5), lib.tri_mul_last_error()
+
+
+def test_pair_update_and_graph_validate_on_the_host(lib):
+    z = tm._Pair(0, 1, 8, 128, tm.BF16)
+    mid = tm._Pair(0, 1, 8, 128, tm.BF16)
+    out = tm._Pair(0, 1, 8, 128, tm.F32)
+    assert lib.tri_mul_pair_update(ctypes.byref(z), None, None, None, ctypes.byref(mid), ctypes.byref(out),
+                                   None) == 1
+    assert lib.tri_mul_pair_update_graph_create(ctypes.byref(z), None, None, None, ctypes.byref(mid),
+                                                ctypes.byref(out), None) == 1
+    assert lib.tri_mul_graph_launch(None, None) == 1
+    lib.tri_mul_graph_destroy(None)          # NULL is ignored
+    assert lib.tri_mul_forward_residual(None, None, None, 0, None, None) != 0
