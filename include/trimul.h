@@ -118,7 +118,8 @@ void tri_mul_layer_destroy(trimul_layer_t *layer);
 
 /* Bytes of workspace tri_mul_forward needs for B x N x N with z of type `dtype`:
  * a, b and x, each [B, c_h, N, N] of the intermediate type (F16 for a BF16 z,
- * F32 for an F32 z), 256-byte aligned. Returns 0 for an invalid layer or size. */
+ * F32 for an F32 z), 256-byte aligned, then the mask extents (2 int32 per batch
+ * element, 256-byte aligned). Returns 0 for an invalid layer or size. */
 size_t tri_mul_workspace_bytes(const trimul_layer_t *layer, int64_t B, int64_t N,
                                trimul_dtype_t dtype);
 
@@ -129,7 +130,12 @@ trimul_status_t tri_mul_layer_bind_workspace(trimul_layer_t *layer, void *worksp
                                              size_t bytes);
 
 /* One triangle multiplicative update (one direction). Returns the update only;
- * the residual add z += update is the caller's.
+ * the residual add z += update is the caller's (or tri_mul_forward_residual's).
+ * With mask skipping switched on (tri_mul_layer_set_mask_skipping), on the tensor-core
+ * path with a mask a first pass finds the mask's extents (the last row and column holding a
+ * nonzero entry, per batch element) and the kernels leave out tiles that are masked in full
+ * and the part of the contraction's k-range beyond them (the results are bitwise the same:
+ * every product left out is an exact zero).
  *   z    : [B, N, N, c_z], dtype F32 (fp32 SIMT path) or BF16 (tensor-core path)
  *   mask : [B, N, N] in z's dtype with values 0 or 1, or NULL for all ones
  *   out  : [B, N, N, c_z]; F32 for the F32 path; F32 or BF16 for the BF16 path
@@ -179,7 +185,8 @@ trimul_status_t tri_mul_output_gate(const trimul_pair_t *z, const void *mask, co
  * loads it, held until the process exits) instead of a bound workspace; the layer's
  * workspace and timing events are not used. It allocates nothing.
  *   - Problems whose a, b and x need more than TRIMUL_NOALLOC_SCRATCH_BYTES (that is,
- *     tri_mul_workspace_bytes() > TRIMUL_NOALLOC_SCRATCH_BYTES; for a BF16 z with
+ *     tri_mul_workspace_bytes() less its mask-extents block > TRIMUL_NOALLOC_SCRATCH_BYTES;
+ *     this path skips no masked tiles; for a BF16 z with
  *     c_h = 128 the limit is B * N * N <= 65536, e.g. N = 256 at B = 1) are rejected
  *     with TRIMUL_ERR_WORKSPACE.
  *   - The first call on each device looks up the array's device address (once, with
@@ -233,13 +240,24 @@ trimul_status_t tri_mul_graph_launch(const trimul_graph_t *graph, void *stream);
 /* Free the graph. NULL is ignored. */
 void tri_mul_graph_destroy(trimul_graph_t *graph);
 
+/* Mask skipping (off by default): when on, tri_mul_forward with a mask on the tensor-core
+ * path first finds the mask's extents {R_b, C_b} per batch element (a memset and one small
+ * kernel) and the kernels then leave out 128-pair tiles that are masked in full (writing
+ * their zeros) and the contraction's k-range beyond the extents ("RFProteina architecture",
+ * section "Kernel support": masks are left-aligned, so a per-row valid count bounds the
+ * work). Worth it when whole rows are padding: measured on B200 it makes B=4 N=256 c_z=384
+ * (valid lengths 162-237) 8% faster and B=1 N=512 c_z=128 (493 of 512 valid) 9% slower. */
+trimul_status_t tri_mul_layer_set_mask_skipping(trimul_layer_t *layer, int enable);
+
 /* Optional per-kernel timing: when `events` is non-NULL, every later
- * tri_mul_forward on this handle records events[0] before K1, events[1] after
+ * tri_mul_forward on this handle records events[0] before K1 (after the mask-extents
+ * pass), events[1] after
  * K1, events[2] after K2 and events[3] after K3 on its stream. The four values
  * are cudaEvent_t created by the caller; NULL switches recording off. */
 trimul_status_t tri_mul_layer_set_timing_events(trimul_layer_t *layer, void *const *events);
 
-/* Number of kernels one tri_mul_forward launches (for launch accounting). */
+/* Number of kernels one tri_mul_forward launches: K1, K2 and K3 (one more, the mask-extents
+ * pass, on the tensor-core path with a mask and mask skipping switched on). */
 int tri_mul_kernels_per_forward(void);
 
 /* Synchronize the current device, then read and clear the library's device

@@ -60,7 +60,9 @@ struct K1Smem {
     int abort_flag;
 };
 
-template <int CZ>
+// SKIP: the instance that leaves out wholly masked tiles (p.ext set); the other one carries
+// none of that code.
+template <int CZ, bool SKIP>
 __global__ void __launch_bounds__(448, 1) k1_project_kernel(const __grid_constant__ K1Args p) {
     using C = K1Cfg<CZ>;
     extern __shared__ uint8_t smem_raw[];
@@ -127,6 +129,7 @@ __global__ void __launch_bounds__(448, 1) k1_project_kernel(const __grid_constan
             for (int pt = cta_in_group; pt < num_ptiles; pt += ctas_per_group, tw.advance(ctas_per_group, p.tiles_per_batch)) {
                 const int b = tw.b;
                 const int p0 = tw.t * 128;
+                if (SKIP && tile_masked_out(p.ext, b, p0, p.N, p.NN, p.rowdiv)) continue;   // nothing to load
                 for (int kc = 0; kc < C::KC; ++kc) {
                     if (!mbar_wait(&s.empty[stage], phase ^ 1, abort_flag, kErrTimeoutProducer)) goto producer_abort;
                     mbar_arrive_expect_tx(&s.full[stage], C::CHUNK);
@@ -152,7 +155,9 @@ __global__ void __launch_bounds__(448, 1) k1_project_kernel(const __grid_constan
             uint32_t phase = 0;
             int abuf = 0;
             uint32_t aphase = 0;
-            for (int pt = cta_in_group; ok && pt < num_ptiles; pt += ctas_per_group) {
+            TileWalk tw(cta_in_group, p.tiles_per_batch);
+            for (int pt = cta_in_group; ok && pt < num_ptiles; pt += ctas_per_group, tw.advance(ctas_per_group, p.tiles_per_batch)) {
+                if (SKIP && tile_masked_out(p.ext, tw.b, tw.t * 128, p.N, p.NN, p.rowdiv)) continue;
                 if (!mbar_wait(&s.tempty[abuf], aphase ^ 1, abort_flag, kErrTimeoutMma)) break;
                 tc_fence_after();
                 const uint32_t d_tmem = tmem_base + abuf * C::NCOL;
@@ -188,6 +193,7 @@ __global__ void __launch_bounds__(448, 1) k1_project_kernel(const __grid_constan
         for (int pt = cta_in_group; pt < num_ptiles; pt += ctas_per_group, tw.advance(ctas_per_group, p.tiles_per_batch)) {
             const int b = tw.b;
             const int p0 = tw.t * 128;
+            if (SKIP && tile_masked_out(p.ext, b, p0, p.N, p.NN, p.rowdiv)) continue;
             // shifted sums in packed pairs: s1 = sum(v - shift), s2 = sum((v - shift)^2), with
             // the row's first entry as the shift
             float shift = 0.f;
@@ -247,6 +253,19 @@ __global__ void __launch_bounds__(448, 1) k1_project_kernel(const __grid_constan
         for (int pt = cta_in_group; pt < num_ptiles; pt += ctas_per_group, tw.advance(ctas_per_group, p.tiles_per_batch)) {
             const int b = tw.b;
             const int p0 = tw.t * 128;
+            if (SKIP && tile_masked_out(p.ext, b, p0, p.N, p.NN, p.rowdiv)) {
+                // every pair of the tile is masked: a and b are 0 there (the contraction reads them)
+                if (leader) tma_store_wait_read<0>();
+                named_bar_sync(1 + wg, 128);
+                for (int ch = 0; ch < C::CH_WG; ++ch) stg[ch * 128 + row] = 0;
+                fence_proxy_async_smem();
+                named_bar_sync(1 + wg, 128);
+                if (leader) {
+                    tma_store_3d(tm_out, stg, p0, ch0 + wg * C::CH_WG, b);
+                    tma_store_commit();
+                }
+                continue;
+            }
             if (!group_all(mbar_wait(&s.sfull[sbuf], sphase, abort_flag, kErrTimeoutEpilogue), 1 + wg, 128)) break;
             const float4 st = stats[sbuf * 128 + row];
             __syncwarp();
@@ -338,6 +357,7 @@ __device__ __forceinline__ __half2 tanh_h2(__half2 x) {
     return u32_as_h2(t);
 }
 
+template <bool SKIP>
 __global__ void __launch_bounds__(K1CmCfg::THREADS, 1) k1_project_cm_kernel(const __grid_constant__ K1Args p) {
     using C = K1CmCfg;
     extern __shared__ uint8_t smem_raw[];
@@ -403,6 +423,7 @@ __global__ void __launch_bounds__(K1CmCfg::THREADS, 1) k1_project_cm_kernel(cons
             for (int pt = cta_in_group; pt < num_ptiles; pt += ctas_per_group, tw.advance(ctas_per_group, p.tiles_per_batch)) {
                 const int b = tw.b;
                 const int p0 = tw.t * 128;
+                if (SKIP && tile_masked_out(p.ext, b, p0, p.N, p.NN, p.rowdiv)) continue;   // nothing to load
                 for (int kc = 0; kc < C::KC; ++kc) {
                     if (!mbar_wait(&s.empty[stage], phase ^ 1, abort_flag, kErrTimeoutProducer)) goto producer_abort;
                     mbar_arrive_expect_tx(&s.full[stage], C::CHUNK);
@@ -426,10 +447,14 @@ __global__ void __launch_bounds__(K1CmCfg::THREADS, 1) k1_project_cm_kernel(cons
             bool ok = mbar_wait(&s.wbar, 0, abort_flag, kErrTimeoutMma);
             int stage = 0;
             uint32_t phase = 0;
-            int abuf = 0;
-            uint32_t aphase = 0;
-            for (int pt = cta_in_group; ok && pt < num_ptiles; pt += ctas_per_group) {
-                if (!mbar_wait(&s.tempty[abuf], aphase ^ 1, abort_flag, kErrTimeoutMma)) break;
+            uint32_t aphase[2] = {0, 0};           // tile j of this CTA uses TMEM buffer j % 2
+            int j = 0;
+            TileWalk tw(cta_in_group, p.tiles_per_batch);
+            for (int pt = cta_in_group; ok && pt < num_ptiles;
+                 pt += ctas_per_group, tw.advance(ctas_per_group, p.tiles_per_batch), ++j) {
+                if (SKIP && tile_masked_out(p.ext, tw.b, tw.t * 128, p.N, p.NN, p.rowdiv)) continue;
+                const int abuf = j & 1;
+                if (!mbar_wait(&s.tempty[abuf], aphase[abuf] ^ 1, abort_flag, kErrTimeoutMma)) break;
                 tc_fence_after();
                 const uint32_t d_gate = tmem_base + abuf * 256;
                 const uint32_t d_proj = d_gate + 128;
@@ -451,7 +476,7 @@ __global__ void __launch_bounds__(K1CmCfg::THREADS, 1) k1_project_cm_kernel(cons
                 }
                 if (!ok) break;
                 tc_commit(&s.tfull[abuf]);
-                if (++abuf == 2) { abuf = 0; aphase ^= 1; }
+                aphase[abuf] ^= 1;
             }
             tc_commit(&s.drain);
             mbar_drain(&s.drain, 0);
@@ -461,12 +486,15 @@ __global__ void __launch_bounds__(K1CmCfg::THREADS, 1) k1_project_cm_kernel(cons
         const int row = (warp - C::STATS_WARP0) * 32 + lane;
         int stage = 0;
         uint32_t phase = 0;
-        int sbuf = 0;
-        uint32_t sphase = 0;
+        uint32_t sphase[2] = {0, 0};               // tile j of this CTA uses statistics buffer j % 2
+        int j = -1;
         TileWalk tw(cta_in_group, p.tiles_per_batch);
         for (int pt = cta_in_group; pt < num_ptiles; pt += ctas_per_group, tw.advance(ctas_per_group, p.tiles_per_batch)) {
             const int b = tw.b;
             const int p0 = tw.t * 128;
+            ++j;
+            if (SKIP && tile_masked_out(p.ext, b, p0, p.N, p.NN, p.rowdiv)) continue;
+            const int sbuf = j & 1;
             const long long pi = (long long)p0 + row;
             uint16_t mbits = 0x3F80u;   // bf16 1.0; the load is issued first so its latency overlaps
             if (p.mask) mbits = (pi < p.NN) ? p.mask[(long long)b * p.NN + pi] : (uint16_t)0;
@@ -501,13 +529,13 @@ __global__ void __launch_bounds__(K1CmCfg::THREADS, 1) k1_project_cm_kernel(cons
             const float inv_n = 1.0f / (float)C::CZ;
             const float dm = (s1.x + s1.y) * inv_n;
             const float var = fmaxf((s2.x + s2.y) * inv_n - dm * dm, 0.f);
-            if (!__all_sync(0xffffffffu, mbar_wait(&s.sempty[sbuf], sphase ^ 1, abort_flag, kErrTimeoutEpilogue))) break;
+            if (!__all_sync(0xffffffffu, mbar_wait(&s.sempty[sbuf], sphase[sbuf] ^ 1, abort_flag, kErrTimeoutEpilogue))) break;
             st_nmean[sbuf * 128 + row] = -(shift + dm);
             st_rstd[sbuf * 128 + row] = rsqrtf(var + p.eps);
             st_hmask[sbuf * 128 + row] = __float2half_rn(0.5f * __uint_as_float((uint32_t)mbits << 16));
             __syncwarp();
             if (lane == 0) mbar_arrive(&s.sfull[sbuf]);
-            if (++sbuf == C::SNB) { sbuf = 0; sphase ^= 1; }
+            sphase[sbuf] ^= 1;
         }
     } else {
         // epilogue: two teams of eight warps take alternate tiles of this CTA's sequence (team k
@@ -539,6 +567,24 @@ __global__ void __launch_bounds__(K1CmCfg::THREADS, 1) k1_project_cm_kernel(cons
         for (int pt = first; pt < num_ptiles; pt += 2 * ctas_per_group, tw.advance(2 * ctas_per_group, p.tiles_per_batch)) {
             const int b = tw.b;
             const int p0 = tw.t * 128;
+            if (SKIP && tile_masked_out(p.ext, b, p0, p.N, p.NN, p.rowdiv)) {
+                // every pair of the tile is masked: a and b are 0 there (the contraction reads them)
+#pragma unroll 1
+                for (int blk = 0; blk < 2; ++blk) {
+                    const int col = col0 + 32 * blk;
+                    if (lane == 0) tma_store_wait_read<0>();
+                    __syncwarp();
+#pragma unroll
+                    for (int u = 0; u < 4; ++u) *reinterpret_cast<uint4 *>(stg + sw64_offset(lane, u)) = make_uint4(0, 0, 0, 0);
+                    fence_proxy_async_smem();
+                    __syncwarp();
+                    if (lane == 0 && p0 + col < p.NN) {
+                        tma_store_3d(tm_out, stg, p0 + col, q * 32, b);
+                        tma_store_commit();
+                    }
+                }
+                continue;
+            }
             if (!__all_sync(0xffffffffu, mbar_wait(&s.sfull[sbuf], phase, abort_flag, kErrTimeoutEpilogue) &&
                                              mbar_wait(&s.tfull[abuf], phase, abort_flag, kErrTimeoutEpilogue)))
                 break;
@@ -615,36 +661,38 @@ int k1_channels_per_warpgroup(int c_z) { return c_z == 128 ? K1CmCfg::C_H : K1Cf
 int k1_row_mode(int c_z) { return c_z == 128 ? 2 : 1; }
 size_t k1_smem_bytes(int c_z) { return c_z == 128 ? K1CmCfg::SMEM : K1Cfg<384>::SMEM; }
 
-template <int CZ>
+template <int CZ, bool SKIP>
 static cudaError_t k1_launch_t(const K1Args &args, int grid, cudaStream_t stream) {
     static int configured_device = -1;
     int dev = 0;
     cudaGetDevice(&dev);
     if (configured_device != dev) {
-        cudaError_t e = cudaFuncSetAttribute(k1_project_kernel<CZ>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+        cudaError_t e = cudaFuncSetAttribute(k1_project_kernel<CZ, SKIP>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                              (int)K1Cfg<CZ>::SMEM);
         if (e != cudaSuccess) return e;
         configured_device = dev;
     }
-    return launch_pdl(k1_project_kernel<CZ>, grid, K1Cfg<CZ>::THREADS, K1Cfg<CZ>::SMEM, stream, args);
+    return launch_pdl(k1_project_kernel<CZ, SKIP>, grid, K1Cfg<CZ>::THREADS, K1Cfg<CZ>::SMEM, stream, args);
 }
 
+template <bool SKIP>
 static cudaError_t k1_launch_cm(const K1Args &args, int grid, cudaStream_t stream) {
     static int configured_device = -1;
     int dev = 0;
     cudaGetDevice(&dev);
     if (configured_device != dev) {
-        cudaError_t e = cudaFuncSetAttribute(k1_project_cm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+        cudaError_t e = cudaFuncSetAttribute(k1_project_cm_kernel<SKIP>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                              (int)K1CmCfg::SMEM);
         if (e != cudaSuccess) return e;
         configured_device = dev;
     }
-    return launch_pdl(k1_project_cm_kernel, grid, K1CmCfg::THREADS, K1CmCfg::SMEM, stream, args);
+    return launch_pdl(k1_project_cm_kernel<SKIP>, grid, K1CmCfg::THREADS, K1CmCfg::SMEM, stream, args);
 }
 
 cudaError_t k1_launch(int c_z, const K1Args &args, int grid, cudaStream_t stream) {
-    if (c_z == 128) return k1_launch_cm(args, grid, stream);
-    if (c_z == 384) return k1_launch_t<384>(args, grid, stream);
+    const bool skip = args.ext != nullptr;
+    if (c_z == 128) return skip ? k1_launch_cm<true>(args, grid, stream) : k1_launch_cm<false>(args, grid, stream);
+    if (c_z == 384) return skip ? k1_launch_t<384, true>(args, grid, stream) : k1_launch_t<384, false>(args, grid, stream);
     return cudaErrorInvalidValue;
 }
 

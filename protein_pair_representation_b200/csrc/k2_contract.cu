@@ -45,6 +45,22 @@ struct Smem {
 constexpr size_t SMEM_BYTES = 1024 /*align*/ + STAGES * STAGE_BYTES + 2 * STG_BYTES + 1024;
 }  // namespace k2
 
+// Number of 64-deep k chunks the tile (bc, m0, n0) sums over; 0: the tile is not computed.
+// With mask extents {R_b, C_b}, a[., k] and b[., k] vanish for k >= C_b (outgoing: mask
+// column k all zero) or k >= R_b (incoming: mask row k all zero), so the sum stops there with
+// the same result (the products left out are exact zeros). When N is a multiple of 128 the
+// output kernel's 128-pair tiles lie inside one row and one 128 x 256 tile here, so tiles at
+// rows >= R_b or columns >= C_b, which it never reads, are not computed either.
+__device__ __forceinline__ int k2_tile_chunks(const K2Args &p, int bc, int m0, int n0) {
+    if (!p.ext) return p.k_chunks;
+    const int b = bc / p.C;
+    const int R = __ldg(p.ext + 2 * b), Cx = __ldg(p.ext + 2 * b + 1);
+    if ((p.N & 127) == 0 && (m0 >= R || n0 >= Cx)) return 0;
+    const int kend = p.incoming ? R : Cx;
+    const int nk = (kend + k2::BK - 1) / k2::BK;
+    return nk < p.k_chunks ? nk : p.k_chunks;
+}
+
 __global__ void __launch_bounds__(k2::THREADS, 1) k2_contract_kernel(const __grid_constant__ K2Args p) {
     using namespace k2;
     extern __shared__ uint8_t smem_raw[];
@@ -99,7 +115,8 @@ __global__ void __launch_bounds__(k2::THREADS, 1) k2_contract_kernel(const __gri
                 const int r = t - bc * tiles_per_channel;
                 const int m0 = (r / p.n_tiles) * BM;
                 const int n0 = (r % p.n_tiles) * BN;
-                for (int kc = 0; kc < p.k_chunks; ++kc) {
+                const int nk = k2_tile_chunks(p, bc, m0, n0);
+                for (int kc = 0; kc < nk; ++kc) {
                     if (!mbar_wait(&s.empty[stage], phase ^ 1, abort_flag, kErrTimeoutProducer)) goto producer_abort;
                     uint8_t *sa = stages + stage * STAGE_BYTES;
                     uint8_t *sb = sa + A_BYTES;
@@ -137,11 +154,15 @@ __global__ void __launch_bounds__(k2::THREADS, 1) k2_contract_kernel(const __gri
             int abuf = 0;
             uint32_t aphase = 0;
             for (int t = blockIdx.x; t < num_tiles; t += gridDim.x) {
+                const int bc = t / tiles_per_channel;
+                const int r = t - bc * tiles_per_channel;
+                const int nk = k2_tile_chunks(p, bc, (r / p.n_tiles) * BM, (r % p.n_tiles) * BN);
+                if (nk == 0) continue;
                 if (!mbar_wait(&s.tempty[abuf], aphase ^ 1, abort_flag, kErrTimeoutMma)) break;
                 tc_fence_after();
                 const uint32_t d_tmem = tmem_base + abuf * BN;
                 bool ok = true;
-                for (int kc = 0; kc < p.k_chunks; ++kc) {
+                for (int kc = 0; kc < nk; ++kc) {
                     if (!mbar_wait(&s.full[stage], phase, abort_flag, kErrTimeoutMma)) { ok = false; break; }
                     tc_fence_after();
                     const uint8_t *sa = stages + stage * STAGE_BYTES;
@@ -183,6 +204,7 @@ __global__ void __launch_bounds__(k2::THREADS, 1) k2_contract_kernel(const __gri
             const int r = t - bc * tiles_per_channel;
             const int m0 = (r / p.n_tiles) * BM;
             const int n0 = (r % p.n_tiles) * BN;
+            if (k2_tile_chunks(p, bc, m0, n0) == 0) continue;
             if (!group_all(mbar_wait(&s.tfull[abuf], aphase, abort_flag, kErrTimeoutEpilogue), 1 + wg, 128)) break;
             tc_fence_after();
 #pragma unroll 1

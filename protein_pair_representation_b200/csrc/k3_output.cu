@@ -62,7 +62,9 @@ struct K3Stats {
     float nmean_z, hrstd_z, nmean_x, rstd_x, hmask, pad0, pad1, pad2;
 };
 
-template <int CZ, bool OUT_F32, bool RES>
+// RES: out = z + update; SKIP: wholly masked tiles written as zeros without any work (p.ext
+// set; never with RES). Instances without them carry none of that code.
+template <int CZ, bool OUT_F32, bool RES, bool SKIP>
 __global__ void __launch_bounds__(576, 1) k3_output_kernel(const __grid_constant__ K3Args p) {
     using C = K3Cfg<CZ, OUT_F32>;
     extern __shared__ uint8_t smem_raw[];
@@ -141,6 +143,7 @@ __global__ void __launch_bounds__(576, 1) k3_output_kernel(const __grid_constant
             for (int pt = cta_in_group; pt < num_ptiles; pt += ctas_per_group, tw.advance(ctas_per_group, p.tiles_per_batch)) {
                 const int b = tw.b;
                 const int p0 = tw.t * 128;
+                if (SKIP && tile_masked_out(p.ext, b, p0, p.N, p.NN, p.rowdiv)) continue;   // nothing to load
                 for (int c = 0; c < C::CPT; ++c) {
                     if (!mbar_wait(&s.empty[stage], phase ^ 1, abort_flag, kErrTimeoutProducer)) goto producer_abort;
                     uint8_t *dst = chunks + stage * C::CHUNK;
@@ -174,7 +177,9 @@ __global__ void __launch_bounds__(576, 1) k3_output_kernel(const __grid_constant
             uint32_t phase = 0;
             int abuf = 0;
             uint32_t aphase = 0;
-            for (int pt = cta_in_group; ok && pt < num_ptiles; pt += ctas_per_group) {
+            TileWalk tw(cta_in_group, p.tiles_per_batch);
+            for (int pt = cta_in_group; ok && pt < num_ptiles; pt += ctas_per_group, tw.advance(ctas_per_group, p.tiles_per_batch)) {
+                if (SKIP && tile_masked_out(p.ext, tw.b, tw.t * 128, p.N, p.NN, p.rowdiv)) continue;
                 if (!mbar_wait(&s.tempty[abuf], aphase ^ 1, abort_flag, kErrTimeoutMma)) break;
                 tc_fence_after();
                 const uint32_t d1 = tmem_base + abuf * 256;     // x . W_o'
@@ -229,6 +234,7 @@ __global__ void __launch_bounds__(576, 1) k3_output_kernel(const __grid_constant
         for (int pt = cta_in_group; pt < num_ptiles; pt += ctas_per_group, tw.advance(ctas_per_group, p.tiles_per_batch)) {
             const int b = tw.b;
             const int p0 = tw.t * 128;
+            if (SKIP && tile_masked_out(p.ext, b, p0, p.N, p.NN, p.rowdiv)) continue;
             const long long pi = (long long)p0 + row;
             uint16_t mbits = 0x3F80u;      // bf16 1.0; issued first so its latency overlaps the sums
             if (!xrole && p.mask) mbits = (pi < p.NN) ? p.mask[(long long)b * p.NN + pi] : (uint16_t)0;
@@ -367,6 +373,23 @@ __global__ void __launch_bounds__(576, 1) k3_output_kernel(const __grid_constant
         for (int pt = cta_in_group; pt < num_ptiles; pt += ctas_per_group, tw.advance(ctas_per_group, p.tiles_per_batch)) {
             const int b = tw.b;
             const int p0 = tw.t * 128;
+            if (SKIP && tile_masked_out(p.ext, b, p0, p.N, p.NN, p.rowdiv)) {
+                // every pair of the tile is masked: out is 0 there
+#pragma unroll 1
+                for (int sc = 0; sc < 64 / C::COLS_PER_STORE; ++sc) {
+                    if (lane == 0) tma_store_wait_read<0>();
+                    __syncwarp();
+#pragma unroll
+                    for (int u = 0; u < 8; ++u) *reinterpret_cast<uint4 *>(stg + sw128_offset(row, u)) = make_uint4(0, 0, 0, 0);
+                    fence_proxy_async_smem();
+                    __syncwarp();
+                    if (lane == 0 && p0 + q * 32 < p.NN) {
+                        tma_store_3d(&p.tm_out, wstg, n0 + wg * 64 + sc * C::COLS_PER_STORE, p0 + q * 32, b);
+                        tma_store_commit();
+                    }
+                }
+                continue;
+            }
             if (!__all_sync(0xffffffffu, mbar_wait(&s.sfull[sbuf], sphase, abort_flag, kErrTimeoutEpilogue))) break;
             const K3Stats st = stats[sbuf * 128 + row];
             const float2 nmx = make_float2(st.nmean_x, st.nmean_x), rx = make_float2(st.rstd_x, st.rstd_x);
@@ -487,25 +510,31 @@ size_t k3_smem_bytes(int c_z, bool out_f32) {
     return out_f32 ? K3Cfg<384, true>::SMEM : K3Cfg<384, false>::SMEM;
 }
 
-template <int CZ, bool F32, bool RES>
+template <int CZ, bool F32, bool RES, bool SKIP>
 static cudaError_t k3_launch_t(const K3Args &args, int grid, cudaStream_t stream) {
     static int configured_device = -1;
     int dev = 0;
     cudaGetDevice(&dev);
     if (configured_device != dev) {
-        cudaError_t e = cudaFuncSetAttribute(k3_output_kernel<CZ, F32, RES>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                             (int)K3Cfg<CZ, F32>::SMEM);
+        cudaError_t e = cudaFuncSetAttribute(k3_output_kernel<CZ, F32, RES, SKIP>,
+                                             cudaFuncAttributeMaxDynamicSharedMemorySize, (int)K3Cfg<CZ, F32>::SMEM);
         if (e != cudaSuccess) return e;
         configured_device = dev;
     }
-    return launch_pdl(k3_output_kernel<CZ, F32, RES>, grid, K3Cfg<CZ, F32>::THREADS, K3Cfg<CZ, F32>::SMEM, stream, args);
+    return launch_pdl(k3_output_kernel<CZ, F32, RES, SKIP>, grid, K3Cfg<CZ, F32>::THREADS, K3Cfg<CZ, F32>::SMEM, stream,
+                      args);
 }
 
 template <int CZ>
 static cudaError_t k3_launch_cz(bool out_f32, const K3Args &args, int grid, cudaStream_t stream) {
     if (args.zres)
-        return out_f32 ? k3_launch_t<CZ, true, true>(args, grid, stream) : k3_launch_t<CZ, false, true>(args, grid, stream);
-    return out_f32 ? k3_launch_t<CZ, true, false>(args, grid, stream) : k3_launch_t<CZ, false, false>(args, grid, stream);
+        return out_f32 ? k3_launch_t<CZ, true, true, false>(args, grid, stream)
+                       : k3_launch_t<CZ, false, true, false>(args, grid, stream);
+    if (args.ext)
+        return out_f32 ? k3_launch_t<CZ, true, false, true>(args, grid, stream)
+                       : k3_launch_t<CZ, false, false, true>(args, grid, stream);
+    return out_f32 ? k3_launch_t<CZ, true, false, false>(args, grid, stream)
+                   : k3_launch_t<CZ, false, false, false>(args, grid, stream);
 }
 
 cudaError_t k3_launch(int c_z, bool out_f32, const K3Args &args, int grid, cudaStream_t stream) {

@@ -23,6 +23,8 @@ struct K1Args {
     long long NN;
     int tiles_per_batch;   // ceil(NN / 128)
     float eps;
+    const int *ext;        // mask extents [B][2] {R_b, C_b} (tiles wholly beyond them skipped), or nullptr
+    uint64_t rowdiv;       // multiplier dividing by N / 8 (div_by_magic)
 };
 
 struct K2Args {
@@ -32,6 +34,10 @@ struct K2Args {
     bool incoming;
     bool f16;              // operands and result in fp16 (else bf16)
     float x_scale;         // result = x_scale * sum_k ...
+    const int *ext;        // mask extents [B][2] {R_b, C_b}, or nullptr: the sum runs over k < C_b
+                           // (outgoing) or k < R_b (incoming); output tiles at rows >= R_b or
+                           // columns >= C_b are not written (the output kernel never reads them)
+    int C;                 // channels per batch element (bc / C = batch element)
 };
 
 struct K3Args {
@@ -48,6 +54,8 @@ struct K3Args {
     float eps;             // input LayerNorm
     float eps_x;           // output LayerNorm on the stored (scaled) x: eps * x_scale^2
     const uint16_t *zres;  // residual: z (bf16, [B][N*N][c_z]) added to the output; null = none
+    const int *ext;        // mask extents (as K1Args); ignored with a residual (masked pairs then copy z)
+    uint64_t rowdiv;
 };
 
 // Launch with programmatic stream serialization: the kernel may begin while the previous
@@ -79,6 +87,15 @@ int k1_row_mode(int c_z);
 
 size_t k2_smem_bytes();
 cudaError_t k2_launch(const K2Args &args, int grid, cudaStream_t stream);
+
+// Mask extents {R_b, C_b} into ext[2B] (zeroed first), for a bf16 mask [B][N*N]; rowdiv
+// divides by N / 8 (host_rowdiv).
+cudaError_t mask_extents_launch(const uint16_t *mask, int B, int N, uint64_t rowdiv, int *ext, cudaStream_t stream);
+
+// Multiplier for div_by_magic dividing by d >= 1, or 0 for d = 1: floor((2^64 - 1) / d) + 1,
+// which is floor(2^64 / d) + 1 when d does not divide 2^64 and exactly 2^64 / d when it does
+// (then the division is exact outright).
+inline uint64_t host_rowdiv(uint64_t d) { return d <= 1 ? 0 : ~0ull / d + 1; }
 
 size_t k3_smem_bytes(int c_z, bool out_f32);
 int k3_groups(int c_z);

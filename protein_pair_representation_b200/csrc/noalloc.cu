@@ -58,8 +58,10 @@ extern "C" trimul_status_t tri_mul_forward_noalloc(const trimul_pair_t *z, const
     if (direction != TRIMUL_OUTGOING && direction != TRIMUL_INCOMING)
         return trimul::set_last_error(TRIMUL_ERR_INVALID_ARG, "unknown direction");
     // a, b and x: three planes, the same layout tri_mul_forward uses in a bound workspace
-    const size_t need = tri_mul_workspace_bytes(layer, z->B, z->N, z->dtype);
-    if (need == 0) return trimul::set_last_error(TRIMUL_ERR_INVALID_ARG, "invalid layer or size");
+    // (which also holds the mask extents after them; this path skips no tiles and needs none)
+    const size_t ws = tri_mul_workspace_bytes(layer, z->B, z->N, z->dtype);
+    if (ws == 0) return trimul::set_last_error(TRIMUL_ERR_INVALID_ARG, "invalid layer or size");
+    const size_t need = ws - (((size_t)z->B * 2 * sizeof(int) + 255) & ~size_t(255));
     if (need > (size_t)TRIMUL_NOALLOC_SCRATCH_BYTES)
         return trimul::set_last_error(TRIMUL_ERR_WORKSPACE,
                                       "problem needs more intermediate memory than the built-in "

@@ -41,6 +41,7 @@ struct trimul_layer {
     size_t ws_bytes;
     cudaEvent_t events[4];
     bool timing;
+    bool skip_masked;            // find mask extents and leave out wholly masked tiles
 };
 
 // ------------------------------------------------------------------ error plumbing
@@ -330,9 +331,12 @@ static size_t ws_plane_bytes(int64_t B, int64_t N, int c_h, trimul_dtype_t dt) {
     return (((size_t)B * c_h * N * N * dtype_size(dt)) + 255) & ~size_t(255);
 }
 
+// The mask extents {R_b, C_b} (int32) of a forward, after the three planes.
+static size_t ws_ext_bytes(int64_t B) { return ((size_t)B * 2 * sizeof(int) + 255) & ~size_t(255); }
+
 extern "C" size_t tri_mul_workspace_bytes(const trimul_layer_t *L, int64_t B, int64_t N, trimul_dtype_t dt) {
     if (!L || B < 1 || N < 1 || (dt != TRIMUL_F32 && dt != TRIMUL_BF16)) return 0;
-    return 3 * ws_plane_bytes(B, N, L->c_h, dt);
+    return 3 * ws_plane_bytes(B, N, L->c_h, dt) + ws_ext_bytes(B);
 }
 
 extern "C" trimul_status_t tri_mul_layer_bind_workspace(trimul_layer_t *L, void *ws, size_t bytes) {
@@ -359,6 +363,12 @@ extern "C" trimul_status_t tri_mul_layer_set_timing_events(trimul_layer_t *L, vo
 
 extern "C" int tri_mul_kernels_per_forward(void) { return 3; }
 
+extern "C" trimul_status_t tri_mul_layer_set_mask_skipping(trimul_layer_t *L, int enable) {
+    if (!L) return fail(TRIMUL_ERR_INVALID_ARG, "layer is NULL");
+    L->skip_masked = enable != 0;
+    return TRIMUL_OK;
+}
+
 // ------------------------------------------------------------------ kernel drivers
 
 static int grid_for(int sms, long long work_units, int multiple) {
@@ -369,7 +379,7 @@ static int grid_for(int sms, long long work_units, int multiple) {
 }
 
 static trimul_status_t run_project_bf16(const trimul_layer_t *L, const void *z, const void *mask, void *a, void *b,
-                                        int B, int N, cudaStream_t st) {
+                                        int B, int N, cudaStream_t st, const int *ext) {
     DeviceInfo d;
     TRY(require_sm100(&d));
     const uint64_t NN = (uint64_t)N * N;
@@ -406,6 +416,8 @@ static trimul_status_t run_project_bf16(const trimul_layer_t *L, const void *z, 
     p.NN = (long long)NN;
     p.tiles_per_batch = (int)((NN + 127) / 128);
     p.eps = L->eps;
+    p.ext = ext;
+    p.rowdiv = host_rowdiv((uint64_t)N / 8);
     const int G = k1_groups(cz);
     const int grid = grid_for(d.sms, (long long)G * B * p.tiles_per_batch, G);
     TRY_CUDA(k1_launch(cz, p, grid, st), "K1 launch");
@@ -413,7 +425,7 @@ static trimul_status_t run_project_bf16(const trimul_layer_t *L, const void *z, 
 }
 
 static trimul_status_t run_contract_tc(const void *a, const void *b, void *x, int64_t BC, int N, bool incoming,
-                                       bool f16, float x_scale, cudaStream_t st) {
+                                       bool f16, float x_scale, cudaStream_t st, const int *ext, int C) {
     DeviceInfo d;
     TRY(require_sm100(&d));
     K2Args p{};
@@ -435,6 +447,8 @@ static trimul_status_t run_contract_tc(const void *a, const void *b, void *x, in
     }
     p.f16 = f16;
     p.x_scale = x_scale;
+    p.ext = ext;
+    p.C = C;
     p.BC = (int)BC;
     p.N = N;
     p.m_tiles = (N + 127) / 128;
@@ -449,7 +463,7 @@ static trimul_status_t run_contract_tc(const void *a, const void *b, void *x, in
 
 static trimul_status_t run_output_bf16(const trimul_layer_t *L, const void *z, const void *mask, const void *x,
                                        float x_scale, void *out, bool out_f32, bool residual, int B, int N,
-                                       cudaStream_t st) {
+                                       cudaStream_t st, const int *ext) {
     DeviceInfo d;
     TRY(require_sm100(&d));
     const uint64_t NN = (uint64_t)N * N;
@@ -498,6 +512,8 @@ static trimul_status_t run_output_bf16(const trimul_layer_t *L, const void *z, c
     p.eps = L->eps;
     p.eps_x = L->eps * x_scale * x_scale;
     p.zres = residual ? reinterpret_cast<const uint16_t *>(z) : nullptr;
+    p.ext = residual ? nullptr : ext;        // with a residual a masked pair copies z: nothing is skipped
+    p.rowdiv = host_rowdiv((uint64_t)N / 8);
     const int G = k3_groups(cz);
     const int grid = grid_for(d.sms, (long long)G * B * p.tiles_per_batch, G);
     TRY_CUDA(k3_launch(cz, out_f32, p, grid, st), "K3 launch");
@@ -506,8 +522,8 @@ static trimul_status_t run_output_bf16(const trimul_layer_t *L, const void *z, c
 
 // ------------------------------------------------------------------ public entry points
 
-extern "C" trimul_status_t tri_mul_project(const trimul_pair_t *z, const void *mask, const trimul_layer_t *L, void *a_out,
-                                           void *b_out, void *stream) {
+static trimul_status_t project_impl(const trimul_pair_t *z, const void *mask, const trimul_layer_t *L, void *a_out,
+                                    void *b_out, const int *ext, void *stream) {
     TRY(check_problem(z, mask, L));
     if (!a_out || !b_out) return fail(TRIMUL_ERR_INVALID_ARG, "a_out / b_out NULL");
     if (!aligned16(a_out) || !aligned16(b_out)) return fail(TRIMUL_ERR_ALIGNMENT, "a_out / b_out not 16-byte aligned");
@@ -517,12 +533,17 @@ extern "C" trimul_status_t tri_mul_project(const trimul_pair_t *z, const void *m
         return fail(TRIMUL_ERR_INVALID_ARG, "a_out, b_out and z overlap");
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
     if (z->dtype == TRIMUL_BF16)
-        return run_project_bf16(L, z->data, mask, a_out, b_out, (int)z->B, (int)z->N, st);
+        return run_project_bf16(L, z->data, mask, a_out, b_out, (int)z->B, (int)z->N, st, ext);
     TRY_CUDA(f32_project_launch(reinterpret_cast<const float *>(z->data), reinterpret_cast<const float *>(mask), L->f32,
                                 L->c_z, L->c_h, (int)z->B, (int)z->N, L->eps, reinterpret_cast<float *>(a_out),
                                 reinterpret_cast<float *>(b_out), st),
              "fp32 projection launch");
     return TRIMUL_OK;
+}
+
+extern "C" trimul_status_t tri_mul_project(const trimul_pair_t *z, const void *mask, const trimul_layer_t *L, void *a_out,
+                                           void *b_out, void *stream) {
+    return project_impl(z, mask, L, a_out, b_out, nullptr, stream);
 }
 
 extern "C" float tri_mul_contract_scale(int64_t N) {
@@ -532,8 +553,9 @@ extern "C" float tri_mul_contract_scale(int64_t N) {
     return ldexpf(1.0f, -((lg + 1) / 2));       // 2^-ceil(log2(N) / 2)
 }
 
-extern "C" trimul_status_t tri_mul_contract(const void *a, const void *b, void *x, int64_t B, int64_t C, int64_t N,
-                                            trimul_dtype_t dtype, trimul_direction_t dir, float x_scale, void *stream) {
+static trimul_status_t contract_impl(const void *a, const void *b, void *x, int64_t B, int64_t C, int64_t N,
+                                     trimul_dtype_t dtype, trimul_direction_t dir, float x_scale, const int *ext,
+                                     void *stream) {
     if (!a || !b || !x) return fail(TRIMUL_ERR_INVALID_ARG, "NULL tensor");
     if (dtype != TRIMUL_F32 && dtype != TRIMUL_BF16 && dtype != TRIMUL_F16) return fail(TRIMUL_ERR_INVALID_ARG, "unknown dtype");
     if (!(x_scale > 0.f) || !(x_scale < 3.0e38f)) return fail(TRIMUL_ERR_INVALID_ARG, "x_scale must be positive and finite");
@@ -546,15 +568,22 @@ extern "C" trimul_status_t tri_mul_contract(const void *a, const void *b, void *
     if (overlap(x, bytes, a, bytes) || overlap(x, bytes, b, bytes)) return fail(TRIMUL_ERR_INVALID_ARG, "x overlaps a or b");
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
     if (dtype != TRIMUL_F32)
-        return run_contract_tc(a, b, x, B * C, (int)N, dir == TRIMUL_INCOMING, dtype == TRIMUL_F16, x_scale, st);
+        return run_contract_tc(a, b, x, B * C, (int)N, dir == TRIMUL_INCOMING, dtype == TRIMUL_F16, x_scale, st, ext,
+                               (int)C);
     TRY_CUDA(f32_contract_launch(reinterpret_cast<const float *>(a), reinterpret_cast<const float *>(b),
                                  reinterpret_cast<float *>(x), (int)(B * C), (int)N, dir == TRIMUL_INCOMING, x_scale, st),
              "fp32 contraction launch");
     return TRIMUL_OK;
 }
 
+extern "C" trimul_status_t tri_mul_contract(const void *a, const void *b, void *x, int64_t B, int64_t C, int64_t N,
+                                            trimul_dtype_t dtype, trimul_direction_t dir, float x_scale, void *stream) {
+    return contract_impl(a, b, x, B, C, N, dtype, dir, x_scale, nullptr, stream);
+}
+
 static trimul_status_t output_gate_impl(const trimul_pair_t *z, const void *mask, const void *x, float x_scale,
-                                        const trimul_layer_t *L, trimul_pair_t *out, bool residual, void *stream) {
+                                        const trimul_layer_t *L, trimul_pair_t *out, bool residual, const int *ext,
+                                        void *stream) {
     TRY(check_problem(z, mask, L));
     if (!(x_scale > 0.f) || !(x_scale < 3.0e38f)) return fail(TRIMUL_ERR_INVALID_ARG, "x_scale must be positive and finite");
     TRY(check_pair(out, "out"));
@@ -568,7 +597,7 @@ static trimul_status_t output_gate_impl(const trimul_pair_t *z, const void *mask
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
     if (z->dtype == TRIMUL_BF16)
         return run_output_bf16(L, z->data, mask, x, x_scale, out->data, out->dtype == TRIMUL_F32, residual, (int)z->B,
-                               (int)z->N, st);
+                               (int)z->N, st, ext);
     TRY_CUDA(f32_output_launch(reinterpret_cast<const float *>(z->data), reinterpret_cast<const float *>(mask),
                                reinterpret_cast<const float *>(x), L->f32, L->c_z, L->c_h, (int)z->B, (int)z->N, L->eps,
                                L->eps * x_scale * x_scale, residual, reinterpret_cast<float *>(out->data), st),
@@ -578,7 +607,7 @@ static trimul_status_t output_gate_impl(const trimul_pair_t *z, const void *mask
 
 extern "C" trimul_status_t tri_mul_output_gate(const trimul_pair_t *z, const void *mask, const void *x, float x_scale,
                                                const trimul_layer_t *L, trimul_pair_t *out, void *stream) {
-    return output_gate_impl(z, mask, x, x_scale, L, out, false, stream);
+    return output_gate_impl(z, mask, x, x_scale, L, out, false, nullptr, stream);
 }
 
 static trimul_status_t forward_impl(const trimul_pair_t *z, const void *mask, const trimul_layer_t *L,
@@ -589,22 +618,30 @@ static trimul_status_t forward_impl(const trimul_pair_t *z, const void *mask, co
     if (out->B != z->B || out->N != z->N || out->C != z->C) return fail(TRIMUL_ERR_INVALID_ARG, "out shape differs from z");
     if (z->dtype == TRIMUL_F32 && out->dtype != TRIMUL_F32) return fail(TRIMUL_ERR_INVALID_ARG, "fp32 path writes fp32 out");
     const size_t plane = ws_plane_bytes(z->B, z->N, L->c_h, z->dtype);
-    if (!L->ws || L->ws_bytes < 3 * plane)
-        return fail(TRIMUL_ERR_WORKSPACE, "workspace of %zu bytes needed, %zu bound", 3 * plane, L->ws_bytes);
+    const size_t need = 3 * plane + ws_ext_bytes(z->B);
+    if (!L->ws || L->ws_bytes < need)
+        return fail(TRIMUL_ERR_WORKSPACE, "workspace of %zu bytes needed, %zu bound", need, L->ws_bytes);
     if (overlap(out->data, pair_bytes(out), z->data, pair_bytes(z))) return fail(TRIMUL_ERR_INVALID_ARG, "out overlaps z");
-    if (overlap(out->data, pair_bytes(out), L->ws, 3 * plane) || overlap(z->data, pair_bytes(z), L->ws, 3 * plane))
+    if (overlap(out->data, pair_bytes(out), L->ws, need) || overlap(z->data, pair_bytes(z), L->ws, need))
         return fail(TRIMUL_ERR_INVALID_ARG, "z or out overlaps the workspace");
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
     uint8_t *ws = reinterpret_cast<uint8_t *>(L->ws);
     void *a = ws, *b = ws + plane, *x = ws + 2 * plane;
-    if (L->timing) TRY_CUDA(cudaEventRecord(L->events[0], st), "event record");
-    TRY(tri_mul_project(z, mask, L, a, b, stream));
-    if (L->timing) TRY_CUDA(cudaEventRecord(L->events[1], st), "event record");
     const bool tc = z->dtype == TRIMUL_BF16;
+    // tensor-core path with a mask, skipping switched on: the mask's extents let the kernels
+    // leave out wholly masked tiles
+    int *ext = (tc && mask && L->skip_masked) ? reinterpret_cast<int *>(ws + 3 * plane) : nullptr;
+    if (ext)
+        TRY_CUDA(mask_extents_launch(reinterpret_cast<const uint16_t *>(mask), (int)z->B, (int)z->N,
+                                     host_rowdiv((uint64_t)z->N / 8), ext, st),
+                 "mask extents launch");
+    if (L->timing) TRY_CUDA(cudaEventRecord(L->events[0], st), "event record");
+    TRY(project_impl(z, mask, L, a, b, ext, stream));
+    if (L->timing) TRY_CUDA(cudaEventRecord(L->events[1], st), "event record");
     const float x_scale = tc ? tri_mul_contract_scale(z->N) : 1.0f;
-    TRY(tri_mul_contract(a, b, x, z->B, L->c_h, z->N, tc ? TRIMUL_F16 : TRIMUL_F32, dir, x_scale, stream));
+    TRY(contract_impl(a, b, x, z->B, L->c_h, z->N, tc ? TRIMUL_F16 : TRIMUL_F32, dir, x_scale, ext, stream));
     if (L->timing) TRY_CUDA(cudaEventRecord(L->events[2], st), "event record");
-    TRY(output_gate_impl(z, mask, x, x_scale, L, out, residual, stream));
+    TRY(output_gate_impl(z, mask, x, x_scale, L, out, residual, ext, stream));
     if (L->timing) TRY_CUDA(cudaEventRecord(L->events[3], st), "event record");
     return TRIMUL_OK;
 }

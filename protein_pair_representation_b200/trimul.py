@@ -91,6 +91,7 @@ def load_library():
         lib.tri_mul_contract_scale.restype = ctypes.c_float
         lib.tri_mul_output_gate.argtypes = [P(_Pair), vp, vp, ctypes.c_float, vp, P(_Pair), vp]
         lib.tri_mul_layer_set_timing_events.argtypes = [vp, P(vp)]
+        lib.tri_mul_layer_set_mask_skipping.argtypes = [vp, st]
         lib.tri_mul_kernels_per_forward.argtypes = []
         lib.tri_mul_check_device_status.argtypes = []
         lib.tri_mul_status_string.argtypes = [st]
@@ -100,7 +101,7 @@ def load_library():
         lib.tri_mul_abi_version.argtypes = []
         for name in ("tri_mul_layer_create", "tri_mul_layer_bind_workspace", "tri_mul_forward",
                      "tri_mul_forward_residual", "tri_mul_pair_update", "tri_mul_pair_update_graph_create",
-                     "tri_mul_graph_launch",
+                     "tri_mul_graph_launch", "tri_mul_layer_set_mask_skipping",
                      "tri_mul_project", "tri_mul_contract", "tri_mul_output_gate",
                      "tri_mul_layer_set_timing_events", "tri_mul_check_device_status"):
             getattr(lib, name).restype = ctypes.c_int
@@ -215,6 +216,10 @@ class TriMulLayer:
         need = self.workspace_bytes(B, N, dtype)
         if self._ws is None or self._ws.numel() < need:
             self.bind_workspace(torch.empty(need, dtype=torch.uint8, device=self.device))
+
+    def set_mask_skipping(self, enable: bool = True):
+        """Leave out wholly masked tiles (mask extents found by a first pass); off by default."""
+        _check(self._lib.tri_mul_layer_set_mask_skipping(self.handle, 1 if enable else 0))
 
     def set_timing_events(self, events):
         """events: four torch.cuda.Event(enable_timing=True) or None."""

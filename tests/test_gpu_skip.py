@@ -1,0 +1,69 @@
+"""Skipping of wholly masked tiles (needs a B200).
+
+With mask skipping switched on, tri_mul_forward with a mask finds the mask's extents and
+leaves out tiles that are masked in full and the k-range beyond them; the stage entry points
+(project, contract, output_gate) called one by one skip nothing. Every product left out is an exact zero, so the two must
+agree bitwise, for masks of any pattern (here: a valid block [0, R) x [0, C) with R != C and
+random holes inside it, the second batch element with the block transposed), and both must
+match the oracle.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import trimul_inputs as ti
+from gpu_helpers import assert_close_rms, upload
+from protein_pair_representation_b200 import trimul as tm
+
+pytestmark = pytest.mark.gpu
+
+
+def _holey_mask(N, R, C, seed):
+    rng = np.random.default_rng(seed)
+    m = np.zeros((2, N, N), dtype=np.float32)
+    m[0, :R, :C] = rng.random((R, C)) > 0.1
+    m[1, :C, :R] = rng.random((C, R)) > 0.1
+    return m
+
+
+@pytest.mark.parametrize("N,R,C,c_z,check_oracle", [
+    (256, 100, 100, 128, True),     # rows and k-chunks past 100 left out; an output m-tile too
+    (256, 130, 70, 128, True),      # R != C: outgoing and incoming bound k differently
+    (136, 100, 60, 128, True),      # N % 128 != 0: tiles straddle rows, no output tile skipped
+    (128, 60, 90, 384, True),       # c_z = 384 kernels
+    (512, 493, 200, 128, False),    # headline size, columns cut short
+])
+def test_forward_with_extents_matches_stages_bitwise(N, R, C, c_z, check_oracle):
+    inp = ti.generate(2, N, c_z, 128, dtype="bf16", seed=N + R + C, mask=("all",), biases=True)
+    inp.mask = _holey_mask(N, R, C, seed=R * C)
+    z, m, w = upload(inp)
+    layer = tm.TriMulLayer(w, eps=inp.eps)
+    layer.set_mask_skipping(True)
+    scale = tm.contract_scale(N)
+    for d in ("outgoing", "incoming"):
+        full = layer.forward(z, m, d)
+        a, b = layer.project(z, m)
+        x = tm.contract(a, b, d, x_scale=scale)
+        staged = layer.output_gate(z, x, m, x_scale=scale)
+        torch.cuda.synchronize()
+        tm.check_device_status()
+        assert torch.equal(full, staged), d
+        got = full.cpu().numpy()
+        assert not np.any(got[inp.mask == 0]), "masked pairs must be exactly 0"
+        if check_oracle:
+            ref = oracle.trimul(inp.z, inp.mask, inp.weights, d, inp.eps)
+            assert_close_rms(got, ref, 2e-2, what=f"N={N} R={R} C={C} {d}")
+
+
+def test_all_masked_element_next_to_a_full_one():
+    inp = ti.generate(2, 256, 128, 128, dtype="bf16", seed=3, mask=("lengths", [0, 256]))
+    z, m, w = upload(inp)
+    layer = tm.TriMulLayer(w, eps=inp.eps)
+    layer.set_mask_skipping(True)
+    for d in ("outgoing", "incoming"):
+        got = layer.forward(z, m, d)
+        torch.cuda.synchronize()
+        tm.check_device_status()
+        assert not torch.any(got[0])
+        assert torch.isfinite(got[1]).all()
