@@ -51,6 +51,7 @@ def parse_args():
     ap.add_argument("--no-cpu-baseline", action="store_true", help="skip timing the CPU oracle")
     ap.add_argument("--skip-masked", action="store_true",
                     help="switch mask skipping on (leave out wholly masked tiles; off by default)")
+    ap.add_argument("--no-transition", action="store_true", help="skip the pair-transition leg")
     ap.add_argument("--no-pair-update", action="store_true",
                     help="skip the pair-update leg (outgoing + incoming with residuals, eager and as a CUDA graph)")
     return ap.parse_args()
@@ -275,6 +276,43 @@ def pair_update_leg(tm, layer, zs, ms_, n_sets, args, dev):
         return {"error": f"{type(exc).__name__}: {exc}"}
 
 
+def transition_leg(tm, zs, ms_, n_sets, args, dev):
+    """The fused pair transition (out = z + m (relu(z W1^T + b1) W2^T + b2), c = 128, hidden 256)
+    on this rank's pair tensors, bf16 in and out, seeded random weights; per-call ms from CUDA
+    events over `steps` calls, inputs cycling through the L2-defeating copies."""
+    import numpy as np
+    import torch
+    try:
+        rng = np.random.default_rng(1234)
+        mk = lambda *shape, scale: torch.from_numpy((rng.standard_normal(shape) * scale).astype(np.float32)).to(
+            dev).to(torch.bfloat16)
+        pt = tm.PairTransition(mk(256, 128, scale=128 ** -0.5), mk(128, 256, scale=256 ** -0.5),
+                               mk(256, scale=0.1), mk(128, scale=0.1))
+        outs = [torch.empty_like(zs[0]) for _ in range(n_sets)]
+        for s_ in range(max(3, args.warmup)):
+            pt.forward(zs[s_ % n_sets], ms_[s_ % n_sets], out=outs[s_ % n_sets])
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        for s_ in range(args.steps):
+            pt.forward(zs[s_ % n_sets], ms_[s_ % n_sets], out=outs[s_ % n_sets])
+        e1.record()
+        torch.cuda.synchronize()
+        tm.check_device_status()
+        ms = e0.elapsed_time(e1) / args.steps
+        P = zs[0].shape[0] * zs[0].shape[1] * zs[0].shape[2]
+        nbytes = P * (2 * 128 + 2 + 2 * 128)           # z in, mask, out (bf16)
+        flops = P * 2 * 2 * 128 * 256
+        peaks = measured_peaks()
+        gbs, tfs = nbytes / (ms * 1e-3) / 1e9, flops / (ms * 1e-3) / 1e12
+        pt.close()
+        return {"ms": ms, "GB_s": gbs, "TFLOP_s": tfs, "hbm_frac": gbs / peaks["hbm_gbs"],
+                "tensor_frac": tfs / peaks["bf16_tflops"], "bytes": nbytes, "flops": flops,
+                "shape": "c=128, hidden=256, bf16 in/out, fp16 hidden activation on chip"}
+    except Exception as exc:       # the headline line must not depend on this leg
+        return {"error": f"{type(exc).__name__}: {exc}"}
+
+
 def workload_config(inp, compute):
     lengths = [int(v) for v in inp.lengths]
     mask = "all-ones mask" if min(lengths) == inp.N else f"ragged mask (L={lengths if inp.B > 1 else lengths[0]})"
@@ -392,6 +430,7 @@ def run_ours(args):
                "d2h_bytes_per_step": sum(o.numel() * o.element_size() for o in out_host)}
 
     pair = None if args.no_pair_update else pair_update_leg(tm, layer, zs, ms_, n_sets, args, dev)
+    trans = None if (args.no_transition or inp.c_z != 128) else transition_leg(tm, zs, ms_, n_sets, args, dev)
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline and args.workload in CPU_BASELINE_WORKLOADS:
@@ -443,6 +482,7 @@ def run_ours(args):
         "effective_tflops": sum(flops.values()) / (layer_ms_single * 1e-3) / 1e12 * world,
         "layer_roofline_frac": t_ideal / (layer_ms_single * 1e-3),
         "roofline": roof, "kernels": kernels, "cpu_baseline": cpu, "e2e": e2e, "pair_update": pair,
+        "pair_transition": trans,
         "gpu_launches": args.steps * len(dirs) * (tm.kernels_per_forward() + (1 if args.skip_masked else 0)),
         "clocks": clock_info,
     }

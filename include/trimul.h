@@ -249,6 +249,26 @@ void tri_mul_graph_destroy(trimul_graph_t *graph);
  * (valid lengths 162-237) 8% faster and B=1 N=512 c_z=128 (493 of 512 valid) 9% slower. */
 trimul_status_t tri_mul_layer_set_mask_skipping(trimul_layer_t *layer, int enable);
 
+/* The fused pair transition, the step that follows the two triangle updates in a pair
+ * update ("RFProteina architecture", section "Kernel support": one launch runs both linears,
+ * the ReLU, the mask and the residual and keeps the hidden activation on chip):
+ *   out_ij = z_ij + m_ij * (relu(z_ij . W1^T + b1) . W2^T + b2)
+ * Weights [out, in] as for the triangle layer: W1 [hidden, c], b1 [hidden], W2 [c, hidden],
+ * b2 [c]; biases may be NULL (0). Supported: bf16, c = 128, hidden = 256 (the pages' expansion
+ * of 2); anything else returns TRIMUL_ERR_UNSUPPORTED_SHAPE. Creation copies the weights
+ * into the handle (biases kept in fp32) and synchronizes `stream`. The forward takes z
+ * [B, N, N, 128] bf16, a mask as tri_mul_forward, and writes out [B, N, N, 128] in F32 or
+ * BF16 (not overlapping z); fp32 accumulation, the hidden activation rounded to f16 on
+ * chip (W2 kept in f16 for that product); N % 8 == 0; sm_100 only. */
+typedef struct trimul_transition trimul_transition_t;
+trimul_status_t tri_mul_transition_create(int c, int hidden, trimul_dtype_t dtype, const void *w1,
+                                          const void *b1, const void *w2, const void *b2,
+                                          void *stream, trimul_transition_t **transition_out);
+void tri_mul_transition_destroy(trimul_transition_t *transition);
+trimul_status_t tri_mul_transition_forward(const trimul_pair_t *z, const void *mask,
+                                           const trimul_transition_t *transition,
+                                           trimul_pair_t *out, void *stream);
+
 /* Optional per-kernel timing: when `events` is non-NULL, every later
  * tri_mul_forward on this handle records events[0] before K1 (after the mask-extents
  * pass), events[1] after

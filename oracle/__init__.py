@@ -210,3 +210,22 @@ def pair_update(z, mask, weights_out, weights_in, eps=1e-5, lib=None):
     z_mid = z + trimul(z, mask, weights_out, "outgoing", eps, lib=lib)
     out = z_mid + trimul(z_mid, mask, weights_in, "incoming", eps, lib=lib)
     return z_mid, out
+
+
+def pair_transition(z, mask, w1, b1, w2, b2):
+    """The fused pair transition, in fp64 ("RFProteina architecture", section "Kernel support":
+    both linears, the ReLU, the mask and the residual in one step):
+        out_ij = z_ij + m_ij * (relu(z_ij . W1^T + b1) . W2^T + b2)
+    z [B, N, N, c], mask [B, N, N] (None: all ones), W1 [h, c], b1 [h], W2 [c, h], b2 [c]
+    (None biases: 0). A masked pair keeps its z bitwise."""
+    z = _f64(z)
+    hid = z @ _f64(w1).T
+    if b1 is not None:
+        hid = hid + _f64(b1)
+    hid = np.maximum(hid, 0.0)
+    upd = hid @ _f64(w2).T
+    if b2 is not None:
+        upd = upd + _f64(b2)
+    if mask is not None:
+        upd = upd * _f64(mask)[..., None]
+    return z + upd

@@ -88,6 +88,23 @@ int k1_row_mode(int c_z);
 size_t k2_smem_bytes();
 cudaError_t k2_launch(const K2Args &args, int grid, cudaStream_t stream);
 
+// The fused pair transition (c = 128, hidden 256): out = z + m * (relu(z W1^T + b1) W2^T + b2).
+struct PtArgs {
+    CUtensorMap tm_z;      // z [B][N*N][128] bf16 viewed {64 ch, N*N, 2 halves, B}, box {64, 64, 2, 1}, 128B swizzle
+    CUtensorMap tm_w1;     // W1 [256][128] bf16, box {64, 256}, 128B swizzle
+    CUtensorMap tm_w2;     // W2 [128][256] f16, box {64, 128}, 128B swizzle
+    CUtensorMap tm_out;    // out [B][N*N][128] f32 or bf16, box {128, 32, 1}, no swizzle
+    const uint16_t *mask;  // [B][N*N] bf16 bits, or nullptr
+    const float *b1;       // [256] fp32 (zeros when the layer has no bias)
+    const float *b2;       // [128] fp32
+    int B;
+    long long NN;
+    int tiles_per_batch;   // NN / 64
+};
+cudaError_t pt_launch(bool out_f32, const PtArgs &args, int grid, cudaStream_t stream);
+cudaError_t bf16_to_f16_launch(const void *src, void *dst, long long n, cudaStream_t stream);
+size_t pt_smem_bytes(bool out_f32);
+
 // Mask extents {R_b, C_b} into ext[2B] (zeroed first), for a bf16 mask [B][N*N]; rowdiv
 // divides by N / 8 (host_rowdiv).
 cudaError_t mask_extents_launch(const uint16_t *mask, int B, int N, uint64_t rowdiv, int *ext, cudaStream_t stream);

@@ -778,6 +778,124 @@ extern "C" trimul_status_t tri_mul_check_device_status(void) {
     return TRIMUL_OK;
 }
 
+// ------------------------------------------------------------------ pair transition
+
+struct trimul_transition {
+    int c, hidden;
+    void *mem;                   // W1 [hidden][c] bf16, W2 [c][hidden] f16, b1 [hidden] f32, b2 [c] f32
+    uint16_t *w1, *w2;
+    float *b1, *b2;
+    CUtensorMap tm_w1, tm_w2;
+};
+
+extern "C" trimul_status_t tri_mul_transition_create(int c, int hidden, trimul_dtype_t dtype, const void *w1,
+                                                     const void *b1, const void *w2, const void *b2, void *stream,
+                                                     trimul_transition_t **out) {
+    if (!out) return fail(TRIMUL_ERR_INVALID_ARG, "out is NULL");
+    *out = nullptr;
+    if (!w1 || !w2) return fail(TRIMUL_ERR_INVALID_ARG, "W1 and W2 are required");
+    if (dtype != TRIMUL_BF16) return fail(TRIMUL_ERR_UNSUPPORTED_SHAPE, "the pair transition runs on bf16 weights");
+    if (c != 128 || hidden != 256)
+        return fail(TRIMUL_ERR_UNSUPPORTED_SHAPE, "pair transition supports c = 128, hidden = 256 (got %d, %d)", c, hidden);
+    DeviceInfo d;
+    TRY(require_sm100(&d));
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    trimul_transition *T = new (std::nothrow) trimul_transition();
+    if (!T) return fail(TRIMUL_ERR_INVALID_ARG, "out of host memory");
+    T->c = c;
+    T->hidden = hidden;
+    const size_t wbytes = (size_t)c * hidden * 2;
+    const size_t total = 2 * wbytes + (size_t)(hidden + c) * sizeof(float);
+    if (cudaMalloc(&T->mem, total) != cudaSuccess) {
+        delete T;
+        return fail(TRIMUL_ERR_CUDA, "cudaMalloc of %zu bytes failed", total);
+    }
+    uint8_t *m = reinterpret_cast<uint8_t *>(T->mem);
+    T->w1 = reinterpret_cast<uint16_t *>(m);
+    T->w2 = reinterpret_cast<uint16_t *>(m + wbytes);
+    T->b1 = reinterpret_cast<float *>(m + 2 * wbytes);
+    T->b2 = T->b1 + hidden;
+    trimul_status_t status = TRIMUL_OK;
+    cudaError_t e = cudaMemcpyAsync(T->w1, w1, wbytes, cudaMemcpyDeviceToDevice, st);
+    if (e == cudaSuccess) e = bf16_to_f16_launch(w2, T->w2, (long long)c * hidden, st);   // GEMM2 runs in f16
+    if (e == cudaSuccess) e = b1 ? to_f32_launch(b1, 1, T->b1, 1, hidden, 0, st) : cudaMemsetAsync(T->b1, 0, hidden * 4, st);
+    if (e == cudaSuccess) e = b2 ? to_f32_launch(b2, 1, T->b2, 1, c, 0, st) : cudaMemsetAsync(T->b2, 0, c * 4, st);
+    if (e == cudaSuccess) e = cudaStreamSynchronize(st);
+    if (e != cudaSuccess) status = cuda_fail(e, "transition weights copy");
+    if (status == TRIMUL_OK) {
+        uint64_t dims1[2] = {(uint64_t)c, (uint64_t)hidden}, strides1[1] = {(uint64_t)c * 2};
+        uint32_t box1[2] = {64, (uint32_t)hidden};
+        status = make_map(&T->tm_w1, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, T->w1, dims1, strides1, box1,
+                          CU_TENSOR_MAP_SWIZZLE_128B, "transition W1");
+    }
+    if (status == TRIMUL_OK) {
+        uint64_t dims2[2] = {(uint64_t)hidden, (uint64_t)c}, strides2[1] = {(uint64_t)hidden * 2};
+        uint32_t box2[2] = {64, (uint32_t)c};
+        status = make_map(&T->tm_w2, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, T->w2, dims2, strides2, box2,
+                          CU_TENSOR_MAP_SWIZZLE_128B, "transition W2");
+    }
+    if (status != TRIMUL_OK) {
+        cudaFree(T->mem);
+        delete T;
+        return status;
+    }
+    *out = T;
+    return TRIMUL_OK;
+}
+
+extern "C" void tri_mul_transition_destroy(trimul_transition_t *T) {
+    if (!T) return;
+    if (T->mem) cudaFree(T->mem);
+    delete T;
+}
+
+extern "C" trimul_status_t tri_mul_transition_forward(const trimul_pair_t *z, const void *mask,
+                                                      const trimul_transition_t *T, trimul_pair_t *out, void *stream) {
+    if (!T) return fail(TRIMUL_ERR_INVALID_ARG, "transition handle is NULL");
+    TRY(check_pair(z, "z"));
+    TRY(check_pair(out, "out"));
+    if (z->dtype != TRIMUL_BF16) return fail(TRIMUL_ERR_UNSUPPORTED_SHAPE, "the pair transition takes a bf16 z");
+    if (z->C != T->c) return fail(TRIMUL_ERR_INVALID_ARG, "z has %lld channels, the transition %d", (long long)z->C, T->c);
+    if (z->N < 8 || z->N % 8 != 0) return fail(TRIMUL_ERR_UNSUPPORTED_SHAPE, "N=%lld must be a positive multiple of 8", (long long)z->N);
+    if (mask && !aligned16(mask)) return fail(TRIMUL_ERR_ALIGNMENT, "mask not 16-byte aligned");
+    if (out->B != z->B || out->N != z->N || out->C != z->C) return fail(TRIMUL_ERR_INVALID_ARG, "out shape differs from z");
+    if (overlap(out->data, pair_bytes(out), z->data, pair_bytes(z))) return fail(TRIMUL_ERR_INVALID_ARG, "out overlaps z");
+    DeviceInfo d;
+    TRY(require_sm100(&d));
+    const uint64_t NN = (uint64_t)z->N * z->N;
+    const uint64_t B = (uint64_t)z->B;
+    PtArgs p{};
+    {
+        // z [B][NN][128] viewed as {64 channels, NN pairs, 2 halves, B}: one copy brings both
+        // 64-channel halves of 64 pairs, laid out [half][pair][64]
+        uint64_t dims[4] = {64, NN, 2, B};
+        uint64_t strides[3] = {(uint64_t)T->c * 2, 128, NN * T->c * 2};
+        uint32_t box[4] = {64, 64, 2, 1};
+        TRY(make_map(&p.tm_z, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, z->data, dims, strides, box,
+                     CU_TENSOR_MAP_SWIZZLE_128B, "transition z"));
+    }
+    {
+        const bool f32 = out->dtype == TRIMUL_F32;
+        const uint64_t es = f32 ? 4 : 2;
+        uint64_t dims[3] = {(uint64_t)T->c, NN, B};
+        uint64_t strides[2] = {(uint64_t)T->c * es, NN * T->c * es};
+        uint32_t box[3] = {(uint32_t)T->c, 32, 1};
+        TRY(make_map(&p.tm_out, f32 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, out->data,
+                     dims, strides, box, CU_TENSOR_MAP_SWIZZLE_NONE, "transition out"));
+    }
+    p.tm_w1 = T->tm_w1;
+    p.tm_w2 = T->tm_w2;
+    p.mask = reinterpret_cast<const uint16_t *>(mask);
+    p.b1 = T->b1;
+    p.b2 = T->b2;
+    p.B = (int)z->B;
+    p.NN = (long long)NN;
+    p.tiles_per_batch = (int)(NN / 64);
+    const int grid = grid_for(d.sms, (long long)B * p.tiles_per_batch, 1);
+    TRY_CUDA(pt_launch(out->dtype == TRIMUL_F32, p, grid, reinterpret_cast<cudaStream_t>(stream)), "transition launch");
+    return TRIMUL_OK;
+}
+
 extern "C" const char *tri_mul_status_string(trimul_status_t s) {
     switch (s) {
         case TRIMUL_OK: return "ok";

@@ -92,6 +92,10 @@ def load_library():
         lib.tri_mul_output_gate.argtypes = [P(_Pair), vp, vp, ctypes.c_float, vp, P(_Pair), vp]
         lib.tri_mul_layer_set_timing_events.argtypes = [vp, P(vp)]
         lib.tri_mul_layer_set_mask_skipping.argtypes = [vp, st]
+        lib.tri_mul_transition_create.argtypes = [st, st, st, vp, vp, vp, vp, vp, P(vp)]
+        lib.tri_mul_transition_destroy.argtypes = [vp]
+        lib.tri_mul_transition_destroy.restype = None
+        lib.tri_mul_transition_forward.argtypes = [P(_Pair), vp, vp, P(_Pair), vp]
         lib.tri_mul_kernels_per_forward.argtypes = []
         lib.tri_mul_check_device_status.argtypes = []
         lib.tri_mul_status_string.argtypes = [st]
@@ -101,7 +105,8 @@ def load_library():
         lib.tri_mul_abi_version.argtypes = []
         for name in ("tri_mul_layer_create", "tri_mul_layer_bind_workspace", "tri_mul_forward",
                      "tri_mul_forward_residual", "tri_mul_pair_update", "tri_mul_pair_update_graph_create",
-                     "tri_mul_graph_launch", "tri_mul_layer_set_mask_skipping",
+                     "tri_mul_graph_launch", "tri_mul_layer_set_mask_skipping", "tri_mul_transition_create",
+                     "tri_mul_transition_forward",
                      "tri_mul_project", "tri_mul_contract", "tri_mul_output_gate",
                      "tri_mul_layer_set_timing_events", "tri_mul_check_device_status"):
             getattr(lib, name).restype = ctypes.c_int
@@ -285,6 +290,52 @@ def contract(a: torch.Tensor, b: torch.Tensor, direction="outgoing", out: torch.
     _check(lib.tri_mul_contract(a.data_ptr(), b.data_ptr(), out.data_ptr(), B, C, N, _dtype_code(a.dtype),
                                 _DIRS[direction], x_scale, _stream_ptr(stream)))
     return out
+
+
+class PairTransition:
+    """The fused pair transition out = z + m * (relu(z W1^T + b1) W2^T + b2) (bf16, c = 128,
+    hidden = 256). Weights: CUDA bf16 tensors W1 [256, 128], W2 [128, 256], biases or None."""
+
+    def __init__(self, w1: torch.Tensor, w2: torch.Tensor, b1: torch.Tensor | None = None,
+                 b2: torch.Tensor | None = None, stream=None):
+        self._lib = load_library()
+        hidden, c = w1.shape
+        for t in (w1, w2, b1, b2):
+            if t is not None and (t.dtype != torch.bfloat16 or not t.is_cuda):
+                raise ValueError("pair transition weights must be bfloat16 CUDA tensors")
+        keep = [t.contiguous() for t in (w1, w2) + tuple(x for x in (b1, b2) if x is not None)]
+        w1c, w2c = keep[0], keep[1]
+        b1c = b1.contiguous() if b1 is not None else None
+        b2c = b2.contiguous() if b2 is not None else None
+        handle = ctypes.c_void_p()
+        _check(self._lib.tri_mul_transition_create(c, hidden, BF16, w1c.data_ptr(),
+                                                   None if b1c is None else b1c.data_ptr(), w2c.data_ptr(),
+                                                   None if b2c is None else b2c.data_ptr(), _stream_ptr(stream),
+                                                   ctypes.byref(handle)))
+        self.handle = handle
+        self.c, self.hidden = c, hidden
+
+    def forward(self, z: torch.Tensor, mask: torch.Tensor | None = None, out: torch.Tensor | None = None,
+                out_dtype: torch.dtype | None = None, stream=None) -> torch.Tensor:
+        if out is None:
+            out = torch.empty(z.shape, dtype=out_dtype or z.dtype, device=z.device)
+        zp, op = _pair(z), _pair(out)
+        _check(self._lib.tri_mul_transition_forward(ctypes.byref(zp), _mask_ptr(mask, z), self.handle,
+                                                    ctypes.byref(op), _stream_ptr(stream)))
+        return out
+
+    __call__ = forward
+
+    def close(self):
+        if getattr(self, "handle", None):
+            self._lib.tri_mul_transition_destroy(self.handle)
+            self.handle = None
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
 
 
 def pair_update(z: torch.Tensor, mask: torch.Tensor | None, layer_out: TriMulLayer, layer_in: TriMulLayer,

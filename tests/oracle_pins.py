@@ -382,6 +382,39 @@ def pin_pair_update_second_step_is_incoming(lib):
     assert np.max(np.abs(out - wrong)) > 1e-6
 
 
+# ---------------------------------------------------------------- pair transition
+
+
+def _transition_inputs(seed=61, B=2, N=5, c=12, h=24):
+    rng = np.random.default_rng(seed)
+    z = rng.standard_normal((B, N, N, c))
+    mask = (rng.random((B, N, N)) > 0.3).astype(np.float64)
+    w1 = rng.standard_normal((h, c)) / math.sqrt(c)
+    b1 = rng.standard_normal(h) * 0.1
+    w2 = rng.standard_normal((c, h)) / math.sqrt(h)
+    b2 = rng.standard_normal(c) * 0.1
+    return z, mask, w1, b1, w2, b2
+
+
+def pin_pair_transition_library(lib):
+    """Against torch's float64 linear and relu, composed as the pages list the steps."""
+    z, mask, w1, b1, w2, b2 = _transition_inputs()
+    ref = _t(z) + _t(mask)[..., None] * F.linear(torch.relu(F.linear(_t(z), _t(w1), _t(b1))), _t(w2), _t(b2))
+    _close(oracle.pair_transition(z, mask, w1, b1, w2, b2), ref.numpy(), what="pair transition")
+
+
+def pin_pair_transition_closed_forms(lib):
+    """With b1 so negative that every hidden unit is cut by the ReLU, out = z + m b2; masked
+    pairs keep z bitwise; scaling W2 and b2 by s scales the update by s."""
+    z, mask, w1, b1, w2, b2 = _transition_inputs()
+    out = oracle.pair_transition(z, mask, w1, np.full_like(b1, -1e6), w2, b2)
+    _close(out, z + mask[..., None] * b2, what="all hidden units cut")
+    out = oracle.pair_transition(z, mask, w1, b1, w2, b2)
+    assert np.array_equal(out[mask == 0], z[mask == 0])
+    out2 = oracle.pair_transition(z, mask, w1, b1, 3.0 * w2, 3.0 * b2)
+    _close(out2 - z, 3.0 * (out - z), what="update linear in W2, b2")
+
+
 ALL_PINS = [
     pin_layernorm_library, pin_linear_library, pin_gated_projection_library, pin_contract_library,
     pin_output_gate_library, pin_full_update_library, pin_constant_field_closed_form,
@@ -389,5 +422,5 @@ ALL_PINS = [
     pin_masked_k_contributes_nothing, pin_padding_equals_truncation, pin_sampled_equals_full,
     pin_b_projection_scale_invariance, pin_single_residue_directions_agree,
     pin_pair_update_masked_pairs_keep_z, pin_pair_update_first_step_is_outgoing,
-    pin_pair_update_second_step_is_incoming,
+    pin_pair_update_second_step_is_incoming, pin_pair_transition_library, pin_pair_transition_closed_forms,
 ]
