@@ -15,10 +15,11 @@
 // exact copy of the bf16 weights except below 2^-14 in magnitude, where the absolute error is
 // under 2^-25.)
 //   WG1    out[p, n] = z[p, n] + m_p (D2 + b2[n]), rows of 128 channels through TMA stores
-// Warps: 0-3 (WG0) the hidden activation, 4-7 (WG1) the output, 8 TMA producer, 9 TMEM and MMA
-// issuer. TMEM: two buffers of [D1: 128 columns | D2: 64 columns]. H is single-buffered: the
-// MMA thread issues GEMM1 of tile t+1 before GEMM2 of tile t, so WG0 works on the next tile's
-// activation while WG1 writes this tile's output.
+// Warps: 0-7 the hidden activation (warpgroup k: hidden half k), 8-15 the output (warpgroup k:
+// pairs [32k, 32k + 32), its own staging and store), 16 TMA producer, 17 TMEM and MMA issuer.
+// TMEM: two buffers of [D1: 128 columns | D2: 64 columns]. H is single-buffered: the MMA thread
+// issues GEMM1 of tile t+1 before GEMM2 of tile t, so the activation warpgroups work on the next
+// tile while the output warpgroups write this one.
 #include "kernels.h"
 #include "sm100.cuh"
 
@@ -29,16 +30,18 @@ constexpr int C = 128, HID = 256, TP = 64;                 // channels, hidden u
 constexpr int W1_BYTES = HID * C * 2;                      // 64 KB: 2 K-chunks of [256 rows][64]
 constexpr int W2_BYTES = C * HID * 2;                      // 64 KB: 4 K-chunks of [128 rows][64]
 constexpr int ZT_BYTES = TP * C * 2;                       // 16 KB: [2 halves][64 pairs][64 ch]
-constexpr int S = 3;                                       // z tiles in flight (held until WG1 is done)
+// z tiles in flight (each held until the output warpgroups have read its residual): 3, or 2
+// with fp32 output, whose staging is twice as large
 constexpr int H_BYTES = HID * TP * 2;                      // 32 KB: [256 rows][64 pairs]
-constexpr int OUT_ROWS = 32;                               // pairs per output store
+constexpr int OUT_ROWS = 32;                               // pairs per output warpgroup
 constexpr int TMEM_COLS = 512;
-constexpr int THREADS = 320;
-constexpr int TMA_WARP = 8, MMA_WARP = 9;
+constexpr int THREADS = 576;
+constexpr int TMA_WARP = 16, MMA_WARP = 17;
+constexpr int SMAX = 3;
 
 struct Smem {
     uint64_t wbar;
-    uint64_t zfull[S], zempty[S];
+    uint64_t zfull[SMAX], zempty[SMAX];
     uint64_t d1full[2], d1empty[2];
     uint64_t d2full[2], d2empty[2];
     uint64_t hfull, hempty;
@@ -49,22 +52,25 @@ struct Smem {
 
 template <bool OUT_F32>
 struct Cfg {
-    static constexpr int STG_BYTES = OUT_ROWS * C * (OUT_F32 ? 4 : 2);
-    static constexpr size_t SMEM = 1024 + W1_BYTES + W2_BYTES + S * ZT_BYTES + H_BYTES + STG_BYTES + TP * 4 + 1024;
+    static constexpr int S = OUT_F32 ? 2 : 3;
+    static constexpr int STG_BYTES = OUT_ROWS * C * (OUT_F32 ? 4 : 2);   // per output warpgroup
+    static constexpr size_t SMEM = 1024 + W1_BYTES + W2_BYTES + S * ZT_BYTES + H_BYTES + 2 * STG_BYTES + TP * 4 + 1024;
+    static_assert(SMEM <= 232448, "shared memory");
 };
 }  // namespace pt
 
 template <bool OUT_F32>
 __global__ void __launch_bounds__(pt::THREADS, 1) pair_transition_kernel(const __grid_constant__ PtArgs p) {
     using namespace pt;
+    constexpr int S = Cfg<OUT_F32>::S;
     extern __shared__ uint8_t smem_raw[];
     uint8_t *base = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint8_t *w1_s = base;
     uint8_t *w2_s = w1_s + W1_BYTES;
     uint8_t *zt = w2_s + W2_BYTES;                         // S z tiles
     uint8_t *h_s = zt + S * ZT_BYTES;                      // hidden activation (GEMM2's B)
-    uint8_t *stg = h_s + H_BYTES;                          // output rows for one store
-    float *mask_s = reinterpret_cast<float *>(stg + Cfg<OUT_F32>::STG_BYTES);   // [64] this tile's mask
+    uint8_t *stg0 = h_s + H_BYTES;                         // output rows, one block per output warpgroup
+    float *mask_s = reinterpret_cast<float *>(stg0 + 2 * Cfg<OUT_F32>::STG_BYTES);   // [64] this tile's mask
     Smem &s = *reinterpret_cast<Smem *>(mask_s + TP);
 
     const int warp = threadIdx.x >> 5;
@@ -76,15 +82,15 @@ __global__ void __launch_bounds__(pt::THREADS, 1) pair_transition_kernel(const _
         mbar_init(&s.wbar, 1);
         for (int i = 0; i < S; ++i) {
             mbar_init(&s.zfull[i], 1);
-            mbar_init(&s.zempty[i], 4);                    // WG1, once it has read the residual
+            mbar_init(&s.zempty[i], 8);                    // output warps, once they have read the residual
         }
         for (int i = 0; i < 2; ++i) {
             mbar_init(&s.d1full[i], 1);
-            mbar_init(&s.d1empty[i], 4);                   // WG0
+            mbar_init(&s.d1empty[i], 8);                   // activation warps
             mbar_init(&s.d2full[i], 1);
-            mbar_init(&s.d2empty[i], 4);                   // WG1
+            mbar_init(&s.d2empty[i], 8);                   // output warps
         }
-        mbar_init(&s.hfull, 4);                            // WG0
+        mbar_init(&s.hfull, 8);                            // activation warps
         mbar_init(&s.hempty, 1);                           // GEMM2's commit
         mbar_init(&s.drain, 1);
         s.abort_flag = 0;
@@ -185,53 +191,55 @@ __global__ void __launch_bounds__(pt::THREADS, 1) pair_transition_kernel(const _
             tc_commit(&s.drain);
             mbar_drain(&s.drain, 0);
         }
-    } else if (warp < 4) {
-        // WG0: H[h, p] = f16(relu(D1[h, p] + b1[h])); thread = TMEM lane r of each hidden half
-        const int r = warp * 32 + lane;
-        const uint32_t lane_off = (uint32_t)(warp * 32) << 16;
-        const float bias[2] = {p.b1[r], p.b1[128 + r]};
+    } else if (warp < 8) {
+        // activation warpgroup hf: H[h, p] = f16(relu(D1[h, p] + b1[h])) for the hidden units
+        // h = 128 hf + r of its half; thread = TMEM lane r
+        const int hf = warp >> 2;
+        const int r = (warp & 3) * 32 + lane;
+        const uint32_t lane_off = (uint32_t)((warp & 3) * 32) << 16;
+        const uint32_t bar_id = 1 + hf;
+        const float bh = p.b1[hf * 128 + r];
+        const int row = hf * 128 + r;                          // K index of GEMM2 = hidden unit
         const int my_tiles = blockIdx.x < num_tiles ? (num_tiles - 1 - blockIdx.x) / gridDim.x + 1 : 0;
         for (int j = 0; j < my_tiles; ++j) {
             const int u = j & 1;
-            if (!group_all(mbar_wait(&s.d1full[u], (uint32_t)(j >> 1) & 1, abort_flag, kErrTimeoutEpilogue), 1, 128)) break;
+            if (!group_all(mbar_wait(&s.d1full[u], (uint32_t)(j >> 1) & 1, abort_flag, kErrTimeoutEpilogue), bar_id, 128)) break;
             // GEMM2 of the previous tile has read H
-            if (!group_all(mbar_wait(&s.hempty, ((uint32_t)j & 1) ^ 1, abort_flag, kErrTimeoutEpilogue), 1, 128)) break;
+            if (!group_all(mbar_wait(&s.hempty, ((uint32_t)j & 1) ^ 1, abort_flag, kErrTimeoutEpilogue), bar_id, 128)) break;
             tc_fence_after();
-#pragma unroll 1
-            for (int hf = 0; hf < 2; ++hf) {
-                float v0[32], v1[32];
-                tmem_ld32(tmem_base + u * 192 + hf * 64 + lane_off, v0);
-                tmem_ld32(tmem_base + u * 192 + hf * 64 + lane_off + 32, v1);
-                tc_wait_ld();
-                const int row = hf * 128 + r;                  // K index of GEMM2 = hidden unit
-                const float bh = hf == 0 ? bias[0] : bias[1];
-#pragma unroll
-                for (int uu = 0; uu < 8; ++uu) {               // 8 pairs per 16-byte unit
-                    uint32_t w[4];
-#pragma unroll
-                    for (int e = 0; e < 4; ++e) {
-                        const int i = 8 * (uu & 3) + 2 * e;
-                        const float a0 = uu < 4 ? v0[i] : v1[i], a1 = uu < 4 ? v0[i + 1] : v1[i + 1];
-                        w[e] = pack_f16x2(fmaxf(a0 + bh, 0.f), fmaxf(a1 + bh, 0.f));
-                    }
-                    *reinterpret_cast<uint4 *>(h_s + sw128_offset(row, uu)) = make_uint4(w[0], w[1], w[2], w[3]);
-                }
-            }
+            float v0[32], v1[32];                              // pairs 0-31 and 32-63
+            tmem_ld32(tmem_base + u * 192 + hf * 64 + lane_off, v0);
+            tmem_ld32(tmem_base + u * 192 + hf * 64 + lane_off + 32, v1);
+            tc_wait_ld();
             tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&s.d1empty[u]);         // D1 read in full
+#pragma unroll
+            for (int uu = 0; uu < 8; ++uu) {                   // 8 pairs per 16-byte unit
+                uint32_t w[4];
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    const int i = 8 * (uu & 3) + 2 * e;
+                    const float a0 = uu < 4 ? v0[i] : v1[i], a1 = uu < 4 ? v0[i + 1] : v1[i + 1];
+                    w[e] = pack_f16x2(fmaxf(a0 + bh, 0.f), fmaxf(a1 + bh, 0.f));
+                }
+                *reinterpret_cast<uint4 *>(h_s + sw128_offset(row, uu)) = make_uint4(w[0], w[1], w[2], w[3]);
+            }
             fence_proxy_async_smem();                          // H is read by the tensor core
             __syncwarp();
-            if (lane == 0) {
-                mbar_arrive(&s.d1empty[u]);
-                mbar_arrive(&s.hfull);
-            }
+            if (lane == 0) mbar_arrive(&s.hfull);
         }
-    } else {
-        // WG1: out[p, n] = z[p, n] + m_p (D2[n, p] + b2[n]); thread = output channel n
-        const int q = warp - 4;
+    } else if (warp < 16) {
+        // output warpgroup k: out[p, n] = z[p, n] + m_p (D2[n, p] + b2[n]) for the pairs
+        // [32k, 32k + 32) of the tile; thread = output channel n
+        const int k = (warp - 8) >> 2;
+        const int q = warp & 3;
         const int n = q * 32 + lane;
-        const int t128 = threadIdx.x - 128;
+        const int tk = (warp - 8 - 4 * k) * 32 + lane;         // thread index within the warpgroup
         const uint32_t lane_off = (uint32_t)(q * 32) << 16;
-        const bool leader = t128 == 0;
+        const uint32_t bar_id = 3 + k;
+        const bool leader = tk == 0;
+        uint8_t *stg = stg0 + k * Cfg<OUT_F32>::STG_BYTES;
         const float bias = p.b2[n];
         const uint32_t zoff = (uint32_t)(n >> 6) * (TP * 128) + (uint32_t)(n & 7) * 2;   // half block, element
         const uint32_t zunit = (uint32_t)(n & 63) >> 3;
@@ -241,47 +249,41 @@ __global__ void __launch_bounds__(pt::THREADS, 1) pair_transition_kernel(const _
             const int b = tw.b;
             const int p0 = tw.t * TP;
             const int u = j & 1, st = j % S;
-            if (t128 < TP) {
+            if (tk < OUT_ROWS) {
                 float m = 1.f;
-                if (p.mask) m = __uint_as_float((uint32_t)p.mask[(long long)b * p.NN + p0 + t128] << 16);
-                mask_s[t128] = m;
+                if (p.mask) m = __uint_as_float((uint32_t)p.mask[(long long)b * p.NN + p0 + k * OUT_ROWS + tk] << 16);
+                mask_s[k * OUT_ROWS + tk] = m;
             }
-            if (!group_all(mbar_wait(&s.d2full[u], (uint32_t)(j >> 1) & 1, abort_flag, kErrTimeoutEpilogue), 2, 128)) break;
+            if (leader) tma_store_wait_read<0>();              // this warpgroup's previous store has read its rows
+            if (!group_all(mbar_wait(&s.d2full[u], (uint32_t)(j >> 1) & 1, abort_flag, kErrTimeoutEpilogue), bar_id, 128)) break;
             tc_fence_after();
             (void)mbar_try_wait(&s.zfull[st], (uint32_t)(j / S) & 1);   // completed phase: acquire the z tile
-            float d0[32], d1[32];                               // pairs 0-31 and 32-63
-            tmem_ld32(tmem_base + u * 192 + 128 + lane_off, d0);
-            tmem_ld32(tmem_base + u * 192 + 128 + lane_off + 32, d1);
+            float d[32];
+            tmem_ld32(tmem_base + u * 192 + 128 + lane_off + k * OUT_ROWS, d);
             tc_wait_ld();
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(&s.d2empty[u]);
             const uint8_t *zb = zt + st * ZT_BYTES + zoff;
-            static_assert(TP == 2 * OUT_ROWS, "two output stores per tile");
 #pragma unroll
-            for (int rr = 0; rr < 2; ++rr) {
-                if (leader) tma_store_wait_read<0>();
-                named_bar_sync(2, 128);
-#pragma unroll
-                for (int pp = 0; pp < OUT_ROWS; ++pp) {
-                    const int pair = rr * OUT_ROWS + pp;
-                    const float zv = __uint_as_float((uint32_t)*reinterpret_cast<const uint16_t *>(
-                                                         zb + sw128_offset(pair, zunit)) << 16);
-                    const float o = fmaf(mask_s[pair], (rr == 0 ? d0[pp] : d1[pp]) + bias, zv);
-                    if (OUT_F32)
-                        reinterpret_cast<float *>(stg)[pp * C + n] = o;
-                    else
-                        reinterpret_cast<__nv_bfloat16 *>(stg)[pp * C + n] = __float2bfloat16_rn(o);
-                }
-                fence_proxy_async_smem();
-                named_bar_sync(2, 128);
-                if (leader) {
-                    tma_store_3d(&p.tm_out, stg, 0, p0 + rr * OUT_ROWS, b);
-                    tma_store_commit();
-                }
+            for (int pp = 0; pp < OUT_ROWS; ++pp) {
+                const int pair = k * OUT_ROWS + pp;
+                const float zv = __uint_as_float((uint32_t)*reinterpret_cast<const uint16_t *>(
+                                                     zb + sw128_offset(pair, zunit)) << 16);
+                const float o = fmaf(mask_s[pair], d[pp] + bias, zv);
+                if (OUT_F32)
+                    reinterpret_cast<float *>(stg)[pp * C + n] = o;
+                else
+                    reinterpret_cast<__nv_bfloat16 *>(stg)[pp * C + n] = __float2bfloat16_rn(o);
             }
+            fence_proxy_async_smem();
             __syncwarp();
-            if (lane == 0) mbar_arrive(&s.zempty[st]);          // the residual has been read
+            if (lane == 0) mbar_arrive(&s.zempty[st]);          // this warp has read the residual
+            named_bar_sync(bar_id, 128);
+            if (leader) {
+                tma_store_3d(&p.tm_out, stg, 0, p0 + k * OUT_ROWS, b);
+                tma_store_commit();
+            }
         }
         if (leader) tma_store_wait_all<0>();
     }
