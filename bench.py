@@ -34,7 +34,7 @@ CPU_BASELINE_WORKLOADS = ("bf16_n512_ragged", "bf16_n256_tail10", "bf16_b4_n256_
 L2_BYTES = 126 * 1024 * 1024
 KERNEL_NAMES = ("k1_project_kernel", "k2_contract_kernel", "k3_output_kernel")
 KERNEL_SOURCES = {"k1_project_kernel": "k1_project.cu", "k2_contract_kernel": "k2_contract.cu",
-                  "k3_output_kernel": "k3_output.cu"}
+                  "k3_output_kernel": "k3_output.cu", "pair_transition_kernel": "transition.cu"}
 
 
 def parse_args():
@@ -308,6 +308,7 @@ def transition_leg(tm, zs, ms_, n_sets, args, dev):
         pt.close()
         return {"ms": ms, "GB_s": gbs, "TFLOP_s": tfs, "hbm_frac": gbs / peaks["hbm_gbs"],
                 "tensor_frac": tfs / peaks["bf16_tflops"], "bytes": nbytes, "flops": flops,
+                "traffic": recorded_traffic("pair_transition_kernel"),
                 "shape": "c=128, hidden=256, bf16 in/out, fp16 hidden activation on chip"}
     except Exception as exc:       # the headline line must not depend on this leg
         return {"error": f"{type(exc).__name__}: {exc}"}
