@@ -33,12 +33,16 @@ struct K3Cfg {
     static constexpr int WO_BYTES = NCOL * C_H * 2;
     static constexpr int WG_BYTES = NCOL * CZ * 2;
     static constexpr int CHUNK = 128 * 64 * 2;
-    static constexpr int STG_BYTES = 128 * 128;      // per warpgroup: 128 rows x 128 bytes
+    static constexpr int STG_BYTES = 128 * 128;      // per warpgroup and buffer: 128 rows x 128 bytes
     static constexpr int COLS_PER_STORE = OUT_F32 ? 32 : 64;
+    // staging buffers per warpgroup: fp32 out takes two stores per tile, and a second buffer
+    // lets the second block be written while the first one's store still reads (c_z = 128:
+    // c_z = 384 keeps its room for the input ring)
+    static constexpr int NSTG = (OUT_F32 && CZ == 128) ? 2 : 1;
     static constexpr int SNB = 2;
     static constexpr int VEC_BYTES = NCOL * 16;          // folding constants of this group's columns
     static constexpr int XPART_BYTES = 4 * 128 * 8;      // x partial sums: [4 warps][128 pairs] float2
-    static constexpr int FIXED = 1024 + WO_BYTES + WG_BYTES + 2 * STG_BYTES + SNB * 128 * 32 + VEC_BYTES + XPART_BYTES + 1024;
+    static constexpr int FIXED = 1024 + WO_BYTES + WG_BYTES + 2 * NSTG * STG_BYTES + SNB * 128 * 32 + VEC_BYTES + XPART_BYTES + 1024;
     static constexpr int S = (232448 - FIXED) / CHUNK > 8 ? 8 : (232448 - FIXED) / CHUNK;
     static constexpr size_t SMEM = FIXED + (size_t)S * CHUNK;
     static constexpr int THREADS = 576;
@@ -56,6 +60,13 @@ struct K3Smem {
     int abort_flag;
 };
 
+// 16-byte global -> shared copy through L2 (cp.async); `bytes` 0 writes zeros and reads nothing.
+__device__ __forceinline__ void cp_async_16(void *dst, const void *src, uint32_t bytes) {
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(smem_u32(dst)), "l"(src), "r"(bytes) : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+__device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_group 0;" ::: "memory"); }
+
 // Per-pair values the epilogue needs, in the form it uses them: negated means, the x rstd,
 // half the z rstd (the gate is evaluated as tanh of half its argument) and half the mask.
 struct K3Stats {
@@ -72,8 +83,8 @@ __global__ void __launch_bounds__(576, 1) k3_output_kernel(const __grid_constant
     uint8_t *wo_s = base;                              // XC chunks of [128 rows][64] bf16
     uint8_t *wg_s = wo_s + C::WO_BYTES;                // ZC chunks of [128 rows][64] bf16
     uint8_t *chunks = wg_s + C::WG_BYTES;              // S chunks
-    uint8_t *staging = chunks + C::S * C::CHUNK;       // 2 x 16 KB
-    K3Stats *stats = reinterpret_cast<K3Stats *>(staging + 2 * C::STG_BYTES);
+    uint8_t *staging = chunks + C::S * C::CHUNK;       // [NSTG][2 warpgroups] x 16 KB
+    K3Stats *stats = reinterpret_cast<K3Stats *>(staging + 2 * C::NSTG * C::STG_BYTES);
     // folding constants of this group's columns, one array each: sum W_o', shift_o,
     // sum W_g', shift_g / 2
     float *vec_s = reinterpret_cast<float *>(stats + C::SNB * 128);   // [4][NCOL]
@@ -357,12 +368,12 @@ __global__ void __launch_bounds__(576, 1) k3_output_kernel(const __grid_constant
         // epilogue: warpgroup wg handles output channels n0 + wg*64 .. +63; warp q of it the
         // pairs [32q, 32q + 32) of the tile. Every warp runs on its own: it waits on the
         // barriers itself, stages its 32 pair rows in its own 4 KB of the warpgroup's staging
-        // buffer and issues the TMA store of that block.
+        // buffer (store block sc in buffer sc % NSTG) and issues the TMA store of that block.
+        // With a residual and bf16 out, the residual rows are copied into the staging rows
+        // (cp.async) before the accumulators are ready, and the output overwrites them in place.
         const int wg = warp >> 2;
         const int q = warp & 3;
         const int row = q * 32 + lane;
-        uint8_t *stg = staging + wg * C::STG_BYTES;   // rows [32q, 32q + 32) belong to this warp
-        uint8_t *wstg = stg + q * 32 * 128;
         const float *v_sum_o = vec_s + wg * 64, *v_shift_o = v_sum_o + C::NCOL;
         const float *v_sum_g = v_sum_o + 2 * C::NCOL, *v_hshift_g = v_sum_o + 3 * C::NCOL;
         int abuf = 0;
@@ -377,15 +388,16 @@ __global__ void __launch_bounds__(576, 1) k3_output_kernel(const __grid_constant
                 // every pair of the tile is masked: out is 0 there
 #pragma unroll 1
                 for (int sc = 0; sc < 64 / C::COLS_PER_STORE; ++sc) {
-                    if (lane == 0) tma_store_wait_read<0>();
+                    uint8_t *stg = staging + ((sc % C::NSTG) * 2 + wg) * C::STG_BYTES;
+                    if (lane == 0) tma_store_wait_read<C::NSTG - 1>();
                     __syncwarp();
 #pragma unroll
                     for (int u = 0; u < 8; ++u) *reinterpret_cast<uint4 *>(stg + sw128_offset(row, u)) = make_uint4(0, 0, 0, 0);
                     fence_proxy_async_smem();
                     __syncwarp();
-                    if (lane == 0 && p0 + q * 32 < p.NN) {
-                        tma_store_3d(&p.tm_out, wstg, n0 + wg * 64 + sc * C::COLS_PER_STORE, p0 + q * 32, b);
-                        tma_store_commit();
+                    if (lane == 0) {
+                        if (p0 + q * 32 < p.NN) tma_store_3d(&p.tm_out, stg + q * 32 * 128, n0 + wg * 64 + sc * C::COLS_PER_STORE, p0 + q * 32, b);
+                        tma_store_commit();   // a group per block, empty or not
                     }
                 }
                 continue;
@@ -399,12 +411,30 @@ __global__ void __launch_bounds__(576, 1) k3_output_kernel(const __grid_constant
             if (lane == 0) mbar_arrive(&s.sempty[sbuf]);
             if (++sbuf == C::SNB) { sbuf = 0; sphase ^= 1; }
 
+            constexpr bool RES_STAGED = RES && !OUT_F32;
+            if (RES_STAGED) {
+                // this warp's 32 residual rows (64 channels, 128 bytes each) into its staging
+                // rows, 4 rows per instruction; rows past the last pair are zero-filled
+                if (lane == 0) tma_store_wait_read<0>();   // the previous tile's store has read them
+                __syncwarp();
+                uint8_t *stg = staging + wg * C::STG_BYTES;
+                const int u = lane & 7;
+#pragma unroll
+                for (int i = 0; i < 8; ++i) {
+                    const int r = q * 32 + 4 * i + (lane >> 3);
+                    const bool in = (long long)p0 + r < p.NN;
+                    const uint16_t *src = p.zres + (in ? ((long long)b * p.NN + p0 + r) * CZ + n0 + wg * 64 + 8 * u : 0);
+                    cp_async_16(stg + sw128_offset(r, u), src, in ? 16u : 0u);
+                }
+                cp_async_commit();
+            }
             if (!__all_sync(0xffffffffu, mbar_wait(&s.tfull[abuf], aphase, abort_flag, kErrTimeoutEpilogue))) break;
             tc_fence_after();
             const uint32_t t1 = tmem_base + abuf * 256 + ((uint32_t)(q * 32) << 16) + wg * 64;
             const uint32_t t2 = t1 + 128;
 #pragma unroll 1
             for (int sc = 0; sc < 64 / C::COLS_PER_STORE; ++sc) {
+                uint8_t *stg = staging + ((sc % C::NSTG) * 2 + wg) * C::STG_BYTES;
 #pragma unroll 1
                 for (int h = 0; h < C::COLS_PER_STORE / 32; ++h) {
                     const int col = sc * C::COLS_PER_STORE + h * 32;   // within this warpgroup's 64
@@ -413,8 +443,10 @@ __global__ void __launch_bounds__(576, 1) k3_output_kernel(const __grid_constant
                     tmem_ld16(t1 + col + 16, *reinterpret_cast<float(*)[16]>(&o[16]));
                     tmem_ld16(t2 + col, *reinterpret_cast<float(*)[16]>(&g[0]));
                     tmem_ld16(t2 + col + 16, *reinterpret_cast<float(*)[16]>(&g[16]));
-                    if (h == 0) {
-                        if (lane == 0) tma_store_wait_read<0>();   // this warp's previous store has read its rows
+                    if (h == 0 && !RES_STAGED) {
+                        // the store of this buffer's previous block has read its rows (with two
+                        // buffers the store just issued, from the other one, may still read)
+                        if (lane == 0) tma_store_wait_read<C::NSTG - 1>();
                         __syncwarp();
                     }
                     tc_wait_ld();
@@ -448,7 +480,7 @@ __global__ void __launch_bounds__(576, 1) k3_output_kernel(const __grid_constant
                             o[i + 1] = r.y;
                         }
                     }
-                    if (RES && (long long)p0 + row < p.NN) {
+                    if (RES && OUT_F32 && (long long)p0 + row < p.NN) {
                         // residual: this pair's z at the block's 32 output channels (from L2: K1
                         // and this kernel's own z chunk loads have just read it)
                         const uint4 *zp = reinterpret_cast<const uint4 *>(
@@ -472,8 +504,21 @@ __global__ void __launch_bounds__(576, 1) k3_output_kernel(const __grid_constant
                             *reinterpret_cast<float4 *>(stg + sw128_offset(row, u)) =
                                 make_float4(o[4 * u], o[4 * u + 1], o[4 * u + 2], o[4 * u + 3]);
                     } else {
+                        if (RES_STAGED) {
+                            cp_async_wait_all();
+                            __syncwarp();                      // rows copied by the other lanes
+                        }
 #pragma unroll
                         for (int u = 0; u < 4; ++u) {
+                            if (RES_STAGED) {
+                                const uint4 zr = *reinterpret_cast<const uint4 *>(stg + sw128_offset(row, h * 4 + u));
+                                const uint32_t zw[4] = {zr.x, zr.y, zr.z, zr.w};
+#pragma unroll
+                                for (int e = 0; e < 4; ++e) {
+                                    o[8 * u + 2 * e] += bf16_lo(zw[e]);
+                                    o[8 * u + 2 * e + 1] += bf16_hi(zw[e]);
+                                }
+                            }
                             uint4 w;
                             w.x = pack_bf16x2(o[8 * u + 0], o[8 * u + 1]);
                             w.y = pack_bf16x2(o[8 * u + 2], o[8 * u + 3]);
@@ -485,8 +530,10 @@ __global__ void __launch_bounds__(576, 1) k3_output_kernel(const __grid_constant
                 }
                 fence_proxy_async_smem();
                 __syncwarp();
-                if (lane == 0 && p0 + q * 32 < p.NN) {   // blocks wholly past the last pair are not stored
-                    tma_store_3d(&p.tm_out, wstg, n0 + wg * 64 + sc * C::COLS_PER_STORE, p0 + q * 32, b);
+                if (lane == 0) {
+                    // blocks wholly past the last pair are not stored; the group is committed
+                    // all the same (empty), so the most recent group is always the last block's
+                    if (p0 + q * 32 < p.NN) tma_store_3d(&p.tm_out, stg + q * 32 * 128, n0 + wg * 64 + sc * C::COLS_PER_STORE, p0 + q * 32, b);
                     tma_store_commit();
                 }
             }

@@ -38,7 +38,7 @@ def _bound(ref_mid, ref_out, z, tol, mid_rel, out_rel):
 
 
 @pytest.mark.parametrize("c_z,N,B,out_dtype", [(128, 96, 2, torch.float32), (128, 96, 2, torch.bfloat16),
-                                               (384, 64, 2, torch.float32)])
+                                               (128, 88, 2, torch.bfloat16), (384, 64, 2, torch.float32)])
 def test_pair_update_bf16_against_oracle(c_z, N, B, out_dtype):
     inp, w_in, z, m, lo, li = _layers(B, N, c_z, "bf16", seed=7 * N + c_z, mask=("uniform_len", N // 2, N))
     z_mid = torch.empty_like(z)
@@ -79,6 +79,19 @@ def test_residual_forward_is_z_plus_update_bitwise(dtype):
         r = lo.forward(z, m, d, out_dtype=torch.float32, residual=True)
         torch.cuda.synchronize()
         assert torch.equal(r, z.float() + u), d
+
+
+@pytest.mark.parametrize("N,B", [(64, 1), (88, 2)])
+def test_residual_forward_bf16_out_is_rounded_z_plus_update(N, B):
+    """bf16 out with the fused residual is bf16(z + update) of the same fp32 update. N=88 has
+    7744 pairs per batch element: the last 128-pair tile holds 64, and the next tile belongs to
+    the second element."""
+    inp, _, z, m, lo, _ = _layers(B, N, 128, "bf16", seed=17 + N, mask=("uniform_len", N // 2, N))
+    for d in ("outgoing", "incoming"):
+        u = lo.forward(z, m, d, out_dtype=torch.float32)
+        r = lo.forward(z, m, d, out_dtype=torch.bfloat16, residual=True)
+        torch.cuda.synchronize()
+        assert torch.equal(r, (z.float() + u).to(torch.bfloat16)), d
 
 
 def test_graph_replay_equals_eager_and_follows_new_inputs():
