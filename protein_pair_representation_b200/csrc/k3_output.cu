@@ -60,13 +60,6 @@ struct K3Smem {
     int abort_flag;
 };
 
-// 16-byte global -> shared copy through L2 (cp.async); `bytes` 0 writes zeros and reads nothing.
-__device__ __forceinline__ void cp_async_16(void *dst, const void *src, uint32_t bytes) {
-    asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(smem_u32(dst)), "l"(src), "r"(bytes) : "memory");
-}
-__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
-__device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_group 0;" ::: "memory"); }
-
 // Per-pair values the epilogue needs, in the form it uses them: negated means, the x rstd,
 // half the z rstd (the gate is evaluated as tanh of half its argument) and half the mask.
 struct K3Stats {

@@ -94,6 +94,7 @@ struct PtArgs {
     CUtensorMap tm_w1;     // W1 [256][128] bf16, box {64, 256}, 128B swizzle
     CUtensorMap tm_w2;     // W2 [128][256] f16, box {64, 128}, 128B swizzle
     CUtensorMap tm_out;    // out [B][N*N][128] f32 or bf16, box {128, 32, 1}, no swizzle
+    const uint16_t *z;     // the same z, bf16 bits, for the residual
     const uint16_t *mask;  // [B][N*N] bf16 bits, or nullptr
     const float *b1;       // [256] fp32 (zeros when the layer has no bias)
     const float *b2;       // [128] fp32

@@ -19,7 +19,10 @@
 // pairs [32k, 32k + 32), its own staging and store), 16 TMA producer, 17 TMEM and MMA issuer.
 // TMEM: two buffers of [D1: 128 columns | D2: 64 columns]. H is single-buffered: the MMA thread
 // issues GEMM1 of tile t+1 before GEMM2 of tile t, so the activation warpgroups work on the next
-// tile while the output warpgroups write this one.
+// tile while the output warpgroups write this one. A z tile is released as soon as GEMM1 has
+// read it, so the input ring runs ahead of the whole pipeline; the output warpgroups load the
+// residual from L2 (GEMM1's copy brought it in a few microseconds earlier), one coalesced
+// 64-byte row segment per warp and pair, before they wait for the accumulators.
 #include "kernels.h"
 #include "sm100.cuh"
 
@@ -30,8 +33,7 @@ constexpr int C = 128, HID = 256, TP = 64;                 // channels, hidden u
 constexpr int W1_BYTES = HID * C * 2;                      // 64 KB: 2 K-chunks of [256 rows][64]
 constexpr int W2_BYTES = C * HID * 2;                      // 64 KB: 4 K-chunks of [128 rows][64]
 constexpr int ZT_BYTES = TP * C * 2;                       // 16 KB: [2 halves][64 pairs][64 ch]
-// z tiles in flight (each held until the output warpgroups have read its residual): 3, or 2
-// with fp32 output, whose staging is twice as large
+// z tiles in flight: 3, or 2 with fp32 output, whose staging is twice as large
 constexpr int H_BYTES = HID * TP * 2;                      // 32 KB: [256 rows][64 pairs]
 constexpr int OUT_ROWS = 32;                               // pairs per output warpgroup
 constexpr int TMEM_COLS = 512;
@@ -54,7 +56,7 @@ template <bool OUT_F32>
 struct Cfg {
     static constexpr int S = OUT_F32 ? 2 : 3;
     static constexpr int STG_BYTES = OUT_ROWS * C * (OUT_F32 ? 4 : 2);   // per output warpgroup
-    static constexpr size_t SMEM = 1024 + W1_BYTES + W2_BYTES + S * ZT_BYTES + H_BYTES + 2 * STG_BYTES + TP * 4 + 1024;
+    static constexpr size_t SMEM = 1024 + W1_BYTES + W2_BYTES + S * ZT_BYTES + H_BYTES + 2 * STG_BYTES + 1024;
     static_assert(SMEM <= 232448, "shared memory");
 };
 }  // namespace pt
@@ -70,8 +72,7 @@ __global__ void __launch_bounds__(pt::THREADS, 1) pair_transition_kernel(const _
     uint8_t *zt = w2_s + W2_BYTES;                         // S z tiles
     uint8_t *h_s = zt + S * ZT_BYTES;                      // hidden activation (GEMM2's B)
     uint8_t *stg0 = h_s + H_BYTES;                         // output rows, one block per output warpgroup
-    float *mask_s = reinterpret_cast<float *>(stg0 + 2 * Cfg<OUT_F32>::STG_BYTES);   // [64] this tile's mask
-    Smem &s = *reinterpret_cast<Smem *>(mask_s + TP);
+    Smem &s = *reinterpret_cast<Smem *>(stg0 + 2 * Cfg<OUT_F32>::STG_BYTES);
 
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
@@ -82,7 +83,7 @@ __global__ void __launch_bounds__(pt::THREADS, 1) pair_transition_kernel(const _
         mbar_init(&s.wbar, 1);
         for (int i = 0; i < S; ++i) {
             mbar_init(&s.zfull[i], 1);
-            mbar_init(&s.zempty[i], 8);                    // output warps, once they have read the residual
+            mbar_init(&s.zempty[i], 1);                    // GEMM1's commit
         }
         for (int i = 0; i < 2; ++i) {
             mbar_init(&s.d1full[i], 1);
@@ -161,6 +162,7 @@ __global__ void __launch_bounds__(pt::THREADS, 1) pair_transition_kernel(const _
                         }
                 }
                 tc_commit(&s.d1full[u]);
+                tc_commit(&s.zempty[st]);                            // GEMM1 has read the z tile
                 return true;
             };
             // GEMM2 of the CTA's tile j (H of tile j in shared memory)
@@ -235,55 +237,58 @@ __global__ void __launch_bounds__(pt::THREADS, 1) pair_transition_kernel(const _
         const int k = (warp - 8) >> 2;
         const int q = warp & 3;
         const int n = q * 32 + lane;
-        const int tk = (warp - 8 - 4 * k) * 32 + lane;         // thread index within the warpgroup
+        const int tk = q * 32 + lane;                          // thread index within the warpgroup
         const uint32_t lane_off = (uint32_t)(q * 32) << 16;
         const uint32_t bar_id = 3 + k;
         const bool leader = tk == 0;
         uint8_t *stg = stg0 + k * Cfg<OUT_F32>::STG_BYTES;
         const float bias = p.b2[n];
-        const uint32_t zoff = (uint32_t)(n >> 6) * (TP * 128) + (uint32_t)(n & 7) * 2;   // half block, element
-        const uint32_t zunit = (uint32_t)(n & 63) >> 3;
         int j = 0;
         TileWalk tw(blockIdx.x, p.tiles_per_batch);
+        uint32_t mbits = 0x3F80u;
+        if (p.mask && blockIdx.x < num_tiles) mbits = p.mask[(long long)tw.b * p.NN + tw.t * TP + k * OUT_ROWS + lane];
         for (int t = blockIdx.x; t < num_tiles; t += gridDim.x, tw.advance(gridDim.x, p.tiles_per_batch), ++j) {
             const int b = tw.b;
-            const int p0 = tw.t * TP;
-            const int u = j & 1, st = j % S;
-            if (tk < OUT_ROWS) {
-                float m = 1.f;
-                if (p.mask) m = __uint_as_float((uint32_t)p.mask[(long long)b * p.NN + p0 + k * OUT_ROWS + tk] << 16);
-                mask_s[k * OUT_ROWS + tk] = m;
+            const long long row0 = (long long)b * p.NN + tw.t * TP + k * OUT_ROWS;   // first pair of the block
+            const int u = j & 1;
+            const float mreg = __uint_as_float(mbits << 16);
+            uint32_t mbits_next = 0x3F80u;
+            if (p.mask && t + (int)gridDim.x < num_tiles) {
+                TileWalk tn = tw;
+                tn.advance(gridDim.x, p.tiles_per_batch);
+                mbits_next = p.mask[(long long)tn.b * p.NN + tn.t * TP + k * OUT_ROWS + lane];
             }
             if (leader) tma_store_wait_read<0>();              // this warpgroup's previous store has read its rows
+            // the residual, z[p, n] for the block's 32 pairs (one 64-byte row segment per warp and
+            // pair, from L2: GEMM1's load has just brought the tile in), issued before the
+            // accumulator wait so that its latency overlaps it
+            uint32_t zr[OUT_ROWS];
+            const uint16_t *zp = p.z + row0 * C + n;
+#pragma unroll
+            for (int pp = 0; pp < OUT_ROWS; ++pp) zr[pp] = __ldg(zp + pp * C);
             if (!group_all(mbar_wait(&s.d2full[u], (uint32_t)(j >> 1) & 1, abort_flag, kErrTimeoutEpilogue), bar_id, 128)) break;
             tc_fence_after();
-            (void)mbar_try_wait(&s.zfull[st], (uint32_t)(j / S) & 1);   // completed phase: acquire the z tile
             float d[32];
             tmem_ld32(tmem_base + u * 192 + 128 + lane_off + k * OUT_ROWS, d);
             tc_wait_ld();
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(&s.d2empty[u]);
-            const uint8_t *zb = zt + st * ZT_BYTES + zoff;
 #pragma unroll
             for (int pp = 0; pp < OUT_ROWS; ++pp) {
-                const int pair = k * OUT_ROWS + pp;
-                const float zv = __uint_as_float((uint32_t)*reinterpret_cast<const uint16_t *>(
-                                                     zb + sw128_offset(pair, zunit)) << 16);
-                const float o = fmaf(mask_s[pair], d[pp] + bias, zv);
+                const float o = fmaf(__shfl_sync(0xffffffffu, mreg, pp), d[pp] + bias, __uint_as_float(zr[pp] << 16));
                 if (OUT_F32)
                     reinterpret_cast<float *>(stg)[pp * C + n] = o;
                 else
-                    reinterpret_cast<__nv_bfloat16 *>(stg)[pp * C + n] = __float2bfloat16_rn(o);
+                    reinterpret_cast<uint16_t *>(stg)[pp * C + n] = __bfloat16_as_ushort(__float2bfloat16_rn(o));
             }
             fence_proxy_async_smem();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&s.zempty[st]);          // this warp has read the residual
             named_bar_sync(bar_id, 128);
             if (leader) {
-                tma_store_3d(&p.tm_out, stg, 0, p0 + k * OUT_ROWS, b);
+                tma_store_3d(&p.tm_out, stg, 0, (int)(row0 - (long long)b * p.NN), b);
                 tma_store_commit();
             }
+            mbits = mbits_next;
         }
         if (leader) tma_store_wait_all<0>();
     }

@@ -885,6 +885,7 @@ extern "C" trimul_status_t tri_mul_transition_forward(const trimul_pair_t *z, co
     }
     p.tm_w1 = T->tm_w1;
     p.tm_w2 = T->tm_w2;
+    p.z = reinterpret_cast<const uint16_t *>(z->data);
     p.mask = reinterpret_cast<const uint16_t *>(mask);
     p.b1 = T->b1;
     p.b2 = T->b2;
