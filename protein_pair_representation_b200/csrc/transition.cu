@@ -20,9 +20,10 @@
 // TMEM: two buffers of [D1: 128 columns | D2: 64 columns]. H is single-buffered: the MMA thread
 // issues GEMM1 of tile t+1 before GEMM2 of tile t, so the activation warpgroups work on the next
 // tile while the output warpgroups write this one. A z tile is released as soon as GEMM1 has
-// read it, so the input ring runs ahead of the whole pipeline; the output warpgroups load the
-// residual from L2 (GEMM1's copy brought it in a few microseconds earlier), one coalesced
-// 64-byte row segment per warp and pair, before they wait for the accumulators.
+// read it, so the input ring runs ahead of the whole pipeline. The output warpgroups take the
+// residual from global memory (L2: GEMM1's copy has just brought it in), one tile ahead, as
+// 16-byte row segments: thread = channel puts m_p (D2 + b2) in fp32 staging rows, then thread =
+// row segment adds z and rounds in place.
 #include "kernels.h"
 #include "sm100.cuh"
 
@@ -33,13 +34,12 @@ constexpr int C = 128, HID = 256, TP = 64;                 // channels, hidden u
 constexpr int W1_BYTES = HID * C * 2;                      // 64 KB: 2 K-chunks of [256 rows][64]
 constexpr int W2_BYTES = C * HID * 2;                      // 64 KB: 4 K-chunks of [128 rows][64]
 constexpr int ZT_BYTES = TP * C * 2;                       // 16 KB: [2 halves][64 pairs][64 ch]
-// z tiles in flight: 3, or 2 with fp32 output, whose staging is twice as large
 constexpr int H_BYTES = HID * TP * 2;                      // 32 KB: [256 rows][64 pairs]
 constexpr int OUT_ROWS = 32;                               // pairs per output warpgroup
 constexpr int TMEM_COLS = 512;
 constexpr int THREADS = 576;
 constexpr int TMA_WARP = 16, MMA_WARP = 17;
-constexpr int SMAX = 3;
+constexpr int SMAX = 2;                                    // z tiles in flight (each freed by GEMM1)
 
 struct Smem {
     uint64_t wbar;
@@ -54,8 +54,8 @@ struct Smem {
 
 template <bool OUT_F32>
 struct Cfg {
-    static constexpr int S = OUT_F32 ? 2 : 3;
-    static constexpr int STG_BYTES = OUT_ROWS * C * (OUT_F32 ? 4 : 2);   // per output warpgroup
+    static constexpr int S = SMAX;
+    static constexpr int STG_BYTES = OUT_ROWS * C * 4;     // per output warpgroup: [32 pairs][128] fp32
     static constexpr size_t SMEM = 1024 + W1_BYTES + W2_BYTES + S * ZT_BYTES + H_BYTES + 2 * STG_BYTES + 1024;
     static_assert(SMEM <= 232448, "shared memory");
 };
@@ -233,7 +233,9 @@ __global__ void __launch_bounds__(pt::THREADS, 1) pair_transition_kernel(const _
         }
     } else if (warp < 16) {
         // output warpgroup k: out[p, n] = z[p, n] + m_p (D2[n, p] + b2[n]) for the pairs
-        // [32k, 32k + 32) of the tile; thread = output channel n
+        // [32k, 32k + 32) of the tile. Phase 1, thread = output channel n: m_p (D2 + b2[n]) into
+        // the fp32 staging rows. Phase 2, thread = 8-channel row segments (4 of the block's 512):
+        // + z, rounded to the output type, in place.
         const int k = (warp - 8) >> 2;
         const int q = warp & 3;
         const int n = q * 32 + lane;
@@ -241,31 +243,41 @@ __global__ void __launch_bounds__(pt::THREADS, 1) pair_transition_kernel(const _
         const uint32_t lane_off = (uint32_t)(q * 32) << 16;
         const uint32_t bar_id = 3 + k;
         const bool leader = tk == 0;
-        uint8_t *stg = stg0 + k * Cfg<OUT_F32>::STG_BYTES;
+        float *stg = reinterpret_cast<float *>(stg0 + k * Cfg<OUT_F32>::STG_BYTES);
         const float bias = p.b2[n];
+        constexpr int SEGS = OUT_ROWS * C / 8 / 128;           // row segments per thread
+        // segment r of this thread: pair tk / 16 + 8 r of the block, channels 8 (tk % 16) + 0..7
+        const int seg_pair = tk >> 4, seg_ch = (tk & 15) * 8;
+        auto load_residual = [&](const TileWalk &w, uint4 (&dst)[SEGS]) {
+            const uint16_t *src = p.z + ((long long)w.b * p.NN + w.t * TP + k * OUT_ROWS + seg_pair) * C + seg_ch;
+#pragma unroll
+            for (int r = 0; r < SEGS; ++r) dst[r] = __ldg(reinterpret_cast<const uint4 *>(src + r * 8 * C));
+        };
         int j = 0;
         TileWalk tw(blockIdx.x, p.tiles_per_batch);
+        // one tile ahead: lane l of every warp holds the mask of pair 32k + l (bf16 bits), and
+        // zn the residual segments
         uint32_t mbits = 0x3F80u;
-        if (p.mask && blockIdx.x < num_tiles) mbits = p.mask[(long long)tw.b * p.NN + tw.t * TP + k * OUT_ROWS + lane];
+        uint4 zn[SEGS];
+        if (blockIdx.x < num_tiles) {
+            if (p.mask) mbits = p.mask[(long long)tw.b * p.NN + tw.t * TP + k * OUT_ROWS + lane];
+            load_residual(tw, zn);
+        }
         for (int t = blockIdx.x; t < num_tiles; t += gridDim.x, tw.advance(gridDim.x, p.tiles_per_batch), ++j) {
             const int b = tw.b;
-            const long long row0 = (long long)b * p.NN + tw.t * TP + k * OUT_ROWS;   // first pair of the block
             const int u = j & 1;
             const float mreg = __uint_as_float(mbits << 16);
+            uint4 zc[SEGS];
+#pragma unroll
+            for (int r = 0; r < SEGS; ++r) zc[r] = zn[r];
             uint32_t mbits_next = 0x3F80u;
-            if (p.mask && t + (int)gridDim.x < num_tiles) {
+            if (t + (int)gridDim.x < num_tiles) {
                 TileWalk tn = tw;
                 tn.advance(gridDim.x, p.tiles_per_batch);
-                mbits_next = p.mask[(long long)tn.b * p.NN + tn.t * TP + k * OUT_ROWS + lane];
+                if (p.mask) mbits_next = p.mask[(long long)tn.b * p.NN + tn.t * TP + k * OUT_ROWS + lane];
+                load_residual(tn, zn);
             }
             if (leader) tma_store_wait_read<0>();              // this warpgroup's previous store has read its rows
-            // the residual, z[p, n] for the block's 32 pairs (one 64-byte row segment per warp and
-            // pair, from L2: GEMM1's load has just brought the tile in), issued before the
-            // accumulator wait so that its latency overlaps it
-            uint32_t zr[OUT_ROWS];
-            const uint16_t *zp = p.z + row0 * C + n;
-#pragma unroll
-            for (int pp = 0; pp < OUT_ROWS; ++pp) zr[pp] = __ldg(zp + pp * C);
             if (!group_all(mbar_wait(&s.d2full[u], (uint32_t)(j >> 1) & 1, abort_flag, kErrTimeoutEpilogue), bar_id, 128)) break;
             tc_fence_after();
             float d[32];
@@ -275,17 +287,41 @@ __global__ void __launch_bounds__(pt::THREADS, 1) pair_transition_kernel(const _
             __syncwarp();
             if (lane == 0) mbar_arrive(&s.d2empty[u]);
 #pragma unroll
-            for (int pp = 0; pp < OUT_ROWS; ++pp) {
-                const float o = fmaf(__shfl_sync(0xffffffffu, mreg, pp), d[pp] + bias, __uint_as_float(zr[pp] << 16));
-                if (OUT_F32)
-                    reinterpret_cast<float *>(stg)[pp * C + n] = o;
-                else
-                    reinterpret_cast<uint16_t *>(stg)[pp * C + n] = __bfloat16_as_ushort(__float2bfloat16_rn(o));
+            for (int pp = 0; pp < OUT_ROWS; ++pp) stg[pp * C + n] = __shfl_sync(0xffffffffu, mreg, pp) * (d[pp] + bias);
+            named_bar_sync(bar_id, 128);
+            float v[SEGS][8];
+#pragma unroll
+            for (int r = 0; r < SEGS; ++r) {
+                const float4 *src = reinterpret_cast<const float4 *>(stg + (seg_pair + 8 * r) * C + seg_ch);
+                const float4 lo = src[0], hi = src[1];
+                const uint32_t zw[4] = {zc[r].x, zc[r].y, zc[r].z, zc[r].w};
+                const float f[8] = {lo.x, lo.y, lo.z, lo.w, hi.x, hi.y, hi.z, hi.w};
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    v[r][2 * e] = f[2 * e] + __uint_as_float(zw[e] << 16);
+                    v[r][2 * e + 1] = f[2 * e + 1] + __uint_as_float(zw[e] & 0xFFFF0000u);
+                }
+            }
+            if (OUT_F32) {
+#pragma unroll
+                for (int r = 0; r < SEGS; ++r) {               // the same addresses this thread read
+                    float4 *dst = reinterpret_cast<float4 *>(stg + (seg_pair + 8 * r) * C + seg_ch);
+                    dst[0] = make_float4(v[r][0], v[r][1], v[r][2], v[r][3]);
+                    dst[1] = make_float4(v[r][4], v[r][5], v[r][6], v[r][7]);
+                }
+            } else {
+                named_bar_sync(bar_id, 128);                   // every fp32 row is read before bf16 rows overwrite them
+                uint16_t *ob = reinterpret_cast<uint16_t *>(stg);
+#pragma unroll
+                for (int r = 0; r < SEGS; ++r)
+                    *reinterpret_cast<uint4 *>(ob + (seg_pair + 8 * r) * C + seg_ch) =
+                        make_uint4(pack_bf16x2(v[r][0], v[r][1]), pack_bf16x2(v[r][2], v[r][3]),
+                                   pack_bf16x2(v[r][4], v[r][5]), pack_bf16x2(v[r][6], v[r][7]));
             }
             fence_proxy_async_smem();
             named_bar_sync(bar_id, 128);
             if (leader) {
-                tma_store_3d(&p.tm_out, stg, 0, (int)(row0 - (long long)b * p.NN), b);
+                tma_store_3d(&p.tm_out, stg, 0, tw.t * TP + k * OUT_ROWS, b);
                 tma_store_commit();
             }
             mbits = mbits_next;
