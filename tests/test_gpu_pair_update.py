@@ -58,6 +58,25 @@ def test_pair_update_bf16_against_oracle(c_z, N, B, out_dtype):
     assert np.array_equal(got_mid[masked], z64[masked]) and np.array_equal(got[masked], z64[masked])
 
 
+def test_pair_update_full_size_bench_workload():
+    """The bench's pair-update leg: B=1 N=512 c_z=128, bf16 z, z_mid and out, ragged mask,
+    every entry against the oracle."""
+    inp, w_in, z, m, lo, li = _layers(1, 512, 128, "bf16", seed=512, mask=("uniform_len", 384, 512))
+    z_mid = torch.empty_like(z)
+    out = tm.pair_update(z, m, lo, li, z_mid=z_mid, out_dtype=torch.bfloat16)
+    torch.cuda.synchronize()
+    tm.check_device_status()
+    ref_mid, ref_out = oracle.pair_update(inp.z, inp.mask, inp.weights, w_in, inp.eps)
+    z64 = np.asarray(inp.z, dtype=np.float64)
+    half_ulp = 2.0 ** -8
+    b_mid, b_out = _bound(ref_mid, ref_out, z64, 2e-2, half_ulp, half_ulp)
+    got_mid, got = z_mid.float().cpu().numpy(), out.float().cpu().numpy()
+    assert np.all(np.abs(got_mid - ref_mid) <= b_mid), f"z_mid: worst excess {np.max(np.abs(got_mid - ref_mid) - b_mid):.3e}"
+    assert np.all(np.abs(got - ref_out) <= b_out), f"out: worst excess {np.max(np.abs(got - ref_out) - b_out):.3e}"
+    masked = inp.mask == 0
+    assert np.array_equal(got[masked], z64[masked])
+
+
 def test_pair_update_fp32_against_oracle():
     inp, w_in, z, m, lo, li = _layers(2, 48, 128, "f32", seed=5, mask=("uniform_len", 20, 48))
     out = tm.pair_update(z, m, lo, li)

@@ -56,6 +56,46 @@ def test_pair_transition_against_oracle(B, N, out_dtype, biases):
     print(f"pair transition B={B} N={N} {out_dtype}: max|err| / RMS(update) = {np.max(err) / rms(ref - z64):.3e}")
 
 
+def test_pair_transition_full_size_sampled():
+    """The bench's launch: B=1 N=512 (67 MB of z, 28 tiles per CTA), bf16 in and out, the
+    ragged mask of length 493; 4096 sampled pairs against the oracle (the transition acts on
+    each pair alone), every masked pair bitwise z."""
+    z, mask, w1, b1, w2, b2 = _problem(1, 512, seed=512, lengths=[493])
+    zd, md = _cuda(z), _cuda(mask)
+    pt = tm.PairTransition(_cuda(w1), _cuda(w2), _cuda(b1), _cuda(b2))
+    out = pt.forward(zd, md, out_dtype=torch.bfloat16)
+    torch.cuda.synchronize()
+    tm.check_device_status()
+    rng = np.random.default_rng(7)
+    flat = rng.choice(512 * 512, size=4096, replace=False)
+    i, j = flat // 512, flat % 512
+    zs, ms = z[0, i, j][None, None], mask[0, i, j][None, None]
+    ref = oracle.pair_transition(zs, ms, w1, b1, w2, b2)[0, 0]
+    got = out[0, torch.from_numpy(i).cuda(), torch.from_numpy(j).cuda()].float().cpu().numpy()
+    z64 = zs[0, 0].astype(np.float64)
+    upd = ref - z64
+    bound = 2e-2 * rms(upd) + 2.0 ** -8 * np.abs(ref)
+    assert np.all(np.abs(got - ref) <= bound), f"worst excess {np.max(np.abs(got - ref) - bound):.3e}"
+    masked = md == 0
+    assert bool(masked.any()) and torch.equal(out[masked], zd[masked])
+
+
+def test_pair_transition_tiles_across_batch_elements():
+    """B=3 N=200: 625 tiles per batch element, about 13 per CTA, so a CTA's tiles (and the
+    next-tile loads of the output warpgroups) cross from one batch element to the next."""
+    z, mask, w1, b1, w2, b2 = _problem(3, 200, seed=200, lengths=[200, 131, 77])
+    pt = tm.PairTransition(_cuda(w1), _cuda(w2), _cuda(b1), _cuda(b2))
+    out = pt.forward(_cuda(z), _cuda(mask), out_dtype=torch.float32)
+    torch.cuda.synchronize()
+    tm.check_device_status()
+    ref = oracle.pair_transition(z, mask, w1, b1, w2, b2)
+    got = out.cpu().numpy()
+    z64 = z.astype(np.float64)
+    err = np.abs(got - ref)
+    assert np.max(err) <= 2e-2 * rms(ref - z64), f"max err / RMS(update) {np.max(err) / rms(ref - z64):.3e}"
+    assert np.array_equal(got[mask == 0], z64[mask == 0])
+
+
 def test_pair_transition_without_mask_and_rejections():
     z, _, w1, b1, w2, b2 = _problem(1, 32, seed=3)
     pt = tm.PairTransition(_cuda(w1), _cuda(w2), _cuda(b1), _cuda(b2))
