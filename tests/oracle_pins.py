@@ -14,9 +14,9 @@ Sources of truth used here:
     projections exchanged, residue-permutation equivariance, masked residues k
     contribute nothing, padding equals truncation, sampled entries equal the
     full computation, invariance of the output under scaling of the b projection,
-  * the pair update (two residual steps): masked pairs keep z bitwise, and with one
-    step's output projection zeroed it reduces to the other step's single update in
-    its own direction.
+  * the pair update (two residual steps): masked pairs keep z bitwise, with one step's
+    output projection zeroed it reduces to the other step's single update in its own
+    direction, and a constant field goes through both steps in closed form.
 """
 from __future__ import annotations
 
@@ -144,27 +144,32 @@ def pin_full_update_library(lib):
 
 # ---------------------------------------------------------------- closed forms
 
-def pin_constant_field_closed_form(lib):
-    """z_ij = v everywhere, all-ones mask: every a_ik = alpha, b_jk = beta, so x_ij = N alpha*beta.
+def _constant_field_update(v, weights, N):
+    """The update of the constant field z_ij = v (all-ones mask) at every pair: every
+    a_ik = alpha, b_jk = beta, so x_ij = N alpha*beta. alpha, beta, the LayerNorm of
+    N alpha*beta and the gate are torch library calls on a single pair; the N^3 contraction
+    is replaced by the scalar N."""
+    w = {k: _t(x) for k, x in weights.items()}
+    c_z, c_h = w["w_ag"].shape[1], w["w_ag"].shape[0]
+    zh = F.layer_norm(_t(v), (c_z,), w["ln_in_g"], w["ln_in_b"], 1e-5)
+    alpha = torch.sigmoid(F.linear(zh, w["w_ag"], w["b_ag"])) * F.linear(zh, w["w_ap"], w["b_ap"])
+    beta = torch.sigmoid(F.linear(zh, w["w_bg"], w["b_bg"])) * F.linear(zh, w["w_bp"], w["b_bp"])
+    xv = N * alpha * beta
+    o = torch.sigmoid(F.linear(zh, w["w_g"], w["b_g"])) * F.linear(
+        F.layer_norm(xv, (c_h,), w["ln_out_g"], w["ln_out_b"], 1e-5), w["w_o"], w["b_o"])
+    return o.numpy()
 
-    alpha, beta, the LayerNorm of N alpha*beta and the gate are evaluated with
-    torch library calls on a single pair; the N^3 contraction is replaced by the
-    scalar N.
-    """
+
+def pin_constant_field_closed_form(lib):
+    """z_ij = v everywhere, all-ones mask: the update is the closed form above at every pair,
+    in both directions."""
     rng = np.random.default_rng(21)
     c_z, c_h = 6, 5
     base = ti.generate(1, 1, c_z, c_h, dtype="f32", seed=21, affine=True, biases=True)
-    w = {k: _t(v) for k, v in base.weights.items()}
     v = rng.standard_normal(c_z) * 2 + 0.5
     for N in (1, 4, 9):
         z = np.broadcast_to(v, (1, N, N, c_z)).copy()
-        zh = F.layer_norm(_t(v), (c_z,), w["ln_in_g"], w["ln_in_b"], 1e-5)
-        alpha = torch.sigmoid(F.linear(zh, w["w_ag"], w["b_ag"])) * F.linear(zh, w["w_ap"], w["b_ap"])
-        beta = torch.sigmoid(F.linear(zh, w["w_bg"], w["b_bg"])) * F.linear(zh, w["w_bp"], w["b_bp"])
-        xv = N * alpha * beta
-        o = torch.sigmoid(F.linear(zh, w["w_g"], w["b_g"])) * F.linear(
-            F.layer_norm(xv, (c_h,), w["ln_out_g"], w["ln_out_b"], 1e-5), w["w_o"], w["b_o"])
-        expect = np.broadcast_to(o.numpy(), (1, N, N, c_z))
+        expect = np.broadcast_to(_constant_field_update(v, base.weights, N), (1, N, N, c_z))
         for d in ("outgoing", "incoming"):
             _close(oracle.trimul(z, None, base.weights, d, 1e-5, lib=lib), expect,
                    rtol=1e-11, what=f"constant field N={N} {d}")
@@ -382,6 +387,23 @@ def pin_pair_update_second_step_is_incoming(lib):
     assert np.max(np.abs(out - wrong)) > 1e-6
 
 
+def pin_pair_update_constant_field(lib):
+    """A constant field stays constant through both steps: z_mid = v + u1(v) and
+    out = z_mid + u2(z_mid), with u1, u2 the closed-form constant-field updates of the two
+    layers. The second step must see z_mid, not z."""
+    rng = np.random.default_rng(23)
+    c_z, c_h, N = 6, 5, 4
+    l1 = ti.generate(1, 1, c_z, c_h, dtype="f32", seed=23, affine=True, biases=True).weights
+    l2 = ti.generate(1, 1, c_z, c_h, dtype="f32", seed=24, affine=True, biases=True).weights
+    v = rng.standard_normal(c_z) * 2 + 0.5
+    z = np.broadcast_to(v, (1, N, N, c_z)).copy()
+    mid = v + _constant_field_update(v, l1, N)
+    out = mid + _constant_field_update(mid, l2, N)
+    z_mid, got = oracle.pair_update(z, None, l1, l2, 1e-5, lib=lib)
+    _close(z_mid, np.broadcast_to(mid, z.shape), rtol=1e-11, what="pair update z_mid, constant field")
+    _close(got, np.broadcast_to(out, z.shape), rtol=1e-11, what="pair update out, constant field")
+
+
 # ---------------------------------------------------------------- pair transition
 
 
@@ -422,5 +444,6 @@ ALL_PINS = [
     pin_masked_k_contributes_nothing, pin_padding_equals_truncation, pin_sampled_equals_full,
     pin_b_projection_scale_invariance, pin_single_residue_directions_agree,
     pin_pair_update_masked_pairs_keep_z, pin_pair_update_first_step_is_outgoing,
-    pin_pair_update_second_step_is_incoming, pin_pair_transition_library, pin_pair_transition_closed_forms,
+    pin_pair_update_second_step_is_incoming, pin_pair_update_constant_field, pin_pair_transition_library,
+    pin_pair_transition_closed_forms,
 ]

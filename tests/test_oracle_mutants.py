@@ -3,8 +3,12 @@
 Each mutant is a single textual edit of oracle/trimul_oracle.c (a dropped term, a
 wrong sign, a transposed index, a swapped operand). The edited copy is compiled
 into a temporary library and the whole pin battery of oracle_pins.py runs
-against it. The real oracle source is never modified.
+against it. The steps written in Python (the pair update and the pair transition)
+are mutated the same way: the edited function is compiled from its source text and
+stands in for the real one while the pins run. The real oracle source is never
+modified.
 """
+import inspect
 import os
 
 import pytest
@@ -49,6 +53,53 @@ def test_mutant_is_caught(name, tmp_path):
     path = tmp_path / "mutant.c"
     path.write_text(src.replace(old, new))
     lib = oracle.load_library(oracle.compile_library(str(path), str(tmp_path / "libmutant.so"), force=True))
+    failed = []
+    for pin in oracle_pins.ALL_PINS:
+        try:
+            pin(lib)
+        except AssertionError:
+            failed.append(pin.__name__)
+    assert failed, f"no pin caught the planted mistake {name}"
+
+
+PY_MUTANTS = {
+    "pair_update_second_step_reads_z": ("pair_update", [
+        ('out = z_mid + trimul(z_mid, mask, weights_in, "incoming", eps, lib=lib)',
+         'out = z_mid + trimul(z, mask, weights_in, "incoming", eps, lib=lib)')]),
+    "pair_update_first_residual_dropped": ("pair_update", [
+        ('z_mid = z + trimul(z, mask, weights_out, "outgoing", eps, lib=lib)',
+         'z_mid = trimul(z, mask, weights_out, "outgoing", eps, lib=lib)')]),
+    "pair_update_second_residual_from_z": ("pair_update", [
+        ('out = z_mid + trimul(z_mid,', 'out = z + trimul(z_mid,')]),
+    "pair_update_directions_swapped": ("pair_update", [
+        ('weights_out, "outgoing", eps', 'weights_out, "incoming", eps'),
+        ('weights_in, "incoming", eps', 'weights_in, "outgoing", eps')]),
+    "pair_update_weights_swapped": ("pair_update", [
+        ('mask, weights_out, "outgoing"', 'mask, weights_in, "outgoing"'),
+        ('mask, weights_in, "incoming"', 'mask, weights_out, "incoming"')]),
+    "transition_relu_dropped": ("pair_transition", [("hid = np.maximum(hid, 0.0)", "hid = hid")]),
+    "transition_relu_as_abs": ("pair_transition", [("hid = np.maximum(hid, 0.0)", "hid = np.abs(hid)")]),
+    "transition_b1_dropped": ("pair_transition", [("hid = hid + _f64(b1)", "hid = hid")]),
+    "transition_b2_dropped": ("pair_transition", [("upd = upd + _f64(b2)", "upd = upd")]),
+    "transition_mask_dropped": ("pair_transition", [("upd = upd * _f64(mask)[..., None]", "upd = upd")]),
+    "transition_residual_dropped": ("pair_transition", [("return z + upd", "return upd")]),
+    "transition_b2_outside_mask": ("pair_transition", [
+        ("upd = upd + _f64(b2)", "pass"),
+        ("return z + upd", "return z + upd + (_f64(b2) if b2 is not None else 0.0)")]),
+}
+
+
+@pytest.mark.parametrize("name", sorted(PY_MUTANTS))
+def test_python_mutant_is_caught(name, monkeypatch):
+    func, edits = PY_MUTANTS[name]
+    src = inspect.getsource(getattr(oracle, func))
+    for old, new in edits:
+        assert src.count(old) == 1, f"mutation site for {name} must match exactly once: {old}"
+        src = src.replace(old, new)
+    namespace = dict(vars(oracle))
+    exec(compile(src, f"<mutant {name}>", "exec"), namespace)
+    monkeypatch.setattr(oracle, func, namespace[func])
+    lib = oracle.load_library()
     failed = []
     for pin in oracle_pins.ALL_PINS:
         try:
