@@ -259,7 +259,9 @@ trimul_status_t tri_mul_layer_set_mask_skipping(trimul_layer_t *layer, int enabl
  * into the handle (biases kept in fp32) and synchronizes `stream`. The forward takes z
  * [B, N, N, 128] bf16, a mask as tri_mul_forward, and writes out [B, N, N, 128] in F32 or
  * BF16 (not overlapping z); fp32 accumulation, the hidden activation rounded to f16 on
- * chip (W2 kept in f16 for that product); N % 8 == 0; sm_100 only. */
+ * chip (W2 kept in f16 for that product); N a multiple of 8 in [8, 16384] and
+ * B * N^2 / 64 < 2^31 (TRIMUL_ERR_UNSUPPORTED_SHAPE otherwise, checked before the handle);
+ * sm_100 only. */
 typedef struct trimul_transition trimul_transition_t;
 trimul_status_t tri_mul_transition_create(int c, int hidden, trimul_dtype_t dtype, const void *w1,
                                           const void *b1, const void *w2, const void *b2,

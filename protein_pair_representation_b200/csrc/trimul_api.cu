@@ -851,12 +851,17 @@ extern "C" void tri_mul_transition_destroy(trimul_transition_t *T) {
 
 extern "C" trimul_status_t tri_mul_transition_forward(const trimul_pair_t *z, const void *mask,
                                                       const trimul_transition_t *T, trimul_pair_t *out, void *stream) {
-    if (!T) return fail(TRIMUL_ERR_INVALID_ARG, "transition handle is NULL");
+    // shapes first (no handle needed), so that every size rule is checked before anything else
     TRY(check_pair(z, "z"));
     TRY(check_pair(out, "out"));
     if (z->dtype != TRIMUL_BF16) return fail(TRIMUL_ERR_UNSUPPORTED_SHAPE, "the pair transition takes a bf16 z");
+    if (z->N < 8 || z->N % 8 != 0 || z->N > 16384)
+        return fail(TRIMUL_ERR_UNSUPPORTED_SHAPE, "N=%lld must be a multiple of 8 in [8, 16384]", (long long)z->N);
+    // the kernel walks B * N^2 / 64 tiles with int indices and int pair coordinates
+    if ((long long)z->B * (z->N * z->N / 64) >= (1LL << 31))
+        return fail(TRIMUL_ERR_UNSUPPORTED_SHAPE, "problem too large: B * N^2 / 64 must stay below 2^31");
+    if (!T) return fail(TRIMUL_ERR_INVALID_ARG, "transition handle is NULL");
     if (z->C != T->c) return fail(TRIMUL_ERR_INVALID_ARG, "z has %lld channels, the transition %d", (long long)z->C, T->c);
-    if (z->N < 8 || z->N % 8 != 0) return fail(TRIMUL_ERR_UNSUPPORTED_SHAPE, "N=%lld must be a positive multiple of 8", (long long)z->N);
     if (mask && !aligned16(mask)) return fail(TRIMUL_ERR_ALIGNMENT, "mask not 16-byte aligned");
     if (out->B != z->B || out->N != z->N || out->C != z->C) return fail(TRIMUL_ERR_INVALID_ARG, "out shape differs from z");
     if (overlap(out->data, pair_bytes(out), z->data, pair_bytes(z))) return fail(TRIMUL_ERR_INVALID_ARG, "out overlaps z");

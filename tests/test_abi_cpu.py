@@ -110,6 +110,25 @@ def test_adjacent_f16_planes_pass_validation(lib):
     assert st in (3, 5), lib.tri_mul_last_error()
 
 
+def test_transition_validates_sizes_on_the_host(lib):
+    """Size rules are checked before the handle and before any device call: N a multiple of
+    8 in [8, 16384] (int pair coordinates in the kernel), B * N^2 / 64 tiles below 2^31."""
+    fake = 1 << 24                             # aligned, never dereferenced
+    def status(B, N, dtype=tm.BF16):
+        z = tm._Pair(fake, B, N, 128, dtype)
+        out = tm._Pair(fake << 8, B, N, 128, tm.BF16)
+        return lib.tri_mul_transition_forward(ctypes.byref(z), None, None, ctypes.byref(out), None)
+    assert status(1, 16392) == 2 and b"[8, 16384]" in lib.tri_mul_last_error()
+    assert status(1, 12) == 2
+    assert status(1, 64, tm.F32) == 2
+    assert status(600, 16384) == 2 and b"too large" in lib.tri_mul_last_error()
+    assert status(1, 16384) == 1 and b"handle is NULL" in lib.tri_mul_last_error()
+    z = tm._Pair(fake, 1, 64, 128, tm.BF16)
+    out = tm._Pair(fake, 1, 64, 128, tm.BF16)
+    assert lib.tri_mul_transition_forward(ctypes.byref(z), None, None, ctypes.byref(out), None) == 1
+    assert lib.tri_mul_transition_forward(None, None, None, None, None) == 1
+
+
 def test_pair_update_and_graph_validate_on_the_host(lib):
     z = tm._Pair(0, 1, 8, 128, tm.BF16)
     mid = tm._Pair(0, 1, 8, 128, tm.BF16)
