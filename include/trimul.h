@@ -140,9 +140,12 @@ trimul_status_t tri_mul_layer_bind_workspace(trimul_layer_t *layer, void *worksp
  *   mask : [B, N, N] in z's dtype with values 0 or 1, or NULL for all ones
  *   out  : [B, N, N, c_z]; F32 for the F32 path; F32 or BF16 for the BF16 path
  *          (must not overlap z or the workspace)
- * Requirements: N % 8 == 0 and N >= 8 (the pages pad token axes to multiples
- * of 8); B >= 1; every pointer 16-byte aligned; a workspace of at least
- * tri_mul_workspace_bytes() bound. The BF16 path needs an sm_100 device. */
+ * Requirements: N % 8 == 0 and 8 <= N <= 16384 (the pages pad token axes to
+ * multiples of 8); B >= 1 and B * c_h <= 65535; on the BF16 path B * N^2 / 128
+ * <= 2^30; every pointer 16-byte aligned; a workspace of at least
+ * tri_mul_workspace_bytes() bound. The BF16 path needs an sm_100 device. The N and
+ * tile rules are checked before the layer handle, B * c_h right after it; a violation
+ * returns TRIMUL_ERR_UNSUPPORTED_SHAPE with nothing launched. */
 trimul_status_t tri_mul_forward(const trimul_pair_t *z, const void *mask,
                                 const trimul_layer_t *layer, trimul_direction_t direction,
                                 trimul_pair_t *out, void *stream);

@@ -175,16 +175,20 @@ static size_t pair_bytes(const trimul_pair_t *t) {
 }
 
 static trimul_status_t check_problem(const trimul_pair_t *z, const void *mask, const trimul_layer_t *L) {
-    if (!L) return fail(TRIMUL_ERR_INVALID_ARG, "layer is NULL");
+    // the size rules first: they need no layer
     TRY(check_pair(z, "z"));
-    if (z->C != L->c_z) return fail(TRIMUL_ERR_INVALID_ARG, "z has %lld channels, layer expects c_z=%d", (long long)z->C, L->c_z);
     if (z->N < 8 || z->N % 8 != 0) return fail(TRIMUL_ERR_UNSUPPORTED_SHAPE, "N=%lld must be a positive multiple of 8", (long long)z->N);
     if (z->N > 16384) return fail(TRIMUL_ERR_UNSUPPORTED_SHAPE, "N=%lld exceeds 16384", (long long)z->N);
+    if (z->dtype == TRIMUL_BF16 && (long long)z->B * z->N * z->N / 128 > (1LL << 30))
+        return fail(TRIMUL_ERR_UNSUPPORTED_SHAPE, "problem too large: B * N^2 / 128 must not exceed 2^30");
+    if (!L) return fail(TRIMUL_ERR_INVALID_ARG, "layer is NULL");
+    if (z->C != L->c_z) return fail(TRIMUL_ERR_INVALID_ARG, "z has %lld channels, layer expects c_z=%d", (long long)z->C, L->c_z);
+    // the contraction's limit (B * c_h planes), checked here so that no stage has run when it fails
+    if ((long long)z->B * L->c_h > 65535)
+        return fail(TRIMUL_ERR_UNSUPPORTED_SHAPE, "B*c_h=%lld exceeds 65535", (long long)z->B * L->c_h);
     if (mask && !aligned16(mask)) return fail(TRIMUL_ERR_ALIGNMENT, "mask pointer not 16-byte aligned");
-    if (z->dtype == TRIMUL_BF16) {
-        if (!L->has_bf16) return fail(TRIMUL_ERR_UNSUPPORTED_SHAPE, "bf16 path supports (c_z, c_h) = (128,128) or (384,128); layer is (%d,%d)", L->c_z, L->c_h);
-        if ((long long)z->B * z->N * z->N / 128 > (1LL << 30)) return fail(TRIMUL_ERR_UNSUPPORTED_SHAPE, "problem too large");
-    }
+    if (z->dtype == TRIMUL_BF16 && !L->has_bf16)
+        return fail(TRIMUL_ERR_UNSUPPORTED_SHAPE, "bf16 path supports (c_z, c_h) = (128,128) or (384,128); layer is (%d,%d)", L->c_z, L->c_h);
     return TRIMUL_OK;
 }
 

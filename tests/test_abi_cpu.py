@@ -59,7 +59,25 @@ def test_null_arguments_are_rejected_on_the_host(lib):
     z = tm._Pair(0, 1, 8, 128, tm.BF16)
     out = tm._Pair(0, 1, 8, 128, tm.F32)
     assert lib.tri_mul_forward(ctypes.byref(z), None, None, 0, ctypes.byref(out), None) == 1
+    assert b"z: NULL tensor" in lib.tri_mul_last_error()
+    z = tm._Pair(1 << 24, 1, 8, 128, tm.BF16)        # aligned, never dereferenced
+    assert lib.tri_mul_forward(ctypes.byref(z), None, None, 0, ctypes.byref(out), None) == 1
     assert b"layer is NULL" in lib.tri_mul_last_error()
+
+
+def test_forward_validates_sizes_before_the_layer(lib):
+    """N a multiple of 8 in [8, 16384]; on the bf16 path B * N^2 / 128 tiles at most 2^30
+    (int tile indices in the kernels). Checked before the layer and any device call."""
+    out = tm._Pair(1 << 40, 1, 8, 128, tm.F32)
+    def status(B, N, dtype=tm.BF16):
+        z = tm._Pair(1 << 24, B, N, 128, dtype)
+        return lib.tri_mul_forward(ctypes.byref(z), None, None, 0, ctypes.byref(out), None)
+    assert status(1, 4) == 2
+    assert status(1, 100) == 2
+    assert status(1, 16392) == 2 and b"exceeds 16384" in lib.tri_mul_last_error()
+    assert status(513, 16384) == 2 and b"too large" in lib.tri_mul_last_error()
+    assert status(513, 16384, tm.F32) == 1               # the fp32 path has no tile limit
+    assert status(512, 16384) == 1 and b"layer is NULL" in lib.tri_mul_last_error()
 
 
 def test_contract_validation_happens_before_any_launch(lib):
