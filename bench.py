@@ -52,6 +52,8 @@ def parse_args():
     ap.add_argument("--skip-masked", action="store_true",
                     help="switch mask skipping on (leave out wholly masked tiles; off by default)")
     ap.add_argument("--no-transition", action="store_true", help="skip the pair-transition leg")
+    ap.add_argument("--no-torch-context", action="store_true",
+                    help="skip timing the eager PyTorch composition of the same math (context only)")
     ap.add_argument("--no-pair-update", action="store_true",
                     help="skip the pair-update leg (outgoing + incoming with residuals, eager and as a CUDA graph)")
     return ap.parse_args()
@@ -276,6 +278,49 @@ def pair_update_leg(tm, layer, zs, ms_, n_sets, args, dev):
         return {"error": f"{type(exc).__name__}: {exc}"}
 
 
+def torch_composition(z, mask, w, direction, eps):
+    """The same update as a plain eager PyTorch composition (layer_norm, linear, sigmoid,
+    einsum): a context figure for the hand-written kernels, not part of the library.
+    w holds the layer's sixteen arrays under the ABI names; biases and affines may be None."""
+    import torch
+    F = torch.nn.functional
+    zh = F.layer_norm(z, (z.shape[-1],), w["ln_in_g"], w["ln_in_b"], eps)
+    m = 1.0 if mask is None else mask[..., None]
+    a = m * torch.sigmoid(F.linear(zh, w["w_ag"], w["b_ag"])) * F.linear(zh, w["w_ap"], w["b_ap"])
+    b = m * torch.sigmoid(F.linear(zh, w["w_bg"], w["b_bg"])) * F.linear(zh, w["w_bp"], w["b_bp"])
+    if direction == "outgoing":
+        x = torch.einsum("bikc,bjkc->bijc", a, b)
+    else:
+        x = torch.einsum("bkic,bkjc->bijc", a, b)
+    xn = F.layer_norm(x, (x.shape[-1],), w["ln_out_g"], w["ln_out_b"], eps)
+    return m * torch.sigmoid(F.linear(zh, w["w_g"], w["b_g"])) * F.linear(xn, w["w_o"], w["b_o"])
+
+
+def torch_composition_leg(zs, ms_, w, eps, dirs, n_sets, args):
+    """ms per layer of torch_composition on the same bf16 inputs and weights (cuBLAS GEMMs and
+    a batched-GEMM einsum, all eager), timed like the main leg: context, not a target."""
+    import torch
+    try:
+        def step(s):
+            for d in dirs:
+                torch_composition(zs[s % n_sets], ms_[s % n_sets], w, d, eps)
+
+        for s in range(max(3, args.warmup)):
+            step(s)
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        for s in range(args.steps):
+            step(s)
+        e1.record()
+        torch.cuda.synchronize()
+        return {"ms_per_layer": e0.elapsed_time(e1) / (args.steps * len(dirs)),
+                "what": "eager PyTorch composition of the same math (layer_norm, linear, sigmoid, einsum) "
+                        "on the same bf16 inputs; context, not a target"}
+    except Exception as exc:       # the headline line must not depend on this leg
+        return {"error": f"{type(exc).__name__}: {exc}"}
+
+
 def transition_leg(tm, zs, ms_, n_sets, args, dev):
     """The fused pair transition (out = z + m (relu(z W1^T + b1) W2^T + b2), c = 128, hidden 256)
     on this rank's pair tensors, bf16 in and out, seeded random weights; per-call ms from CUDA
@@ -432,6 +477,7 @@ def run_ours(args):
 
     pair = None if args.no_pair_update else pair_update_leg(tm, layer, zs, ms_, n_sets, args, dev)
     trans = None if (args.no_transition or inp.c_z != 128) else transition_leg(tm, zs, ms_, n_sets, args, dev)
+    context = None if args.no_torch_context else torch_composition_leg(zs, ms_, w, inp.eps, dirs, n_sets, args)
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline and args.workload in CPU_BASELINE_WORKLOADS:
@@ -483,7 +529,7 @@ def run_ours(args):
         "effective_tflops": sum(flops.values()) / (layer_ms_single * 1e-3) / 1e12 * world,
         "layer_roofline_frac": t_ideal / (layer_ms_single * 1e-3),
         "roofline": roof, "kernels": kernels, "cpu_baseline": cpu, "e2e": e2e, "pair_update": pair,
-        "pair_transition": trans,
+        "pair_transition": trans, "torch_composition": context,
         "gpu_launches": args.steps * len(dirs) * (tm.kernels_per_forward() + (1 if args.skip_masked else 0)),
         "clocks": clock_info,
     }
