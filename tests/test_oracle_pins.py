@@ -18,15 +18,20 @@ def test_pin(pin):
 
 
 def test_golden_regression_fixture():
-    """The oracle still reproduces the values its own committed script wrote (drift guard)."""
+    """The oracle still reproduces the values its own committed script wrote (drift guard):
+    the update in both directions, the pair update and the pair transition."""
+    import importlib.util
+    spec = importlib.util.spec_from_file_location("make_oracle_small", os.path.join(GOLDEN, "make_oracle_small.py"))
+    maker = importlib.util.module_from_spec(spec)
+    spec.loader.exec_module(maker)
     with open(os.path.join(GOLDEN, "oracle_small.json")) as f:
         g = json.load(f)
-    inp = ti.generate(g["B"], g["N"], g["c_z"], g["c_h"], dtype=g["dtype"], seed=g["seed"],
-                      mask=tuple(g["mask"]), affine=True, biases=True)
-    for d in ("outgoing", "incoming"):
-        out = oracle.trimul(inp.z, inp.mask, inp.weights, d, inp.eps)
-        idx = tuple(np.array(g["index"]).T)
-        np.testing.assert_allclose(out[idx], np.array(g[d]), rtol=1e-12, atol=1e-14)
+    idx = tuple(np.array(g["index"]).T)
+    vals = maker.oracle_values({k: g[k] for k in ("B", "N", "c_z", "c_h", "dtype", "seed", "mask")})
+    keys = ("outgoing", "incoming", "pair_update_mid", "pair_update_out", "pair_transition")
+    assert set(keys) <= set(g) and set(vals) == set(keys)
+    for k in keys:
+        np.testing.assert_allclose(vals[k][idx], np.array(g[k]), rtol=1e-12, atol=1e-14, err_msg=k)
 
 
 def test_empty_problem():
