@@ -1,10 +1,14 @@
 """Benchmark of the triangle multiplicative update on B200 (one JSON line on rank 0).
 
 A step is one pass of the hot path over one batch of synthetic input: the outgoing and
-the incoming update (tri_mul_forward twice, three kernels each) on the OpenFold-shaped
-pair workload B=1, N=512, c_z=c_h=128, bf16 z with a ragged padding mask. `value` is
-milliseconds per layer (one direction) for the whole job; several GPUs run independent
-replicas (weak scaling, no collective on the data path).
+the incoming update (tri_mul_forward twice: K1, the offsets pass, K2 and K3 each) on the
+OpenFold-shaped pair workload B=1, N=512, c_z=c_h=128, bf16 z with a ragged padding mask.
+`value` is milliseconds per layer (one direction) for the whole job, timed with nothing but
+the forwards in the timed region; a second, instrumented pass records CUDA events between
+the kernels for the per-kernel breakdown and the roofline. Several GPUs run independent
+replicas (weak scaling, no collective on the data path). On one GPU the line also carries
+`workloads`: the same two measurements for the other seeded configurations (N=256 with its
+tail mask, B=4 N=256 c_z=384, and N=2048 incoming then outgoing).
 
   python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
 
@@ -31,6 +35,12 @@ METRIC = "ms/layer and effective TFLOP/s (fraction of bf16 roofline) for tri-mul
 WORKLOAD = "bf16_n512_ragged"
 WORKLOADS = ("bf16_n512_ragged", "bf16_n256_tail10", "bf16_b4_n256_cz384", "bf16_n2048")
 CPU_BASELINE_WORKLOADS = ("bf16_n512_ragged", "bf16_n256_tail10", "bf16_b4_n256_cz384")
+# the other configurations timed on one GPU next to the headline (the N=64 fp32 one is launch-bound)
+EXTRA_WORKLOADS = ("bf16_n256_tail10", "bf16_b4_n256_cz384", "bf16_n2048")
+# oracle timings on the host: (workload, threads) pairs run by default; --cpu-full runs all of
+# fp32_n64 ... bf16_b4_n256_cz384 on all threads and on one
+CPU_DEFAULT_RUNS = (("fp32_n64", 0), ("bf16_n256_tail10", 0), ("bf16_n512_ragged", 0), ("bf16_b4_n256_cz384", 0),
+                    ("fp32_n64", 1), ("bf16_n256_tail10", 1))
 L2_BYTES = 126 * 1024 * 1024
 KERNEL_NAMES = ("k1_project_kernel", "k2_contract_kernel", "k3_output_kernel")
 KERNEL_SOURCES = {"k1_project_kernel": "k1_project.cu", "k2_contract_kernel": "k2_contract.cu",
@@ -56,7 +66,22 @@ def parse_args():
                     help="skip timing the eager PyTorch composition of the same math (context only)")
     ap.add_argument("--no-pair-update", action="store_true",
                     help="skip the pair-update leg (outgoing + incoming with residuals, eager and as a CUDA graph)")
+    ap.add_argument("--no-workloads", action="store_true", help="skip timing the other seeded configurations")
+    ap.add_argument("--cpu-full", action="store_true",
+                    help="time the oracle on every CPU configuration on all threads and on one thread")
+    ap.add_argument("--cpu-oracle-probe", nargs=2, metavar=("WORKLOAD", "DIRECTION"), default=None,
+                    help=argparse.SUPPRESS)   # internal: one oracle layer in a fresh process (OMP_NUM_THREADS set)
     return ap.parse_args()
+
+
+def valid_work(lengths, c_z, c_h):
+    """Flops of one layer counting only the valid residues (the work a length-L problem needs):
+    the dense formulas of layer_work with N replaced by each batch element's valid length L_b."""
+    total = 0
+    for L in lengths:
+        f, _ = layer_work(1, int(L), c_z, c_h)
+        total += sum(f.values())
+    return total
 
 
 def layer_work(B, N, c_z, c_h, out_bytes=4):
@@ -202,6 +227,48 @@ def cpu_oracle_layer_ms(inp, directions):
     return statistics.mean(times), oracle.num_threads()
 
 
+def cpu_model():
+    try:
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.startswith("model name"):
+                    return line.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    import platform
+    return platform.processor() or "unknown"
+
+
+def cpu_oracle_probe(workload, direction):
+    """One oracle layer of `workload` in this (fresh) process; prints its JSON timing."""
+    import oracle
+    import trimul_inputs as ti
+    inp = ti.make_config(workload)
+    t0 = time.perf_counter()
+    oracle.trimul(inp.z, inp.mask, inp.weights, direction, inp.eps)
+    print(json.dumps({"ms": (time.perf_counter() - t0) * 1e3, "threads": oracle.num_threads()}), flush=True)
+
+
+def cpu_oracle_runs(runs):
+    """Oracle wall-clock ms per layer for (workload, threads) pairs, each in a fresh process
+    (threads 0: all of the host's, else OMP_NUM_THREADS=threads), outgoing direction."""
+    out = []
+    for workload, threads in runs:
+        env = dict(os.environ)
+        if threads:
+            env["OMP_NUM_THREADS"] = str(threads)
+        else:
+            env.pop("OMP_NUM_THREADS", None)
+        try:
+            r = subprocess.run([sys.executable, os.path.abspath(__file__), "--cpu-oracle-probe", workload, "outgoing"],
+                               env=env, capture_output=True, text=True, timeout=900, cwd=ROOT)
+            rec = json.loads(r.stdout.strip().splitlines()[-1])
+            out.append({"workload": workload, "threads": rec["threads"], "ms_per_layer": rec["ms"]})
+        except Exception as exc:                  # the line must not depend on this leg
+            out.append({"workload": workload, "threads": threads or None, "error": f"{type(exc).__name__}: {exc}"})
+    return out
+
+
 def run_reference(args):
     """The oracle on the host cores: each step computes one full layer (directions alternate)."""
     rank, world, _ = dist_setup(args.gpus)
@@ -232,7 +299,8 @@ def run_reference(args):
         "higher_is_better": False, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
         "config": workload_config(inp, "f64"),
         "effective_tflops": sum(flops.values()) / (ms_layer * 1e-3) / 1e12,
-        "cpu_baseline": {"value": ms_layer, "unit": "ms/layer", "cores": cores, "kind": "oracle", "sample": sample},
+        "cpu_baseline": {"value": ms_layer, "unit": "ms/layer", "cores": cores, "kind": "oracle", "sample": sample,
+                         "cpu_model": cpu_model(), "nproc": os.cpu_count()},
         "e2e": {"value": ms_layer, "unit": "ms/layer", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
         "gpu_launches": 0,
     }
@@ -346,15 +414,16 @@ def transition_leg(tm, zs, ms_, n_sets, args, dev):
         tm.check_device_status()
         ms = e0.elapsed_time(e1) / args.steps
         P = zs[0].shape[0] * zs[0].shape[1] * zs[0].shape[2]
-        nbytes = P * (2 * 128 + 2 + 2 * 128)           # z in, mask, out (bf16)
-        flops = P * 2 * 2 * 128 * 256
+        c, hidden = pt.c, pt.hidden
+        nbytes = P * (2 * c + 2 + 2 * c)               # z in, mask, out (bf16)
+        flops = P * 2 * 2 * c * hidden
         peaks = measured_peaks()
         gbs, tfs = nbytes / (ms * 1e-3) / 1e9, flops / (ms * 1e-3) / 1e12
         pt.close()
         return {"ms": ms, "GB_s": gbs, "TFLOP_s": tfs, "hbm_frac": gbs / peaks["hbm_gbs"],
                 "tensor_frac": tfs / peaks["bf16_tflops"], "bytes": nbytes, "flops": flops,
                 "traffic": recorded_traffic("pair_transition_kernel"),
-                "shape": "c=128, hidden=256, bf16 in/out, fp16 hidden activation on chip"}
+                "shape": f"c={c}, hidden={hidden}, bf16 in/out, fp16 hidden activation on chip"}
     except Exception as exc:       # the headline line must not depend on this leg
         return {"error": f"{type(exc).__name__}: {exc}"}
 
@@ -369,13 +438,112 @@ def workload_config(inp, compute):
             "directions": ["outgoing", "incoming"], "compute": compute}
 
 
+class Workload:
+    """One seeded configuration on this rank's GPU: inputs (cycled through enough copies that
+    every step reads z and the mask from outside L2), the layer with its workspace, outputs."""
+
+    def __init__(self, tm, name, seed, dev, out_dt, skip_masked):
+        import numpy as np
+        import torch
+
+        import trimul_inputs as ti
+        self.name = name
+        self.inp = inp = ti.make_config(name, seed=seed)
+        self.dirs = ti.CONFIGS[name]["directions"]
+        self.z0 = torch.from_numpy(inp.z).to(dev).to(torch.bfloat16)
+        self.m0 = torch.from_numpy(inp.mask).to(dev).to(torch.bfloat16)
+        self.w = {k: torch.from_numpy(np.ascontiguousarray(v)).to(dev).to(torch.bfloat16) for k, v in inp.weights.items()}
+        self.layer = tm.TriMulLayer(self.w, eps=inp.eps)
+        self.layer.ensure_workspace(inp.B, inp.N, torch.bfloat16)
+        if skip_masked:
+            self.layer.set_mask_skipping(True)
+        self.set_bytes = self.z0.numel() * 2 + self.m0.numel() * 2
+        # one copy when it alone is over twice the L2, else enough copies to be
+        self.n_sets = 1 if self.set_bytes >= 2 * L2_BYTES else max(2, -(-2 * L2_BYTES // self.set_bytes))
+        self.zs = [self.z0] + [self.z0.clone() for _ in range(self.n_sets - 1)]
+        self.ms = [self.m0] + [self.m0.clone() for _ in range(self.n_sets - 1)]
+        self.outs = [torch.empty(self.z0.shape, dtype=out_dt, device=dev) for _ in self.dirs]
+        self.out_bytes = 4 if out_dt == torch.float32 else 2
+
+    def step(self, s, evs=None):
+        for di, d in enumerate(self.dirs):
+            if evs is not None:
+                self.layer.set_timing_events(evs[di])
+            self.layer.forward(self.zs[s % self.n_sets], self.ms[s % self.n_sets], d, out=self.outs[di])
+        if evs is not None:
+            self.layer.set_timing_events(None)
+
+    def l2_note(self):
+        if self.n_sets == 1:
+            return f"z and mask ({self.set_bytes / 2**20:.0f} MiB) larger than twice the 126 MiB L2"
+        return f"z and mask cycle through {self.n_sets} copies ({self.n_sets * self.set_bytes / 2**20:.0f} MiB > 126 MiB L2)"
+
+
+def time_steps(wl, steps, first, sync_all, dist=None, dev=None, instrumented=False):
+    """Device ms of `steps` steps (CUDA events on the launching stream, barrier + synchronize on
+    both sides, max over ranks) and, when instrumented, the per-kernel mean ms from the four
+    events each forward records between its kernels."""
+    import torch
+    kev = None
+    if instrumented:
+        kev = [[[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in wl.dirs] for _ in range(steps)]
+        for ev in kev:                   # torch creates the CUDA event on first record
+            for row in ev:
+                for e in row:
+                    e.record()
+        torch.cuda.synchronize()
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    sync_all()
+    t0.record()
+    for s in range(steps):
+        wl.step(first + s, kev[s] if instrumented else None)
+    t1.record()
+    sync_all()
+    elapsed = max_over_ranks(t0.elapsed_time(t1), dist, dev)
+    kernel_ms = None
+    if instrumented:
+        kernel_ms = {k: statistics.mean(ev[d][i].elapsed_time(ev[d][i + 1]) for ev in kev for d in range(len(wl.dirs)))
+                     for i, k in enumerate(KERNEL_NAMES)}
+    return elapsed, kernel_ms
+
+
+def kernel_record(inp, kernel_ms, peaks, out_bytes):
+    flops, nbytes = layer_work(inp.B, inp.N, inp.c_z, inp.c_h, out_bytes)
+    kernels = {}
+    for k in KERNEL_NAMES:
+        t = kernel_ms[k] * 1e-3
+        t_hbm = nbytes[k] / (peaks["hbm_gbs"] * 1e9)
+        t_tc = flops[k] / (peaks["bf16_tflops"] * 1e12)
+        kernels[k] = {"ms": kernel_ms[k], "GB_s": nbytes[k] / t / 1e9, "TFLOP_s": flops[k] / t / 1e12,
+                      "hbm_frac": nbytes[k] / t / 1e9 / peaks["hbm_gbs"],
+                      "tensor_frac": flops[k] / t / 1e12 / peaks["bf16_tflops"],
+                      "bound": "hbm" if t_hbm >= t_tc else "tensor", "roofline_frac": max(t_hbm, t_tc) / t,
+                      "bytes": nbytes[k], "flops": flops[k]}
+    t_ideal = sum(max(nbytes[k] / (peaks["hbm_gbs"] * 1e9), flops[k] / (peaks["bf16_tflops"] * 1e12))
+                  for k in KERNEL_NAMES)
+    return kernels, flops, t_ideal
+
+
+def workload_summary(wl, layer_ms, kernel_ms, instr_layer_ms, peaks):
+    """The record of one configuration: clean and instrumented ms per layer, per-kernel
+    figures, the layer's roofline fraction and its flops dense and at the valid lengths."""
+    inp = wl.inp
+    kernels, flops, t_ideal = kernel_record(inp, kernel_ms, peaks, wl.out_bytes)
+    dense = sum(flops.values())
+    at_l = valid_work(inp.lengths, inp.c_z, inp.c_h)
+    return {"config": workload_config(inp, "bf16 operands, fp16 a/b/x, fp32 accumulation"),
+            "directions": list(wl.dirs), "ms_per_layer": layer_ms, "ms_per_layer_instrumented": instr_layer_ms,
+            "effective_tflops": dense / (layer_ms * 1e-3) / 1e12,
+            "flops_dense": dense, "flops_at_valid_length": at_l,
+            "tflops_at_valid_length": at_l / (layer_ms * 1e-3) / 1e12,
+            "layer_roofline_frac": t_ideal / (layer_ms * 1e-3), "kernels": kernels, "l2": wl.l2_note()}
+
+
 def run_ours(args):
     import datetime
 
-    import numpy as np
     import torch
 
-    import trimul_inputs as ti
     from protein_pair_representation_b200 import trimul as tm
 
     rank, world, local = dist_setup(args.gpus)
@@ -386,46 +554,17 @@ def run_ours(args):
         import torch.distributed as dist
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
 
-    inp = ti.make_config(args.workload, seed=rank)     # every replica its own seeded problem
-    dirs = ti.CONFIGS[args.workload]["directions"]
-    out_dt = torch.float32 if args.out_dtype == "f32" else torch.bfloat16
-    z0 = torch.from_numpy(inp.z).to(dev).to(torch.bfloat16)
-    m0 = torch.from_numpy(inp.mask).to(dev).to(torch.bfloat16)
-    w = {k: torch.from_numpy(np.ascontiguousarray(v)).to(dev).to(torch.bfloat16) for k, v in inp.weights.items()}
-    layer = tm.TriMulLayer(w, eps=inp.eps)
-    layer.ensure_workspace(inp.B, inp.N, torch.bfloat16)
-    if args.skip_masked:
-        layer.set_mask_skipping(True)
-    # inputs cycle through enough copies that every step reads z from outside L2
-    set_bytes = z0.numel() * 2 + m0.numel() * 2
-    n_sets = max(2, -(-2 * L2_BYTES // set_bytes))
-    zs = [z0] + [z0.clone() for _ in range(n_sets - 1)]
-    ms_ = [m0] + [m0.clone() for _ in range(n_sets - 1)]
-    outs = [torch.empty(z0.shape, dtype=out_dt, device=dev) for _ in dirs]
-
-    def step(s, evs=None):
-        for di, d in enumerate(dirs):
-            if evs is not None:
-                layer.set_timing_events(evs[di])
-            layer.forward(zs[s % n_sets], ms_[s % n_sets], d, out=outs[di])
-        if evs is not None:
-            layer.set_timing_events(None)
-
     def sync_all():
         if dist is not None:
             dist.barrier()
         torch.cuda.synchronize()
 
+    out_dt = torch.float32 if args.out_dtype == "f32" else torch.bfloat16
+    wl = Workload(tm, args.workload, rank, dev, out_dt, args.skip_masked)   # every replica its own seeded problem
+    inp, dirs = wl.inp, wl.dirs
     for s in range(args.warmup):
-        step(s)
+        wl.step(s)
     tm.check_device_status()
-    kev = [[[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in dirs] for _ in range(args.steps)]
-    for ev in kev:                       # torch creates the CUDA event on first record
-        for row in ev:
-            for e in row:
-                e.record()
-    torch.cuda.synchronize()
-    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     smi_index = local
     if os.environ.get("CUDA_VISIBLE_DEVICES"):
         try:
@@ -435,31 +574,28 @@ def run_ours(args):
     clocks = ClockSampler(smi_index)
     clocks.start()
     time.sleep(0.4)
-    sync_all()
-    t0.record()
-    for s in range(args.steps):
-        step(args.warmup + s, kev[s])
-    t1.record()
-    sync_all()
+    # the headline: nothing but the forwards in the timed region
+    elapsed, _ = time_steps(wl, args.steps, args.warmup, sync_all, dist, dev)
     clock_info = clocks.stop()
     tm.check_device_status()
-    elapsed = max_over_ranks(t0.elapsed_time(t1), dist, dev)
-    kernel_ms = {k: statistics.mean(ev[d][i].elapsed_time(ev[d][i + 1]) for ev in kev for d in range(len(dirs)))
-                 for i, k in enumerate(KERNEL_NAMES)}
+    # the per-kernel breakdown: the same steps with events between the kernels
+    instr_elapsed, kernel_ms = time_steps(wl, args.steps, args.warmup + args.steps, sync_all, dist, dev,
+                                          instrumented=True)
+    tm.check_device_status()
 
     # host-buffer end to end: pinned inputs in, results out, every step
     e2e = None
     if not args.no_e2e:
-        z_host = z0.cpu().pin_memory()
-        m_host = m0.cpu().pin_memory()
-        out_host = [torch.empty(z0.shape, dtype=out_dt, pin_memory=True) for _ in dirs]
+        z_host = wl.z0.cpu().pin_memory()
+        m_host = wl.m0.cpu().pin_memory()
+        out_host = [torch.empty(wl.z0.shape, dtype=out_dt, pin_memory=True) for _ in dirs]
 
         def e2e_step():
-            zs[0].copy_(z_host, non_blocking=True)
-            ms_[0].copy_(m_host, non_blocking=True)
+            wl.zs[0].copy_(z_host, non_blocking=True)
+            wl.ms[0].copy_(m_host, non_blocking=True)
             for di, d in enumerate(dirs):
-                layer.forward(zs[0], ms_[0], d, out=outs[di])
-                out_host[di].copy_(outs[di], non_blocking=True)
+                wl.layer.forward(wl.zs[0], wl.ms[0], d, out=wl.outs[di])
+                out_host[di].copy_(wl.outs[di], non_blocking=True)
 
         for _ in range(max(1, args.warmup)):
             e2e_step()
@@ -475,16 +611,41 @@ def run_ours(args):
                "h2d_bytes_per_step": z_host.numel() * 2 + m_host.numel() * 2,
                "d2h_bytes_per_step": sum(o.numel() * o.element_size() for o in out_host)}
 
-    pair = None if args.no_pair_update else pair_update_leg(tm, layer, zs, ms_, n_sets, args, dev)
-    trans = None if (args.no_transition or inp.c_z != 128) else transition_leg(tm, zs, ms_, n_sets, args, dev)
-    context = None if args.no_torch_context else torch_composition_leg(zs, ms_, w, inp.eps, dirs, n_sets, args)
+    pair = None if args.no_pair_update else pair_update_leg(tm, wl.layer, wl.zs, wl.ms, wl.n_sets, args, dev)
+    trans = None if (args.no_transition or inp.c_z != 128) else transition_leg(tm, wl.zs, wl.ms, wl.n_sets, args, dev)
+    context = None if args.no_torch_context else torch_composition_leg(wl.zs, wl.ms, wl.w, inp.eps, dirs, wl.n_sets, args)
+
+    peaks = measured_peaks()
+    workloads = None
+    if world == 1 and not args.no_workloads:
+        workloads = {}
+        for name in EXTRA_WORKLOADS:
+            if name == args.workload:
+                continue
+            try:
+                other = Workload(tm, name, 0, dev, out_dt, args.skip_masked)
+                for s in range(max(3, args.warmup)):
+                    other.step(s)
+                w_el, _ = time_steps(other, args.steps, 0, sync_all)
+                w_iel, w_kms = time_steps(other, args.steps, args.steps, sync_all, instrumented=True)
+                tm.check_device_status()
+                n_layers = args.steps * len(other.dirs)
+                workloads[name] = workload_summary(other, w_el / n_layers, w_kms, w_iel / n_layers, peaks)
+                del other
+                torch.cuda.empty_cache()
+            except Exception as exc:        # the headline line must not depend on this leg
+                workloads[name] = {"error": f"{type(exc).__name__}: {exc}"}
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline and args.workload in CPU_BASELINE_WORKLOADS:
         ms_cpu, cores = cpu_oracle_layer_ms(inp, dirs)
+        runs = ([(w, t) for w in ("fp32_n64",) + CPU_BASELINE_WORKLOADS for t in (0, 1)] if args.cpu_full
+                else list(CPU_DEFAULT_RUNS))
         cpu = {"value": ms_cpu, "unit": "ms/layer", "cores": cores, "kind": "oracle",
                "sample": f"one full layer per direction ({', '.join(dirs)}) of the same workload, fp64, "
-                         f"wall clock on {cores} threads"}
+                         f"wall clock on {cores} threads",
+               "cpu_model": cpu_model(), "nproc": os.cpu_count(),
+               "per_config": cpu_oracle_runs(runs)}
 
     if dist is not None:
         dist.barrier()
@@ -492,20 +653,11 @@ def run_ours(args):
     if rank != 0:
         return
 
-    peaks = measured_peaks()
-    out_bytes = 4 if out_dt == torch.float32 else 2
-    flops, nbytes = layer_work(inp.B, inp.N, inp.c_z, inp.c_h, out_bytes)
+    n_layers = args.steps * len(dirs)
     layer_ms = job_ms_per_layer(elapsed, args.steps, len(dirs), world)
-    layer_ms_single = elapsed / (args.steps * len(dirs))
-    kernels = {}
-    for k in KERNEL_NAMES:
-        t = kernel_ms[k] * 1e-3
-        t_hbm = nbytes[k] / (peaks["hbm_gbs"] * 1e9)
-        t_tc = flops[k] / (peaks["bf16_tflops"] * 1e12)
-        kernels[k] = {"ms": kernel_ms[k], "GB_s": nbytes[k] / t / 1e9, "TFLOP_s": flops[k] / t / 1e12,
-                      "hbm_frac": nbytes[k] / t / 1e9 / peaks["hbm_gbs"],
-                      "tensor_frac": flops[k] / t / 1e12 / peaks["bf16_tflops"],
-                      "bound": "hbm" if t_hbm >= t_tc else "tensor", "roofline_frac": max(t_hbm, t_tc) / t}
+    layer_ms_single = elapsed / n_layers
+    kernels, flops, t_ideal = kernel_record(inp, kernel_ms, peaks, wl.out_bytes)
+    nbytes = {k: kernels[k]["bytes"] for k in KERNEL_NAMES}
     dom = max(KERNEL_NAMES, key=lambda k: kernel_ms[k])
     kd = kernels[dom]
     if kd["bound"] == "hbm":
@@ -514,23 +666,28 @@ def run_ours(args):
     else:
         roof = {"kernel": dom, "bound": "tensor", "achieved": kd["TFLOP_s"], "peak": peaks["bf16_tflops"],
                 "unit": "TFLOP/s", "frac": kd["tensor_frac"], "peak_source": f"{peaks['source']} (bf16 burst; fp16 equal)"}
-    tr = recorded_traffic(dom)
-    roof["traffic"] = tr
+    roof["traffic"] = recorded_traffic(dom)
     roof["algorithmic_bytes"] = nbytes[dom]
-    t_ideal = sum(max(nbytes[k] / (peaks["hbm_gbs"] * 1e9), flops[k] / (peaks["bf16_tflops"] * 1e12))
-                  for k in KERNEL_NAMES)
+    roof["timing"] = ("mean of the kernel's CUDA-event interval in the instrumented pass"
+                      + (" (K1's interval also holds the small offsets pass that follows it)" if dom == KERNEL_NAMES[0] else ""))
+    dense = sum(flops.values())
+    at_l = valid_work(inp.lengths, inp.c_z, inp.c_h)
     cfg = workload_config(inp, "bf16 operands, fp16 a/b/x, fp32 accumulation")
     cfg.update({"out_dtype": args.out_dtype, "parallelism": f"replicas x{world}", "mask_skipping": args.skip_masked,
-                "l2": f"z and mask cycle through {n_sets} copies ({n_sets * set_bytes / 2**20:.0f} MiB > 126 MiB L2)"})
+                "l2": wl.l2_note()})
+    launches_per_forward = tm.kernels_per_forward() + (1 if args.skip_masked else 0)
     line = {
         "metric": METRIC, "value": layer_ms, "unit": "ms/layer", "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": elapsed / args.steps, "higher_is_better": False, "scaling": "weak",
         "vs_baseline": None, "dtype": "bf16", "data": "synthetic", "config": cfg,
-        "effective_tflops": sum(flops.values()) / (layer_ms_single * 1e-3) / 1e12 * world,
+        "effective_tflops": dense / (layer_ms_single * 1e-3) / 1e12 * world,
+        "flops_dense": dense, "flops_at_valid_length": at_l,
+        "tflops_at_valid_length": at_l / (layer_ms_single * 1e-3) / 1e12 * world,
         "layer_roofline_frac": t_ideal / (layer_ms_single * 1e-3),
+        "ms_per_layer_instrumented": instr_elapsed / n_layers,
         "roofline": roof, "kernels": kernels, "cpu_baseline": cpu, "e2e": e2e, "pair_update": pair,
-        "pair_transition": trans, "torch_composition": context,
-        "gpu_launches": args.steps * len(dirs) * (tm.kernels_per_forward() + (1 if args.skip_masked else 0)),
+        "pair_transition": trans, "torch_composition": context, "workloads": workloads,
+        "gpu_launches": args.steps * len(dirs) * launches_per_forward,
         "clocks": clock_info,
     }
     print(json.dumps(line), flush=True)
@@ -538,6 +695,9 @@ def run_ours(args):
 
 def main():
     args = parse_args()
+    if args.cpu_oracle_probe:
+        cpu_oracle_probe(*args.cpu_oracle_probe)
+        return
     if args.impl == "reference":
         run_reference(args)
     else:

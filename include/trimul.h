@@ -118,19 +118,29 @@ void tri_mul_layer_destroy(trimul_layer_t *layer);
 
 /* Bytes of workspace tri_mul_forward needs for B x N x N with z of type `dtype`:
  * a, b and x, each [B, c_h, N, N] of the intermediate type (F16 for a BF16 z,
- * F32 for an F32 z), 256-byte aligned, then the mask extents (2 int32 per batch
- * element, 256-byte aligned). Returns 0 for an invalid layer or size. */
+ * F32 for an F32 z), 256-byte aligned, then, each 256-byte aligned, the mask extents
+ * (2 int32 per batch element), the offsets of the stored x (c_h fp32 per batch
+ * element) and their share of the output projection (c_z fp32 per batch element).
+ * Returns 0 for an invalid layer or size. */
 size_t tri_mul_workspace_bytes(const trimul_layer_t *layer, int64_t B, int64_t N,
                                trimul_dtype_t dtype);
 
 /* Attach caller-owned device workspace to the handle (replaces any earlier one).
  * The handle does not own it. Two forwards that run concurrently on different
- * streams must use different handles (or different workspaces). */
+ * streams must use different handles: besides the workspace, the handle holds the
+ * channel sums its projection step gathers during a forward. */
 trimul_status_t tri_mul_layer_bind_workspace(trimul_layer_t *layer, void *workspace,
                                              size_t bytes);
 
 /* One triangle multiplicative update (one direction). Returns the update only;
  * the residual add z += update is the caller's (or tri_mul_forward_residual's).
+ * On the tensor-core path four kernels run: K1 (projection), a small pass that turns
+ * K1's per-channel sums of a and b into per-(batch, channel) offsets o, K2 (contraction,
+ * storing x - o) and K3 (output gate, adding o back exactly). o = Sa Sb / P^1.5 (Sa, Sb the
+ * channel sums over the batch element, P its unmasked pairs) estimates the common mode of x
+ * that a large mean of a and b produces; storing x - o keeps the F16 rounding of x small
+ * next to the spread the output LayerNorm divides by. Any o gives the same function; the
+ * sums are integers (fixed point), so results do not depend on the order tiles finish in.
  * With mask skipping switched on (tri_mul_layer_set_mask_skipping), on the tensor-core
  * path with a mask a first pass finds the mask's extents (the last row and column holding a
  * nonzero entry, per batch element) and the kernels leave out tiles that are masked in full
@@ -183,22 +193,24 @@ trimul_status_t tri_mul_output_gate(const trimul_pair_t *z, const void *mask, co
 /* tri_mul_forward for callers that cannot allocate device memory (for example a plug-in
  * inside a framework that owns the allocator and gives it no way to ask for memory, or
  * a path that must not risk an allocation failing or stalling mid-work). Same arguments,
- * kernels and results as tri_mul_forward, but a, b and x live in a fixed array built
- * into the library (TRIMUL_NOALLOC_SCRATCH_BYTES of device memory on every GPU that
- * loads it, held until the process exits) instead of a bound workspace; the layer's
- * workspace and timing events are not used. It allocates nothing.
- *   - Problems whose a, b and x need more than TRIMUL_NOALLOC_SCRATCH_BYTES (that is,
- *     tri_mul_workspace_bytes() less its mask-extents block > TRIMUL_NOALLOC_SCRATCH_BYTES;
- *     this path skips no masked tiles; for a BF16 z with
- *     c_h = 128 the limit is B * N * N <= 65536, e.g. N = 256 at B = 1) are rejected
- *     with TRIMUL_ERR_WORKSPACE.
- *   - The first call on each device looks up the array's device address (once, with
- *     that device current); make that first call before any stream capture.
+ * checks, kernels and results as tri_mul_forward, but the intermediates (a, b, x and the
+ * small per-batch vectors tri_mul_workspace_bytes() counts) live in a fixed array built
+ * into the library (TRIMUL_NOALLOC_SCRATCH_BYTES of device memory on every GPU that loads
+ * it, held until the process exits) instead of a bound workspace; the layer's workspace
+ * and timing events are not used. It allocates nothing.
+ *   - Every argument is checked before anything touches the device; a problem with
+ *     tri_mul_workspace_bytes() > TRIMUL_NOALLOC_SCRATCH_BYTES (for a BF16 z with
+ *     c_h = 128: B * N * N > 65536, e.g. N = 256 at B = 1 fits) is rejected with
+ *     TRIMUL_ERR_WORKSPACE.
+ *   - The first call in each device context looks up the array's device address (with
+ *     that device current) and keeps it for that context; a reset device gets a new
+ *     lookup. Make the first call before any stream capture.
  *   - All calls share the one array and it keeps the last call's contents (nothing in
  *     it needs to start at zero). Calls that overlap on the GPU (different streams
- *     without ordering between them, or concurrent host threads) race on it: order them.
+ *     without ordering between them, or concurrent host threads) race on it, and so do
+ *     overlapping calls with one layer handle: order them.
  * This entry point is an engineering addition with no counterpart in the pages. */
-#define TRIMUL_NOALLOC_SCRATCH_BYTES (48u * 1024u * 1024u)
+#define TRIMUL_NOALLOC_SCRATCH_BYTES (48u * 1024u * 1024u + 64u * 1024u)
 trimul_status_t tri_mul_forward_noalloc(const trimul_pair_t *z, const void *mask,
                                         const trimul_layer_t *layer, trimul_direction_t direction,
                                         trimul_pair_t *out, void *stream);
@@ -276,13 +288,16 @@ trimul_status_t tri_mul_transition_forward(const trimul_pair_t *z, const void *m
 
 /* Optional per-kernel timing: when `events` is non-NULL, every later
  * tri_mul_forward on this handle records events[0] before K1 (after the mask-extents
- * pass), events[1] after
- * K1, events[2] after K2 and events[3] after K3 on its stream. The four values
- * are cudaEvent_t created by the caller; NULL switches recording off. */
+ * pass), events[1] after K1 and the offsets pass, events[2] after K2 and events[3]
+ * after K3 on its stream. The four values are cudaEvent_t created by the caller;
+ * NULL switches recording off. Recording an event between two kernels ends the
+ * overlap of one kernel's start with the previous one's end, so timed forwards run
+ * a little slower than untimed ones. */
 trimul_status_t tri_mul_layer_set_timing_events(trimul_layer_t *layer, void *const *events);
 
-/* Number of kernels one tri_mul_forward launches: K1, K2 and K3 (one more, the mask-extents
- * pass, on the tensor-core path with a mask and mask skipping switched on). */
+/* Number of kernels one tri_mul_forward launches on the tensor-core path: K1, the offsets
+ * pass, K2 and K3 (one more, the mask-extents pass, with a mask and mask skipping switched
+ * on). The fp32 path launches three (no offsets pass). */
 int tri_mul_kernels_per_forward(void);
 
 /* Synchronize the current device, then read and clear the library's device
@@ -310,7 +325,7 @@ const char *tri_mul_last_error(void);
 /* ABI version of this header (major * 100 + minor). */
 int tri_mul_abi_version(void);
 
-#define TRIMUL_ABI_VERSION 101
+#define TRIMUL_ABI_VERSION 102
 
 #ifdef __cplusplus
 }

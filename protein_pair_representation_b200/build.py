@@ -13,8 +13,8 @@ INCLUDE = os.path.join(ROOT, "include")
 LIB_DIR = os.path.join(PKG, "lib")
 LIB_PATH = os.path.join(LIB_DIR, "libtrimul.so")
 
-SOURCES = ["trimul_api.cu", "k1_project.cu", "k2_contract.cu", "k3_output.cu", "extents.cu", "transition.cu", "fold.cu", "f32_path.cu",
-           "noalloc.cu"]
+SOURCES = ["trimul_api.cu", "k1_project.cu", "k2_contract.cu", "k3_output.cu", "offsets.cu", "extents.cu",
+           "transition.cu", "fold.cu", "f32_path.cu", "noalloc.cu"]
 HEADERS = ["kernels.h", "sm100.cuh"]
 
 NVCC_FLAGS = [

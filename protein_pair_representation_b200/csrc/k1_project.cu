@@ -13,8 +13,9 @@
 // so the tensor cores multiply the raw bf16 z tile, and the epilogue applies the
 // per-pair (mean, rstd) and the per-channel (sum W', shift) pair of constants.
 //
-// Two kernels. c_z = 128 (k1_project_cm_kernel, further below) puts one hidden channel
-// on each TMEM lane. c_z = 384 (k1_project_kernel) puts one pair on each TMEM lane:
+// Two kernels. c_z = 128 (k1_project_ab_kernel, further below) puts one hidden channel
+// on each TMEM lane and makes both operands from each z tile. c_z = 384 (k1_project_kernel)
+// puts one pair on each TMEM lane:
 // 128 consecutive pairs of one batch element times NCOL = 128 packed weight rows, laid
 // out in 32-row blocks of [16 gate rows, 16 projection rows] for 16 channels so one
 // 32-column TMEM load gives a thread both factors of 16 outputs, with four column groups
@@ -189,6 +190,10 @@ __global__ void __launch_bounds__(448, 1) k1_project_kernel(const __grid_constan
         uint32_t phase = 0;
         int sbuf = 0;
         uint32_t sphase = 0;
+        // unmasked pairs of batch element cnt_b seen so far (group 0's CTAs count them)
+        const bool counting = p.acc != nullptr && group == 0;
+        int cnt_b = -1;
+        unsigned int cnt = 0;
         TileWalk tw(cta_in_group, p.tiles_per_batch);
         for (int pt = cta_in_group; pt < num_ptiles; pt += ctas_per_group, tw.advance(ctas_per_group, p.tiles_per_batch)) {
             const int b = tw.b;
@@ -228,14 +233,26 @@ __global__ void __launch_bounds__(448, 1) k1_project_kernel(const __grid_constan
             const float mean = shift + dm;
             const float rstd = rsqrtf(var + p.eps);
             const long long pi = (long long)p0 + row;
-            float m = 1.f;
-            if (p.mask) m = (pi < p.NN) ? __uint_as_float((uint32_t)p.mask[(long long)b * p.NN + pi] << 16) : 0.f;
+            // 1 (no mask), the mask entry, or 0 past the last pair
+            float m = pi < p.NN ? 1.f : 0.f;
+            if (p.mask && pi < p.NN) m = __uint_as_float((uint32_t)p.mask[(long long)b * p.NN + pi] << 16);
+            if (counting) {
+                const unsigned int valid = __ballot_sync(0xffffffffu, m != 0.f);
+                if (b != cnt_b) {
+                    if (cnt_b >= 0 && lane == 0) atomicAdd(p.acc + (size_t)cnt_b * (2 * C::C_H + 1) + 2 * C::C_H, (unsigned long long)cnt);
+                    cnt_b = b;
+                    cnt = 0;
+                }
+                cnt += __popc(valid);
+            }
             if (!__all_sync(0xffffffffu, mbar_wait(&s.sempty[sbuf], sphase ^ 1, abort_flag, kErrTimeoutEpilogue))) break;
             stats[sbuf * 128 + row] = make_float4(mean, rstd, m, 0.f);
             __syncwarp();
             if (lane == 0) mbar_arrive(&s.sfull[sbuf]);
             if (++sbuf == C::SNB) { sbuf = 0; sphase ^= 1; }
         }
+        if (counting && cnt_b >= 0 && lane == 0)
+            atomicAdd(p.acc + (size_t)cnt_b * (2 * C::C_H + 1) + 2 * C::C_H, (unsigned long long)cnt);
     } else {
         // epilogue: warpgroup wg handles channels [ch0 + wg*CH_WG, +CH_WG)
         const int wg = warp >> 2;
@@ -249,10 +266,31 @@ __global__ void __launch_bounds__(448, 1) k1_project_kernel(const __grid_constan
         uint32_t aphase = 0;
         int sbuf = 0;
         uint32_t sphase = 0;
+        // running sums of this thread's outputs per channel over batch element sum_b; summed over
+        // the warp and added to the channel sums when the batch element changes and at the end
+        unsigned long long *acc_w = p.acc ? p.acc + operand * C::C_H + ch0 + wg * C::CH_WG : nullptr;
+        int sum_b = -1;
+        float run[C::CH_WG];
+#pragma unroll
+        for (int t = 0; t < C::CH_WG; ++t) run[t] = 0.f;
+        auto flush = [&](int fb) {
+#pragma unroll
+            for (int t = 0; t < C::CH_WG; ++t) {
+                float v = run[t];
+#pragma unroll
+                for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+                if (lane == 0) atomicAdd(acc_w + (size_t)fb * (2 * C::C_H + 1) + t, (unsigned long long)llrintf(v * kAccScale));
+                run[t] = 0.f;
+            }
+        };
         TileWalk tw(cta_in_group, p.tiles_per_batch);
         for (int pt = cta_in_group; pt < num_ptiles; pt += ctas_per_group, tw.advance(ctas_per_group, p.tiles_per_batch)) {
             const int b = tw.b;
             const int p0 = tw.t * 128;
+            if (acc_w && b != sum_b) {
+                if (sum_b >= 0) flush(sum_b);
+                sum_b = b;
+            }
             if (SKIP && tile_masked_out(p.ext, b, p0, p.N, p.NN, p.rowdiv)) {
                 // every pair of the tile is masked: a and b are 0 there (the contraction reads them)
                 if (leader) tma_store_wait_read<0>();
@@ -277,8 +315,8 @@ __global__ void __launch_bounds__(448, 1) k1_project_kernel(const __grid_constan
             tc_fence_after();
             if (leader) tma_store_wait_read<0>();
             named_bar_sync(1 + wg, 128);
-#pragma unroll 1
-            for (int blk = 0; blk < C::BLK_WG; ++blk) {
+#pragma unroll
+            for (int blk = 0; blk < C::BLK_WG; ++blk) {   // unrolled: run[] stays in registers
                 float v[32];
                 tmem_ld32(tmem_base + abuf * C::NCOL + ((uint32_t)(q * 32) << 16) + (wg * C::BLK_WG + blk) * 32, v);
                 tc_wait_ld();
@@ -287,8 +325,9 @@ __global__ void __launch_bounds__(448, 1) k1_project_kernel(const __grid_constan
                     const float4 cv = __ldg(&vec[blk * 16 + e]);
                     const float g = fmaf(rstd, fmaf(-mean, cv.x, v[e]), cv.y);
                     const float pr = fmaf(rstd, fmaf(-mean, cv.z, v[16 + e]), cv.w);
-                    const float out = sigmoid_tanh(g) * pr * m;
-                    stg[(blk * 16 + e) * 128 + row] = __half_as_ushort(__float2half_rn(out));
+                    const __half oh = __float2half_rn(sigmoid_tanh(g) * pr * m);
+                    stg[(blk * 16 + e) * 128 + row] = __half_as_ushort(oh);
+                    if (acc_w) run[blk * 16 + e] += __half2float(oh);
                 }
             }
             tc_fence_before();
@@ -302,6 +341,7 @@ __global__ void __launch_bounds__(448, 1) k1_project_kernel(const __grid_constan
                 tma_store_commit();
             }
         }
+        if (acc_w && sum_b >= 0) flush(sum_b);
         if (leader) tma_store_wait_all<0>();
     }
 
@@ -314,37 +354,38 @@ __global__ void __launch_bounds__(448, 1) k1_project_kernel(const __grid_constan
 }
 
 // ------------------------------------------------------------------------------------------
-// K1 for c_z = 128: accumulators with one TMEM lane per hidden channel.
+// K1 for c_z = 128: both operands from each z tile, one TMEM lane per hidden channel.
 //
-// D_gate[c, p] = W'_gate[c] . z_p and D_proj[c, p] = W'_proj[c] . z_p for the 128 channels
-// of one operand (a or b) and 128 pairs: A = folded weights [128 channels x c_z], B = the z
-// tile [128 pairs x c_z], both K-major. A thread of the epilogue owns one channel for the
-// whole kernel, so that channel's four folding constants stay in registers; the per-pair
-// LayerNorm statistics are read from shared memory (broadcast, four pairs per load); and
-// consecutive pairs of one channel are consecutive columns, which pack directly into
-// 16-byte rows of the channel-major output tile.
-// The gate is evaluated in f16x2 (tanh.approx.f16x2 on g/2, the gate rows being folded
-// with an extra factor 1/2), as are the products with the projection and the mask.
-// Warps: 0-15 epilogue (two teams of two warpgroups that take alternate tiles; warpgroup
-// s of a team: pairs [64s, 64s+64) of its tiles), 16-19 LayerNorm statistics, 20 TMA
-// producer, 21 TMEM allocator + MMA issuer.
-struct K1CmCfg {
-    static constexpr int CZ = 128, C_H = kHidden, KC = CZ / 64;
-    static constexpr int G = 2;                               // one group per operand
-    static constexpr int W_CHUNK = 2 * C_H * 64 * 2;          // [gate 128 rows, proj 128 rows] x 64 k
-    static constexpr int W_BYTES = KC * W_CHUNK;              // 64 KB
-    static constexpr int CHUNK = 128 * 64 * 2;                // z chunk: 128 pairs x 64 channels
+// A 64-pair tile of z (16 KB, one TMA box) is read once per CTA, its LayerNorm statistics are
+// computed once, and four accumulators are filled from it: D_r[c, p] = W'_r[c] . z_p for the
+// four weight blocks r = a-gate, a-projection, b-gate, b-projection (A = the folded weights,
+// 128 channels x c_z, resident in shared memory for the whole kernel: 128 KB; B = the z tile,
+// 64 pairs x c_z; both K-major; M = 128, N = 64). The four accumulators of a tile take 256 TMEM
+// columns, so two tiles are in flight.
+// A thread of the epilogue owns one channel of one operand for the whole kernel, so that
+// channel's four folding constants stay in registers; the per-pair LayerNorm statistics are
+// read from shared memory (broadcast); and consecutive pairs of one channel are consecutive
+// TMEM columns, which pack directly into 16-byte rows of the channel-major output tile.
+// The gate is evaluated in f16x2 (tanh.approx.f16x2 on g/2, the gate rows being folded with
+// an extra factor 1/2), as are the products with the projection and the mask.
+// Warps: 0-15 epilogue (two teams of eight warps that take alternate tiles; warp 4o + q of a
+// team: operand o, channels [32q, 32q + 32)), 16-17 LayerNorm statistics (one thread per
+// pair), 18 TMA producer, 19 TMEM allocator + MMA issuer.
+struct K1AbCfg {
+    static constexpr int CZ = 128, C_H = kHidden, TP = 64;   // pairs per tile
+    static constexpr int W_CHUNK = 4 * C_H * 64 * 2;          // [a-gate, a-proj, b-gate, b-proj rows] x 64 k: 64 KB
+    static constexpr int W_BYTES = (CZ / 64) * W_CHUNK;       // 128 KB
+    static constexpr int TILE = TP * CZ * 2;                  // z tile: [2 halves][64 pairs][64 ch], 16 KB
     static constexpr int WARP_STG = 32 * 32 * 2;              // per epilogue warp: [32 ch][32 pairs] f16
-    static constexpr int STG_TOTAL = 16 * WARP_STG;           // 32 KB for the 16 epilogue warps
-    static constexpr int SNB = 2;
-    static constexpr int STATS_BYTES = SNB * 128 * (4 + 4 + 2);   // mean, rstd (f32), mask (f16) per pair
-    static constexpr int FIXED = 1024 + W_BYTES + STG_TOTAL + STATS_BYTES + 1024;
-    static constexpr int S = (232448 - FIXED) / CHUNK > 8 ? 8 : (232448 - FIXED) / CHUNK;
-    static constexpr size_t SMEM = FIXED + (size_t)S * CHUNK;
-    static constexpr int EPI_WARPS = 16;                      // four warpgroups, 32 pairs each
-    static constexpr int STATS_WARP0 = 16, STATS_WARPS = 4;
-    static constexpr int TMA_WARP = 20, MMA_WARP = 21;
-    static constexpr int THREADS = 22 * 32;
+    static constexpr int EPI_WARPS = 16;
+    static constexpr int STG_TOTAL = EPI_WARPS * WARP_STG;    // 32 KB
+    static constexpr int STATS_WARP0 = 16, STATS_WARPS = 2;
+    static constexpr int TMA_WARP = 18, MMA_WARP = 19;
+    static constexpr int THREADS = 20 * 32;
+    static constexpr int STATS_BYTES = 2 * TP * (4 + 4 + 2);  // -mean, rstd (f32), mask / 2 (f16) per pair
+    static constexpr int FIXED = 1024 + W_BYTES + STG_TOTAL + STATS_BYTES + 512;
+    static constexpr int S = (232448 - FIXED) / TILE > 8 ? 8 : (232448 - FIXED) / TILE;
+    static constexpr size_t SMEM = FIXED + (size_t)S * TILE;
 };
 
 __device__ __forceinline__ uint32_t h2_as_u32(__half2 h) { return *reinterpret_cast<uint32_t *>(&h); }
@@ -358,38 +399,33 @@ __device__ __forceinline__ __half2 tanh_h2(__half2 x) {
 }
 
 template <bool SKIP>
-__global__ void __launch_bounds__(K1CmCfg::THREADS, 1) k1_project_cm_kernel(const __grid_constant__ K1Args p) {
-    using C = K1CmCfg;
+__global__ void __launch_bounds__(K1AbCfg::THREADS, 1) k1_project_ab_kernel(const __grid_constant__ K1Args p) {
+    using C = K1AbCfg;
+    static_assert(sizeof(K1Smem) <= 512, "barrier block");
     extern __shared__ uint8_t smem_raw[];
     uint8_t *base = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-    uint8_t *w_s = base;                                  // KC chunks of [256 rows][64] bf16
-    uint8_t *chunks = w_s + C::W_BYTES;                   // S chunks of [128 pairs][64] bf16
-    uint8_t *staging = chunks + C::S * C::CHUNK;          // 16 x [32 ch][32 pairs] f16, 64B swizzle
-    float *st_nmean = reinterpret_cast<float *>(staging + C::STG_TOTAL);     // [SNB][128] -mean
-    float *st_rstd = st_nmean + C::SNB * 128;
-    __half *st_hmask = reinterpret_cast<__half *>(st_rstd + C::SNB * 128);    // [SNB][128] mask / 2
-    K1Smem &s = *reinterpret_cast<K1Smem *>(st_hmask + C::SNB * 128);
+    uint8_t *w_s = base;                                  // 2 k-chunks of [512 rows][64] bf16
+    uint8_t *tiles = w_s + C::W_BYTES;                    // S tiles of [2][64 pairs][64] bf16
+    uint8_t *staging = tiles + C::S * C::TILE;            // 16 x [32 ch][32 pairs] f16, 64B swizzle
+    float *st_nmean = reinterpret_cast<float *>(staging + C::STG_TOTAL);   // [2][64] -mean
+    float *st_rstd = st_nmean + 2 * C::TP;
+    __half *st_hmask = reinterpret_cast<__half *>(st_rstd + 2 * C::TP);    // [2][64] mask / 2
+    K1Smem &s = *reinterpret_cast<K1Smem *>(st_hmask + 2 * C::TP);
 
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
     volatile int *abort_flag = &s.abort_flag;
-
-    const int operand = blockIdx.x % C::G;
-    const int cta_in_group = blockIdx.x / C::G;
-    const int ctas_per_group = gridDim.x / C::G;
-    const int num_ptiles = p.B * p.tiles_per_batch;
+    const int num_tiles = p.B * p.tiles_per_batch;
 
     if (threadIdx.x == 0) {
         mbar_init(&s.wbar, 1);
         for (int i = 0; i < C::S; ++i) {
             mbar_init(&s.full[i], 1);
-            mbar_init(&s.empty[i], 1 + C::STATS_WARPS);  // MMA commit + stats warps
+            mbar_init(&s.empty[i], 1 + C::STATS_WARPS);   // MMA commit + statistics warps
         }
         for (int i = 0; i < 2; ++i) {
             mbar_init(&s.tfull[i], 1);
             mbar_init(&s.tempty[i], C::EPI_WARPS / 2);     // the team that drains buffer i
-        }
-        for (int i = 0; i < C::SNB; ++i) {
             mbar_init(&s.sfull[i], C::STATS_WARPS);
             mbar_init(&s.sempty[i], C::EPI_WARPS / 2);
         }
@@ -413,24 +449,24 @@ __global__ void __launch_bounds__(K1CmCfg::THREADS, 1) k1_project_cm_kernel(cons
             tma_prefetch_desc(&p.tm_z);
             tma_prefetch_desc(&p.tm_w);
             mbar_arrive_expect_tx(&s.wbar, C::W_BYTES);
-            for (int kc = 0; kc < C::KC; ++kc)
-                tma_load_2d(w_s + kc * C::W_CHUNK, &p.tm_w, &s.wbar, kc * 64, operand * 2 * C::C_H);
+            for (int kc = 0; kc < C::CZ / 64; ++kc)
+                for (int h = 0; h < 2; ++h)          // rows [256 h, 256 h + 256) of the 512
+                    tma_load_2d(w_s + kc * C::W_CHUNK + h * 256 * 128, &p.tm_w, &s.wbar, kc * 64, h * 256);
             pdl_wait();
             int stage = 0;
             uint32_t phase = 0;
             uint32_t filled = 0;
-            TileWalk tw(cta_in_group, p.tiles_per_batch);
-            for (int pt = cta_in_group; pt < num_ptiles; pt += ctas_per_group, tw.advance(ctas_per_group, p.tiles_per_batch)) {
+            TileWalk tw(blockIdx.x, p.tiles_per_batch);
+            for (int t = blockIdx.x; t < num_tiles; t += gridDim.x, tw.advance(gridDim.x, p.tiles_per_batch)) {
                 const int b = tw.b;
-                const int p0 = tw.t * 128;
-                if (SKIP && tile_masked_out(p.ext, b, p0, p.N, p.NN, p.rowdiv)) continue;   // nothing to load
-                for (int kc = 0; kc < C::KC; ++kc) {
-                    if (!mbar_wait(&s.empty[stage], phase ^ 1, abort_flag, kErrTimeoutProducer)) goto producer_abort;
-                    mbar_arrive_expect_tx(&s.full[stage], C::CHUNK);
-                    tma_load_3d(chunks + stage * C::CHUNK, &p.tm_z, &s.full[stage], kc * 64, p0, b);
-                    ++filled;
-                    if (++stage == C::S) { stage = 0; phase ^= 1; }
-                }
+                const int p0 = tw.t * C::TP;
+                if (SKIP && tile_masked_out<C::TP>(p.ext, b, p0, p.N, p.NN, p.rowdiv)) continue;   // nothing to load
+                if (!mbar_wait(&s.empty[stage], phase ^ 1, abort_flag, kErrTimeoutProducer)) goto producer_abort;
+                mbar_arrive_expect_tx(&s.full[stage], C::TILE);
+                // both 64-channel halves of the tile's 64 pairs in one copy
+                tma_load_4d(tiles + stage * C::TILE, &p.tm_z, &s.full[stage], 0, p0, 0, b);
+                ++filled;
+                if (++stage == C::S) { stage = 0; phase ^= 1; }
             }
             goto producer_done;
         producer_abort:
@@ -443,38 +479,31 @@ __global__ void __launch_bounds__(K1CmCfg::THREADS, 1) k1_project_cm_kernel(cons
         }
     } else if (warp == C::MMA_WARP) {
         if (lane == 0) {
-            const uint32_t idesc = idesc_f32acc(128, 128, false, false, false);
+            const uint32_t idesc = idesc_f32acc(128, C::TP, false, false, false);
             bool ok = mbar_wait(&s.wbar, 0, abort_flag, kErrTimeoutMma);
             int stage = 0;
             uint32_t phase = 0;
             uint32_t aphase[2] = {0, 0};           // tile j of this CTA uses TMEM buffer j % 2
             int j = 0;
-            TileWalk tw(cta_in_group, p.tiles_per_batch);
-            for (int pt = cta_in_group; ok && pt < num_ptiles;
-                 pt += ctas_per_group, tw.advance(ctas_per_group, p.tiles_per_batch), ++j) {
-                if (SKIP && tile_masked_out(p.ext, tw.b, tw.t * 128, p.N, p.NN, p.rowdiv)) continue;
+            TileWalk tw(blockIdx.x, p.tiles_per_batch);
+            for (int t = blockIdx.x; ok && t < num_tiles; t += gridDim.x, tw.advance(gridDim.x, p.tiles_per_batch), ++j) {
+                if (SKIP && tile_masked_out<C::TP>(p.ext, tw.b, tw.t * C::TP, p.N, p.NN, p.rowdiv)) continue;
                 const int abuf = j & 1;
                 if (!mbar_wait(&s.tempty[abuf], aphase[abuf] ^ 1, abort_flag, kErrTimeoutMma)) break;
+                if (!mbar_wait(&s.full[stage], phase, abort_flag, kErrTimeoutMma)) break;
                 tc_fence_after();
-                const uint32_t d_gate = tmem_base + abuf * 256;
-                const uint32_t d_proj = d_gate + 128;
-                for (int kc = 0; kc < C::KC; ++kc) {
-                    if (!mbar_wait(&s.full[stage], phase, abort_flag, kErrTimeoutMma)) { ok = false; break; }
-                    tc_fence_after();
-                    const uint8_t *zc = chunks + stage * C::CHUNK;
-                    const uint8_t *wg = w_s + kc * C::W_CHUNK;
+                const uint8_t *zt = tiles + stage * C::TILE;
 #pragma unroll
-                    for (int kk = 0; kk < 4; ++kk) {
-                        const uint64_t bd = smem_desc_sw128(zc + kk * 32, 16, 1024);
-                        const uint64_t ag = smem_desc_sw128(wg + kk * 32, 16, 1024);
-                        const uint64_t ap = smem_desc_sw128(wg + C::C_H * 128 + kk * 32, 16, 1024);
-                        tc_mma_bf16(d_gate, ag, bd, idesc, (kc | kk) != 0);
-                        tc_mma_bf16(d_proj, ap, bd, idesc, (kc | kk) != 0);
-                    }
-                    tc_commit(&s.empty[stage]);
-                    if (++stage == C::S) { stage = 0; phase ^= 1; }
+                for (int kk = 0; kk < C::CZ / 16; ++kk) {
+                    const uint64_t bd = smem_desc_sw128(zt + (kk >> 2) * 8192 + (kk & 3) * 32, 16, 1024);
+                    const uint8_t *wk = w_s + (kk >> 2) * C::W_CHUNK + (kk & 3) * 32;
+#pragma unroll
+                    for (int r = 0; r < 4; ++r)
+                        tc_mma_bf16(tmem_base + abuf * 256 + r * C::TP, smem_desc_sw128(wk + r * C::C_H * 128, 16, 1024),
+                                    bd, idesc, kk != 0);
                 }
-                if (!ok) break;
+                tc_commit(&s.empty[stage]);
+                if (++stage == C::S) { stage = 0; phase ^= 1; }
                 tc_commit(&s.tfull[abuf]);
                 aphase[abuf] ^= 1;
             }
@@ -488,29 +517,42 @@ __global__ void __launch_bounds__(K1CmCfg::THREADS, 1) k1_project_cm_kernel(cons
         uint32_t phase = 0;
         uint32_t sphase[2] = {0, 0};               // tile j of this CTA uses statistics buffer j % 2
         int j = -1;
-        TileWalk tw(cta_in_group, p.tiles_per_batch);
-        for (int pt = cta_in_group; pt < num_ptiles; pt += ctas_per_group, tw.advance(ctas_per_group, p.tiles_per_batch)) {
+        // unmasked pairs of batch element cnt_b seen so far
+        const bool counting = p.acc != nullptr;
+        int cnt_b = -1;
+        unsigned int cnt = 0;
+        TileWalk tw(blockIdx.x, p.tiles_per_batch);
+        for (int t = blockIdx.x; t < num_tiles; t += gridDim.x, tw.advance(gridDim.x, p.tiles_per_batch)) {
             const int b = tw.b;
-            const int p0 = tw.t * 128;
+            const int p0 = tw.t * C::TP;
             ++j;
-            if (SKIP && tile_masked_out(p.ext, b, p0, p.N, p.NN, p.rowdiv)) continue;
+            if (SKIP && tile_masked_out<C::TP>(p.ext, b, p0, p.N, p.NN, p.rowdiv)) continue;
             const int sbuf = j & 1;
-            const long long pi = (long long)p0 + row;
-            uint16_t mbits = 0x3F80u;   // bf16 1.0; the load is issued first so its latency overlaps
-            if (p.mask) mbits = (pi < p.NN) ? p.mask[(long long)b * p.NN + pi] : (uint16_t)0;
+            const long long pi = (long long)p0 + row;   // < NN: NN is a multiple of 64
+            // bf16 1.0 (no mask) or the mask entry; the load is issued first so its latency overlaps
+            const uint16_t mbits = p.mask ? p.mask[(long long)b * p.NN + pi] : (uint16_t)0x3F80u;
+            if (counting) {
+                const unsigned int valid = __ballot_sync(0xffffffffu, (mbits & 0x7FFFu) != 0);
+                if (b != cnt_b) {
+                    if (cnt_b >= 0 && lane == 0) atomicAdd(p.acc + (size_t)cnt_b * (2 * C::C_H + 1) + 2 * C::C_H, (unsigned long long)cnt);
+                    cnt_b = b;
+                    cnt = 0;
+                }
+                cnt += __popc(valid);
+            }
+            if (!__all_sync(0xffffffffu, mbar_wait(&s.full[stage], phase, abort_flag, kErrTimeoutEpilogue))) break;
+            const uint8_t *zt = tiles + stage * C::TILE;
             // shifted sums in packed pairs: s1 = sum(v - shift), s2 = sum((v - shift)^2), with
             // the row's first entry as the shift
             float shift = 0.f;
             float2 nsh = make_float2(0.f, 0.f), s1 = make_float2(0.f, 0.f), s2 = make_float2(0.f, 0.f);
-            bool ok = true;
-            for (int kc = 0; kc < C::KC; ++kc) {
-                if (!__all_sync(0xffffffffu, mbar_wait(&s.full[stage], phase, abort_flag, kErrTimeoutEpilogue))) { ok = false; break; }
-                const uint8_t *zc = chunks + stage * C::CHUNK;
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
 #pragma unroll
                 for (int u = 0; u < 8; ++u) {
-                    const uint4 w = *reinterpret_cast<const uint4 *>(zc + sw128_offset(row, u));
+                    const uint4 w = *reinterpret_cast<const uint4 *>(zt + h * 8192 + sw128_offset(row, u));
                     const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
-                    if (kc == 0 && u == 0) {
+                    if (h == 0 && u == 0) {
                         shift = bf16_lo(w.x);
                         nsh = make_float2(-shift, -shift);
                     }
@@ -521,129 +563,140 @@ __global__ void __launch_bounds__(K1CmCfg::THREADS, 1) k1_project_cm_kernel(cons
                         s2 = f2_fma(d, d, s2);
                     }
                 }
-                __syncwarp();
-                if (lane == 0) mbar_arrive(&s.empty[stage]);
-                if (++stage == C::S) { stage = 0; phase ^= 1; }
             }
-            if (!ok) break;
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&s.empty[stage]);
+            if (++stage == C::S) { stage = 0; phase ^= 1; }
             const float inv_n = 1.0f / (float)C::CZ;
             const float dm = (s1.x + s1.y) * inv_n;
             const float var = fmaxf((s2.x + s2.y) * inv_n - dm * dm, 0.f);
             if (!__all_sync(0xffffffffu, mbar_wait(&s.sempty[sbuf], sphase[sbuf] ^ 1, abort_flag, kErrTimeoutEpilogue))) break;
-            st_nmean[sbuf * 128 + row] = -(shift + dm);
-            st_rstd[sbuf * 128 + row] = rsqrtf(var + p.eps);
-            st_hmask[sbuf * 128 + row] = __float2half_rn(0.5f * __uint_as_float((uint32_t)mbits << 16));
+            st_nmean[sbuf * C::TP + row] = -(shift + dm);
+            st_rstd[sbuf * C::TP + row] = rsqrtf(var + p.eps);
+            st_hmask[sbuf * C::TP + row] = __float2half_rn(0.5f * __uint_as_float((uint32_t)mbits << 16));
             __syncwarp();
             if (lane == 0) mbar_arrive(&s.sfull[sbuf]);
             sphase[sbuf] ^= 1;
         }
+        if (counting && cnt_b >= 0 && lane == 0)
+            atomicAdd(p.acc + (size_t)cnt_b * (2 * C::C_H + 1) + 2 * C::C_H, (unsigned long long)cnt);
     } else {
-        // epilogue: two teams of eight warps take alternate tiles of this CTA's sequence (team k
-        // drains TMEM buffer k and statistics buffer k), so that one team's waits and TMEM
-        // loads overlap the other team's arithmetic. Thread = hidden channel c; warpgroup s of
-        // a team owns the 64 pairs [64 s, 64 s + 64) of its tiles. Every warp runs on its own:
-        // it waits on the barriers itself and stages each [32 channels][32 pairs] block of its
-        // output in its own 2 KB of shared memory (64-byte rows, 64-byte swizzle) for a TMA
-        // store.
-        const int wg = warp >> 2;
-        const int team = wg >> 1;
+        // epilogue: team k (warps 8k .. 8k + 7) drains TMEM buffer k and statistics buffer k, i.e.
+        // the tiles j = k, k + 2, ... of this CTA, so that one team's waits and TMEM loads overlap
+        // the other team's arithmetic. Warp 4o + q of a team: operand o, channels [32q, 32q + 32);
+        // thread = channel c; it covers the tile's 64 pairs in two store blocks of 32. Every warp
+        // runs on its own: it waits on the barriers itself and stages each [32 channels][32 pairs]
+        // block in its own 2 KB of shared memory (64-byte rows, 64-byte swizzle) for a TMA store.
+        const int team = warp >> 3;
+        const int operand = (warp >> 2) & 1;
         const int q = warp & 3;
         const int c = q * 32 + lane;
-        const int col0 = 64 * (wg & 1);
         uint8_t *stg = staging + warp * C::WARP_STG;
         const CUtensorMap *tm_out = operand == 0 ? &p.tm_a : &p.tm_b;
         // {sum W'_gate, shift_gate, sum W'_proj, shift_proj}; the gate entries are for g / 2
         const float4 cv = p.vec[operand * C::C_H + c];
         const float2 cg_sum = make_float2(cv.x, cv.x), cg_shift = make_float2(cv.y, cv.y);
         const float2 cp_sum = make_float2(cv.z, cv.z), cp_shift = make_float2(cv.w, cv.w);
-        static_assert(C::SNB == 2, "one statistics buffer per epilogue team");
-        const int abuf = team, sbuf = team;
-        const uint32_t tbase = tmem_base + abuf * 256 + ((uint32_t)(q * 32) << 16);
-        const float *snmean0 = st_nmean + sbuf * 128 + col0, *srstd0 = st_rstd + sbuf * 128 + col0;
-        const __half *shmask0 = st_hmask + sbuf * 128 + col0;
+        const int buf = team;
+        const uint32_t tbase = tmem_base + buf * 256 + operand * 2 * C::TP + ((uint32_t)(q * 32) << 16);
+        const float *snmean = st_nmean + buf * C::TP, *srstd = st_rstd + buf * C::TP;
+        const __half *shmask = st_hmask + buf * C::TP;
+        // running sum of this channel's stored outputs over batch element sum_b
+        unsigned long long *acc_c = p.acc ? p.acc + operand * C::C_H + c : nullptr;
+        int sum_b = -1;
+        float run = 0.f;
         uint32_t phase = 0;
-        const int first = cta_in_group + team * ctas_per_group;
+        const int first = blockIdx.x + team * gridDim.x;
         TileWalk tw(first, p.tiles_per_batch);
-        for (int pt = first; pt < num_ptiles; pt += 2 * ctas_per_group, tw.advance(2 * ctas_per_group, p.tiles_per_batch)) {
+        for (int t = first; t < num_tiles; t += 2 * gridDim.x, tw.advance(2 * gridDim.x, p.tiles_per_batch)) {
             const int b = tw.b;
-            const int p0 = tw.t * 128;
-            if (SKIP && tile_masked_out(p.ext, b, p0, p.N, p.NN, p.rowdiv)) {
+            const int p0 = tw.t * C::TP;
+            if (acc_c && b != sum_b) {
+                if (sum_b >= 0) atomicAdd(acc_c + (size_t)sum_b * (2 * C::C_H + 1), (unsigned long long)llrintf(run * kAccScale));
+                sum_b = b;
+                run = 0.f;
+            }
+            if (SKIP && tile_masked_out<C::TP>(p.ext, b, p0, p.N, p.NN, p.rowdiv)) {
                 // every pair of the tile is masked: a and b are 0 there (the contraction reads them)
 #pragma unroll 1
                 for (int blk = 0; blk < 2; ++blk) {
-                    const int col = col0 + 32 * blk;
                     if (lane == 0) tma_store_wait_read<0>();
                     __syncwarp();
 #pragma unroll
                     for (int u = 0; u < 4; ++u) *reinterpret_cast<uint4 *>(stg + sw64_offset(lane, u)) = make_uint4(0, 0, 0, 0);
                     fence_proxy_async_smem();
                     __syncwarp();
-                    if (lane == 0 && p0 + col < p.NN) {
-                        tma_store_3d(tm_out, stg, p0 + col, q * 32, b);
+                    if (lane == 0) {
+                        tma_store_3d(tm_out, stg, p0 + 32 * blk, q * 32, b);
                         tma_store_commit();
                     }
                 }
                 continue;
             }
-            if (!__all_sync(0xffffffffu, mbar_wait(&s.sfull[sbuf], phase, abort_flag, kErrTimeoutEpilogue) &&
-                                             mbar_wait(&s.tfull[abuf], phase, abort_flag, kErrTimeoutEpilogue)))
+            if (!__all_sync(0xffffffffu, mbar_wait(&s.sfull[buf], phase, abort_flag, kErrTimeoutEpilogue) &&
+                                             mbar_wait(&s.tfull[buf], phase, abort_flag, kErrTimeoutEpilogue)))
                 break;
             tc_fence_after();
 #pragma unroll 1
             for (int blk = 0; blk < 2; ++blk) {         // two store blocks of 32 pairs
-                const int col = col0 + 32 * blk;
                 if (lane == 0) tma_store_wait_read<0>();   // this warp's previous store has read its block
                 __syncwarp();
 #pragma unroll 1
                 for (int hh = 0; hh < 2; ++hh) {      // two halves of 16 pairs
+                    const int o = 32 * blk + 16 * hh;
                     float g[16], pr[16];
-                    tmem_ld16(tbase + col + 16 * hh, g);
-                    tmem_ld16(tbase + 128 + col + 16 * hh, pr);
+                    tmem_ld16(tbase + o, g);
+                    tmem_ld16(tbase + C::TP + o, pr);
                     tc_wait_ld();
                     if (blk == 1 && hh == 1) {
                         // the last TMEM load of the tile has landed: hand the buffer back to the
                         // MMA now, not after this warp's arithmetic and store
                         tc_fence_before();
                         __syncwarp();
-                        if (lane == 0) mbar_arrive(&s.tempty[abuf]);
+                        if (lane == 0) mbar_arrive(&s.tempty[buf]);
                     }
-                    const int o = 32 * blk + 16 * hh;
                     uint32_t outw[8];
 #pragma unroll
-                    for (int j = 0; j < 16; j += 4) {
-                        const float4 nm = *reinterpret_cast<const float4 *>(snmean0 + o + j);
-                        const float4 rs = *reinterpret_cast<const float4 *>(srstd0 + o + j);
-                        const uint2 mk = *reinterpret_cast<const uint2 *>(shmask0 + o + j);
+                    for (int jj = 0; jj < 16; jj += 4) {
+                        const float4 nm = *reinterpret_cast<const float4 *>(snmean + o + jj);
+                        const float4 rs = *reinterpret_cast<const float4 *>(srstd + o + jj);
+                        const uint2 mk = *reinterpret_cast<const uint2 *>(shmask + o + jj);
 #pragma unroll
                         for (int h = 0; h < 2; ++h) {
                             // two consecutive pairs of this channel in one packed lane pair
                             const float2 nm2 = h == 0 ? make_float2(nm.x, nm.y) : make_float2(nm.z, nm.w);
                             const float2 rs2 = h == 0 ? make_float2(rs.x, rs.y) : make_float2(rs.z, rs.w);
-                            const float2 gv = f2_fma(rs2, f2_fma(nm2, cg_sum, make_float2(g[j + 2 * h], g[j + 2 * h + 1])), cg_shift);
-                            const float2 pv = f2_fma(rs2, f2_fma(nm2, cp_sum, make_float2(pr[j + 2 * h], pr[j + 2 * h + 1])), cp_shift);
+                            const float2 gv = f2_fma(rs2, f2_fma(nm2, cg_sum, make_float2(g[jj + 2 * h], g[jj + 2 * h + 1])), cg_shift);
+                            const float2 pv = f2_fma(rs2, f2_fma(nm2, cp_sum, make_float2(pr[jj + 2 * h], pr[jj + 2 * h + 1])), cp_shift);
                             // mask * sigmoid(2 x) = (mask / 2) tanh(x) + mask / 2, x being the halved gate
                             const __half2 hm = u32_as_h2(h == 0 ? mk.x : mk.y);
                             const __half2 gm = __hfma2(tanh_h2(__floats2half2_rn(gv.x, gv.y)), hm, hm);
-                            outw[j / 2 + h] = h2_as_u32(__hmul2(gm, __floats2half2_rn(pv.x, pv.y)));
+                            outw[jj / 2 + h] = h2_as_u32(__hmul2(gm, __floats2half2_rn(pv.x, pv.y)));
                         }
                     }
 #pragma unroll
                     for (int u = 0; u < 2; ++u)
                         *reinterpret_cast<uint4 *>(stg + sw64_offset(lane, 2 * hh + u)) =
                             make_uint4(outw[4 * u], outw[4 * u + 1], outw[4 * u + 2], outw[4 * u + 3]);
+                    if (acc_c) {
+                        __half2 hs = u32_as_h2(outw[0]);
+#pragma unroll
+                        for (int u = 1; u < 8; ++u) hs = __hadd2(hs, u32_as_h2(outw[u]));
+                        const float2 hf = __half22float2(hs);
+                        run += hf.x + hf.y;
+                    }
                 }
                 fence_proxy_async_smem();
                 __syncwarp();
                 if (lane == 0) {
-                    if (blk == 1) mbar_arrive(&s.sempty[sbuf]);   // statistics read in full
-                    if (p0 + col < p.NN) {              // blocks wholly past the last pair are not stored
-                        tma_store_3d(tm_out, stg, p0 + col, q * 32, b);
-                        tma_store_commit();
-                    }
+                    if (blk == 1) mbar_arrive(&s.sempty[buf]);   // statistics read in full
+                    tma_store_3d(tm_out, stg, p0 + 32 * blk, q * 32, b);
+                    tma_store_commit();
                 }
             }
             phase ^= 1;
         }
+        if (acc_c && sum_b >= 0) atomicAdd(acc_c + (size_t)sum_b * (2 * C::C_H + 1), (unsigned long long)llrintf(run * kAccScale));
         if (lane == 0) tma_store_wait_all<0>();
     }
 
@@ -655,11 +708,12 @@ __global__ void __launch_bounds__(K1CmCfg::THREADS, 1) k1_project_cm_kernel(cons
     }
 }
 
-int k1_ncol(int c_z) { return c_z == 128 ? 2 * K1CmCfg::C_H : K1Cfg<384>::NCOL; }
-int k1_groups(int c_z) { return c_z == 128 ? K1CmCfg::G : K1Cfg<384>::G; }
-int k1_channels_per_warpgroup(int c_z) { return c_z == 128 ? K1CmCfg::C_H : K1Cfg<384>::CH_WG; }
+int k1_ncol(int c_z) { return c_z == 128 ? 256 : K1Cfg<384>::NCOL; }
+int k1_groups(int c_z) { return c_z == 128 ? 1 : K1Cfg<384>::G; }
+int k1_channels_per_warpgroup(int c_z) { return c_z == 128 ? K1AbCfg::C_H : K1Cfg<384>::CH_WG; }
 int k1_row_mode(int c_z) { return c_z == 128 ? 2 : 1; }
-size_t k1_smem_bytes(int c_z) { return c_z == 128 ? K1CmCfg::SMEM : K1Cfg<384>::SMEM; }
+int k1_tile_pairs(int c_z) { return c_z == 128 ? K1AbCfg::TP : 128; }
+size_t k1_smem_bytes(int c_z) { return c_z == 128 ? K1AbCfg::SMEM : K1Cfg<384>::SMEM; }
 
 template <int CZ, bool SKIP>
 static cudaError_t k1_launch_t(const K1Args &args, int grid, cudaStream_t stream) {
@@ -676,22 +730,22 @@ static cudaError_t k1_launch_t(const K1Args &args, int grid, cudaStream_t stream
 }
 
 template <bool SKIP>
-static cudaError_t k1_launch_cm(const K1Args &args, int grid, cudaStream_t stream) {
+static cudaError_t k1_launch_ab(const K1Args &args, int grid, cudaStream_t stream) {
     static int configured_device = -1;
     int dev = 0;
     cudaGetDevice(&dev);
     if (configured_device != dev) {
-        cudaError_t e = cudaFuncSetAttribute(k1_project_cm_kernel<SKIP>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                             (int)K1CmCfg::SMEM);
+        cudaError_t e = cudaFuncSetAttribute(k1_project_ab_kernel<SKIP>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                             (int)K1AbCfg::SMEM);
         if (e != cudaSuccess) return e;
         configured_device = dev;
     }
-    return launch_pdl(k1_project_cm_kernel<SKIP>, grid, K1CmCfg::THREADS, K1CmCfg::SMEM, stream, args);
+    return launch_pdl(k1_project_ab_kernel<SKIP>, grid, K1AbCfg::THREADS, K1AbCfg::SMEM, stream, args);
 }
 
 cudaError_t k1_launch(int c_z, const K1Args &args, int grid, cudaStream_t stream) {
     const bool skip = args.ext != nullptr;
-    if (c_z == 128) return skip ? k1_launch_cm<true>(args, grid, stream) : k1_launch_cm<false>(args, grid, stream);
+    if (c_z == 128) return skip ? k1_launch_ab<true>(args, grid, stream) : k1_launch_ab<false>(args, grid, stream);
     if (c_z == 384) return skip ? k1_launch_t<384, true>(args, grid, stream) : k1_launch_t<384, false>(args, grid, stream);
     return cudaErrorInvalidValue;
 }

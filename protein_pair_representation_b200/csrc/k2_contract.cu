@@ -6,9 +6,10 @@
 //   outgoing  X_c = A_c B_c^T   (x_ij = sum_k a_ik b_jk; both operands K-major)
 //   incoming  X_c = A_c^T B_c   (x_ij = sum_k a_ki b_kj; both operands MN-major)
 // a, b, x are [B*c_h][N][N] of one 16-bit type (fp16 on the update path, bf16 also
-// supported), with fp32 accumulation and an optional power-of-two scale applied to
-// the result before rounding. The two directions differ only in the TMA boxes and
-// in the major-ness bits of the shared-memory descriptors.
+// supported), with fp32 accumulation, an optional power-of-two scale and a per-channel
+// offset applied to the result before rounding (x = round(scale * sum - offset)). The
+// two directions differ only in the TMA boxes and in the major-ness bits of the
+// shared-memory descriptors.
 //
 // Persistent kernel, one CTA per SM, 128 x 256 output tiles, 64-deep k chunks:
 //   warp 8      TMA producer (one elected lane) filling a 4-stage ring
@@ -205,6 +206,7 @@ __global__ void __launch_bounds__(k2::THREADS, 1) k2_contract_kernel(const __gri
             const int m0 = (r / p.n_tiles) * BM;
             const int n0 = (r % p.n_tiles) * BN;
             if (k2_tile_chunks(p, bc, m0, n0) == 0) continue;
+            const float nq = -__ldg(p.xoff + (size_t)bc * p.xoff_stride);   // minus this channel's offset
             if (!group_all(mbar_wait(&s.tfull[abuf], aphase, abort_flag, kErrTimeoutEpilogue), 1 + wg, 128)) break;
             tc_fence_after();
 #pragma unroll 1
@@ -225,7 +227,7 @@ __global__ void __launch_bounds__(k2::THREADS, 1) k2_contract_kernel(const __gri
                         if (lane == 0) mbar_arrive(&s.tempty[abuf]);
                     }
 #pragma unroll
-                    for (int e = 0; e < 32; ++e) v[e] *= p.x_scale;
+                    for (int e = 0; e < 32; ++e) v[e] = fmaf(v[e], p.x_scale, nq);
 #pragma unroll
                     for (int u = 0; u < 4; ++u) {
                         uint4 w;

@@ -12,7 +12,8 @@ constexpr int kHidden = 128;  // c_h of the tensor-core path
 // ---- bf16 tensor-core path ---------------------------------------------------------
 
 struct K1Args {
-    CUtensorMap tm_z;      // z [B][N*N][c_z] bf16, box {64, 128, 1}, 128B swizzle
+    CUtensorMap tm_z;      // z: c_z = 128: {64 ch, N*N, 2 halves, B}, box {64, 64, 2, 1}; c_z = 384:
+                           // [B][N*N][c_z], box {64, 128, 1}; bf16, 128B swizzle
     CUtensorMap tm_w;      // packed weights [4*c_h][c_z] bf16, box {64, NCOL}, 128B swizzle
     CUtensorMap tm_a;      // a [B][c_h][N*N] f16; c_z = 128: box {64, 128, 1} 128B swizzle,
                            // c_z = 384: box {128, channels per warpgroup, 1} no swizzle
@@ -21,11 +22,17 @@ struct K1Args {
     const float4 *vec;     // [2][c_h] {sum W'_gate, shift_gate, sum W'_proj, shift_proj}
     int B, N;
     long long NN;
-    int tiles_per_batch;   // ceil(NN / 128)
+    int tiles_per_batch;   // ceil(NN / k1_tile_pairs(c_z))
     float eps;
     const int *ext;        // mask extents [B][2] {R_b, C_b} (tiles wholly beyond them skipped), or nullptr
     uint64_t rowdiv;       // multiplier dividing by N / 8 (div_by_magic)
+    unsigned long long *acc;   // per batch element [2*c_h + 1]: fixed-point (x kAccScale) sums of the
+                               // stored a and b per channel and the count of unmasked pairs, added
+                               // with integer atomics (order-independent); nullptr: not gathered
 };
+
+// Fixed-point scale of the a / b channel sums (K1Args::acc).
+constexpr float kAccScale = 256.0f;
 
 struct K2Args {
     CUtensorMap tm_a, tm_b, tm_x;
@@ -38,6 +45,9 @@ struct K2Args {
                            // (outgoing) or k < R_b (incoming); output tiles at rows >= R_b or
                            // columns >= C_b are not written (the output kernel never reads them)
     int C;                 // channels per batch element (bc / C = batch element)
+    const float *xoff;     // per (batch, channel) offset q subtracted after the scaling, before the
+                           // rounding: x = round(x_scale * sum - xoff[bc * xoff_stride])
+    int xoff_stride;       // 1, or 0 with xoff pointing at a single zero
 };
 
 struct K3Args {
@@ -56,6 +66,12 @@ struct K3Args {
     const uint16_t *zres;  // residual: z (bf16, [B][N*N][c_z]) added to the output; null = none
     const int *ext;        // mask extents (as K1Args); ignored with a residual (masked pairs then copy z)
     uint64_t rowdiv;
+    // The stored x is x_scale * x - q[b][c]: the LayerNorm statistics add q back per channel
+    // (q = xoff + b * xoff_stride, c_h entries) and the x-GEMM adds Q[b][n] = sum_c q[b][c] W_o'[n][c]
+    // (xoff_w + b * xoffw_stride, c_z entries). Strides 0 with pointers at zeros: no offsets.
+    const float *xoff;
+    const float *xoff_w;
+    int xoff_stride, xoffw_stride;
 };
 
 // Launch with programmatic stream serialization: the kernel may begin while the previous
@@ -84,6 +100,7 @@ int k1_ncol(int c_z);
 int k1_channels_per_warpgroup(int c_z);
 cudaError_t k1_launch(int c_z, const K1Args &args, int grid, cudaStream_t stream);
 int k1_row_mode(int c_z);
+int k1_tile_pairs(int c_z);        // pairs per K1 tile (64 at c_z = 128, 128 at c_z = 384)
 
 size_t k2_smem_bytes();
 cudaError_t k2_launch(const K2Args &args, int grid, cudaStream_t stream);
@@ -118,6 +135,13 @@ inline uint64_t host_rowdiv(uint64_t d) { return d <= 1 ? 0 : ~0ull / d + 1; }
 size_t k3_smem_bytes(int c_z, bool out_f32);
 int k3_groups(int c_z);
 cudaError_t k3_launch(int c_z, bool out_f32, const K3Args &args, int grid, cudaStream_t stream);  // residual iff args.zres
+
+// The per-(batch, channel) offsets of the stored x from K1's sums: q[b][c] = x_scale * Sa Sb / P^1.5
+// (Sa, Sb the channel sums of a and b over batch element b, P its unmasked pairs; 0 when P = 0),
+// Q[b][n] = sum_c q[b][c] wo[n][c] (wo the folded f16 W_o' [c_z][c_h]); the sums are zeroed for the
+// next forward. One CTA per batch element.
+cudaError_t xoffsets_launch(unsigned long long *acc, int B, int c_h, int c_z, float x_scale, const uint16_t *wo,
+                            float *q, float *Q, cudaStream_t stream);
 
 // ---- weight folding (layer creation) -----------------------------------------------
 

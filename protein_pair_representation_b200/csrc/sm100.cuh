@@ -149,18 +149,19 @@ __device__ __forceinline__ uint32_t div_by_magic(uint32_t x, uint64_t m) {
     return m ? (uint32_t)__umul64hi((uint64_t)x, m) : x;
 }
 
-// Whether every pair of the 128-pair tile starting at pair p0 of batch element b is masked,
-// from the mask's extents ext[2b] = R_b (1 + the last row holding a nonzero mask entry) and
-// ext[2b + 1] = C_b (1 + the last such column): the tile lies in rows >= R_b, or within one
-// row at columns >= C_b. ext = null: no extents, nothing is skipped. rowdiv divides by N / 8
-// (p0 and N are multiples of 8).
+// Whether every pair of the TP-pair tile (128 by default) starting at pair p0 of batch element b
+// is masked, from the mask's extents ext[2b] = R_b (1 + the last row holding a nonzero mask
+// entry) and ext[2b + 1] = C_b (1 + the last such column): the tile lies in rows >= R_b, or
+// within one row at columns >= C_b. ext = null: no extents, nothing is skipped. rowdiv divides
+// by N / 8 (p0 and N are multiples of 8).
+template <int TP = 128>
 __device__ __forceinline__ bool tile_masked_out(const int *ext, int b, long long p0, int N, long long NN,
                                                 uint64_t rowdiv) {
     if (!ext) return false;
     const int R = __ldg(ext + 2 * b), C = __ldg(ext + 2 * b + 1);
     const int i0 = (int)div_by_magic((uint32_t)(p0 >> 3), rowdiv);
     if (i0 >= R) return true;
-    const long long last = (p0 + 127 < NN - 1) ? p0 + 127 : NN - 1;
+    const long long last = (p0 + TP - 1 < NN - 1) ? p0 + TP - 1 : NN - 1;
     const int i1 = (int)div_by_magic((uint32_t)(last >> 3), rowdiv);
     return i1 == i0 && (int)(p0 - (long long)i0 * N) >= C;
 }

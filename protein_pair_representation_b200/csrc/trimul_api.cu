@@ -20,6 +20,8 @@
 namespace trimul {
 __device__ unsigned int g_device_error = 0;
 }
+// The offset of the stand-alone contraction, which has none.
+static __device__ __align__(16) float g_zero_float[4] = {0.f, 0.f, 0.f, 0.f};
 
 using namespace trimul;
 
@@ -34,6 +36,10 @@ struct trimul_layer {
     uint16_t *k3_wo;             // [c_z][c_h] folded
     uint16_t *k3_wg;             // [c_z][c_z] folded
     float4 *k3_vec;              // [c_z]
+    // K1's per-(batch, channel) sums of a and b and unmasked-pair counts, [65535 / c_h + 1][2 c_h + 1]
+    // (zero between forwards: the offsets kernel clears what it has read)
+    unsigned long long *acc;
+    float *zeros;                // kZeros zero floats: the offsets of the stand-alone stages
     // fp32 path
     F32Weights f32;
     // workspace
@@ -151,6 +157,12 @@ static trimul_status_t make_map(CUtensorMap *m, CUtensorMapDataType dt, int rank
         if (_s != TRIMUL_OK) return _s;           \
     } while (0)
 
+// Zero floats kept in each layer, enough for any offset vector a kernel reads with stride 0.
+static constexpr int kZeros = 512;
+
+// Batch elements the layer's channel sums have room for: B * c_h <= 65535 is enforced.
+static int acc_batches(int c_h) { return 65535 / c_h + 1; }
+
 // ------------------------------------------------------------------ validation helpers
 
 static bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
@@ -174,13 +186,27 @@ static size_t pair_bytes(const trimul_pair_t *t) {
     return (size_t)t->B * t->N * t->N * t->C * dtype_size(t->dtype);
 }
 
-static trimul_status_t check_problem(const trimul_pair_t *z, const void *mask, const trimul_layer_t *L) {
-    // the size rules first: they need no layer
+// The size rules of z: they need no layer.
+static trimul_status_t check_sizes(const trimul_pair_t *z) {
     TRY(check_pair(z, "z"));
     if (z->N < 8 || z->N % 8 != 0) return fail(TRIMUL_ERR_UNSUPPORTED_SHAPE, "N=%lld must be a positive multiple of 8", (long long)z->N);
     if (z->N > 16384) return fail(TRIMUL_ERR_UNSUPPORTED_SHAPE, "N=%lld exceeds 16384", (long long)z->N);
     if (z->dtype == TRIMUL_BF16 && (long long)z->B * z->N * z->N / 128 > (1LL << 30))
         return fail(TRIMUL_ERR_UNSUPPORTED_SHAPE, "problem too large: B * N^2 / 128 must not exceed 2^30");
+    return TRIMUL_OK;
+}
+
+// The rules on out that need no layer: present, aligned, z's shape, fp32 on the fp32 path, apart from z.
+static trimul_status_t check_out(const trimul_pair_t *z, const trimul_pair_t *out) {
+    TRY(check_pair(out, "out"));
+    if (out->B != z->B || out->N != z->N || out->C != z->C) return fail(TRIMUL_ERR_INVALID_ARG, "out shape differs from z");
+    if (z->dtype == TRIMUL_F32 && out->dtype != TRIMUL_F32) return fail(TRIMUL_ERR_INVALID_ARG, "fp32 path writes fp32 out");
+    if (overlap(out->data, pair_bytes(out), z->data, pair_bytes(z))) return fail(TRIMUL_ERR_INVALID_ARG, "out overlaps z");
+    return TRIMUL_OK;
+}
+
+static trimul_status_t check_problem(const trimul_pair_t *z, const void *mask, const trimul_layer_t *L) {
+    TRY(check_sizes(z));
     if (!L) return fail(TRIMUL_ERR_INVALID_ARG, "layer is NULL");
     if (z->C != L->c_z) return fail(TRIMUL_ERR_INVALID_ARG, "z has %lld channels, layer expects c_z=%d", (long long)z->C, L->c_z);
     // the contraction's limit (B * c_h planes), checked here so that no stage has run when it fails
@@ -217,13 +243,16 @@ extern "C" trimul_status_t tri_mul_layer_create(const trimul_weights_desc_t *w, 
     // carve one allocation
     size_t off = 0;
     auto take = [&](size_t bytes) { size_t o = off; off = (off + bytes + 255) & ~size_t(255); return o; };
-    size_t o_k1w = 0, o_k1v = 0, o_k3o = 0, o_k3g = 0, o_k3v = 0;
+    size_t o_k1w = 0, o_k1v = 0, o_k3o = 0, o_k3g = 0, o_k3v = 0, o_acc = 0, o_zero = 0, acc_bytes = 0;
     if (L->has_bf16) {
         o_k1w = take((size_t)4 * ch * cz * 2);
         o_k1v = take((size_t)2 * ch * sizeof(float4));
         o_k3o = take((size_t)cz * ch * 2);
         o_k3g = take((size_t)cz * cz * 2);
         o_k3v = take((size_t)cz * sizeof(float4));
+        acc_bytes = (size_t)acc_batches(ch) * (2 * ch + 1) * sizeof(unsigned long long);
+        o_acc = take(acc_bytes);
+        o_zero = take(kZeros * sizeof(float));
     }
     const size_t o_lig = take(cz * 4), o_lib = take(cz * 4);
     const size_t o_wag = take((size_t)ch * cz * 4), o_wap = take((size_t)ch * cz * 4);
@@ -270,6 +299,9 @@ extern "C" trimul_status_t tri_mul_layer_create(const trimul_weights_desc_t *w, 
         L->k3_wo = reinterpret_cast<uint16_t *>(m + o_k3o);
         L->k3_wg = reinterpret_cast<uint16_t *>(m + o_k3g);
         L->k3_vec = reinterpret_cast<float4 *>(m + o_k3v);
+        L->acc = reinterpret_cast<unsigned long long *>(m + o_acc);
+        L->zeros = reinterpret_cast<float *>(m + o_zero);
+        ce = cudaMemsetAsync(m + o_acc, 0, (o_zero - o_acc) + kZeros * sizeof(float), st);
         const int ncol = k1_ncol(cz);
         const void *srcs[2][2] = {{w->w_ag, w->w_ap}, {w->w_bg, w->w_bp}};
         const void *biases[2][2] = {{w->b_ag, w->b_ap}, {w->b_bg, w->b_bp}};
@@ -331,16 +363,25 @@ extern "C" void tri_mul_layer_destroy(trimul_layer_t *L) {
     delete L;
 }
 
+static size_t align256(size_t n) { return (n + 255) & ~size_t(255); }
+
 static size_t ws_plane_bytes(int64_t B, int64_t N, int c_h, trimul_dtype_t dt) {
-    return (((size_t)B * c_h * N * N * dtype_size(dt)) + 255) & ~size_t(255);
+    return align256((size_t)B * c_h * N * N * dtype_size(dt));
 }
 
-// The mask extents {R_b, C_b} (int32) of a forward, after the three planes.
-static size_t ws_ext_bytes(int64_t B) { return ((size_t)B * 2 * sizeof(int) + 255) & ~size_t(255); }
+// After the three planes: the mask extents {R_b, C_b} (int32), then the offsets q [B][c_h] and
+// their projections Q [B][c_z] (fp32) of the stored x.
+static size_t ws_ext_bytes(int64_t B) { return align256((size_t)B * 2 * sizeof(int)); }
+static size_t ws_q_bytes(int64_t B, int c_h) { return align256((size_t)B * c_h * sizeof(float)); }
+static size_t ws_Q_bytes(int64_t B, int c_z) { return align256((size_t)B * c_z * sizeof(float)); }
+
+static size_t ws_total_bytes(const trimul_layer_t *L, int64_t B, int64_t N, trimul_dtype_t dt) {
+    return 3 * ws_plane_bytes(B, N, L->c_h, dt) + ws_ext_bytes(B) + ws_q_bytes(B, L->c_h) + ws_Q_bytes(B, L->c_z);
+}
 
 extern "C" size_t tri_mul_workspace_bytes(const trimul_layer_t *L, int64_t B, int64_t N, trimul_dtype_t dt) {
     if (!L || B < 1 || N < 1 || (dt != TRIMUL_F32 && dt != TRIMUL_BF16)) return 0;
-    return 3 * ws_plane_bytes(B, N, L->c_h, dt) + ws_ext_bytes(B);
+    return ws_total_bytes(L, B, N, dt);
 }
 
 extern "C" trimul_status_t tri_mul_layer_bind_workspace(trimul_layer_t *L, void *ws, size_t bytes) {
@@ -365,7 +406,7 @@ extern "C" trimul_status_t tri_mul_layer_set_timing_events(trimul_layer_t *L, vo
     return TRIMUL_OK;
 }
 
-extern "C" int tri_mul_kernels_per_forward(void) { return 3; }
+extern "C" int tri_mul_kernels_per_forward(void) { return 4; }
 
 extern "C" trimul_status_t tri_mul_layer_set_mask_skipping(trimul_layer_t *L, int enable) {
     if (!L) return fail(TRIMUL_ERR_INVALID_ARG, "layer is NULL");
@@ -383,16 +424,24 @@ static int grid_for(int sms, long long work_units, int multiple) {
 }
 
 static trimul_status_t run_project_bf16(const trimul_layer_t *L, const void *z, const void *mask, void *a, void *b,
-                                        int B, int N, cudaStream_t st, const int *ext) {
+                                        int B, int N, cudaStream_t st, const int *ext, unsigned long long *acc) {
     DeviceInfo d;
     TRY(require_sm100(&d));
     const uint64_t NN = (uint64_t)N * N;
     const int cz = L->c_z, ch = L->c_h;
     K1Args p{};
-    {
+    const int tp = k1_tile_pairs(cz);
+    if (cz == 128) {
+        // z [B][NN][128] viewed as {64 channels, NN pairs, 2 halves, B}: one copy brings both
+        // 64-channel halves of a 64-pair tile, laid out [half][pair][64]
+        uint64_t dims[4] = {64, NN, 2, (uint64_t)B};
+        uint64_t strides[3] = {(uint64_t)cz * 2, 128, NN * cz * 2};
+        uint32_t box[4] = {64, (uint32_t)tp, 2, 1};
+        TRY(make_map(&p.tm_z, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, z, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_128B, "K1 z"));
+    } else {
         uint64_t dims[3] = {(uint64_t)cz, NN, (uint64_t)B};
         uint64_t strides[2] = {(uint64_t)cz * 2, NN * cz * 2};
-        uint32_t box[3] = {64, 128, 1};
+        uint32_t box[3] = {64, (uint32_t)tp, 1};
         TRY(make_map(&p.tm_z, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, z, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_128B, "K1 z"));
     }
     {
@@ -418,10 +467,11 @@ static trimul_status_t run_project_bf16(const trimul_layer_t *L, const void *z, 
     p.B = B;
     p.N = N;
     p.NN = (long long)NN;
-    p.tiles_per_batch = (int)((NN + 127) / 128);
+    p.tiles_per_batch = (int)((NN + tp - 1) / tp);
     p.eps = L->eps;
     p.ext = ext;
     p.rowdiv = host_rowdiv((uint64_t)N / 8);
+    p.acc = acc;
     const int G = k1_groups(cz);
     const int grid = grid_for(d.sms, (long long)G * B * p.tiles_per_batch, G);
     TRY_CUDA(k1_launch(cz, p, grid, st), "K1 launch");
@@ -429,7 +479,8 @@ static trimul_status_t run_project_bf16(const trimul_layer_t *L, const void *z, 
 }
 
 static trimul_status_t run_contract_tc(const void *a, const void *b, void *x, int64_t BC, int N, bool incoming,
-                                       bool f16, float x_scale, cudaStream_t st, const int *ext, int C) {
+                                       bool f16, float x_scale, cudaStream_t st, const int *ext, int C,
+                                       const float *xoff, int xoff_stride) {
     DeviceInfo d;
     TRY(require_sm100(&d));
     K2Args p{};
@@ -451,6 +502,8 @@ static trimul_status_t run_contract_tc(const void *a, const void *b, void *x, in
     }
     p.f16 = f16;
     p.x_scale = x_scale;
+    p.xoff = xoff;
+    p.xoff_stride = xoff_stride;
     p.ext = ext;
     p.C = C;
     p.BC = (int)BC;
@@ -467,7 +520,7 @@ static trimul_status_t run_contract_tc(const void *a, const void *b, void *x, in
 
 static trimul_status_t run_output_bf16(const trimul_layer_t *L, const void *z, const void *mask, const void *x,
                                        float x_scale, void *out, bool out_f32, bool residual, int B, int N,
-                                       cudaStream_t st, const int *ext) {
+                                       cudaStream_t st, const int *ext, const float *q, const float *Q) {
     DeviceInfo d;
     TRY(require_sm100(&d));
     const uint64_t NN = (uint64_t)N * N;
@@ -518,6 +571,10 @@ static trimul_status_t run_output_bf16(const trimul_layer_t *L, const void *z, c
     p.zres = residual ? reinterpret_cast<const uint16_t *>(z) : nullptr;
     p.ext = residual ? nullptr : ext;        // with a residual a masked pair copies z: nothing is skipped
     p.rowdiv = host_rowdiv((uint64_t)N / 8);
+    p.xoff = q ? q : L->zeros;
+    p.xoff_stride = q ? ch : 0;
+    p.xoff_w = Q ? Q : L->zeros;
+    p.xoffw_stride = Q ? cz : 0;
     const int G = k3_groups(cz);
     const int grid = grid_for(d.sms, (long long)G * B * p.tiles_per_batch, G);
     TRY_CUDA(k3_launch(cz, out_f32, p, grid, st), "K3 launch");
@@ -527,7 +584,7 @@ static trimul_status_t run_output_bf16(const trimul_layer_t *L, const void *z, c
 // ------------------------------------------------------------------ public entry points
 
 static trimul_status_t project_impl(const trimul_pair_t *z, const void *mask, const trimul_layer_t *L, void *a_out,
-                                    void *b_out, const int *ext, void *stream) {
+                                    void *b_out, const int *ext, unsigned long long *acc, void *stream) {
     TRY(check_problem(z, mask, L));
     if (!a_out || !b_out) return fail(TRIMUL_ERR_INVALID_ARG, "a_out / b_out NULL");
     if (!aligned16(a_out) || !aligned16(b_out)) return fail(TRIMUL_ERR_ALIGNMENT, "a_out / b_out not 16-byte aligned");
@@ -537,7 +594,7 @@ static trimul_status_t project_impl(const trimul_pair_t *z, const void *mask, co
         return fail(TRIMUL_ERR_INVALID_ARG, "a_out, b_out and z overlap");
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
     if (z->dtype == TRIMUL_BF16)
-        return run_project_bf16(L, z->data, mask, a_out, b_out, (int)z->B, (int)z->N, st, ext);
+        return run_project_bf16(L, z->data, mask, a_out, b_out, (int)z->B, (int)z->N, st, ext, acc);
     TRY_CUDA(f32_project_launch(reinterpret_cast<const float *>(z->data), reinterpret_cast<const float *>(mask), L->f32,
                                 L->c_z, L->c_h, (int)z->B, (int)z->N, L->eps, reinterpret_cast<float *>(a_out),
                                 reinterpret_cast<float *>(b_out), st),
@@ -547,7 +604,7 @@ static trimul_status_t project_impl(const trimul_pair_t *z, const void *mask, co
 
 extern "C" trimul_status_t tri_mul_project(const trimul_pair_t *z, const void *mask, const trimul_layer_t *L, void *a_out,
                                            void *b_out, void *stream) {
-    return project_impl(z, mask, L, a_out, b_out, nullptr, stream);
+    return project_impl(z, mask, L, a_out, b_out, nullptr, nullptr, stream);
 }
 
 extern "C" float tri_mul_contract_scale(int64_t N) {
@@ -557,9 +614,10 @@ extern "C" float tri_mul_contract_scale(int64_t N) {
     return ldexpf(1.0f, -((lg + 1) / 2));       // 2^-ceil(log2(N) / 2)
 }
 
+// q: per (batch, channel) offsets subtracted from x_scale * x before rounding, or nullptr (none)
 static trimul_status_t contract_impl(const void *a, const void *b, void *x, int64_t B, int64_t C, int64_t N,
                                      trimul_dtype_t dtype, trimul_direction_t dir, float x_scale, const int *ext,
-                                     void *stream) {
+                                     const float *q, void *stream) {
     if (!a || !b || !x) return fail(TRIMUL_ERR_INVALID_ARG, "NULL tensor");
     if (dtype != TRIMUL_F32 && dtype != TRIMUL_BF16 && dtype != TRIMUL_F16) return fail(TRIMUL_ERR_INVALID_ARG, "unknown dtype");
     if (!(x_scale > 0.f) || !(x_scale < 3.0e38f)) return fail(TRIMUL_ERR_INVALID_ARG, "x_scale must be positive and finite");
@@ -571,9 +629,26 @@ static trimul_status_t contract_impl(const void *a, const void *b, void *x, int6
     const size_t bytes = (size_t)B * C * N * N * dtype_size(dtype);
     if (overlap(x, bytes, a, bytes) || overlap(x, bytes, b, bytes)) return fail(TRIMUL_ERR_INVALID_ARG, "x overlaps a or b");
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
-    if (dtype != TRIMUL_F32)
+    if (dtype != TRIMUL_F32) {
+        static float *zero_dev[64];                 // one zero float per device for the offset-free call
+        const float *xo = q;
+        if (!xo) {
+            int dev = 0;
+            TRY_CUDA(cudaGetDevice(&dev), "cudaGetDevice");
+            if (dev < 0 || dev >= 64) return fail(TRIMUL_ERR_UNSUPPORTED_DEVICE, "device index %d", dev);
+            {
+                std::lock_guard<std::mutex> lk(g_dev_mu);
+                if (!zero_dev[dev]) {
+                    void *pz = nullptr;
+                    TRY_CUDA(cudaGetSymbolAddress(&pz, g_zero_float), "zero offset address");
+                    zero_dev[dev] = reinterpret_cast<float *>(pz);
+                }
+                xo = zero_dev[dev];
+            }
+        }
         return run_contract_tc(a, b, x, B * C, (int)N, dir == TRIMUL_INCOMING, dtype == TRIMUL_F16, x_scale, st, ext,
-                               (int)C);
+                               (int)C, xo, q ? 1 : 0);
+    }
     TRY_CUDA(f32_contract_launch(reinterpret_cast<const float *>(a), reinterpret_cast<const float *>(b),
                                  reinterpret_cast<float *>(x), (int)(B * C), (int)N, dir == TRIMUL_INCOMING, x_scale, st),
              "fp32 contraction launch");
@@ -582,26 +657,24 @@ static trimul_status_t contract_impl(const void *a, const void *b, void *x, int6
 
 extern "C" trimul_status_t tri_mul_contract(const void *a, const void *b, void *x, int64_t B, int64_t C, int64_t N,
                                             trimul_dtype_t dtype, trimul_direction_t dir, float x_scale, void *stream) {
-    return contract_impl(a, b, x, B, C, N, dtype, dir, x_scale, nullptr, stream);
+    return contract_impl(a, b, x, B, C, N, dtype, dir, x_scale, nullptr, nullptr, stream);
 }
 
 static trimul_status_t output_gate_impl(const trimul_pair_t *z, const void *mask, const void *x, float x_scale,
                                         const trimul_layer_t *L, trimul_pair_t *out, bool residual, const int *ext,
-                                        void *stream) {
+                                        const float *q, const float *Q, void *stream) {
+    TRY(check_sizes(z));
+    TRY(check_out(z, out));
     TRY(check_problem(z, mask, L));
     if (!(x_scale > 0.f) || !(x_scale < 3.0e38f)) return fail(TRIMUL_ERR_INVALID_ARG, "x_scale must be positive and finite");
-    TRY(check_pair(out, "out"));
     if (!x) return fail(TRIMUL_ERR_INVALID_ARG, "x is NULL");
     if (!aligned16(x)) return fail(TRIMUL_ERR_ALIGNMENT, "x not 16-byte aligned");
-    if (out->B != z->B || out->N != z->N || out->C != z->C) return fail(TRIMUL_ERR_INVALID_ARG, "out shape differs from z");
-    if (z->dtype == TRIMUL_F32 && out->dtype != TRIMUL_F32) return fail(TRIMUL_ERR_INVALID_ARG, "fp32 path writes fp32 out");
-    if (overlap(out->data, pair_bytes(out), z->data, pair_bytes(z))) return fail(TRIMUL_ERR_INVALID_ARG, "out overlaps z");
     const size_t xbytes = (size_t)z->B * L->c_h * z->N * z->N * dtype_size(z->dtype);
     if (overlap(out->data, pair_bytes(out), x, xbytes)) return fail(TRIMUL_ERR_INVALID_ARG, "out overlaps x");
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
     if (z->dtype == TRIMUL_BF16)
         return run_output_bf16(L, z->data, mask, x, x_scale, out->data, out->dtype == TRIMUL_F32, residual, (int)z->B,
-                               (int)z->N, st, ext);
+                               (int)z->N, st, ext, q, Q);
     TRY_CUDA(f32_output_launch(reinterpret_cast<const float *>(z->data), reinterpret_cast<const float *>(mask),
                                reinterpret_cast<const float *>(x), L->f32, L->c_z, L->c_h, (int)z->B, (int)z->N, L->eps,
                                L->eps * x_scale * x_scale, residual, reinterpret_cast<float *>(out->data), st),
@@ -611,43 +684,64 @@ static trimul_status_t output_gate_impl(const trimul_pair_t *z, const void *mask
 
 extern "C" trimul_status_t tri_mul_output_gate(const trimul_pair_t *z, const void *mask, const void *x, float x_scale,
                                                const trimul_layer_t *L, trimul_pair_t *out, void *stream) {
-    return output_gate_impl(z, mask, x, x_scale, L, out, false, nullptr, stream);
+    return output_gate_impl(z, mask, x, x_scale, L, out, false, nullptr, nullptr, nullptr, stream);
 }
 
-static trimul_status_t forward_impl(const trimul_pair_t *z, const void *mask, const trimul_layer_t *L,
-                                    trimul_direction_t dir, trimul_pair_t *out, bool residual, void *stream) {
-    TRY(check_problem(z, mask, L));
-    TRY(check_pair(out, "out"));
+namespace trimul {
+// One update with its intermediates in `ws` (ws_bytes long; the layer's bound workspace, or the
+// no-allocation array). Every argument rule is checked before anything is launched: the sizes of
+// z, then out, then the layer, then the buffer. timing: record the layer's timing events.
+// check_only: run every check that does not need the buffer's address (ws_ptr is ignored) and
+// return without touching the device.
+trimul_status_t forward_buffers(const trimul_pair_t *z, const void *mask, const trimul_layer_t *L,
+                                trimul_direction_t dir, trimul_pair_t *out, bool residual, void *ws_ptr,
+                                size_t ws_bytes, bool timing, void *stream, bool check_only) {
+    TRY(check_sizes(z));
+    TRY(check_out(z, out));
     if (dir != TRIMUL_OUTGOING && dir != TRIMUL_INCOMING) return fail(TRIMUL_ERR_INVALID_ARG, "unknown direction");
-    if (out->B != z->B || out->N != z->N || out->C != z->C) return fail(TRIMUL_ERR_INVALID_ARG, "out shape differs from z");
-    if (z->dtype == TRIMUL_F32 && out->dtype != TRIMUL_F32) return fail(TRIMUL_ERR_INVALID_ARG, "fp32 path writes fp32 out");
+    TRY(check_problem(z, mask, L));
     const size_t plane = ws_plane_bytes(z->B, z->N, L->c_h, z->dtype);
-    const size_t need = 3 * plane + ws_ext_bytes(z->B);
-    if (!L->ws || L->ws_bytes < need)
-        return fail(TRIMUL_ERR_WORKSPACE, "workspace of %zu bytes needed, %zu bound", need, L->ws_bytes);
-    if (overlap(out->data, pair_bytes(out), z->data, pair_bytes(z))) return fail(TRIMUL_ERR_INVALID_ARG, "out overlaps z");
-    if (overlap(out->data, pair_bytes(out), L->ws, need) || overlap(z->data, pair_bytes(z), L->ws, need))
+    const size_t need = ws_total_bytes(L, z->B, z->N, z->dtype);
+    if ((!check_only && !ws_ptr) || ws_bytes < need)
+        return fail(TRIMUL_ERR_WORKSPACE, "workspace of %zu bytes needed, %zu available", need,
+                    (check_only || ws_ptr) ? ws_bytes : (size_t)0);
+    if (check_only) return TRIMUL_OK;
+    if (!aligned16(ws_ptr)) return fail(TRIMUL_ERR_ALIGNMENT, "workspace not 16-byte aligned");
+    if (overlap(out->data, pair_bytes(out), ws_ptr, need) || overlap(z->data, pair_bytes(z), ws_ptr, need))
         return fail(TRIMUL_ERR_INVALID_ARG, "z or out overlaps the workspace");
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
-    uint8_t *ws = reinterpret_cast<uint8_t *>(L->ws);
+    uint8_t *ws = reinterpret_cast<uint8_t *>(ws_ptr);
     void *a = ws, *b = ws + plane, *x = ws + 2 * plane;
     const bool tc = z->dtype == TRIMUL_BF16;
+    uint8_t *aux = ws + 3 * plane;
     // tensor-core path with a mask, skipping switched on: the mask's extents let the kernels
     // leave out wholly masked tiles
-    int *ext = (tc && mask && L->skip_masked) ? reinterpret_cast<int *>(ws + 3 * plane) : nullptr;
+    int *ext = (tc && mask && L->skip_masked) ? reinterpret_cast<int *>(aux) : nullptr;
+    float *q = reinterpret_cast<float *>(aux + ws_ext_bytes(z->B));
+    float *Q = reinterpret_cast<float *>(aux + ws_ext_bytes(z->B) + ws_q_bytes(z->B, L->c_h));
     if (ext)
         TRY_CUDA(mask_extents_launch(reinterpret_cast<const uint16_t *>(mask), (int)z->B, (int)z->N,
                                      host_rowdiv((uint64_t)z->N / 8), ext, st),
                  "mask extents launch");
-    if (L->timing) TRY_CUDA(cudaEventRecord(L->events[0], st), "event record");
-    TRY(project_impl(z, mask, L, a, b, ext, stream));
-    if (L->timing) TRY_CUDA(cudaEventRecord(L->events[1], st), "event record");
+    timing = timing && L->timing;
+    if (timing) TRY_CUDA(cudaEventRecord(L->events[0], st), "event record");
+    TRY(project_impl(z, mask, L, a, b, ext, tc ? L->acc : nullptr, stream));
     const float x_scale = tc ? tri_mul_contract_scale(z->N) : 1.0f;
-    TRY(contract_impl(a, b, x, z->B, L->c_h, z->N, tc ? TRIMUL_F16 : TRIMUL_F32, dir, x_scale, ext, stream));
-    if (L->timing) TRY_CUDA(cudaEventRecord(L->events[2], st), "event record");
-    TRY(output_gate_impl(z, mask, x, x_scale, L, out, residual, ext, stream));
-    if (L->timing) TRY_CUDA(cudaEventRecord(L->events[3], st), "event record");
+    // the offsets of the stored x from K1's channel sums (the fp32 path stores x as it is)
+    if (tc) TRY_CUDA(xoffsets_launch(L->acc, (int)z->B, L->c_h, L->c_z, x_scale, L->k3_wo, q, Q, st), "offsets launch");
+    if (timing) TRY_CUDA(cudaEventRecord(L->events[1], st), "event record");
+    TRY(contract_impl(a, b, x, z->B, L->c_h, z->N, tc ? TRIMUL_F16 : TRIMUL_F32, dir, x_scale, ext, tc ? q : nullptr, stream));
+    if (timing) TRY_CUDA(cudaEventRecord(L->events[2], st), "event record");
+    TRY(output_gate_impl(z, mask, x, x_scale, L, out, residual, ext, tc ? q : nullptr, tc ? Q : nullptr, stream));
+    if (timing) TRY_CUDA(cudaEventRecord(L->events[3], st), "event record");
     return TRIMUL_OK;
+}
+
+}  // namespace trimul
+
+static trimul_status_t forward_impl(const trimul_pair_t *z, const void *mask, const trimul_layer_t *L,
+                                    trimul_direction_t dir, trimul_pair_t *out, bool residual, void *stream) {
+    return forward_buffers(z, mask, L, dir, out, residual, L ? L->ws : nullptr, L ? L->ws_bytes : 0, true, stream, false);
 }
 
 extern "C" trimul_status_t tri_mul_forward(const trimul_pair_t *z, const void *mask, const trimul_layer_t *L,

@@ -49,8 +49,8 @@ def test_status_strings_and_versions(lib):
     for code in range(9):
         assert lib.tri_mul_status_string(code)
     assert lib.tri_mul_status_string(99) == b"unknown status"
-    assert lib.tri_mul_abi_version() == 101
-    assert lib.tri_mul_kernels_per_forward() == 3
+    assert lib.tri_mul_abi_version() == 102
+    assert lib.tri_mul_kernels_per_forward() == 4
 
 
 def test_null_arguments_are_rejected_on_the_host(lib):
@@ -62,15 +62,18 @@ def test_null_arguments_are_rejected_on_the_host(lib):
     assert b"z: NULL tensor" in lib.tri_mul_last_error()
     z = tm._Pair(1 << 24, 1, 8, 128, tm.BF16)        # aligned, never dereferenced
     assert lib.tri_mul_forward(ctypes.byref(z), None, None, 0, ctypes.byref(out), None) == 1
+    assert b"out: NULL tensor" in lib.tri_mul_last_error()
+    out = tm._Pair(1 << 30, 1, 8, 128, tm.F32)
+    assert lib.tri_mul_forward(ctypes.byref(z), None, None, 0, ctypes.byref(out), None) == 1
     assert b"layer is NULL" in lib.tri_mul_last_error()
 
 
 def test_forward_validates_sizes_before_the_layer(lib):
     """N a multiple of 8 in [8, 16384]; on the bf16 path B * N^2 / 128 tiles at most 2^30
     (int tile indices in the kernels). Checked before the layer and any device call."""
-    out = tm._Pair(1 << 40, 1, 8, 128, tm.F32)
     def status(B, N, dtype=tm.BF16):
         z = tm._Pair(1 << 24, B, N, 128, dtype)
+        out = tm._Pair(1 << 46, B, N, 128, tm.F32)
         return lib.tri_mul_forward(ctypes.byref(z), None, None, 0, ctypes.byref(out), None)
     assert status(1, 4) == 2
     assert status(1, 100) == 2
@@ -158,3 +161,33 @@ def test_pair_update_and_graph_validate_on_the_host(lib):
     assert lib.tri_mul_graph_launch(None, None) == 1
     lib.tri_mul_graph_destroy(None)          # NULL is ignored
     assert lib.tri_mul_forward_residual(None, None, None, 0, None, None) != 0
+
+
+def test_forward_and_noalloc_check_out_before_the_layer_and_the_device(lib):
+    """Every rule on `out` that needs no layer (present, aligned, z's shape, fp32 on the fp32
+    path, apart from z) is checked before the layer handle, so a bad `out` is reported with
+    nothing launched (here: no device at all) by both the workspace and the no-allocation
+    entry points."""
+    fn = lib.tri_mul_forward_noalloc
+    fn.argtypes = [ctypes.POINTER(tm._Pair), ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int,
+                   ctypes.POINTER(tm._Pair), ctypes.c_void_p]
+    fn.restype = ctypes.c_int
+    z = tm._Pair(1 << 24, 1, 64, 128, tm.BF16)           # aligned, never dereferenced
+    bad_outs = {
+        b"out shape differs": tm._Pair(1 << 32, 1, 32, 128, tm.F32),
+        b"fp32 path writes fp32 out": None,
+        b"out overlaps z": tm._Pair((1 << 24) + 4096, 1, 64, 128, tm.F32),
+        b"not 16-byte aligned": tm._Pair((1 << 32) + 8, 1, 64, 128, tm.F32),
+        b"out: NULL tensor": tm._Pair(0, 1, 64, 128, tm.F32),
+    }
+    for entry in (lib.tri_mul_forward, fn):
+        for msg, out in bad_outs.items():
+            zz = z
+            if out is None:                               # an fp32 z with a bf16 out
+                zz = tm._Pair(1 << 24, 1, 64, 128, tm.F32)
+                out = tm._Pair(1 << 32, 1, 64, 128, tm.BF16)
+            st = entry(ctypes.byref(zz), None, None, 0, ctypes.byref(out), None)
+            assert st in (1, 7) and msg in lib.tri_mul_last_error(), (entry, msg, lib.tri_mul_last_error())
+        good = tm._Pair(1 << 32, 1, 64, 128, tm.F32)
+        assert entry(ctypes.byref(z), None, None, 0, ctypes.byref(good), None) == 1
+        assert b"layer is NULL" in lib.tri_mul_last_error()

@@ -1,11 +1,11 @@
 """Skipping of wholly masked tiles (needs a B200).
 
 With mask skipping switched on, tri_mul_forward with a mask finds the mask's extents and
-leaves out tiles that are masked in full and the k-range beyond them; the stage entry points
-(project, contract, output_gate) called one by one skip nothing. Every product left out is an exact zero, so the two must
-agree bitwise, for masks of any pattern (here: a valid block [0, R) x [0, C) with R != C and
-random holes inside it, the second batch element with the block transposed), and both must
-match the oracle.
+leaves out tiles that are masked in full and the k-range beyond them; with it off nothing is
+left out. Every product left out is an exact zero (and adds nothing to the channel sums the
+offsets of the stored x come from), so the two must agree bitwise, for masks of any pattern
+(here: a valid block [0, R) x [0, C) with R != C and random holes inside it, the second batch
+element with the block transposed), and both must match the oracle.
 """
 import numpy as np
 import pytest
@@ -34,21 +34,19 @@ def _holey_mask(N, R, C, seed):
     (128, 60, 90, 384, True),       # c_z = 384 kernels
     (512, 493, 200, 128, False),    # headline size, columns cut short
 ])
-def test_forward_with_extents_matches_stages_bitwise(N, R, C, c_z, check_oracle):
+def test_forward_with_extents_matches_dense_forward_bitwise(N, R, C, c_z, check_oracle):
     inp = ti.generate(2, N, c_z, 128, dtype="bf16", seed=N + R + C, mask=("all",), biases=True)
     inp.mask = _holey_mask(N, R, C, seed=R * C)
     z, m, w = upload(inp)
     layer = tm.TriMulLayer(w, eps=inp.eps)
+    dense = tm.TriMulLayer(w, eps=inp.eps)
     layer.set_mask_skipping(True)
-    scale = tm.contract_scale(N)
     for d in ("outgoing", "incoming"):
         full = layer.forward(z, m, d)
-        a, b = layer.project(z, m)
-        x = tm.contract(a, b, d, x_scale=scale)
-        staged = layer.output_gate(z, x, m, x_scale=scale)
+        ref_dense = dense.forward(z, m, d)
         torch.cuda.synchronize()
         tm.check_device_status()
-        assert torch.equal(full, staged), d
+        assert torch.equal(full, ref_dense), d
         got = full.cpu().numpy()
         assert not np.any(got[inp.mask == 0]), "masked pairs must be exactly 0"
         if check_oracle:

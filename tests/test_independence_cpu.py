@@ -40,7 +40,9 @@ def test_oracle_includes_nothing_of_the_package():
             assert name not in text, f"{os.path.relpath(path, ROOT)} refers to {name}"
 
 
-ALLOWED = {"bench.py": {"cpu_oracle_layer_ms", "run_reference"}, "__graft_entry__.py": {"build", "smoke"}}
+# bench.py: the cpu_baseline leg (cpu_oracle_layer_ms, and cpu_oracle_probe run in a child process
+# per thread count) and the reference arm
+ALLOWED = {"bench.py": {"cpu_oracle_layer_ms", "cpu_oracle_probe", "run_reference"}, "__graft_entry__.py": {"build", "smoke"}}
 
 
 @pytest.mark.parametrize("name", sorted(ALLOWED))
