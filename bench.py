@@ -626,11 +626,16 @@ def run_ours(args):
                 other = Workload(tm, name, 0, dev, out_dt, args.skip_masked)
                 for s in range(max(3, args.warmup)):
                     other.step(s)
+                w_clocks = ClockSampler(smi_index)
+                w_clocks.start()
+                time.sleep(0.4)
                 w_el, _ = time_steps(other, args.steps, 0, sync_all)
                 w_iel, w_kms = time_steps(other, args.steps, args.steps, sync_all, instrumented=True)
+                w_clock_info = w_clocks.stop()
                 tm.check_device_status()
                 n_layers = args.steps * len(other.dirs)
                 workloads[name] = workload_summary(other, w_el / n_layers, w_kms, w_iel / n_layers, peaks)
+                workloads[name]["clocks"] = w_clock_info
                 del other
                 torch.cuda.empty_cache()
             except Exception as exc:        # the headline line must not depend on this leg

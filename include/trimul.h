@@ -119,9 +119,8 @@ void tri_mul_layer_destroy(trimul_layer_t *layer);
 /* Bytes of workspace tri_mul_forward needs for B x N x N with z of type `dtype`:
  * a, b and x, each [B, c_h, N, N] of the intermediate type (F16 for a BF16 z,
  * F32 for an F32 z), 256-byte aligned, then, each 256-byte aligned, the mask extents
- * (2 int32 per batch element), the offsets of the stored x (c_h fp32 per batch
- * element) and their share of the output projection (c_z fp32 per batch element).
- * Returns 0 for an invalid layer or size. */
+ * (2 int32 per batch element) and the offset of the stored x (c_h fp32 per batch
+ * element). Returns 0 for an invalid layer or size. */
 size_t tri_mul_workspace_bytes(const trimul_layer_t *layer, int64_t B, int64_t N,
                                trimul_dtype_t dtype);
 
@@ -134,13 +133,14 @@ trimul_status_t tri_mul_layer_bind_workspace(trimul_layer_t *layer, void *worksp
 
 /* One triangle multiplicative update (one direction). Returns the update only;
  * the residual add z += update is the caller's (or tri_mul_forward_residual's).
- * On the tensor-core path four kernels run: K1 (projection), a small pass that turns
- * K1's per-channel sums of a and b into per-(batch, channel) offsets o, K2 (contraction,
- * storing x - o) and K3 (output gate, adding o back exactly). o = Sa Sb / P^1.5 (Sa, Sb the
- * channel sums over the batch element, P its unmasked pairs) estimates the common mode of x
- * that a large mean of a and b produces; storing x - o keeps the F16 rounding of x small
- * next to the spread the output LayerNorm divides by. Any o gives the same function; the
- * sums are integers (fixed point), so results do not depend on the order tiles finish in.
+ * On the tensor-core path four kernels run: K1 (projection), a small pass that turns K1's
+ * per-channel sums of a and b into one offset o per batch element, K2 (contraction, storing
+ * x - o) and K3 (output gate). o = (1/c_h) sum_c Sa_c Sb_c / P^1.5 (Sa_c, Sb_c the channel sums
+ * over the batch element, P its unmasked pairs) estimates the common mode of x that a large
+ * mean of a and b produces; storing x - o keeps the F16 rounding of x small next to the
+ * spread the output LayerNorm divides by, and the LayerNorm, which ignores a constant added
+ * to every channel of a pair, needs no correction. The sums are integers (fixed point), so
+ * results do not depend on the order tiles finish in.
  * With mask skipping switched on (tri_mul_layer_set_mask_skipping), on the tensor-core
  * path with a mask a first pass finds the mask's extents (the last row and column holding a
  * nonzero entry, per batch element) and the kernels leave out tiles that are masked in full
@@ -254,6 +254,56 @@ trimul_status_t tri_mul_pair_update_graph_create(const trimul_pair_t *z, const v
 trimul_status_t tri_mul_graph_launch(const trimul_graph_t *graph, void *stream);
 /* Free the graph. NULL is ignored. */
 void tri_mul_graph_destroy(trimul_graph_t *graph);
+
+/* ---- Row-sharded update ("big mode") ----------------------------------------------------
+ * One update split by rows over G shards (GPUs), as the commentary on the AI-refactored
+ * structure-prediction code describes for complexes too large for one GPU: the pair tensor
+ * is sharded across the GPUs of a node by rows, large intermediates chunked. Shard g owns
+ * rows [row0[g], row0[g+1]) of z, of the mask and of the update, and of the a and b planes.
+ *   outgoing: x_ij = sum_k a_ik b_jk needs this shard's a rows and b rows j from every shard;
+ *   incoming: x_ij = sum_k a_ki b_kj needs a and b rows k from every shard (a's columns i of
+ *             this shard's rows).
+ * Phase 1 (tri_mul_shard_project) makes a and b of the shard's rows; between the phases the
+ * caller makes every shard's a (incoming only) and b readable by the others (an all-gather
+ * into local buffers, or peer mappings of the other GPUs' buffers: the contraction reads
+ * them through TMA tensor maps, never with a multicast load); phase 2 (tri_mul_shard_finish)
+ * contracts and gates the shard's rows. Both phases of one update use the same layer handle
+ * and its bound workspace (tri_mul_shard_workspace_bytes: this shard's x and its offset),
+ * in order on one stream; phase 1 computes the offset of the stored x from the shard's own
+ * channel sums (see tri_mul_forward), so shards need not exchange anything else.
+ * Tensor-core path only: bf16 z, (c_z, c_h) = (128, 128) or (384, 128); N a multiple of 128
+ * in [128, 16384]; every shard a whole number of 128-row blocks; 1 <= G <= 8. Results equal
+ * the unsharded update up to the offset's rounding (a per-shard offset instead of one per
+ * batch element). */
+
+/* Rows [row0, row0 + R) of a [B, N, N, C] pair tensor, stored contiguously as [B, R, N, C]. */
+typedef struct {
+    void *data;
+    int64_t B, R, N, C, row0;
+    trimul_dtype_t dtype;
+} trimul_rows_t;
+
+/* Workspace bytes one shard of R rows needs (bound with tri_mul_layer_bind_workspace):
+ * x [B, c_h, R, N] F16 and the offset (c_h fp32 per batch element), each 256-byte aligned.
+ * Returns 0 for an invalid layer or size. */
+size_t tri_mul_shard_workspace_bytes(const trimul_layer_t *layer, int64_t B, int64_t R, int64_t N);
+
+/* Phase 1: K1 on the shard's rows and the offsets pass. z and mask hold the shard's rows
+ * (mask [B, R, N] in z's dtype, or NULL); a_out and b_out receive [B, c_h, R, N] F16 (caller
+ * owned, not overlapping z, each other or the workspace). */
+trimul_status_t tri_mul_shard_project(const trimul_rows_t *z, const void *mask, const trimul_layer_t *layer,
+                                      void *a_out, void *b_out, void *stream);
+
+/* Phase 2: the contraction for the shard's rows, then K3 on them, writing out (the shard's
+ * rows of the update, F32 or BF16, z's shape, not overlapping z or the workspace).
+ * shard_row0[0..G] are the shard boundaries (0 = shard_row0[0] < ... < shard_row0[G] = N, each a
+ * multiple of 128); z's rows must be one of the shards. a_shards[g], b_shards[g]: shard g's
+ * phase-1 a and b ([B, c_h, R_g, N] F16, device pointers readable from this GPU); a_shards is read
+ * only for this shard (outgoing) or all shards (incoming). */
+trimul_status_t tri_mul_shard_finish(const trimul_rows_t *z, const void *mask, const trimul_layer_t *layer,
+                                     trimul_direction_t direction, int G, const int64_t *shard_row0,
+                                     const void *const *a_shards, const void *const *b_shards,
+                                     trimul_rows_t *out, void *stream);
 
 /* Mask skipping (off by default): when on, tri_mul_forward with a mask on the tensor-core
  * path first finds the mask's extents {R_b, C_b} per batch element (a memset and one small

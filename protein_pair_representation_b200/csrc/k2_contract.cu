@@ -62,8 +62,23 @@ __device__ __forceinline__ int k2_tile_chunks(const K2Args &p, int bc, int m0, i
     return nk < p.k_chunks ? nk : p.k_chunks;
 }
 
-__global__ void __launch_bounds__(k2::THREADS, 1) k2_contract_kernel(const __grid_constant__ K2Args p) {
+// The shard holding global row r (row0 ascending, row0[G] = N; rows past N: the last shard,
+// whose box then reads past its rows and is zero-filled).
+__device__ __forceinline__ int shard_of(const K2ShardArgs &s, int r) {
+    int g = 0;
+    while (g + 1 < s.G && r >= s.row0[g + 1]) ++g;
+    return g;
+}
+
+__device__ __forceinline__ const K2Args &base_args(const K2Args &a) { return a; }
+__device__ __forceinline__ const K2Args &base_args(const K2ShardArgs &a) { return a.base; }
+
+// SHARD: the operands of a row-sharded update come from per-shard maps (K2ShardArgs); the
+// other instance carries none of that code.
+template <bool SHARD, typename Args>
+__global__ void __launch_bounds__(k2::THREADS, 1) k2_contract_kernel(const __grid_constant__ Args pa) {
     using namespace k2;
+    const K2Args &p = base_args(pa);
     extern __shared__ uint8_t smem_raw[];
     uint8_t *base = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint8_t *stages = base;
@@ -91,6 +106,12 @@ __global__ void __launch_bounds__(k2::THREADS, 1) k2_contract_kernel(const __gri
         tma_prefetch_desc(&p.tm_a);
         tma_prefetch_desc(&p.tm_b);
         tma_prefetch_desc(&p.tm_x);
+        if constexpr (SHARD) {
+            for (int g = 0; g < pa.G; ++g) {
+                tma_prefetch_desc(&pa.tm_sb[g]);
+                if (p.incoming) tma_prefetch_desc(&pa.tm_sa[g]);
+            }
+        }
     }
     if (warp == MMA_WARP) {
         tmem_alloc(&s.tmem_base, TMEM_COLS);
@@ -123,7 +144,26 @@ __global__ void __launch_bounds__(k2::THREADS, 1) k2_contract_kernel(const __gri
                     uint8_t *sb = sa + A_BYTES;
                     mbar_arrive_expect_tx(&s.full[stage], STAGE_BYTES);
                     const int k0 = kc * BK;
-                    if (!p.incoming) {
+                    if constexpr (SHARD) {
+                        if (!p.incoming) {
+                            tma_load_3d(sa, &p.tm_a, &s.full[stage], k0, m0, bc);
+#pragma unroll
+                            for (int h = 0; h < BN / 128; ++h) {    // b rows j from the shard holding them
+                                const int j = n0 + 128 * h;
+                                const int g = shard_of(pa, j);
+                                tma_load_3d(sb + h * 16384, &pa.tm_sb[g], &s.full[stage], k0, j - pa.row0[g], bc);
+                            }
+                        } else {
+                            const int g = shard_of(pa, k0);         // a 64-row k chunk lies in one shard
+                            const int kl = k0 - pa.row0[g];
+#pragma unroll
+                            for (int h = 0; h < BM / 64; ++h)
+                                tma_load_3d(sa + h * 8192, &pa.tm_sa[g], &s.full[stage], pa.i0 + m0 + 64 * h, kl, bc);
+#pragma unroll
+                            for (int h = 0; h < BN / 64; ++h)
+                                tma_load_3d(sb + h * 8192, &pa.tm_sb[g], &s.full[stage], n0 + 64 * h, kl, bc);
+                        }
+                    } else if (!p.incoming) {
                         tma_load_3d(sa, &p.tm_a, &s.full[stage], k0, m0, bc);
                         tma_load_3d(sb, &p.tm_b, &s.full[stage], k0, n0, bc);
                     } else {
@@ -267,17 +307,26 @@ __global__ void __launch_bounds__(k2::THREADS, 1) k2_contract_kernel(const __gri
 
 size_t k2_smem_bytes() { return k2::SMEM_BYTES; }
 
-cudaError_t k2_launch(const K2Args &args, int grid, cudaStream_t stream) {
+template <bool SHARD, typename Args>
+static cudaError_t k2_launch_t(const Args &args, int grid, cudaStream_t stream) {
     static int configured_device = -1;
     int dev = 0;
     cudaGetDevice(&dev);
     if (configured_device != dev) {
-        cudaError_t e = cudaFuncSetAttribute(k2_contract_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+        cudaError_t e = cudaFuncSetAttribute(k2_contract_kernel<SHARD, Args>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                              (int)k2::SMEM_BYTES);
         if (e != cudaSuccess) return e;
         configured_device = dev;
     }
-    return launch_pdl(k2_contract_kernel, grid, k2::THREADS, k2::SMEM_BYTES, stream, args);
+    return launch_pdl(k2_contract_kernel<SHARD, Args>, grid, k2::THREADS, k2::SMEM_BYTES, stream, args);
+}
+
+cudaError_t k2_launch(const K2Args &args, int grid, cudaStream_t stream) {
+    return k2_launch_t<false>(args, grid, stream);
+}
+
+cudaError_t k2_shard_launch(const K2ShardArgs &args, int grid, cudaStream_t stream) {
+    return k2_launch_t<true>(args, grid, stream);
 }
 
 }  // namespace trimul

@@ -8,8 +8,8 @@
 // section "Triangle multiplication on SM90": K3 with both LayerNorms folded into its
 // weights). Both norms are folded as in K1:
 //   x . W_o' -> rstd_x (acc1 - mean_x sum W_o') + shift_o, with W_o' = W_o * gamma_out
-// where x is held as stored + q[b][c] (the contraction stores x_scale x less a per-channel
-// offset q): the statistics add q per channel, and acc1 gains Q[b][n] = sum_c q[b][c] W_o'[n][c]
+// The LayerNorm over c_h ignores a constant added to every channel of a pair, so x may be
+// stored less any per-pair constant (the forward stores it less a per-batch-element offset).
 //   z . W_g' -> rstd_z (acc2 - mean_z sum W_g') + shift_g, with W_g' = W_g * gamma_in
 //
 // Tile: 128 consecutive pairs (one TMEM lane each) times 128 output channels. x arrives
@@ -256,10 +256,6 @@ __global__ void __launch_bounds__(576, 1) k3_output_kernel(const __grid_constant
             float2 a1[4], a2[4], xnsh[4];
 #pragma unroll
             for (int k = 0; k < 4; ++k) a1[k] = a2[k] = xnsh[k] = make_float2(0.f, 0.f);
-            // the stored x is x_scale x - q[b][c]: the statistics are taken of u = stored + q, this
-            // thread reading channels xg + 8 j of each chunk (q of channel 0 for the shift)
-            const float *qb = p.xoff + (size_t)b * p.xoff_stride;
-            const float q0 = xrole ? __ldg(qb) : 0.f;
             for (int c = 0; c < C::CPT; ++c) {
                 const bool arrived = mbar_wait(&s.full[stage], phase, abort_flag, kErrTimeoutEpilogue);
                 if (xrole ? !group_all(arrived, 1, 128) : !__all_sync(0xffffffffu, arrived)) { ok = false; break; }
@@ -274,24 +270,19 @@ __global__ void __launch_bounds__(576, 1) k3_output_kernel(const __grid_constant
 #pragma unroll
                         for (int k = 0; k < 4; ++k) {
                             const float2 v = __half22float2(*reinterpret_cast<const __half2 *>(&h0[k]));
-                            xnsh[k] = make_float2(-v.x - q0, -v.y - q0);
+                            xnsh[k] = make_float2(-v.x, -v.y);
                         }
                         // this thread's own pair (`row`) shift, for the final mean
                         sh = __half2float(__ushort_as_half(*reinterpret_cast<const uint16_t *>(
-                            ch + mblk * 8192 + sw128_offset(0, r64 >> 3) + (r64 & 7) * 2))) + q0;
+                            ch + mblk * 8192 + sw128_offset(0, r64 >> 3) + (r64 & 7) * 2)));
                     }
-                    float qc[8];
-#pragma unroll
-                    for (int j = 0; j < 8; ++j) qc[j] = __ldg(qb + c * 64 + xg + 8 * j);
 #pragma unroll
                     for (int j = 0; j < 8; ++j) {
                         const uint4 w = *reinterpret_cast<const uint4 *>(xblk_off + sw128_offset(xg + 8 * j, xo & 7));
                         const uint32_t hw[4] = {w.x, w.y, w.z, w.w};
-                        const float q = qc[j];
 #pragma unroll
                         for (int k = 0; k < 4; ++k) {
-                            const float2 d = f2_add(__half22float2(*reinterpret_cast<const __half2 *>(&hw[k])),
-                                                    f2_add(xnsh[k], make_float2(q, q)));
+                            const float2 d = f2_add(__half22float2(*reinterpret_cast<const __half2 *>(&hw[k])), xnsh[k]);
                             a1[k] = f2_add(a1[k], d);
                             a2[k] = f2_fma(d, d, a2[k]);
                         }
@@ -350,7 +341,11 @@ __global__ void __launch_bounds__(576, 1) k3_output_kernel(const __grid_constant
             const float t1 = s1.x + s1.y, t2 = s2.x + s2.y;
             const float inv_n = 1.0f / (float)(xrole ? C::C_H : CZ);
             const float dm = t1 * inv_n;
-            const float rs = rsqrtf(fmaxf(t2 * inv_n - dm * dm, 0.f) + (xrole ? p.eps_x : p.eps));
+            float rs = rsqrtf(fmaxf(t2 * inv_n - dm * dm, 0.f) + (xrole ? p.eps_x : p.eps));
+            // every channel of this pair's x holds the same value (the shifted square sum is
+            // exactly 0): the normalized vector is exactly 0 whatever the scale, so the x-GEMM's
+            // rounding residue in rstd (x . W_o' - mean sum W_o') must not be amplified by 1/sqrt(eps)
+            if (xrole && t2 == 0.f) rs = 0.f;
             // an inf or NaN anywhere in this pair's x makes the shifted square sum inf or NaN
             if (xrole && !(fabsf(t2) <= 3.0e38f)) atomicOr(&g_device_error, (unsigned int)kErrRange);
             const bool freed = mbar_wait(&s.sempty[sbuf], sphase ^ 1, abort_flag, kErrTimeoutEpilogue);
@@ -436,8 +431,6 @@ __global__ void __launch_bounds__(576, 1) k3_output_kernel(const __grid_constant
             tc_fence_after();
             const uint32_t t1 = tmem_base + abuf * 256 + ((uint32_t)(q * 32) << 16) + wg * 64;
             const uint32_t t2 = t1 + 128;
-            // the offsets' share of the x-GEMM for this batch element's output channels
-            const float *Qb = p.xoff_w + (size_t)b * p.xoffw_stride + n0 + wg * 64;
 #pragma unroll 1
             for (int sc = 0; sc < 64 / C::COLS_PER_STORE; ++sc) {
                 uint8_t *stg = staging + ((sc % C::NSTG) * 2 + wg) * C::STG_BYTES;
@@ -469,7 +462,6 @@ __global__ void __launch_bounds__(576, 1) k3_output_kernel(const __grid_constant
                         const float4 ho = *reinterpret_cast<const float4 *>(v_shift_o + col + e);
                         const float4 sg = *reinterpret_cast<const float4 *>(v_sum_g + col + e);
                         const float4 hg = *reinterpret_cast<const float4 *>(v_hshift_g + col + e);
-                        const float4 qw = __ldg(reinterpret_cast<const float4 *>(Qb + col + e));
 #pragma unroll
                         for (int k = 0; k < 2; ++k) {
                             // output channels e + 2k and e + 2k + 1 of this pair, packed
@@ -477,9 +469,8 @@ __global__ void __launch_bounds__(576, 1) k3_output_kernel(const __grid_constant
                             const float2 ho2 = k == 0 ? make_float2(ho.x, ho.y) : make_float2(ho.z, ho.w);
                             const float2 sg2 = k == 0 ? make_float2(sg.x, sg.y) : make_float2(sg.z, sg.w);
                             const float2 hg2 = k == 0 ? make_float2(hg.x, hg.y) : make_float2(hg.z, hg.w);
-                            const float2 qw2 = k == 0 ? make_float2(qw.x, qw.y) : make_float2(qw.z, qw.w);
                             const int i = e + 2 * k;
-                            const float2 ov = f2_fma(rx, f2_fma(nmx, so2, f2_add(make_float2(o[i], o[i + 1]), qw2)), ho2);
+                            const float2 ov = f2_fma(rx, f2_fma(nmx, so2, make_float2(o[i], o[i + 1])), ho2);
                             // half the gate argument; mask * sigmoid(2 y) = (mask / 2) tanh(y) + mask / 2
                             const float2 gh = f2_fma(hrz, f2_fma(nmz, sg2, make_float2(g[i], g[i + 1])), hg2);
                             const float2 gm = f2_fma(hm, make_float2(tanh_approx(gh.x), tanh_approx(gh.y)), hm);

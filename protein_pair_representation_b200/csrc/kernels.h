@@ -45,9 +45,26 @@ struct K2Args {
                            // (outgoing) or k < R_b (incoming); output tiles at rows >= R_b or
                            // columns >= C_b are not written (the output kernel never reads them)
     int C;                 // channels per batch element (bc / C = batch element)
-    const float *xoff;     // per (batch, channel) offset q subtracted after the scaling, before the
-                           // rounding: x = round(x_scale * sum - xoff[bc * xoff_stride])
+    const float *xoff;     // offset q subtracted after the scaling, before the rounding:
+                           // x = round(x_scale * sum - xoff[bc * xoff_stride])
     int xoff_stride;       // 1, or 0 with xoff pointing at a single zero
+};
+
+// The contraction for one shard of a row-sharded update. The N x N planes of a and b are
+// split by rows over G shards, shard g holding rows [row0[g], row0[g + 1]) of every plane
+// ([B*c_h][rows][N], its own buffer: a local copy or another GPU's memory); this shard's
+// output rows are x[., i0 + i, .] for i < R (base.m_tiles covers R, base.tm_x is [B*c_h][R][N]).
+//   outgoing: x_ij = sum_k a_ik b_jk   A = this shard's a rows (base.tm_a), B rows j from their shards
+//   incoming: x_ij = sum_k a_ki b_kj   A columns i and B rows k, both from the shard holding row k
+// Every shard boundary is a multiple of 128 rows, so a 128-row box never spans two shards.
+constexpr int kMaxShards = 8;
+struct K2ShardArgs {
+    K2Args base;
+    CUtensorMap tm_sa[kMaxShards];   // incoming: shard g's a, {N, R_g, B*c_h}, box {64, 64, 1}
+    CUtensorMap tm_sb[kMaxShards];   // shard g's b: outgoing box {64, 128, 1}, incoming box {64, 64, 1}
+    int row0[kMaxShards + 1];
+    int G;
+    int i0;                          // first global row of this shard's output
 };
 
 struct K3Args {
@@ -66,12 +83,6 @@ struct K3Args {
     const uint16_t *zres;  // residual: z (bf16, [B][N*N][c_z]) added to the output; null = none
     const int *ext;        // mask extents (as K1Args); ignored with a residual (masked pairs then copy z)
     uint64_t rowdiv;
-    // The stored x is x_scale * x - q[b][c]: the LayerNorm statistics add q back per channel
-    // (q = xoff + b * xoff_stride, c_h entries) and the x-GEMM adds Q[b][n] = sum_c q[b][c] W_o'[n][c]
-    // (xoff_w + b * xoffw_stride, c_z entries). Strides 0 with pointers at zeros: no offsets.
-    const float *xoff;
-    const float *xoff_w;
-    int xoff_stride, xoffw_stride;
 };
 
 // Launch with programmatic stream serialization: the kernel may begin while the previous
@@ -104,6 +115,7 @@ int k1_tile_pairs(int c_z);        // pairs per K1 tile (64 at c_z = 128, 128 at
 
 size_t k2_smem_bytes();
 cudaError_t k2_launch(const K2Args &args, int grid, cudaStream_t stream);
+cudaError_t k2_shard_launch(const K2ShardArgs &args, int grid, cudaStream_t stream);
 
 // The fused pair transition (c = 128, hidden 256): out = z + m * (relu(z W1^T + b1) W2^T + b2).
 struct PtArgs {
@@ -136,12 +148,11 @@ size_t k3_smem_bytes(int c_z, bool out_f32);
 int k3_groups(int c_z);
 cudaError_t k3_launch(int c_z, bool out_f32, const K3Args &args, int grid, cudaStream_t stream);  // residual iff args.zres
 
-// The per-(batch, channel) offsets of the stored x from K1's sums: q[b][c] = x_scale * Sa Sb / P^1.5
-// (Sa, Sb the channel sums of a and b over batch element b, P its unmasked pairs; 0 when P = 0),
-// Q[b][n] = sum_c q[b][c] wo[n][c] (wo the folded f16 W_o' [c_z][c_h]); the sums are zeroed for the
-// next forward. One CTA per batch element.
-cudaError_t xoffsets_launch(unsigned long long *acc, int B, int c_h, int c_z, float x_scale, const uint16_t *wo,
-                            float *q, float *Q, cudaStream_t stream);
+// The offset of the stored x of each batch element from K1's sums, written to all c_h entries
+// q[b][c]: x_scale * (1 / c_h) sum_c Sa_c Sb_c / P^1.5, rounded to an fp16 value (Sa_c, Sb_c the
+// channel sums of a and b over batch element b, P its unmasked pairs; 0 when P = 0); the sums are
+// zeroed for the next forward. One CTA per batch element.
+cudaError_t xoffsets_launch(unsigned long long *acc, int B, int c_h, float x_scale, float *q, cudaStream_t stream);
 
 // ---- weight folding (layer creation) -----------------------------------------------
 

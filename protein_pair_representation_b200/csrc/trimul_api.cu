@@ -39,7 +39,6 @@ struct trimul_layer {
     // K1's per-(batch, channel) sums of a and b and unmasked-pair counts, [65535 / c_h + 1][2 c_h + 1]
     // (zero between forwards: the offsets kernel clears what it has read)
     unsigned long long *acc;
-    float *zeros;                // kZeros zero floats: the offsets of the stand-alone stages
     // fp32 path
     F32Weights f32;
     // workspace
@@ -157,9 +156,6 @@ static trimul_status_t make_map(CUtensorMap *m, CUtensorMapDataType dt, int rank
         if (_s != TRIMUL_OK) return _s;           \
     } while (0)
 
-// Zero floats kept in each layer, enough for any offset vector a kernel reads with stride 0.
-static constexpr int kZeros = 512;
-
 // Batch elements the layer's channel sums have room for: B * c_h <= 65535 is enforced.
 static int acc_batches(int c_h) { return 65535 / c_h + 1; }
 
@@ -243,7 +239,7 @@ extern "C" trimul_status_t tri_mul_layer_create(const trimul_weights_desc_t *w, 
     // carve one allocation
     size_t off = 0;
     auto take = [&](size_t bytes) { size_t o = off; off = (off + bytes + 255) & ~size_t(255); return o; };
-    size_t o_k1w = 0, o_k1v = 0, o_k3o = 0, o_k3g = 0, o_k3v = 0, o_acc = 0, o_zero = 0, acc_bytes = 0;
+    size_t o_k1w = 0, o_k1v = 0, o_k3o = 0, o_k3g = 0, o_k3v = 0, o_acc = 0, acc_bytes = 0;
     if (L->has_bf16) {
         o_k1w = take((size_t)4 * ch * cz * 2);
         o_k1v = take((size_t)2 * ch * sizeof(float4));
@@ -252,7 +248,6 @@ extern "C" trimul_status_t tri_mul_layer_create(const trimul_weights_desc_t *w, 
         o_k3v = take((size_t)cz * sizeof(float4));
         acc_bytes = (size_t)acc_batches(ch) * (2 * ch + 1) * sizeof(unsigned long long);
         o_acc = take(acc_bytes);
-        o_zero = take(kZeros * sizeof(float));
     }
     const size_t o_lig = take(cz * 4), o_lib = take(cz * 4);
     const size_t o_wag = take((size_t)ch * cz * 4), o_wap = take((size_t)ch * cz * 4);
@@ -300,8 +295,7 @@ extern "C" trimul_status_t tri_mul_layer_create(const trimul_weights_desc_t *w, 
         L->k3_wg = reinterpret_cast<uint16_t *>(m + o_k3g);
         L->k3_vec = reinterpret_cast<float4 *>(m + o_k3v);
         L->acc = reinterpret_cast<unsigned long long *>(m + o_acc);
-        L->zeros = reinterpret_cast<float *>(m + o_zero);
-        ce = cudaMemsetAsync(m + o_acc, 0, (o_zero - o_acc) + kZeros * sizeof(float), st);
+        ce = cudaMemsetAsync(m + o_acc, 0, acc_bytes, st);
         const int ncol = k1_ncol(cz);
         const void *srcs[2][2] = {{w->w_ag, w->w_ap}, {w->w_bg, w->w_bp}};
         const void *biases[2][2] = {{w->b_ag, w->b_ap}, {w->b_bg, w->b_bp}};
@@ -369,14 +363,13 @@ static size_t ws_plane_bytes(int64_t B, int64_t N, int c_h, trimul_dtype_t dt) {
     return align256((size_t)B * c_h * N * N * dtype_size(dt));
 }
 
-// After the three planes: the mask extents {R_b, C_b} (int32), then the offsets q [B][c_h] and
-// their projections Q [B][c_z] (fp32) of the stored x.
+// After the three planes: the mask extents {R_b, C_b} (int32), then the offset of the stored x
+// (fp32, one value per batch element repeated over its c_h channel planes).
 static size_t ws_ext_bytes(int64_t B) { return align256((size_t)B * 2 * sizeof(int)); }
 static size_t ws_q_bytes(int64_t B, int c_h) { return align256((size_t)B * c_h * sizeof(float)); }
-static size_t ws_Q_bytes(int64_t B, int c_z) { return align256((size_t)B * c_z * sizeof(float)); }
 
 static size_t ws_total_bytes(const trimul_layer_t *L, int64_t B, int64_t N, trimul_dtype_t dt) {
-    return 3 * ws_plane_bytes(B, N, L->c_h, dt) + ws_ext_bytes(B) + ws_q_bytes(B, L->c_h) + ws_Q_bytes(B, L->c_z);
+    return 3 * ws_plane_bytes(B, N, L->c_h, dt) + ws_ext_bytes(B) + ws_q_bytes(B, L->c_h);
 }
 
 extern "C" size_t tri_mul_workspace_bytes(const trimul_layer_t *L, int64_t B, int64_t N, trimul_dtype_t dt) {
@@ -423,11 +416,12 @@ static int grid_for(int sms, long long work_units, int multiple) {
     return (int)g;
 }
 
+// K1 on B x R x N pairs (R rows of N: the whole pair tensor, R = N, or one shard's rows).
 static trimul_status_t run_project_bf16(const trimul_layer_t *L, const void *z, const void *mask, void *a, void *b,
-                                        int B, int N, cudaStream_t st, const int *ext, unsigned long long *acc) {
+                                        int B, int R, int N, cudaStream_t st, const int *ext, unsigned long long *acc) {
     DeviceInfo d;
     TRY(require_sm100(&d));
-    const uint64_t NN = (uint64_t)N * N;
+    const uint64_t NN = (uint64_t)R * N;
     const int cz = L->c_z, ch = L->c_h;
     K1Args p{};
     const int tp = k1_tile_pairs(cz);
@@ -518,12 +512,13 @@ static trimul_status_t run_contract_tc(const void *a, const void *b, void *x, in
     return TRIMUL_OK;
 }
 
+// K3 on B x R x N pairs (as run_project_bf16).
 static trimul_status_t run_output_bf16(const trimul_layer_t *L, const void *z, const void *mask, const void *x,
-                                       float x_scale, void *out, bool out_f32, bool residual, int B, int N,
-                                       cudaStream_t st, const int *ext, const float *q, const float *Q) {
+                                       float x_scale, void *out, bool out_f32, bool residual, int B, int R, int N,
+                                       cudaStream_t st, const int *ext) {
     DeviceInfo d;
     TRY(require_sm100(&d));
-    const uint64_t NN = (uint64_t)N * N;
+    const uint64_t NN = (uint64_t)R * N;
     const int cz = L->c_z, ch = L->c_h;
     K3Args p{};
     {
@@ -571,10 +566,6 @@ static trimul_status_t run_output_bf16(const trimul_layer_t *L, const void *z, c
     p.zres = residual ? reinterpret_cast<const uint16_t *>(z) : nullptr;
     p.ext = residual ? nullptr : ext;        // with a residual a masked pair copies z: nothing is skipped
     p.rowdiv = host_rowdiv((uint64_t)N / 8);
-    p.xoff = q ? q : L->zeros;
-    p.xoff_stride = q ? ch : 0;
-    p.xoff_w = Q ? Q : L->zeros;
-    p.xoffw_stride = Q ? cz : 0;
     const int G = k3_groups(cz);
     const int grid = grid_for(d.sms, (long long)G * B * p.tiles_per_batch, G);
     TRY_CUDA(k3_launch(cz, out_f32, p, grid, st), "K3 launch");
@@ -594,7 +585,7 @@ static trimul_status_t project_impl(const trimul_pair_t *z, const void *mask, co
         return fail(TRIMUL_ERR_INVALID_ARG, "a_out, b_out and z overlap");
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
     if (z->dtype == TRIMUL_BF16)
-        return run_project_bf16(L, z->data, mask, a_out, b_out, (int)z->B, (int)z->N, st, ext, acc);
+        return run_project_bf16(L, z->data, mask, a_out, b_out, (int)z->B, (int)z->N, (int)z->N, st, ext, acc);
     TRY_CUDA(f32_project_launch(reinterpret_cast<const float *>(z->data), reinterpret_cast<const float *>(mask), L->f32,
                                 L->c_z, L->c_h, (int)z->B, (int)z->N, L->eps, reinterpret_cast<float *>(a_out),
                                 reinterpret_cast<float *>(b_out), st),
@@ -662,7 +653,7 @@ extern "C" trimul_status_t tri_mul_contract(const void *a, const void *b, void *
 
 static trimul_status_t output_gate_impl(const trimul_pair_t *z, const void *mask, const void *x, float x_scale,
                                         const trimul_layer_t *L, trimul_pair_t *out, bool residual, const int *ext,
-                                        const float *q, const float *Q, void *stream) {
+                                        void *stream) {
     TRY(check_sizes(z));
     TRY(check_out(z, out));
     TRY(check_problem(z, mask, L));
@@ -674,7 +665,7 @@ static trimul_status_t output_gate_impl(const trimul_pair_t *z, const void *mask
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
     if (z->dtype == TRIMUL_BF16)
         return run_output_bf16(L, z->data, mask, x, x_scale, out->data, out->dtype == TRIMUL_F32, residual, (int)z->B,
-                               (int)z->N, st, ext, q, Q);
+                               (int)z->N, (int)z->N, st, ext);
     TRY_CUDA(f32_output_launch(reinterpret_cast<const float *>(z->data), reinterpret_cast<const float *>(mask),
                                reinterpret_cast<const float *>(x), L->f32, L->c_z, L->c_h, (int)z->B, (int)z->N, L->eps,
                                L->eps * x_scale * x_scale, residual, reinterpret_cast<float *>(out->data), st),
@@ -684,7 +675,7 @@ static trimul_status_t output_gate_impl(const trimul_pair_t *z, const void *mask
 
 extern "C" trimul_status_t tri_mul_output_gate(const trimul_pair_t *z, const void *mask, const void *x, float x_scale,
                                                const trimul_layer_t *L, trimul_pair_t *out, void *stream) {
-    return output_gate_impl(z, mask, x, x_scale, L, out, false, nullptr, nullptr, nullptr, stream);
+    return output_gate_impl(z, mask, x, x_scale, L, out, false, nullptr, stream);
 }
 
 namespace trimul {
@@ -718,7 +709,6 @@ trimul_status_t forward_buffers(const trimul_pair_t *z, const void *mask, const 
     // leave out wholly masked tiles
     int *ext = (tc && mask && L->skip_masked) ? reinterpret_cast<int *>(aux) : nullptr;
     float *q = reinterpret_cast<float *>(aux + ws_ext_bytes(z->B));
-    float *Q = reinterpret_cast<float *>(aux + ws_ext_bytes(z->B) + ws_q_bytes(z->B, L->c_h));
     if (ext)
         TRY_CUDA(mask_extents_launch(reinterpret_cast<const uint16_t *>(mask), (int)z->B, (int)z->N,
                                      host_rowdiv((uint64_t)z->N / 8), ext, st),
@@ -727,12 +717,12 @@ trimul_status_t forward_buffers(const trimul_pair_t *z, const void *mask, const 
     if (timing) TRY_CUDA(cudaEventRecord(L->events[0], st), "event record");
     TRY(project_impl(z, mask, L, a, b, ext, tc ? L->acc : nullptr, stream));
     const float x_scale = tc ? tri_mul_contract_scale(z->N) : 1.0f;
-    // the offsets of the stored x from K1's channel sums (the fp32 path stores x as it is)
-    if (tc) TRY_CUDA(xoffsets_launch(L->acc, (int)z->B, L->c_h, L->c_z, x_scale, L->k3_wo, q, Q, st), "offsets launch");
+    // the offset of the stored x from K1's channel sums (the fp32 path stores x as it is)
+    if (tc) TRY_CUDA(xoffsets_launch(L->acc, (int)z->B, L->c_h, x_scale, q, st), "offsets launch");
     if (timing) TRY_CUDA(cudaEventRecord(L->events[1], st), "event record");
     TRY(contract_impl(a, b, x, z->B, L->c_h, z->N, tc ? TRIMUL_F16 : TRIMUL_F32, dir, x_scale, ext, tc ? q : nullptr, stream));
     if (timing) TRY_CUDA(cudaEventRecord(L->events[2], st), "event record");
-    TRY(output_gate_impl(z, mask, x, x_scale, L, out, residual, ext, tc ? q : nullptr, tc ? Q : nullptr, stream));
+    TRY(output_gate_impl(z, mask, x, x_scale, L, out, residual, ext, stream));
     if (timing) TRY_CUDA(cudaEventRecord(L->events[3], st), "event record");
     return TRIMUL_OK;
 }
@@ -752,6 +742,169 @@ extern "C" trimul_status_t tri_mul_forward(const trimul_pair_t *z, const void *m
 extern "C" trimul_status_t tri_mul_forward_residual(const trimul_pair_t *z, const void *mask, const trimul_layer_t *L,
                                                     trimul_direction_t dir, trimul_pair_t *out, void *stream) {
     return forward_impl(z, mask, L, dir, out, true, stream);
+}
+
+// ------------------------------------------------------------------ row-sharded update
+
+// A slab of rows: rows [row0, row0 + R) of a [B, N, N, C] pair tensor, stored [B, R, N, C].
+static trimul_status_t check_rows(const trimul_rows_t *t, const char *name) {
+    if (!t || !t->data) return fail(TRIMUL_ERR_INVALID_ARG, "%s: NULL tensor", name);
+    if (t->dtype != TRIMUL_BF16 && t->dtype != TRIMUL_F32) return fail(TRIMUL_ERR_INVALID_ARG, "%s: unknown dtype", name);
+    if (t->B < 1 || t->R < 1 || t->N < 1 || t->C < 1) return fail(TRIMUL_ERR_INVALID_ARG, "%s: sizes must be positive", name);
+    if (!aligned16(t->data)) return fail(TRIMUL_ERR_ALIGNMENT, "%s: pointer not 16-byte aligned", name);
+    return TRIMUL_OK;
+}
+
+static size_t rows_bytes(const trimul_rows_t *t) { return (size_t)t->B * t->R * t->N * t->C * dtype_size(t->dtype); }
+
+// The size rules of a shard (no layer needed): the tensor-core path, N a multiple of 128 in
+// [128, 16384], the rows a multiple of 128 starting at a multiple of 128 inside [0, N).
+static trimul_status_t check_shard_sizes(const trimul_rows_t *z) {
+    TRY(check_rows(z, "z"));
+    if (z->dtype != TRIMUL_BF16) return fail(TRIMUL_ERR_UNSUPPORTED_SHAPE, "a row-sharded update takes a bf16 z");
+    if (z->N < 128 || z->N % 128 != 0 || z->N > 16384)
+        return fail(TRIMUL_ERR_UNSUPPORTED_SHAPE, "N=%lld must be a multiple of 128 in [128, 16384]", (long long)z->N);
+    if (z->R % 128 != 0 || z->row0 % 128 != 0 || z->row0 < 0 || z->row0 + z->R > z->N)
+        return fail(TRIMUL_ERR_UNSUPPORTED_SHAPE, "shard rows [%lld, %lld) must be whole 128-row blocks inside [0, %lld)",
+                    (long long)z->row0, (long long)(z->row0 + z->R), (long long)z->N);
+    if ((long long)z->B * z->R * z->N / 128 > (1LL << 30))
+        return fail(TRIMUL_ERR_UNSUPPORTED_SHAPE, "problem too large: B * R * N / 128 must not exceed 2^30");
+    return TRIMUL_OK;
+}
+
+static trimul_status_t check_shard_layer(const trimul_rows_t *z, const void *mask, const trimul_layer_t *L) {
+    if (!L) return fail(TRIMUL_ERR_INVALID_ARG, "layer is NULL");
+    if (z->C != L->c_z) return fail(TRIMUL_ERR_INVALID_ARG, "z has %lld channels, layer expects c_z=%d", (long long)z->C, L->c_z);
+    if (!L->has_bf16)
+        return fail(TRIMUL_ERR_UNSUPPORTED_SHAPE, "bf16 path supports (c_z, c_h) = (128,128) or (384,128); layer is (%d,%d)", L->c_z, L->c_h);
+    if ((long long)z->B * L->c_h > 65535)
+        return fail(TRIMUL_ERR_UNSUPPORTED_SHAPE, "B*c_h=%lld exceeds 65535", (long long)z->B * L->c_h);
+    if (mask && !aligned16(mask)) return fail(TRIMUL_ERR_ALIGNMENT, "mask pointer not 16-byte aligned");
+    return TRIMUL_OK;
+}
+
+static size_t shard_x_bytes(const trimul_layer_t *L, int64_t B, int64_t R, int64_t N) {
+    return align256((size_t)B * L->c_h * R * N * 2);
+}
+
+static size_t shard_ws_bytes(const trimul_layer_t *L, int64_t B, int64_t R, int64_t N) {
+    return shard_x_bytes(L, B, R, N) + ws_q_bytes(B, L->c_h);
+}
+
+extern "C" size_t tri_mul_shard_workspace_bytes(const trimul_layer_t *L, int64_t B, int64_t R, int64_t N) {
+    if (!L || B < 1 || R < 1 || N < 1) return 0;
+    return shard_ws_bytes(L, B, R, N);
+}
+
+static trimul_status_t check_shard_workspace(const trimul_rows_t *z, const trimul_layer_t *L) {
+    const size_t need = shard_ws_bytes(L, z->B, z->R, z->N);
+    if (!L->ws || L->ws_bytes < need)
+        return fail(TRIMUL_ERR_WORKSPACE, "workspace of %zu bytes needed, %zu bound", need, L->ws ? L->ws_bytes : (size_t)0);
+    if (overlap(z->data, rows_bytes(z), L->ws, need)) return fail(TRIMUL_ERR_INVALID_ARG, "z overlaps the workspace");
+    return TRIMUL_OK;
+}
+
+extern "C" trimul_status_t tri_mul_shard_project(const trimul_rows_t *z, const void *mask, const trimul_layer_t *L,
+                                                 void *a_out, void *b_out, void *stream) {
+    TRY(check_shard_sizes(z));
+    TRY(check_shard_layer(z, mask, L));
+    if (!a_out || !b_out) return fail(TRIMUL_ERR_INVALID_ARG, "a_out / b_out NULL");
+    if (!aligned16(a_out) || !aligned16(b_out)) return fail(TRIMUL_ERR_ALIGNMENT, "a_out / b_out not 16-byte aligned");
+    const size_t plane = (size_t)z->B * L->c_h * z->R * z->N * 2;
+    if (overlap(a_out, plane, b_out, plane) || overlap(a_out, plane, z->data, rows_bytes(z)) ||
+        overlap(b_out, plane, z->data, rows_bytes(z)))
+        return fail(TRIMUL_ERR_INVALID_ARG, "a_out, b_out and z overlap");
+    TRY(check_shard_workspace(z, L));
+    const size_t need = shard_ws_bytes(L, z->B, z->R, z->N);
+    if (overlap(a_out, plane, L->ws, need) || overlap(b_out, plane, L->ws, need))
+        return fail(TRIMUL_ERR_INVALID_ARG, "a_out / b_out overlap the workspace");
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    float *q = reinterpret_cast<float *>(reinterpret_cast<uint8_t *>(L->ws) + shard_x_bytes(L, z->B, z->R, z->N));
+    TRY(run_project_bf16(L, z->data, mask, a_out, b_out, (int)z->B, (int)z->R, (int)z->N, st, nullptr, L->acc));
+    // the offset of this shard's stored x, from its own rows' channel sums
+    TRY_CUDA(xoffsets_launch(L->acc, (int)z->B, L->c_h, tri_mul_contract_scale(z->N), q, st), "offsets launch");
+    return TRIMUL_OK;
+}
+
+extern "C" trimul_status_t tri_mul_shard_finish(const trimul_rows_t *z, const void *mask, const trimul_layer_t *L,
+                                                trimul_direction_t dir, int G, const int64_t *shard_row0,
+                                                const void *const *a_shards, const void *const *b_shards,
+                                                trimul_rows_t *out, void *stream) {
+    TRY(check_shard_sizes(z));
+    TRY(check_rows(out, "out"));
+    if (out->B != z->B || out->R != z->R || out->N != z->N || out->C != z->C || out->row0 != z->row0)
+        return fail(TRIMUL_ERR_INVALID_ARG, "out rows differ from z's");
+    if (overlap(out->data, rows_bytes(out), z->data, rows_bytes(z))) return fail(TRIMUL_ERR_INVALID_ARG, "out overlaps z");
+    if (dir != TRIMUL_OUTGOING && dir != TRIMUL_INCOMING) return fail(TRIMUL_ERR_INVALID_ARG, "unknown direction");
+    if (G < 1 || G > kMaxShards) return fail(TRIMUL_ERR_UNSUPPORTED_SHAPE, "G=%d shards: 1 to %d are supported", G, kMaxShards);
+    if (!shard_row0 || !a_shards || !b_shards) return fail(TRIMUL_ERR_INVALID_ARG, "shard table is NULL");
+    if (shard_row0[0] != 0 || shard_row0[G] != z->N)
+        return fail(TRIMUL_ERR_INVALID_ARG, "shard rows must start at 0 and end at N");
+    int self = -1;
+    for (int g = 0; g < G; ++g) {
+        if (shard_row0[g + 1] <= shard_row0[g] || shard_row0[g] % 128 != 0)
+            return fail(TRIMUL_ERR_UNSUPPORTED_SHAPE, "shard %d: rows must be ascending whole 128-row blocks", g);
+        if (shard_row0[g] == z->row0 && shard_row0[g + 1] - shard_row0[g] == z->R) self = g;
+        if (!b_shards[g] || !aligned16(b_shards[g]) || (dir == TRIMUL_INCOMING && (!a_shards[g] || !aligned16(a_shards[g]))))
+            return fail(TRIMUL_ERR_INVALID_ARG, "shard %d: a / b missing or not 16-byte aligned", g);
+    }
+    if (self < 0) return fail(TRIMUL_ERR_INVALID_ARG, "z's rows are not one of the shards");
+    if (!a_shards[self] || !aligned16(a_shards[self])) return fail(TRIMUL_ERR_INVALID_ARG, "this shard's a is missing or misaligned");
+    TRY(check_shard_layer(z, mask, L));
+    TRY(check_shard_workspace(z, L));
+    if (overlap(out->data, rows_bytes(out), L->ws, shard_ws_bytes(L, z->B, z->R, z->N)))
+        return fail(TRIMUL_ERR_INVALID_ARG, "out overlaps the workspace");
+    DeviceInfo d;
+    TRY(require_sm100(&d));
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    uint8_t *ws = reinterpret_cast<uint8_t *>(L->ws);
+    void *x = ws;
+    const float *q = reinterpret_cast<const float *>(ws + shard_x_bytes(L, z->B, z->R, z->N));
+    const int64_t BC = z->B * L->c_h;
+    const bool incoming = dir == TRIMUL_INCOMING;
+    K2ShardArgs sa{};
+    K2Args &p = sa.base;
+    const CUtensorMapDataType dt = CU_TENSOR_MAP_DATA_TYPE_FLOAT16;
+    for (int g = 0; g < G; ++g) {
+        const uint64_t Rg = (uint64_t)(shard_row0[g + 1] - shard_row0[g]);
+        uint64_t dims[3] = {(uint64_t)z->N, Rg, (uint64_t)BC};
+        uint64_t strides[2] = {(uint64_t)z->N * 2, Rg * z->N * 2};
+        uint32_t boxb[3] = {64, incoming ? 64u : 128u, 1};
+        TRY(make_map(&sa.tm_sb[g], dt, 3, b_shards[g], dims, strides, boxb, CU_TENSOR_MAP_SWIZZLE_128B, "K2 shard b"));
+        if (incoming) {
+            uint32_t boxa[3] = {64, 64, 1};
+            TRY(make_map(&sa.tm_sa[g], dt, 3, a_shards[g], dims, strides, boxa, CU_TENSOR_MAP_SWIZZLE_128B, "K2 shard a"));
+        }
+        sa.row0[g] = (int)shard_row0[g];
+    }
+    sa.row0[G] = (int)z->N;
+    sa.G = G;
+    sa.i0 = (int)z->row0;
+    {
+        uint64_t dims[3] = {(uint64_t)z->N, (uint64_t)z->R, (uint64_t)BC};
+        uint64_t strides[2] = {(uint64_t)z->N * 2, (uint64_t)z->R * z->N * 2};
+        uint32_t boxa[3] = {64, 128, 1};
+        TRY(make_map(&p.tm_a, dt, 3, a_shards[self], dims, strides, boxa, CU_TENSOR_MAP_SWIZZLE_128B, "K2 shard own a"));
+        TRY(make_map(&p.tm_x, dt, 3, x, dims, strides, boxa, CU_TENSOR_MAP_SWIZZLE_128B, "K2 shard x"));
+        p.tm_b = sa.tm_sb[0];
+    }
+    const float x_scale = tri_mul_contract_scale(z->N);
+    p.f16 = true;
+    p.x_scale = x_scale;
+    p.xoff = q;
+    p.xoff_stride = 1;
+    p.ext = nullptr;
+    p.C = L->c_h;
+    p.BC = (int)BC;
+    p.N = (int)z->N;
+    p.m_tiles = (int)(z->R / 128);
+    p.n_tiles = (int)((z->N + 255) / 256);
+    p.k_chunks = (int)(z->N / 64);
+    p.incoming = incoming;
+    const long long tiles = BC * p.m_tiles * p.n_tiles;
+    TRY_CUDA(k2_shard_launch(sa, grid_for(d.sms, tiles, 1), st), "K2 shard launch");
+    return run_output_bf16(L, z->data, mask, x, x_scale, out->data, out->dtype == TRIMUL_F32, false, (int)z->B, (int)z->R,
+                           (int)z->N, st, nullptr);
 }
 
 // ------------------------------------------------------------------ pair update and its graph

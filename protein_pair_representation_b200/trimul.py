@@ -46,6 +46,11 @@ class _Pair(ctypes.Structure):
                 ("C", ctypes.c_int64), ("dtype", ctypes.c_int)]
 
 
+class _Rows(ctypes.Structure):
+    _fields_ = [("data", ctypes.c_void_p), ("B", ctypes.c_int64), ("R", ctypes.c_int64), ("N", ctypes.c_int64),
+                ("C", ctypes.c_int64), ("row0", ctypes.c_int64), ("dtype", ctypes.c_int)]
+
+
 class _WeightsDesc(ctypes.Structure):
     _fields_ = [("c_z", ctypes.c_int32), ("c_h", ctypes.c_int32), ("dtype", ctypes.c_int),
                 ("eps", ctypes.c_float)] + [(n, ctypes.c_void_p) for n in WEIGHT_ORDER]
@@ -96,6 +101,10 @@ def load_library():
         lib.tri_mul_transition_destroy.argtypes = [vp]
         lib.tri_mul_transition_destroy.restype = None
         lib.tri_mul_transition_forward.argtypes = [P(_Pair), vp, vp, P(_Pair), vp]
+        lib.tri_mul_shard_workspace_bytes.argtypes = [vp, i64, i64, i64]
+        lib.tri_mul_shard_workspace_bytes.restype = ctypes.c_size_t
+        lib.tri_mul_shard_project.argtypes = [P(_Rows), vp, vp, vp, vp, vp]
+        lib.tri_mul_shard_finish.argtypes = [P(_Rows), vp, vp, st, st, P(i64), P(vp), P(vp), P(_Rows), vp]
         lib.tri_mul_kernels_per_forward.argtypes = []
         lib.tri_mul_check_device_status.argtypes = []
         lib.tri_mul_status_string.argtypes = [st]
@@ -108,6 +117,7 @@ def load_library():
                      "tri_mul_graph_launch", "tri_mul_layer_set_mask_skipping", "tri_mul_transition_create",
                      "tri_mul_transition_forward",
                      "tri_mul_project", "tri_mul_contract", "tri_mul_output_gate",
+                     "tri_mul_shard_project", "tri_mul_shard_finish",
                      "tri_mul_layer_set_timing_events", "tri_mul_check_device_status"):
             getattr(lib, name).restype = ctypes.c_int
         _lib = lib
@@ -152,6 +162,27 @@ def _pair(t: torch.Tensor) -> _Pair:
     if not t.is_contiguous():
         raise ValueError("pair tensor must be contiguous")
     return _Pair(t.data_ptr(), t.shape[0], t.shape[1], t.shape[3], _dtype_code(t.dtype))
+
+
+def _rows(t: torch.Tensor, row0: int, N: int) -> _Rows:
+    """[B, R, N, C] rows [row0, row0 + R) of an N x N pair tensor."""
+    if t.dim() != 4 or t.shape[2] != N:
+        raise ValueError(f"row slab must be [B, R, N={N}, C], got {tuple(t.shape)}")
+    if not t.is_contiguous():
+        raise ValueError("row slab must be contiguous")
+    return _Rows(t.data_ptr(), t.shape[0], t.shape[1], N, t.shape[3], row0, _dtype_code(t.dtype))
+
+
+def shard_bounds(N: int, G: int) -> list:
+    """Row boundaries of G shards of an N x N pair tensor: whole 128-row blocks, as even as they go
+    (the first shards take the extra blocks)."""
+    if N % 128 or G < 1 or G > N // 128:
+        raise ValueError(f"N={N} must be a multiple of 128 with at least one 128-row block per shard (G={G})")
+    blocks = N // 128
+    bounds = [0]
+    for g in range(G):
+        bounds.append(bounds[-1] + 128 * (blocks // G + (1 if g < blocks % G else 0)))
+    return bounds
 
 
 def _mask_ptr(mask, z):
@@ -260,6 +291,44 @@ class TriMulLayer:
         _check(self._lib.tri_mul_project(ctypes.byref(zp), _mask_ptr(mask, z), self.handle,
                                          a.data_ptr(), b.data_ptr(), _stream_ptr(stream)))
         return a, b
+
+    # ---- row-sharded update (one shard of the rows; see include/trimul.h) ----
+
+    def ensure_shard_workspace(self, B: int, R: int, N: int):
+        need = int(self._lib.tri_mul_shard_workspace_bytes(self.handle, B, R, N))
+        if self._ws is None or self._ws.numel() < need:
+            self.bind_workspace(torch.empty(need, dtype=torch.uint8, device=self.device))
+
+    def shard_project(self, z_rows: torch.Tensor, mask_rows: torch.Tensor | None, row0: int, N: int, stream=None):
+        """Phase 1 for rows [row0, row0 + R) of an N x N pair tensor: a, b as [B, c_h, R, N] float16."""
+        B, R = z_rows.shape[0], z_rows.shape[1]
+        self.ensure_shard_workspace(B, R, N)
+        a = torch.empty((B, self.c_h, R, N), dtype=torch.float16, device=z_rows.device)
+        b = torch.empty_like(a)
+        zr = _rows(z_rows, row0, N)
+        _check(self._lib.tri_mul_shard_project(ctypes.byref(zr), _mask_ptr(mask_rows, z_rows) if mask_rows is not None
+                                               else None, self.handle, a.data_ptr(), b.data_ptr(), _stream_ptr(stream)))
+        return a, b
+
+    def shard_finish(self, z_rows: torch.Tensor, mask_rows: torch.Tensor | None, row0: int, N: int, direction,
+                     bounds, a_shards, b_shards, out: torch.Tensor | None = None,
+                     out_dtype: torch.dtype | None = None, stream=None):
+        """Phase 2: this shard's rows of the update from every shard's phase-1 a and b (a list of
+        G tensors each; entries of a_shards other than this shard's may be None for outgoing)."""
+        G = len(bounds) - 1
+        B, R = z_rows.shape[0], z_rows.shape[1]
+        self.ensure_shard_workspace(B, R, N)
+        if out is None:
+            out = torch.empty(z_rows.shape, dtype=out_dtype or torch.float32, device=z_rows.device)
+        row_arr = (ctypes.c_int64 * (G + 1))(*bounds)
+        ptr = lambda t: None if t is None else t.data_ptr()
+        a_arr = (ctypes.c_void_p * G)(*[ptr(t) for t in a_shards])
+        b_arr = (ctypes.c_void_p * G)(*[ptr(t) for t in b_shards])
+        zr, orow = _rows(z_rows, row0, N), _rows(out, row0, N)
+        _check(self._lib.tri_mul_shard_finish(ctypes.byref(zr), _mask_ptr(mask_rows, z_rows) if mask_rows is not None
+                                              else None, self.handle, _DIRS[direction], G, row_arr, a_arr, b_arr,
+                                              ctypes.byref(orow), _stream_ptr(stream)))
+        return out
 
     def output_gate(self, z: torch.Tensor, x: torch.Tensor, mask: torch.Tensor | None = None,
                     out: torch.Tensor | None = None, out_dtype: torch.dtype | None = None, x_scale: float = 1.0,

@@ -6,8 +6,9 @@ Zero-mean seeded weights keep |mean_c x| small; gated projections with a large c
 (positive or negative projection biases, as trained trunks often have) make every channel of
 x carry nearly the same large value L * mean(a_c) * mean(b_c), and a plain fp16 x then misses
 the 2e-2 RMS bound (a CPU emulation of the storage roundings alone gives 3e-2 ... 6e-2 at
-N = 256 ... 512 with biases of +3). The update stores x less a per-(batch, channel) offset and
-adds it back in the output kernel; these tests hold that path to the bound:
+N = 256 ... 512 with biases of +3). The update stores x less one offset per batch element,
+which the output LayerNorm (blind to a constant added to every channel of a pair) needs no
+correction for; these tests hold that path to the bound:
 
   - the headline shape (B=1, N=512, ragged mask L ~ U[384, 512]) with projection biases of
     +3 / +4 / -3 (and gate biases), both directions, against the fp64 oracle on every entry;
