@@ -305,14 +305,41 @@ trimul_status_t tri_mul_shard_finish(const trimul_rows_t *z, const void *mask, c
                                      const void *const *a_shards, const void *const *b_shards,
                                      trimul_rows_t *out, void *stream);
 
-/* Mask skipping (off by default): when on, tri_mul_forward with a mask on the tensor-core
- * path first finds the mask's extents {R_b, C_b} per batch element (a memset and one small
- * kernel) and the kernels then leave out 128-pair tiles that are masked in full (writing
- * their zeros) and the contraction's k-range beyond the extents ("RFProteina architecture",
- * section "Kernel support": masks are left-aligned, so a per-row valid count bounds the
- * work). Worth it when whole rows are padding: measured on B200 it makes B=4 N=256 c_z=384
- * (valid lengths 162-237) 8% faster and B=1 N=512 c_z=128 (493 of 512 valid) 9% slower. */
+/* Mask skipping ("RFProteina architecture", section "Kernel support": masks are left-aligned,
+ * so per-row valid counts, computed once, bound the work of every pair update). With a mask's
+ * extents {R_b, C_b} (1 + the last row / column of batch element b holding a nonzero mask
+ * entry) the kernels leave out tiles that are masked in full (writing their zeros) and the
+ * contraction's k-range beyond them; results are bitwise those without skipping. Extents come,
+ * in this order, from a caller (tri_mul_forward_extents), from valid lengths set on the layer
+ * (tri_mul_layer_set_valid_lengths, when they match the problem's B and N), or, with mask
+ * skipping switched on (tri_mul_layer_set_mask_skipping, off by default), from a pass over the
+ * mask (a memset and one small kernel) per forward, or once per tri_mul_pair_update. */
 trimul_status_t tri_mul_layer_set_mask_skipping(trimul_layer_t *layer, int enable);
+
+/* The extents of a bf16 mask [B, N, N] into extents[2B] (int32 on the device, 16-byte aligned):
+ * a memset and one small kernel on `stream`. */
+trimul_status_t tri_mul_mask_extents(const void *mask, int64_t B, int64_t N, trimul_dtype_t dtype,
+                                     int32_t *extents, void *stream);
+
+/* tri_mul_forward with the mask's extents given (device int32 [B][2], for instance from
+ * tri_mul_mask_extents once per mask): skipping applies whatever the layer's settings. Every
+ * nonzero mask entry of batch element b must lie in rows < R_b and columns < C_b. BF16 path. */
+trimul_status_t tri_mul_forward_extents(const trimul_pair_t *z, const void *mask, const int32_t *extents,
+                                        const trimul_layer_t *layer, trimul_direction_t direction,
+                                        trimul_pair_t *out, void *stream);
+
+/* The share of one layer's dense work (its flops at N) that skipping by left-aligned valid
+ * lengths lengths[0..B) leaves out (K1 and K3 scale with L_b^2 pairs, K2 with L_b^3). */
+double tri_mul_skip_saving(const int64_t *lengths, int64_t B, int64_t N, int32_t c_z, int32_t c_h);
+
+/* Per-batch-element valid lengths of a left-aligned padding mask (host int64 [B]: mask entries
+ * of batch element b are 0 at rows or columns >= lengths[b]), set once for all later forwards
+ * of B x N problems on this handle: their extents {L_b, L_b} go to a device buffer the handle
+ * allocates now (the call synchronizes), and skipping is used only when tri_mul_skip_saving
+ * is at least 0.15 (it costs a few percent otherwise; *skipping_out, when not NULL, tells
+ * which). NULL lengths clears them. */
+trimul_status_t tri_mul_layer_set_valid_lengths(trimul_layer_t *layer, const int64_t *lengths, int64_t B, int64_t N,
+                                                int32_t *skipping_out);
 
 /* The fused pair transition, the step that follows the two triangle updates in a pair
  * update ("RFProteina architecture", section "Kernel support": one launch runs both linears,
@@ -375,7 +402,7 @@ const char *tri_mul_last_error(void);
 /* ABI version of this header (major * 100 + minor). */
 int tri_mul_abi_version(void);
 
-#define TRIMUL_ABI_VERSION 102
+#define TRIMUL_ABI_VERSION 103
 
 #ifdef __cplusplus
 }

@@ -13,7 +13,7 @@
 // so the tensor cores multiply the raw bf16 z tile, and the epilogue applies the
 // per-pair (mean, rstd) and the per-channel (sum W', shift) pair of constants.
 //
-// Two kernels. c_z = 128 (k1_project_ab_kernel, further below) puts one hidden channel
+// Two kernels. c_z = 128 (k1_project_tm_kernel, further below) puts one hidden channel
 // on each TMEM lane and makes both operands from each z tile. c_z = 384 (k1_project_kernel)
 // puts one pair on each TMEM lane:
 // 128 consecutive pairs of one batch element times NCOL = 128 packed weight rows, laid
@@ -28,6 +28,37 @@
 #include "sm100.cuh"
 
 namespace trimul {
+
+// Unmasked-pair counts of one batch element for the offset of the stored x (kAccSampled,
+// kAccAll and kAccRows entries after the channel sums), kept by one lane per statistics warp and
+// added with integer atomics when the batch element changes and at the end.
+struct PairCounts {
+    int b = -1;
+    unsigned int sampled = 0, all = 0, rows = 0;
+    __device__ __forceinline__ void flush(unsigned long long *acc) {
+        if (b < 0) return;
+        unsigned long long *a = acc + (size_t)b * kAccStride;
+        atomicAdd(a + kAccSampled, (unsigned long long)sampled);
+        atomicAdd(a + kAccAll, (unsigned long long)all);
+        atomicAdd(a + kAccRows, (unsigned long long)rows);
+    }
+    // valid: this lane's pair is unmasked; samp: it is one of the sampled pairs; first: it is the
+    // first pair of its row (a padding mask's row is valid iff its first pair is)
+    __device__ __forceinline__ void add(unsigned long long *acc, int batch, bool valid, bool samp, bool first, int lane) {
+        const unsigned int v = __ballot_sync(0xffffffffu, valid);
+        const unsigned int s = __ballot_sync(0xffffffffu, valid && samp);
+        const unsigned int f = __ballot_sync(0xffffffffu, valid && first);
+        if (lane != 0) return;
+        if (batch != b) {
+            flush(acc);
+            b = batch;
+            sampled = all = rows = 0;
+        }
+        sampled += __popc(s);
+        all += __popc(v);
+        rows += __popc(f);
+    }
+};
 
 template <int CZ>
 struct K1Cfg {
@@ -190,10 +221,10 @@ __global__ void __launch_bounds__(448, 1) k1_project_kernel(const __grid_constan
         uint32_t phase = 0;
         int sbuf = 0;
         uint32_t sphase = 0;
-        // unmasked pairs of batch element cnt_b seen so far (group 0's CTAs count them)
+        // unmasked pairs seen so far (group 0's CTAs count them); the sampled pairs are each
+        // tile's first 16, the ones whose outputs the epilogue sums
         const bool counting = p.acc != nullptr && group == 0;
-        int cnt_b = -1;
-        unsigned int cnt = 0;
+        PairCounts counts;
         TileWalk tw(cta_in_group, p.tiles_per_batch);
         for (int pt = cta_in_group; pt < num_ptiles; pt += ctas_per_group, tw.advance(ctas_per_group, p.tiles_per_batch)) {
             const int b = tw.b;
@@ -236,23 +267,14 @@ __global__ void __launch_bounds__(448, 1) k1_project_kernel(const __grid_constan
             // 1 (no mask), the mask entry, or 0 past the last pair
             float m = pi < p.NN ? 1.f : 0.f;
             if (p.mask && pi < p.NN) m = __uint_as_float((uint32_t)p.mask[(long long)b * p.NN + pi] << 16);
-            if (counting) {
-                const unsigned int valid = __ballot_sync(0xffffffffu, m != 0.f);
-                if (b != cnt_b) {
-                    if (cnt_b >= 0 && lane == 0) atomicAdd(p.acc + (size_t)cnt_b * (2 * C::C_H + 1) + 2 * C::C_H, (unsigned long long)cnt);
-                    cnt_b = b;
-                    cnt = 0;
-                }
-                cnt += __popc(valid);
-            }
+            if (counting) counts.add(p.acc, b, m != 0.f, row < 16, pi % p.N == 0, lane);
             if (!__all_sync(0xffffffffu, mbar_wait(&s.sempty[sbuf], sphase ^ 1, abort_flag, kErrTimeoutEpilogue))) break;
             stats[sbuf * 128 + row] = make_float4(mean, rstd, m, 0.f);
             __syncwarp();
             if (lane == 0) mbar_arrive(&s.sfull[sbuf]);
             if (++sbuf == C::SNB) { sbuf = 0; sphase ^= 1; }
         }
-        if (counting && cnt_b >= 0 && lane == 0)
-            atomicAdd(p.acc + (size_t)cnt_b * (2 * C::C_H + 1) + 2 * C::C_H, (unsigned long long)cnt);
+        if (counting && lane == 0) counts.flush(p.acc);
     } else {
         // epilogue: warpgroup wg handles channels [ch0 + wg*CH_WG, +CH_WG)
         const int wg = warp >> 2;
@@ -266,8 +288,9 @@ __global__ void __launch_bounds__(448, 1) k1_project_kernel(const __grid_constan
         uint32_t aphase = 0;
         int sbuf = 0;
         uint32_t sphase = 0;
-        // running sums of this thread's outputs per channel over batch element sum_b; summed over
-        // the warp and added to the channel sums when the batch element changes and at the end
+        // running sums of this thread's outputs per channel over batch element sum_b (the first 16
+        // pairs of each tile: the sampled ones); summed over the warp and added to the channel sums
+        // when the batch element changes and at the end
         unsigned long long *acc_w = p.acc ? p.acc + operand * C::C_H + ch0 + wg * C::CH_WG : nullptr;
         int sum_b = -1;
         float run[C::CH_WG];
@@ -279,7 +302,7 @@ __global__ void __launch_bounds__(448, 1) k1_project_kernel(const __grid_constan
                 float v = run[t];
 #pragma unroll
                 for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
-                if (lane == 0) atomicAdd(acc_w + (size_t)fb * (2 * C::C_H + 1) + t, (unsigned long long)llrintf(v * kAccScale));
+                if (lane == 0) atomicAdd(acc_w + (size_t)fb * kAccStride + t, (unsigned long long)llrintf(v * kAccScale));
                 run[t] = 0.f;
             }
         };
@@ -327,7 +350,7 @@ __global__ void __launch_bounds__(448, 1) k1_project_kernel(const __grid_constan
                     const float pr = fmaf(rstd, fmaf(-mean, cv.z, v[16 + e]), cv.w);
                     const float out = sigmoid_tanh(g) * pr * m;
                     stg[(blk * 16 + e) * 128 + row] = __half_as_ushort(__float2half_rn(out));
-                    run[blk * 16 + e] += out;        // the unrounded value: an estimate needs no more
+                    if (row < 16) run[blk * 16 + e] += out;   // sampled pairs, unrounded: an estimate needs no more
                 }
             }
             tc_fence_before();
@@ -356,385 +379,29 @@ __global__ void __launch_bounds__(448, 1) k1_project_kernel(const __grid_constan
 // ------------------------------------------------------------------------------------------
 // K1 for c_z = 128: both operands from each z tile, one TMEM lane per hidden channel.
 //
-// A 128-pair tile of z (32 KB, one TMA box) is read once per CTA, its LayerNorm statistics are
-// computed once, and four accumulators are filled from it: D_r[c, p] = W'_r[c] . z_p for the
-// four weight blocks r = a-gate, a-projection, b-gate, b-projection (A = the folded weights,
-// 128 channels x c_z, resident in shared memory for the whole kernel: 128 KB; B = the z tile,
-// 128 pairs x c_z; both K-major; M = N = 128). The four accumulators take all 512 TMEM columns:
-// operand a's two in the first 256 (region a), operand b's in the last 256 (region b). The MMA
-// fills region a, then region b, of each tile; region a of the next tile is filled while the
-// epilogue still works on region b, so each region is single-buffered and the two alternate.
-// N = 128 keeps the tensor core's operand reads from shared memory at 2 KB per pair (the
-// weights are read once per 128 pairs), which, with the epilogue's traffic, is what bounds
-// this kernel's rate.
+// A 64-pair tile of z (16 KB, one TMA box with both 64-channel halves) is read once per CTA, its
+// LayerNorm statistics are computed once, and four accumulators are filled from it:
+// D_r[c, p] = W'_r[c] . z_p for the four weight blocks r = a-gate, a-projection, b-gate,
+// b-projection (A = the folded weights, 128 channels x c_z, resident in shared memory for the
+// whole kernel: 128 KB; B = the z tile, 64 pairs x c_z; both K-major; M = 128, N = 64).
+// Two teams of eight epilogue warps take alternate tiles, each team with its own TMEM buffer of
+// the four accumulators (256 columns), so the MMA of a tile never waits for the other team;
+// sixteen epilogue warps (four per scheduler) hide the latency of TMEM loads and of the gate
+// arithmetic, and a four-stage z ring covers the HBM latency. (A design with 128-pair tiles,
+// N = 128 and one single-buffered TMEM region per operand, drained by eight warps, read the
+// weights half as often but ran 7% slower at N = 512: its epilogue was latency-bound.)
 // A thread of the epilogue owns one channel of one operand for the whole kernel, so that
 // channel's four folding constants stay in registers; the per-pair LayerNorm statistics are
-// read from shared memory (broadcast); and consecutive pairs of one channel are consecutive
-// TMEM columns, which pack directly into 16-byte rows of the channel-major output tile.
+// read from shared memory (broadcast); consecutive pairs of one channel are consecutive TMEM
+// columns, which pack directly into 16-byte rows of the channel-major output tile.
 // The epilogue's arithmetic is fp32 in packed pairs (f32x2) up to one f16x2 rounding of the
-// result: the gate as (mask/2) tanh(g/2) + mask/2 with one tanh.approx.f32 per output (the
-// gate rows are folded with an extra factor 1/2), times the projection. With 256 gated outputs
-// per pair, the transcendental / conversion pipe (16 lanes per SM) is this kernel's tightest
-// unit: one tanh and half a pack per output keep it under the HBM time per tile, where an
-// f16x2 gate (inputs converted, tanh in halves, products rounded) took about twice as many.
-// Warps: 0-7 epilogue (warp 4o + q: operand o, channels [32q, 32q + 32), all 128 pairs of a
-// tile in four store blocks of 32), 8-11 LayerNorm statistics (one thread per pair), 12 TMA
-// producer, 13 TMEM allocator + MMA issuer.
-#ifndef K1_TILE_PAIRS
-#define K1_TILE_PAIRS 128
-#endif
-struct K1AbCfg {
-    static constexpr int CZ = 128, C_H = kHidden, TP = K1_TILE_PAIRS;   // pairs per tile (64, 96 or 128)
-    static_assert(TP % 32 == 0 && TP >= 64 && TP <= 128, "tile pairs");
-    static constexpr int W_CHUNK = 4 * C_H * 64 * 2;           // [a-gate, a-proj, b-gate, b-proj rows] x 64 k: 64 KB
-    static constexpr int W_BYTES = (CZ / 64) * W_CHUNK;        // 128 KB
-    static constexpr int TILE = TP * CZ * 2;                   // z tile: [2 halves][128 pairs][64 ch], 32 KB
-    static constexpr int HALF = TP * 128;                      // one 64-channel half of a tile
-    static constexpr int WARP_STG = 32 * 32 * 2;               // per epilogue warp: [32 ch][32 pairs] f16
-    static constexpr int EPI_WARPS = 8;
-    static constexpr int STG_TOTAL = EPI_WARPS * WARP_STG;     // 16 KB
-    static constexpr int STATS_WARP0 = 8, STATS_WARPS = TP / 32;   // one thread per pair
-    static constexpr int TMA_WARP = STATS_WARP0 + STATS_WARPS, MMA_WARP = TMA_WARP + 1;
-    static constexpr int THREADS = (MMA_WARP + 1) * 32;
-    static constexpr int STATS_BYTES = 2 * TP * (4 + 4 + 4);   // -mean, rstd, mask / 2 (f32) per pair
-    static constexpr int FIXED = 1024 + W_BYTES + STG_TOTAL + STATS_BYTES + 512;
-    static constexpr int S = (232448 - FIXED) / TILE > 8 ? 8 : (232448 - FIXED) / TILE;
-    static constexpr size_t SMEM = FIXED + (size_t)S * TILE;
-};
-
-template <bool SKIP>
-__global__ void __launch_bounds__(K1AbCfg::THREADS, 1) k1_project_ab_kernel(const __grid_constant__ K1Args p) {
-    using C = K1AbCfg;
-    static_assert(sizeof(K1Smem) <= 512, "barrier block");
-    static_assert(C::S >= 2, "z ring");
-    extern __shared__ uint8_t smem_raw[];
-    uint8_t *base = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-    uint8_t *w_s = base;                                  // 2 k-chunks of [512 rows][64] bf16
-    uint8_t *tiles = w_s + C::W_BYTES;                    // S tiles of [2][128 pairs][64] bf16
-    uint8_t *staging = tiles + C::S * C::TILE;            // 8 x [32 ch][32 pairs] f16, 64B swizzle
-    float *st_nmean = reinterpret_cast<float *>(staging + C::STG_TOTAL);   // [2][128] -mean
-    float *st_rstd = st_nmean + 2 * C::TP;
-    float *st_hmask = st_rstd + 2 * C::TP;                                  // [2][128] mask / 2
-    K1Smem &s = *reinterpret_cast<K1Smem *>(st_hmask + 2 * C::TP);
-
-    const int warp = threadIdx.x >> 5;
-    const int lane = threadIdx.x & 31;
-    volatile int *abort_flag = &s.abort_flag;
-    const int num_tiles = p.B * p.tiles_per_batch;
-
-    if (threadIdx.x == 0) {
-        mbar_init(&s.wbar, 1);
-        for (int i = 0; i < C::S; ++i) {
-            mbar_init(&s.full[i], 1);
-            mbar_init(&s.empty[i], 1 + C::STATS_WARPS);   // MMA commit + statistics warps
-        }
-        for (int i = 0; i < 2; ++i) {
-            mbar_init(&s.tfull[i], 1);                      // region i (operand i) filled
-            mbar_init(&s.tempty[i], C::EPI_WARPS / 2);      // operand i's warps have loaded region i
-            mbar_init(&s.sfull[i], C::STATS_WARPS);
-            mbar_init(&s.sempty[i], C::EPI_WARPS);
-        }
-        mbar_init(&s.drain, 1);
-        s.abort_flag = 0;
-        fence_mbarrier_init();
-    }
-    if (warp == C::MMA_WARP) {
-        tmem_alloc(&s.tmem_base, 512);
-        tmem_relinquish();
-    }
-    tc_fence_before();
-    __syncthreads();
-    tc_fence_after();
-    const uint32_t tmem_base = s.tmem_base;
-    pdl_launch_dependents();
-    if (warp != C::TMA_WARP) pdl_wait();       // the producer waits after its weight loads
-
-    if (warp == C::TMA_WARP) {
-        if (lane == 0) {
-            tma_prefetch_desc(&p.tm_z);
-            tma_prefetch_desc(&p.tm_w);
-            mbar_arrive_expect_tx(&s.wbar, C::W_BYTES);
-            for (int kc = 0; kc < C::CZ / 64; ++kc)
-                for (int h = 0; h < 2; ++h)          // rows [256 h, 256 h + 256) of the 512
-                    tma_load_2d(w_s + kc * C::W_CHUNK + h * 256 * 128, &p.tm_w, &s.wbar, kc * 64, h * 256);
-            pdl_wait();
-            int stage = 0;
-            uint32_t phase = 0;
-            uint32_t filled = 0;
-            TileWalk tw(blockIdx.x, p.tiles_per_batch);
-            for (int t = blockIdx.x; t < num_tiles; t += gridDim.x, tw.advance(gridDim.x, p.tiles_per_batch)) {
-                const int b = tw.b;
-                const int p0 = tw.t * C::TP;
-                if (SKIP && tile_masked_out<C::TP>(p.ext, b, p0, p.N, p.NN, p.rowdiv)) continue;   // nothing to load
-                if (!mbar_wait(&s.empty[stage], phase ^ 1, abort_flag, kErrTimeoutProducer)) goto producer_abort;
-                mbar_arrive_expect_tx(&s.full[stage], C::TILE);
-                // both 64-channel halves of the tile's 128 pairs in one copy (pairs past the
-                // last one are zero-filled)
-                tma_load_4d(tiles + stage * C::TILE, &p.tm_z, &s.full[stage], 0, p0, 0, b);
-                ++filled;
-                if (++stage == C::S) { stage = 0; phase ^= 1; }
-            }
-            goto producer_done;
-        producer_abort:
-            for (uint32_t i = 0; i < (filled < (uint32_t)C::S ? filled : (uint32_t)C::S); ++i) {
-                uint32_t f = filled - 1 - i;
-                mbar_drain(&s.full[f % C::S], (f / C::S) & 1);
-            }
-        producer_done:
-            mbar_drain(&s.wbar, 0);
-        }
-    } else if (warp == C::MMA_WARP) {
-        if (lane == 0) {
-            const uint32_t idesc = idesc_f32acc(128, C::TP, false, false, false);
-            bool ok = mbar_wait(&s.wbar, 0, abort_flag, kErrTimeoutMma);
-            int stage = 0;
-            uint32_t phase = 0;
-            uint32_t rphase = 0;                   // both regions are filled once per tile
-            TileWalk tw(blockIdx.x, p.tiles_per_batch);
-            for (int t = blockIdx.x; ok && t < num_tiles; t += gridDim.x, tw.advance(gridDim.x, p.tiles_per_batch)) {
-                if (SKIP && tile_masked_out<C::TP>(p.ext, tw.b, tw.t * C::TP, p.N, p.NN, p.rowdiv)) continue;
-                if (!mbar_wait(&s.full[stage], phase, abort_flag, kErrTimeoutMma)) break;
-                const uint8_t *zt = tiles + stage * C::TILE;
-#pragma unroll 1
-                for (int o = 0; o < 2; ++o) {      // region o: operand o's gate and projection
-                    if (!mbar_wait(&s.tempty[o], rphase ^ 1, abort_flag, kErrTimeoutMma)) { ok = false; break; }
-                    tc_fence_after();
-#pragma unroll
-                    for (int kk = 0; kk < C::CZ / 16; ++kk) {
-                        const uint64_t bd = smem_desc_sw128(zt + (kk >> 2) * C::HALF + (kk & 3) * 32, 16, 1024);
-                        const uint8_t *wk = w_s + (kk >> 2) * C::W_CHUNK + (kk & 3) * 32 + o * 2 * C::C_H * 128;
-#pragma unroll
-                        for (int r = 0; r < 2; ++r)
-                            tc_mma_bf16(tmem_base + (2 * o + r) * C::TP, smem_desc_sw128(wk + r * C::C_H * 128, 16, 1024),
-                                        bd, idesc, kk != 0);
-                    }
-                    tc_commit(&s.tfull[o]);
-                }
-                if (!ok) break;
-                tc_commit(&s.empty[stage]);
-                if (++stage == C::S) { stage = 0; phase ^= 1; }
-                rphase ^= 1;
-            }
-            tc_commit(&s.drain);
-            mbar_drain(&s.drain, 0);
-        }
-    } else if (warp >= C::STATS_WARP0) {
-        // LayerNorm statistics: thread = pair row of the tile
-        const int row = (warp - C::STATS_WARP0) * 32 + lane;
-        int stage = 0;
-        uint32_t phase = 0;
-        uint32_t sphase[2] = {0, 0};               // tile j of this CTA uses statistics buffer j % 2
-        int j = -1;
-        // unmasked pairs of batch element cnt_b seen so far
-        const bool counting = p.acc != nullptr;
-        int cnt_b = -1;
-        unsigned int cnt = 0;
-        TileWalk tw(blockIdx.x, p.tiles_per_batch);
-        for (int t = blockIdx.x; t < num_tiles; t += gridDim.x, tw.advance(gridDim.x, p.tiles_per_batch)) {
-            const int b = tw.b;
-            const int p0 = tw.t * C::TP;
-            ++j;
-            if (SKIP && tile_masked_out<C::TP>(p.ext, b, p0, p.N, p.NN, p.rowdiv)) continue;
-            const int sbuf = j & 1;
-            const long long pi = (long long)p0 + row;
-            // bf16 1.0 (no mask), the mask entry, or 0 past the last pair (whose outputs then vanish
-            // and add nothing to the channel sums); the load is issued first so its latency overlaps
-            uint16_t mbits = pi < p.NN ? (uint16_t)0x3F80u : (uint16_t)0;
-            if (p.mask && pi < p.NN) mbits = p.mask[(long long)b * p.NN + pi];
-            if (counting) {
-                const unsigned int valid = __ballot_sync(0xffffffffu, (mbits & 0x7FFFu) != 0);
-                if (b != cnt_b) {
-                    if (cnt_b >= 0 && lane == 0) atomicAdd(p.acc + (size_t)cnt_b * (2 * C::C_H + 1) + 2 * C::C_H, (unsigned long long)cnt);
-                    cnt_b = b;
-                    cnt = 0;
-                }
-                cnt += __popc(valid);
-            }
-            if (!__all_sync(0xffffffffu, mbar_wait(&s.full[stage], phase, abort_flag, kErrTimeoutEpilogue))) break;
-            const uint8_t *zt = tiles + stage * C::TILE;
-            // shifted sums in packed pairs: s1 = sum(v - shift), s2 = sum((v - shift)^2), with
-            // the row's first entry as the shift
-            float shift = 0.f;
-            float2 nsh = make_float2(0.f, 0.f), s1 = make_float2(0.f, 0.f), s2 = make_float2(0.f, 0.f);
-#pragma unroll
-            for (int h = 0; h < 2; ++h) {
-#pragma unroll
-                for (int u = 0; u < 8; ++u) {
-                    const uint4 w = *reinterpret_cast<const uint4 *>(zt + h * C::HALF + sw128_offset(row, u));
-                    const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
-                    if (h == 0 && u == 0) {
-                        shift = bf16_lo(w.x);
-                        nsh = make_float2(-shift, -shift);
-                    }
-#pragma unroll
-                    for (int e = 0; e < 4; ++e) {
-                        const float2 d = f2_add(make_float2(bf16_lo(ws[e]), bf16_hi(ws[e])), nsh);
-                        s1 = f2_add(s1, d);
-                        s2 = f2_fma(d, d, s2);
-                    }
-                }
-            }
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&s.empty[stage]);
-            if (++stage == C::S) { stage = 0; phase ^= 1; }
-            const float inv_n = 1.0f / (float)C::CZ;
-            const float dm = (s1.x + s1.y) * inv_n;
-            const float var = fmaxf((s2.x + s2.y) * inv_n - dm * dm, 0.f);
-            if (!__all_sync(0xffffffffu, mbar_wait(&s.sempty[sbuf], sphase[sbuf] ^ 1, abort_flag, kErrTimeoutEpilogue))) break;
-            st_nmean[sbuf * C::TP + row] = -(shift + dm);
-            st_rstd[sbuf * C::TP + row] = rsqrtf(var + p.eps);
-            st_hmask[sbuf * C::TP + row] = 0.5f * __uint_as_float((uint32_t)mbits << 16);
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&s.sfull[sbuf]);
-            sphase[sbuf] ^= 1;
-        }
-        if (counting && cnt_b >= 0 && lane == 0)
-            atomicAdd(p.acc + (size_t)cnt_b * (2 * C::C_H + 1) + 2 * C::C_H, (unsigned long long)cnt);
-    } else {
-        // epilogue: warp 4o + q drains operand o's region for channels [32q, 32q + 32); thread =
-        // channel c; it covers the tile's 128 pairs in four store blocks of 32. Every warp runs
-        // on its own: it waits on the barriers itself and stages each [32 channels][32 pairs]
-        // block in its own 2 KB of shared memory (64-byte rows, 64-byte swizzle) for a TMA store.
-        const int operand = warp >> 2;
-        const int q = warp & 3;
-        const int c = q * 32 + lane;
-        uint8_t *stg = staging + warp * C::WARP_STG;
-        const CUtensorMap *tm_out = operand == 0 ? &p.tm_a : &p.tm_b;
-        // {sum W'_gate, shift_gate, sum W'_proj, shift_proj}; the gate entries are for g / 2
-        const float4 cv = p.vec[operand * C::C_H + c];
-        const float2 cg_sum = make_float2(cv.x, cv.x), cg_shift = make_float2(cv.y, cv.y);
-        const float2 cp_sum = make_float2(cv.z, cv.z), cp_shift = make_float2(cv.w, cv.w);
-        const uint32_t tbase = tmem_base + operand * 2 * C::TP + ((uint32_t)(q * 32) << 16);
-        // running sum of this channel's stored outputs over batch element sum_b
-        unsigned long long *acc_c = p.acc ? p.acc + operand * C::C_H + c : nullptr;
-        int sum_b = -1;
-        float2 run = make_float2(0.f, 0.f);
-        uint32_t rphase = 0;
-        uint32_t sphase[2] = {0, 0};
-        int j = -1;
-        TileWalk tw(blockIdx.x, p.tiles_per_batch);
-        for (int t = blockIdx.x; t < num_tiles; t += gridDim.x, tw.advance(gridDim.x, p.tiles_per_batch)) {
-            const int b = tw.b;
-            const int p0 = tw.t * C::TP;
-            ++j;
-            if (acc_c && b != sum_b) {
-                if (sum_b >= 0)
-                    atomicAdd(acc_c + (size_t)sum_b * (2 * C::C_H + 1), (unsigned long long)llrintf((run.x + run.y) * kAccScale));
-                sum_b = b;
-                run = make_float2(0.f, 0.f);
-            }
-            if (SKIP && tile_masked_out<C::TP>(p.ext, b, p0, p.N, p.NN, p.rowdiv)) {
-                // every pair of the tile is masked: a and b are 0 there (the contraction reads them)
-#pragma unroll 1
-                for (int blk = 0; blk < C::TP / 32; ++blk) {
-                    if (lane == 0) tma_store_wait_read<0>();
-                    __syncwarp();
-#pragma unroll
-                    for (int u = 0; u < 4; ++u) *reinterpret_cast<uint4 *>(stg + sw64_offset(lane, u)) = make_uint4(0, 0, 0, 0);
-                    fence_proxy_async_smem();
-                    __syncwarp();
-                    if (lane == 0 && p0 + 32 * blk < p.NN) {
-                        tma_store_3d(tm_out, stg, p0 + 32 * blk, q * 32, b);
-                        tma_store_commit();
-                    }
-                }
-                continue;
-            }
-            const int sbuf = j & 1;
-            if (!__all_sync(0xffffffffu, mbar_wait(&s.sfull[sbuf], sphase[sbuf], abort_flag, kErrTimeoutEpilogue) &&
-                                             mbar_wait(&s.tfull[operand], rphase, abort_flag, kErrTimeoutEpilogue)))
-                break;
-            sphase[sbuf] ^= 1;
-            rphase ^= 1;
-            tc_fence_after();
-            const float *snmean = st_nmean + sbuf * C::TP, *srstd = st_rstd + sbuf * C::TP;
-            const float *shmask = st_hmask + sbuf * C::TP;
-            // 16-pair steps it = 0 .. NIT - 1 (store block it / 2): the TMEM loads of step it + 1 are
-            // issued before step it's arithmetic, so their latency is hidden behind it
-            constexpr int NIT = C::TP / 16;
-            float g0[16], p0v[16], g1[16], p1v[16];
-            tmem_ld16(tbase, g0);
-            tmem_ld16(tbase + C::TP, p0v);
-            auto step = [&](const int it, float (&gc)[16], float (&pc)[16], float (&gn)[16], float (&pn)[16]) {
-                const int blk = it >> 1, hh = it & 1, o = 16 * it;
-                if (hh == 0) {
-                    if (lane == 0) tma_store_wait_read<0>();    // this warp's previous store has read its block
-                    __syncwarp();
-                }
-                tc_wait_ld_regs(gc, pc);                    // step it's loads (the only ones outstanding)
-                if (it + 1 < NIT) {
-                    tmem_ld16(tbase + o + 16, gn);
-                    tmem_ld16(tbase + C::TP + o + 16, pn);
-                } else {
-                    // the last TMEM load of the tile has landed: hand the region back to the MMA
-                    // now, not after this warp's arithmetic and store
-                    tc_fence_before();
-                    __syncwarp();
-                    if (lane == 0) mbar_arrive(&s.tempty[operand]);
-                }
-                uint32_t outw[8];
-#pragma unroll
-                for (int jj = 0; jj < 16; jj += 4) {
-                    const float4 nm = *reinterpret_cast<const float4 *>(snmean + o + jj);
-                    const float4 rs = *reinterpret_cast<const float4 *>(srstd + o + jj);
-                    const float4 mk = *reinterpret_cast<const float4 *>(shmask + o + jj);
-#pragma unroll
-                    for (int h = 0; h < 2; ++h) {
-                        // two consecutive pairs of this channel in one packed lane pair
-                        const float2 nm2 = h == 0 ? make_float2(nm.x, nm.y) : make_float2(nm.z, nm.w);
-                        const float2 rs2 = h == 0 ? make_float2(rs.x, rs.y) : make_float2(rs.z, rs.w);
-                        const float2 hm2 = h == 0 ? make_float2(mk.x, mk.y) : make_float2(mk.z, mk.w);
-                        const float2 gv = f2_fma(rs2, f2_fma(nm2, cg_sum, make_float2(gc[jj + 2 * h], gc[jj + 2 * h + 1])), cg_shift);
-                        const float2 pv = f2_fma(rs2, f2_fma(nm2, cp_sum, make_float2(pc[jj + 2 * h], pc[jj + 2 * h + 1])), cp_shift);
-                        // mask * sigmoid(2 x) = (mask / 2) tanh(x) + mask / 2, x being the halved gate
-                        const float2 gm = f2_fma(make_float2(tanh_approx(gv.x), tanh_approx(gv.y)), hm2, hm2);
-                        const float2 av = f2_mul(gm, pv);
-                        outw[jj / 2 + h] = pack_f16x2(av.x, av.y);
-                        run = f2_add(run, av);
-                    }
-                }
-#pragma unroll
-                for (int u = 0; u < 2; ++u)
-                    *reinterpret_cast<uint4 *>(stg + sw64_offset(lane, 2 * hh + u)) =
-                        make_uint4(outw[4 * u], outw[4 * u + 1], outw[4 * u + 2], outw[4 * u + 3]);
-                if (hh == 1) {
-                    fence_proxy_async_smem();
-                    __syncwarp();
-                    if (lane == 0) {
-                        if (blk == C::TP / 32 - 1) mbar_arrive(&s.sempty[sbuf]);   // statistics read in full
-                        if (p0 + 32 * blk < p.NN) {     // blocks wholly past the last pair are not stored
-                            tma_store_3d(tm_out, stg, p0 + 32 * blk, q * 32, b);
-                            tma_store_commit();
-                        }
-                    }
-                }
-            };
-#pragma unroll 1
-            for (int it = 0; it < NIT; it += 2) {
-                step(it, g0, p0v, g1, p1v);
-                step(it + 1, g1, p1v, g0, p0v);
-            }
-        }
-        if (acc_c && sum_b >= 0)
-            atomicAdd(acc_c + (size_t)sum_b * (2 * C::C_H + 1), (unsigned long long)llrintf((run.x + run.y) * kAccScale));
-        if (lane == 0) tma_store_wait_all<0>();
-    }
-
-    tc_fence_before();
-    __syncthreads();
-    if (warp == C::MMA_WARP) {
-        tc_fence_after();
-        tmem_dealloc(tmem_base, 512);
-    }
-}
-
-// ------------------------------------------------------------------------------------------
-// K1 for c_z = 128, team design: 64-pair tiles, two teams of eight epilogue warps that take
-// alternate tiles, each team with its own TMEM buffer of the four accumulators (M = 128,
-// N = 64: 256 columns), so the MMA of a tile never waits for the other team. 16 epilogue
-// warps (four per scheduler) hide the latency of TMEM loads and of the gate arithmetic, which
-// sets the pace of the region design above; a four-stage z ring covers the HBM latency. The
-// arithmetic is the same as above, in 8-pair steps whose TMEM loads are issued one step ahead.
+// result: the gate as (mask/2) tanh(g/2) + mask/2 with one tanh.approx.f32 per output (the gate
+// rows are folded with an extra factor 1/2), times the projection. With 256 gated outputs per
+// pair, the transcendental / conversion pipe (16 lanes per SM) is a tight unit: one tanh and
+// half a pack per output keep it under the HBM time per tile, where an f16x2 gate (inputs
+// converted, tanh in halves, products rounded) took about twice as many. The TMEM loads of each
+// 8-pair step are issued one step ahead. The channel sums behind the offset of the stored x are
+// taken over the first 8 pairs of each tile (an estimate needs no more).
 // Warps: 0-15 epilogue (team t = warp / 8; warp 4o + q of a team: operand o, channels
 // [32q, 32q + 32), the tile's 64 pairs in two store blocks of 32), 16-17 LayerNorm statistics,
 // 18 TMA producer, 19 TMEM allocator + MMA issuer.
@@ -875,8 +542,7 @@ __global__ void __launch_bounds__(K1TmCfg::THREADS, 1) k1_project_tm_kernel(cons
         uint32_t sphase[2] = {0, 0};
         int j = -1;
         const bool counting = p.acc != nullptr;
-        int cnt_b = -1;
-        unsigned int cnt = 0;
+        PairCounts counts;              // the sampled pairs are each tile's first 8
         TileWalk tw(blockIdx.x, p.tiles_per_batch);
         for (int t = blockIdx.x; t < num_tiles; t += gridDim.x, tw.advance(gridDim.x, p.tiles_per_batch)) {
             const int b = tw.b;
@@ -886,15 +552,7 @@ __global__ void __launch_bounds__(K1TmCfg::THREADS, 1) k1_project_tm_kernel(cons
             const int sbuf = j & 1;
             const long long pi = (long long)p0 + row;     // < NN: NN is a multiple of 64
             const uint16_t mbits = p.mask ? p.mask[(long long)b * p.NN + pi] : (uint16_t)0x3F80u;
-            if (counting) {
-                const unsigned int valid = __ballot_sync(0xffffffffu, (mbits & 0x7FFFu) != 0);
-                if (b != cnt_b) {
-                    if (cnt_b >= 0 && lane == 0) atomicAdd(p.acc + (size_t)cnt_b * (2 * C::C_H + 1) + 2 * C::C_H, (unsigned long long)cnt);
-                    cnt_b = b;
-                    cnt = 0;
-                }
-                cnt += __popc(valid);
-            }
+            if (counting) counts.add(p.acc, b, (mbits & 0x7FFFu) != 0, row < 8, pi % p.N == 0, lane);
             if (!__all_sync(0xffffffffu, mbar_wait(&s.full[stage], phase, abort_flag, kErrTimeoutEpilogue))) break;
             const uint8_t *zt = tiles + stage * C::TILE;
             float shift = 0.f;
@@ -931,8 +589,7 @@ __global__ void __launch_bounds__(K1TmCfg::THREADS, 1) k1_project_tm_kernel(cons
             if (lane == 0) mbar_arrive(&s.sfull[sbuf]);
             sphase[sbuf] ^= 1;
         }
-        if (counting && cnt_b >= 0 && lane == 0)
-            atomicAdd(p.acc + (size_t)cnt_b * (2 * C::C_H + 1) + 2 * C::C_H, (unsigned long long)cnt);
+        if (counting && lane == 0) counts.flush(p.acc);
     } else {
         const int team = warp >> 3;
         const int operand = (warp >> 2) & 1;
@@ -956,8 +613,7 @@ __global__ void __launch_bounds__(K1TmCfg::THREADS, 1) k1_project_tm_kernel(cons
             const int b = tw.b;
             const int p0 = tw.t * C::TP;
             if (acc_c && b != sum_b) {
-                if (sum_b >= 0)
-                    atomicAdd(acc_c + (size_t)sum_b * (2 * C::C_H + 1), (unsigned long long)llrintf((run.x + run.y) * kAccScale));
+                if (sum_b >= 0) atomicAdd(acc_c + (size_t)sum_b * kAccStride, (unsigned long long)llrintf((run.x + run.y) * kAccScale));
                 sum_b = b;
                 run = make_float2(0.f, 0.f);
             }
@@ -1019,7 +675,7 @@ __global__ void __launch_bounds__(K1TmCfg::THREADS, 1) k1_project_tm_kernel(cons
                         const float2 gm = f2_fma(make_float2(tanh_approx(gv.x), tanh_approx(gv.y)), hm2, hm2);
                         const float2 av = f2_mul(gm, pv);
                         outw[jj / 2 + h] = pack_f16x2(av.x, av.y);
-                        run = f2_add(run, av);
+                        if (it == 0) run = f2_add(run, av);    // the sampled pairs: the tile's first 8
                     }
                 }
                 *reinterpret_cast<uint4 *>(stg + sw64_offset(lane, part)) = make_uint4(outw[0], outw[1], outw[2], outw[3]);
@@ -1039,8 +695,7 @@ __global__ void __launch_bounds__(K1TmCfg::THREADS, 1) k1_project_tm_kernel(cons
                 step(it + 1, g1, p1v, g0, p0v);
             }
         }
-        if (acc_c && sum_b >= 0)
-            atomicAdd(acc_c + (size_t)sum_b * (2 * C::C_H + 1), (unsigned long long)llrintf((run.x + run.y) * kAccScale));
+        if (acc_c && sum_b >= 0) atomicAdd(acc_c + (size_t)sum_b * kAccStride, (unsigned long long)llrintf((run.x + run.y) * kAccScale));
         if (lane == 0) tma_store_wait_all<0>();
     }
 
@@ -1054,13 +709,10 @@ __global__ void __launch_bounds__(K1TmCfg::THREADS, 1) k1_project_tm_kernel(cons
 
 int k1_ncol(int c_z) { return c_z == 128 ? 256 : K1Cfg<384>::NCOL; }
 int k1_groups(int c_z) { return c_z == 128 ? 1 : K1Cfg<384>::G; }
-int k1_channels_per_warpgroup(int c_z) { return c_z == 128 ? K1AbCfg::C_H : K1Cfg<384>::CH_WG; }
+int k1_channels_per_warpgroup(int c_z) { return c_z == 128 ? K1TmCfg::C_H : K1Cfg<384>::CH_WG; }
 int k1_row_mode(int c_z) { return c_z == 128 ? 2 : 1; }
-#ifndef K1_TEAMS
-#define K1_TEAMS 1
-#endif
-int k1_tile_pairs(int c_z) { return c_z == 128 ? (K1_TEAMS ? K1TmCfg::TP : K1AbCfg::TP) : 128; }
-size_t k1_smem_bytes(int c_z) { return c_z == 128 ? (K1_TEAMS ? K1TmCfg::SMEM : K1AbCfg::SMEM) : K1Cfg<384>::SMEM; }
+int k1_tile_pairs(int c_z) { return c_z == 128 ? K1TmCfg::TP : 128; }
+size_t k1_smem_bytes(int c_z) { return c_z == 128 ? K1TmCfg::SMEM : K1Cfg<384>::SMEM; }
 
 template <int CZ, bool SKIP>
 static cudaError_t k1_launch_t(const K1Args &args, int grid, cudaStream_t stream) {
@@ -1077,11 +729,10 @@ static cudaError_t k1_launch_t(const K1Args &args, int grid, cudaStream_t stream
 }
 
 template <bool SKIP>
-static cudaError_t k1_launch_ab(const K1Args &args, int grid, cudaStream_t stream) {
+static cudaError_t k1_launch_tm(const K1Args &args, int grid, cudaStream_t stream) {
     static int configured_device = -1;
     int dev = 0;
     cudaGetDevice(&dev);
-#if K1_TEAMS
     if (configured_device != dev) {
         cudaError_t e = cudaFuncSetAttribute(k1_project_tm_kernel<SKIP>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                              (int)K1TmCfg::SMEM);
@@ -1089,20 +740,11 @@ static cudaError_t k1_launch_ab(const K1Args &args, int grid, cudaStream_t strea
         configured_device = dev;
     }
     return launch_pdl(k1_project_tm_kernel<SKIP>, grid, K1TmCfg::THREADS, K1TmCfg::SMEM, stream, args);
-#else
-    if (configured_device != dev) {
-        cudaError_t e = cudaFuncSetAttribute(k1_project_ab_kernel<SKIP>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                             (int)K1AbCfg::SMEM);
-        if (e != cudaSuccess) return e;
-        configured_device = dev;
-    }
-    return launch_pdl(k1_project_ab_kernel<SKIP>, grid, K1AbCfg::THREADS, K1AbCfg::SMEM, stream, args);
-#endif
 }
 
 cudaError_t k1_launch(int c_z, const K1Args &args, int grid, cudaStream_t stream) {
     const bool skip = args.ext != nullptr;
-    if (c_z == 128) return skip ? k1_launch_ab<true>(args, grid, stream) : k1_launch_ab<false>(args, grid, stream);
+    if (c_z == 128) return skip ? k1_launch_tm<true>(args, grid, stream) : k1_launch_tm<false>(args, grid, stream);
     if (c_z == 384) return skip ? k1_launch_t<384, true>(args, grid, stream) : k1_launch_t<384, false>(args, grid, stream);
     return cudaErrorInvalidValue;
 }

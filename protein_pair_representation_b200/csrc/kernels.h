@@ -26,13 +26,17 @@ struct K1Args {
     float eps;
     const int *ext;        // mask extents [B][2] {R_b, C_b} (tiles wholly beyond them skipped), or nullptr
     uint64_t rowdiv;       // multiplier dividing by N / 8 (div_by_magic)
-    unsigned long long *acc;   // per batch element [2*c_h + 1]: fixed-point (x kAccScale) sums of the
-                               // stored a and b per channel and the count of unmasked pairs, added
+    unsigned long long *acc;   // per batch element kAccStride entries (below): sums and counts added
                                // with integer atomics (order-independent); nullptr: not gathered
 };
 
-// Fixed-point scale of the a / b channel sums (K1Args::acc).
+// The channel sums behind the offset of the stored x (K1Args::acc), per batch element:
+// [c_h sums of a | c_h sums of b | sampled | all | rows], the sums in fixed point (x kAccScale)
+// over a sample of the pairs, then the counts of unmasked pairs in the sample, of all unmasked
+// pairs, and of rows whose first pair is unmasked. The stride is fixed by c_h = kHidden.
 constexpr float kAccScale = 256.0f;
+constexpr int kAccSampled = 2 * kHidden, kAccAll = 2 * kHidden + 1, kAccRows = 2 * kHidden + 2;
+constexpr int kAccStride = 2 * kHidden + 3;
 
 struct K2Args {
     CUtensorMap tm_a, tm_b, tm_x;
@@ -149,9 +153,9 @@ int k3_groups(int c_z);
 cudaError_t k3_launch(int c_z, bool out_f32, const K3Args &args, int grid, cudaStream_t stream);  // residual iff args.zres
 
 // The offset of the stored x of each batch element from K1's sums, written to all c_h entries
-// q[b][c]: x_scale * (1 / c_h) sum_c Sa_c Sb_c / P^1.5, rounded to an fp16 value (Sa_c, Sb_c the
-// channel sums of a and b over batch element b, P its unmasked pairs; 0 when P = 0); the sums are
-// zeroed for the next forward. One CTA per batch element.
+// q[b][c]: x_scale * L * (1 / c_h) sum_c mean(a_c) mean(b_c), rounded to an fp16 value (the means
+// over the sampled unmasked pairs, L = all / rows the estimated contraction length; 0 without
+// sampled pairs); the sums are zeroed for the next forward. One CTA per batch element.
 cudaError_t xoffsets_launch(unsigned long long *acc, int B, int c_h, float x_scale, float *q, cudaStream_t stream);
 
 // ---- weight folding (layer creation) -----------------------------------------------

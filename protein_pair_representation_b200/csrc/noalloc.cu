@@ -19,7 +19,7 @@ namespace trimul {
 trimul_status_t set_last_error(trimul_status_t st, const char *msg);
 trimul_status_t forward_buffers(const trimul_pair_t *z, const void *mask, const trimul_layer_t *L,
                                 trimul_direction_t dir, trimul_pair_t *out, bool residual, void *ws_ptr,
-                                size_t ws_bytes, bool timing, void *stream, bool check_only);
+                                size_t ws_bytes, bool timing, void *stream, bool check_only, const int *given_ext);
 }
 
 // The library's own scratch for the intermediates. Every GPU that loads the library holds
@@ -95,7 +95,7 @@ extern "C" trimul_status_t tri_mul_forward_noalloc(const trimul_pair_t *z, const
                                                    trimul_pair_t *out, void *stream) {
     // every argument rule first, with nothing touched on the device
     trimul_status_t st = trimul::forward_buffers(z, mask, layer, direction, out, false, nullptr,
-                                                 (size_t)TRIMUL_NOALLOC_SCRATCH_BYTES, false, stream, true);
+                                                 (size_t)TRIMUL_NOALLOC_SCRATCH_BYTES, false, stream, true, nullptr);
     if (st == TRIMUL_ERR_WORKSPACE)
         return trimul::set_last_error(TRIMUL_ERR_WORKSPACE,
                                       "problem needs more intermediate memory than the built-in "
@@ -107,5 +107,5 @@ extern "C" trimul_status_t tri_mul_forward_noalloc(const trimul_pair_t *z, const
     // Nothing in the array has to start at zero: a call writes every intermediate it reads
     // (the channel sums that must start at zero live in the layer handle).
     return trimul::forward_buffers(z, mask, layer, direction, out, false, base,
-                                   (size_t)TRIMUL_NOALLOC_SCRATCH_BYTES, false, stream, false);
+                                   (size_t)TRIMUL_NOALLOC_SCRATCH_BYTES, false, stream, false, nullptr);
 }

@@ -36,7 +36,7 @@ struct trimul_layer {
     uint16_t *k3_wo;             // [c_z][c_h] folded
     uint16_t *k3_wg;             // [c_z][c_z] folded
     float4 *k3_vec;              // [c_z]
-    // K1's per-(batch, channel) sums of a and b and unmasked-pair counts, [65535 / c_h + 1][2 c_h + 1]
+    // K1's per-(batch, channel) sums of a and b and unmasked-pair counts, [65535 / c_h + 1][kAccStride]
     // (zero between forwards: the offsets kernel clears what it has read)
     unsigned long long *acc;
     // fp32 path
@@ -47,6 +47,11 @@ struct trimul_layer {
     cudaEvent_t events[4];
     bool timing;
     bool skip_masked;            // find mask extents and leave out wholly masked tiles
+    // valid lengths set by tri_mul_layer_set_valid_lengths: extents {L_b, L_b} on the device for
+    // problems of vl_B x vl_N, and whether the rule chose to skip with them
+    int *vl_ext;
+    int64_t vl_B, vl_N;
+    bool vl_skip;
 };
 
 // ------------------------------------------------------------------ error plumbing
@@ -156,6 +161,12 @@ static trimul_status_t make_map(CUtensorMap *m, CUtensorMapDataType dt, int rank
         if (_s != TRIMUL_OK) return _s;           \
     } while (0)
 
+// Skipping by valid lengths is chosen when it leaves out at least this share of the dense work
+// (measured on B200: the skipping instances and their tile tests cost a few percent; at B=1 N=512
+// with 493 of 512 valid, 9% of the work, skipping did not pay; at B=4 N=256 with 162-237 valid,
+// about 40%, it saved 8.5% of the time).
+static constexpr double kSkipRule = 0.15;
+
 // Batch elements the layer's channel sums have room for: B * c_h <= 65535 is enforced.
 static int acc_batches(int c_h) { return 65535 / c_h + 1; }
 
@@ -246,7 +257,7 @@ extern "C" trimul_status_t tri_mul_layer_create(const trimul_weights_desc_t *w, 
         o_k3o = take((size_t)cz * ch * 2);
         o_k3g = take((size_t)cz * cz * 2);
         o_k3v = take((size_t)cz * sizeof(float4));
-        acc_bytes = (size_t)acc_batches(ch) * (2 * ch + 1) * sizeof(unsigned long long);
+        acc_bytes = (size_t)acc_batches(ch) * kAccStride * sizeof(unsigned long long);
         o_acc = take(acc_bytes);
     }
     const size_t o_lig = take(cz * 4), o_lib = take(cz * 4);
@@ -354,6 +365,7 @@ extern "C" trimul_status_t tri_mul_layer_create(const trimul_weights_desc_t *w, 
 extern "C" void tri_mul_layer_destroy(trimul_layer_t *L) {
     if (!L) return;
     if (L->mem) cudaFree(L->mem);
+    if (L->vl_ext) cudaFree(L->vl_ext);
     delete L;
 }
 
@@ -686,7 +698,7 @@ namespace trimul {
 // return without touching the device.
 trimul_status_t forward_buffers(const trimul_pair_t *z, const void *mask, const trimul_layer_t *L,
                                 trimul_direction_t dir, trimul_pair_t *out, bool residual, void *ws_ptr,
-                                size_t ws_bytes, bool timing, void *stream, bool check_only) {
+                                size_t ws_bytes, bool timing, void *stream, bool check_only, const int *given_ext) {
     TRY(check_sizes(z));
     TRY(check_out(z, out));
     if (dir != TRIMUL_OUTGOING && dir != TRIMUL_INCOMING) return fail(TRIMUL_ERR_INVALID_ARG, "unknown direction");
@@ -705,14 +717,25 @@ trimul_status_t forward_buffers(const trimul_pair_t *z, const void *mask, const 
     void *a = ws, *b = ws + plane, *x = ws + 2 * plane;
     const bool tc = z->dtype == TRIMUL_BF16;
     uint8_t *aux = ws + 3 * plane;
-    // tensor-core path with a mask, skipping switched on: the mask's extents let the kernels
-    // leave out wholly masked tiles
-    int *ext = (tc && mask && L->skip_masked) ? reinterpret_cast<int *>(aux) : nullptr;
+    // tensor-core path with a mask: the mask's extents let the kernels leave out wholly masked
+    // tiles. They come from the caller (given_ext), from the layer's valid lengths when they fit
+    // this problem and the rule chose skipping, or, with mask skipping switched on, from a pass
+    // over the mask into the workspace.
+    const int *ext = nullptr;
     float *q = reinterpret_cast<float *>(aux + ws_ext_bytes(z->B));
-    if (ext)
-        TRY_CUDA(mask_extents_launch(reinterpret_cast<const uint16_t *>(mask), (int)z->B, (int)z->N,
-                                     host_rowdiv((uint64_t)z->N / 8), ext, st),
-                 "mask extents launch");
+    if (tc && mask) {
+        if (given_ext) {
+            ext = given_ext;
+        } else if (L->vl_ext && L->vl_B == z->B && L->vl_N == z->N) {
+            ext = L->vl_skip ? L->vl_ext : nullptr;
+        } else if (L->skip_masked) {
+            int *e = reinterpret_cast<int *>(aux);
+            TRY_CUDA(mask_extents_launch(reinterpret_cast<const uint16_t *>(mask), (int)z->B, (int)z->N,
+                                         host_rowdiv((uint64_t)z->N / 8), e, st),
+                     "mask extents launch");
+            ext = e;
+        }
+    }
     timing = timing && L->timing;
     if (timing) TRY_CUDA(cudaEventRecord(L->events[0], st), "event record");
     TRY(project_impl(z, mask, L, a, b, ext, tc ? L->acc : nullptr, stream));
@@ -731,7 +754,8 @@ trimul_status_t forward_buffers(const trimul_pair_t *z, const void *mask, const 
 
 static trimul_status_t forward_impl(const trimul_pair_t *z, const void *mask, const trimul_layer_t *L,
                                     trimul_direction_t dir, trimul_pair_t *out, bool residual, void *stream) {
-    return forward_buffers(z, mask, L, dir, out, residual, L ? L->ws : nullptr, L ? L->ws_bytes : 0, true, stream, false);
+    return forward_buffers(z, mask, L, dir, out, residual, L ? L->ws : nullptr, L ? L->ws_bytes : 0, true, stream, false,
+                           nullptr);
 }
 
 extern "C" trimul_status_t tri_mul_forward(const trimul_pair_t *z, const void *mask, const trimul_layer_t *L,
@@ -927,8 +951,95 @@ extern "C" trimul_status_t tri_mul_pair_update(const trimul_pair_t *z, const voi
                                                const trimul_layer_t *Li, trimul_pair_t *z_mid, trimul_pair_t *out,
                                                void *stream) {
     TRY(check_pair_update(z, Lo, Li, z_mid, out));
-    TRY(forward_impl(z, mask, Lo, TRIMUL_OUTGOING, z_mid, true, stream));
-    return forward_impl(z_mid, mask, Li, TRIMUL_INCOMING, out, true, stream);
+    // with mask skipping on and no valid lengths set, one pass over the (shared) mask serves both
+    // updates: its extents go to the first layer's workspace and both forwards read them there
+    const int *ext = nullptr;
+    const bool lengths = Lo->vl_ext && Lo->vl_B == z->B && Lo->vl_N == z->N;
+    if (z->dtype == TRIMUL_BF16 && mask && Lo->skip_masked && !lengths) {
+        TRY(forward_buffers(z, mask, Lo, TRIMUL_OUTGOING, z_mid, true, Lo->ws, Lo->ws_bytes, false, stream, true, nullptr));
+        if (!aligned16(mask)) return fail(TRIMUL_ERR_ALIGNMENT, "mask pointer not 16-byte aligned");
+        int *e = reinterpret_cast<int *>(reinterpret_cast<uint8_t *>(Lo->ws) + 3 * ws_plane_bytes(z->B, z->N, Lo->c_h, z->dtype));
+        TRY_CUDA(mask_extents_launch(reinterpret_cast<const uint16_t *>(mask), (int)z->B, (int)z->N,
+                                     host_rowdiv((uint64_t)z->N / 8), e, reinterpret_cast<cudaStream_t>(stream)),
+                 "mask extents launch");
+        ext = e;
+    }
+    TRY(forward_buffers(z, mask, Lo, TRIMUL_OUTGOING, z_mid, true, Lo->ws, Lo->ws_bytes, true, stream, false, ext));
+    return forward_buffers(z_mid, mask, Li, TRIMUL_INCOMING, out, true, Li->ws, Li->ws_bytes, true, stream, false,
+                           Li->skip_masked || Li == Lo ? ext : nullptr);
+}
+
+// ------------------------------------------------------------------ mask extents and valid lengths
+
+extern "C" trimul_status_t tri_mul_mask_extents(const void *mask, int64_t B, int64_t N, trimul_dtype_t dtype,
+                                                int32_t *extents, void *stream) {
+    if (!mask || !extents) return fail(TRIMUL_ERR_INVALID_ARG, "mask / extents NULL");
+    if (dtype != TRIMUL_BF16) return fail(TRIMUL_ERR_UNSUPPORTED_SHAPE, "extents are found for bf16 masks");
+    if (B < 1 || N < 8 || N % 8 || N > 16384) return fail(TRIMUL_ERR_UNSUPPORTED_SHAPE, "N=%lld must be a multiple of 8 in [8, 16384]", (long long)N);
+    if (!aligned16(mask) || !aligned16(extents)) return fail(TRIMUL_ERR_ALIGNMENT, "mask / extents not 16-byte aligned");
+    DeviceInfo d;
+    TRY(require_sm100(&d));
+    TRY_CUDA(mask_extents_launch(reinterpret_cast<const uint16_t *>(mask), (int)B, (int)N, host_rowdiv((uint64_t)N / 8),
+                                 reinterpret_cast<int *>(extents), reinterpret_cast<cudaStream_t>(stream)),
+             "mask extents launch");
+    return TRIMUL_OK;
+}
+
+extern "C" trimul_status_t tri_mul_forward_extents(const trimul_pair_t *z, const void *mask, const int32_t *extents,
+                                                   const trimul_layer_t *L, trimul_direction_t dir, trimul_pair_t *out,
+                                                   void *stream) {
+    if (!mask || !extents) return fail(TRIMUL_ERR_INVALID_ARG, "mask / extents NULL");
+    if (!aligned16(extents)) return fail(TRIMUL_ERR_ALIGNMENT, "extents not 16-byte aligned");
+    if (z && z->dtype != TRIMUL_BF16) return fail(TRIMUL_ERR_UNSUPPORTED_SHAPE, "extents are used on the bf16 path");
+    return forward_buffers(z, mask, L, dir, out, false, L ? L->ws : nullptr, L ? L->ws_bytes : 0, true, stream, false,
+                           reinterpret_cast<const int *>(extents));
+}
+
+// The share of one layer's dense work (its flops at N) that skipping by the valid lengths leaves
+// out: K1 and K3 scale with the valid pairs (L_b^2), K2 with L_b^3.
+extern "C" double tri_mul_skip_saving(const int64_t *lengths, int64_t B, int64_t N, int32_t c_z, int32_t c_h) {
+    if (!lengths || B < 1 || N < 1 || c_z < 1 || c_h < 1) return 0.0;
+    const double n = (double)N;
+    const double dense_pairs = 2.0 * c_z * 4.0 * c_h + 2.0 * c_z * (c_z + c_h);   // K1 + K3 per pair
+    double dense = 0.0, kept = 0.0;
+    for (int64_t b = 0; b < B; ++b) {
+        const double l = (double)(lengths[b] < 0 ? 0 : (lengths[b] > N ? N : lengths[b]));
+        dense += n * n * dense_pairs + 2.0 * c_h * n * n * n;
+        kept += l * l * dense_pairs + 2.0 * c_h * l * l * l;
+    }
+    return dense > 0.0 ? 1.0 - kept / dense : 0.0;
+}
+
+extern "C" trimul_status_t tri_mul_layer_set_valid_lengths(trimul_layer_t *L, const int64_t *lengths, int64_t B,
+                                                           int64_t N, int32_t *skipping_out) {
+    if (!L) return fail(TRIMUL_ERR_INVALID_ARG, "layer is NULL");
+    if (skipping_out) *skipping_out = 0;
+    if (!lengths) {                          // clear
+        L->vl_B = L->vl_N = 0;
+        L->vl_skip = false;
+        return TRIMUL_OK;
+    }
+    if (B < 1 || N < 8 || N % 8 || N > 16384 || B * L->c_h > 65535)
+        return fail(TRIMUL_ERR_UNSUPPORTED_SHAPE, "B=%lld N=%lld outside the supported sizes", (long long)B, (long long)N);
+    for (int64_t b = 0; b < B; ++b)
+        if (lengths[b] < 0 || lengths[b] > N) return fail(TRIMUL_ERR_INVALID_ARG, "length %lld of batch element %lld outside [0, N]",
+                                                          (long long)lengths[b], (long long)b);
+    if (L->vl_ext && L->vl_B < B) {
+        cudaFree(L->vl_ext);
+        L->vl_ext = nullptr;
+    }
+    if (!L->vl_ext) TRY_CUDA(cudaMalloc(&L->vl_ext, (size_t)B * 2 * sizeof(int)), "cudaMalloc(valid lengths)");
+    int *host = new (std::nothrow) int[2 * B];
+    if (!host) return fail(TRIMUL_ERR_INVALID_ARG, "out of host memory");
+    for (int64_t b = 0; b < B; ++b) host[2 * b] = host[2 * b + 1] = (int)lengths[b];
+    cudaError_t e = cudaMemcpy(L->vl_ext, host, (size_t)B * 2 * sizeof(int), cudaMemcpyHostToDevice);
+    delete[] host;
+    TRY_CUDA(e, "copy valid lengths");
+    L->vl_B = B;
+    L->vl_N = N;
+    L->vl_skip = tri_mul_skip_saving(lengths, B, N, L->c_z, L->c_h) >= kSkipRule;
+    if (skipping_out) *skipping_out = L->vl_skip ? 1 : 0;
+    return TRIMUL_OK;
 }
 
 struct trimul_graph {

@@ -105,6 +105,11 @@ def load_library():
         lib.tri_mul_shard_workspace_bytes.restype = ctypes.c_size_t
         lib.tri_mul_shard_project.argtypes = [P(_Rows), vp, vp, vp, vp, vp]
         lib.tri_mul_shard_finish.argtypes = [P(_Rows), vp, vp, st, st, P(i64), P(vp), P(vp), P(_Rows), vp]
+        lib.tri_mul_mask_extents.argtypes = [vp, i64, i64, st, vp, vp]
+        lib.tri_mul_forward_extents.argtypes = [P(_Pair), vp, vp, vp, st, P(_Pair), vp]
+        lib.tri_mul_skip_saving.argtypes = [P(i64), i64, i64, ctypes.c_int32, ctypes.c_int32]
+        lib.tri_mul_skip_saving.restype = ctypes.c_double
+        lib.tri_mul_layer_set_valid_lengths.argtypes = [vp, P(i64), i64, i64, P(ctypes.c_int32)]
         lib.tri_mul_kernels_per_forward.argtypes = []
         lib.tri_mul_check_device_status.argtypes = []
         lib.tri_mul_status_string.argtypes = [st]
@@ -117,7 +122,8 @@ def load_library():
                      "tri_mul_graph_launch", "tri_mul_layer_set_mask_skipping", "tri_mul_transition_create",
                      "tri_mul_transition_forward",
                      "tri_mul_project", "tri_mul_contract", "tri_mul_output_gate",
-                     "tri_mul_shard_project", "tri_mul_shard_finish",
+                     "tri_mul_shard_project", "tri_mul_shard_finish", "tri_mul_mask_extents",
+                     "tri_mul_forward_extents", "tri_mul_layer_set_valid_lengths",
                      "tri_mul_layer_set_timing_events", "tri_mul_check_device_status"):
             getattr(lib, name).restype = ctypes.c_int
         _lib = lib
@@ -256,6 +262,31 @@ class TriMulLayer:
     def set_mask_skipping(self, enable: bool = True):
         """Leave out wholly masked tiles (mask extents found by a first pass); off by default."""
         _check(self._lib.tri_mul_layer_set_mask_skipping(self.handle, 1 if enable else 0))
+
+    def set_valid_lengths(self, lengths, N: int | None = None) -> bool:
+        """Valid lengths of a left-aligned padding mask, one per batch element, for every later
+        forward of len(lengths) x N problems (None clears). Returns whether skipping was chosen."""
+        if lengths is None:
+            _check(self._lib.tri_mul_layer_set_valid_lengths(self.handle, None, 0, 0, None))
+            return False
+        arr = (ctypes.c_int64 * len(lengths))(*[int(v) for v in lengths])
+        chosen = ctypes.c_int32(0)
+        _check(self._lib.tri_mul_layer_set_valid_lengths(self.handle, arr, len(lengths), N, ctypes.byref(chosen)))
+        return bool(chosen.value)
+
+    def forward_extents(self, z: torch.Tensor, mask: torch.Tensor, extents: torch.Tensor, direction="outgoing",
+                        out: torch.Tensor | None = None, out_dtype: torch.dtype | None = None, stream=None):
+        """The update with the mask's extents given (int32 [B, 2] CUDA tensor, e.g. mask_extents())."""
+        B, N = z.shape[0], z.shape[1]
+        self.ensure_workspace(B, N, z.dtype)
+        if extents.dtype != torch.int32 or tuple(extents.shape) != (B, 2) or not extents.is_contiguous():
+            raise ValueError("extents must be a contiguous int32 [B, 2] tensor")
+        if out is None:
+            out = torch.empty(z.shape, dtype=out_dtype or torch.float32, device=z.device)
+        zp, op = _pair(z), _pair(out)
+        _check(self._lib.tri_mul_forward_extents(ctypes.byref(zp), _mask_ptr(mask, z), extents.data_ptr(), self.handle,
+                                                 _DIRS[direction], ctypes.byref(op), _stream_ptr(stream)))
+        return out
 
     def set_timing_events(self, events):
         """events: four torch.cuda.Event(enable_timing=True) or None."""
@@ -462,6 +493,22 @@ class PairUpdateGraph:
             self.close()
         except Exception:
             pass
+
+
+def mask_extents(mask: torch.Tensor, stream=None) -> torch.Tensor:
+    """{R_b, C_b} of a bfloat16 [B, N, N] mask: int32 [B, 2] on its device."""
+    if mask.dtype != torch.bfloat16 or mask.dim() != 3 or not mask.is_contiguous():
+        raise ValueError("mask must be a contiguous bfloat16 [B, N, N] tensor")
+    ext = torch.empty((mask.shape[0], 2), dtype=torch.int32, device=mask.device)
+    _check(load_library().tri_mul_mask_extents(mask.data_ptr(), mask.shape[0], mask.shape[1], BF16, ext.data_ptr(),
+                                               _stream_ptr(stream)))
+    return ext
+
+
+def skip_saving(lengths, N: int, c_z: int = 128, c_h: int = 128) -> float:
+    """The share of a layer's dense work that skipping by these valid lengths leaves out."""
+    arr = (ctypes.c_int64 * len(lengths))(*[int(v) for v in lengths])
+    return float(load_library().tri_mul_skip_saving(arr, len(lengths), N, c_z, c_h))
 
 
 def check_device_status():

@@ -49,7 +49,7 @@ def test_status_strings_and_versions(lib):
     for code in range(9):
         assert lib.tri_mul_status_string(code)
     assert lib.tri_mul_status_string(99) == b"unknown status"
-    assert lib.tri_mul_abi_version() == 102
+    assert lib.tri_mul_abi_version() == 103
     assert lib.tri_mul_kernels_per_forward() == 4
 
 
@@ -191,3 +191,20 @@ def test_forward_and_noalloc_check_out_before_the_layer_and_the_device(lib):
         good = tm._Pair(1 << 32, 1, 64, 128, tm.F32)
         assert entry(ctypes.byref(z), None, None, 0, ctypes.byref(good), None) == 1
         assert b"layer is NULL" in lib.tri_mul_last_error()
+
+
+def test_skip_rule_and_valid_length_validation(lib):
+    """The skipping rule's measure (host only): no saving at full length, all of it at zero
+    length, K2's cubic share in between; the headline's 493 of 512 stays under the 0.15 rule,
+    the c_z = 384 workload's lengths (162-237 of 256) are over it."""
+    assert tm.skip_saving([512], 512) == 0.0
+    assert tm.skip_saving([0, 0], 64) == 1.0
+    half = tm.skip_saving([128], 256)
+    assert 0.75 < half < 0.875                    # between 1 - 1/4 (pairs) and 1 - 1/8 (cube)
+    assert tm.skip_saving([493], 512) < 0.15
+    assert tm.skip_saving([237, 210, 193, 162], 256, 384, 128) > 0.15
+    assert lib.tri_mul_layer_set_valid_lengths(None, None, 0, 0, None) == 1
+    assert lib.tri_mul_forward_extents(None, None, None, None, 0, None, None) == 1
+    fake = ctypes.c_void_p(1 << 24)
+    assert lib.tri_mul_mask_extents(fake, 1, 12, tm.BF16, fake, None) == 2
+    assert lib.tri_mul_mask_extents(fake, 1, 16, tm.F32, fake, None) == 2

@@ -65,3 +65,56 @@ def test_all_masked_element_next_to_a_full_one():
         tm.check_device_status()
         assert not torch.any(got[0])
         assert torch.isfinite(got[1]).all()
+
+
+def test_mask_extents_values():
+    m = _holey_mask(136, 100, 60, seed=1)
+    m = np.concatenate([m, np.zeros((1, 136, 136), np.float32)])       # a third element fully masked
+    mt = torch.from_numpy(m).cuda().to(torch.bfloat16)
+    ext = tm.mask_extents(mt).cpu().numpy()
+    for b in range(3):
+        rows = np.nonzero(m[b].any(axis=1))[0]
+        cols = np.nonzero(m[b].any(axis=0))[0]
+        assert ext[b, 0] == (rows.max() + 1 if rows.size else 0)
+        assert ext[b, 1] == (cols.max() + 1 if cols.size else 0)
+
+
+@pytest.mark.parametrize("c_z", [128, 384])
+def test_given_extents_and_valid_lengths_match_the_dense_forward_bitwise(c_z):
+    lengths = [237, 210, 193, 162] if c_z == 384 else [200, 256, 90, 131]
+    inp = ti.generate(4, 256, c_z, 128, dtype="bf16", seed=c_z + 2, mask=("lengths", lengths), biases=True)
+    z, m, w = upload(inp)
+    dense = tm.TriMulLayer(w, eps=inp.eps)
+    layer = tm.TriMulLayer(w, eps=inp.eps)
+    ext = tm.mask_extents(m)
+    assert ext.cpu().numpy().tolist() == [[L, L] for L in lengths]
+    assert layer.set_valid_lengths(lengths, 256) is (tm.skip_saving(lengths, 256, c_z, 128) >= 0.15)
+    for d in ("outgoing", "incoming"):
+        ref = dense.forward(z, m, d)
+        got_ext = layer.forward_extents(z, m, ext, d)
+        got_len = layer.forward(z, m, d)
+        torch.cuda.synchronize()
+        tm.check_device_status()
+        assert torch.equal(ref, got_ext), d
+        assert torch.equal(ref, got_len), d
+    layer.set_valid_lengths(None)
+
+
+def test_headline_lengths_do_not_choose_skipping():
+    layer_inp = ti.generate(1, 512, 128, 128, dtype="bf16", seed=0, mask=("lengths", [493]))
+    z, m, w = upload(layer_inp)
+    layer = tm.TriMulLayer(w, eps=layer_inp.eps)
+    assert layer.set_valid_lengths([493], 512) is False
+
+
+def test_pair_update_finds_the_extents_once_and_matches_dense():
+    inp = ti.generate(2, 256, 128, 128, dtype="bf16", seed=12, mask=("lengths", [150, 256]), biases=True)
+    z, m, w = upload(inp)
+    dense = tm.TriMulLayer(w, eps=inp.eps)
+    skip = tm.TriMulLayer(w, eps=inp.eps)
+    skip.set_mask_skipping(True)
+    ref = tm.pair_update(z, m, dense, dense, out_dtype=torch.float32)
+    got = tm.pair_update(z, m, skip, skip, out_dtype=torch.float32)
+    torch.cuda.synchronize()
+    tm.check_device_status()
+    assert torch.equal(ref, got)
