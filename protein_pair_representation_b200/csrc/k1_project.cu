@@ -387,9 +387,9 @@ __global__ void __launch_bounds__(448, 1) k1_project_kernel(const __grid_constan
 // Two teams of eight epilogue warps take alternate tiles, each team with its own TMEM buffer of
 // the four accumulators (256 columns), so the MMA of a tile never waits for the other team;
 // sixteen epilogue warps (four per scheduler) hide the latency of TMEM loads and of the gate
-// arithmetic, and a four-stage z ring covers the HBM latency. (A design with 128-pair tiles,
-// N = 128 and one single-buffered TMEM region per operand, drained by eight warps, read the
-// weights half as often but ran 7% slower at N = 512: its epilogue was latency-bound.)
+// arithmetic. (A design with 128-pair tiles, N = 128 and one single-buffered TMEM region per
+// operand, drained by eight warps, read the weights half as often but ran 7% slower at N = 512:
+// its epilogue was latency-bound.)
 // A thread of the epilogue owns one channel of one operand for the whole kernel, so that
 // channel's four folding constants stay in registers; the per-pair LayerNorm statistics are
 // read from shared memory (broadcast); consecutive pairs of one channel are consecutive TMEM
@@ -402,18 +402,21 @@ __global__ void __launch_bounds__(448, 1) k1_project_kernel(const __grid_constan
 // converted, tanh in halves, products rounded) took about twice as many. The TMEM loads of each
 // 8-pair step are issued one step ahead. The channel sums behind the offset of the stored x are
 // taken over the first 8 pairs of each tile (an estimate needs no more).
+// Each epilogue warp stores its [32 channels][64 pairs] block of a tile with one TMA store, so
+// every channel row is written in 128-byte segments: with 64-byte segments (two stores per tile
+// from a 2 KB buffer) K1 at N = 2048, whose a and b cannot stay in L2, took 29% longer, and with
+// 32-byte ones twice as long. The 4 KB blocks leave room for a two-tile z ring.
 // Warps: 0-15 epilogue (team t = warp / 8; warp 4o + q of a team: operand o, channels
-// [32q, 32q + 32), the tile's 64 pairs in two store blocks of 32), 16-17 LayerNorm statistics,
-// 18 TMA producer, 19 TMEM allocator + MMA issuer.
+// [32q, 32q + 32)), 16-17 LayerNorm statistics, 18 TMA producer, 19 TMEM allocator + MMA issuer.
 struct K1TmCfg {
     static constexpr int CZ = 128, C_H = kHidden, TP = 64;
     static constexpr int W_CHUNK = 4 * C_H * 64 * 2;
     static constexpr int W_BYTES = (CZ / 64) * W_CHUNK;        // 128 KB
     static constexpr int TILE = TP * CZ * 2;                   // 16 KB: [2 halves][64 pairs][64 ch]
     static constexpr int HALF = TP * 128;
-    static constexpr int WARP_STG = 32 * 32 * 2;
+    static constexpr int WARP_STG = 32 * TP * 2;                // one [32 channels][64 pairs] block
     static constexpr int EPI_WARPS = 16;
-    static constexpr int STG_TOTAL = EPI_WARPS * WARP_STG;     // 32 KB
+    static constexpr int STG_TOTAL = EPI_WARPS * WARP_STG;     // 64 KB
     static constexpr int STATS_WARP0 = 16, STATS_WARPS = TP / 32;
     static constexpr int TMA_WARP = 18, MMA_WARP = 19;
     static constexpr int THREADS = 20 * 32;
@@ -427,7 +430,7 @@ template <bool SKIP>
 __global__ void __launch_bounds__(K1TmCfg::THREADS, 1) k1_project_tm_kernel(const __grid_constant__ K1Args p) {
     using C = K1TmCfg;
     static_assert(sizeof(K1Smem) <= 512, "barrier block");
-    static_assert(C::S >= 3, "z ring");
+    static_assert(C::S >= 2, "z ring");
     extern __shared__ uint8_t smem_raw[];
     uint8_t *base = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint8_t *w_s = base;
@@ -618,18 +621,15 @@ __global__ void __launch_bounds__(K1TmCfg::THREADS, 1) k1_project_tm_kernel(cons
                 run = make_float2(0.f, 0.f);
             }
             if (SKIP && tile_masked_out<C::TP>(p.ext, b, p0, p.N, p.NN, p.rowdiv)) {
-#pragma unroll 1
-                for (int blk = 0; blk < C::TP / 32; ++blk) {
-                    if (lane == 0) tma_store_wait_read<0>();
-                    __syncwarp();
+                if (lane == 0) tma_store_wait_read<0>();
+                __syncwarp();
 #pragma unroll
-                    for (int u = 0; u < 4; ++u) *reinterpret_cast<uint4 *>(stg + sw64_offset(lane, u)) = make_uint4(0, 0, 0, 0);
-                    fence_proxy_async_smem();
-                    __syncwarp();
-                    if (lane == 0) {
-                        tma_store_3d(tm_out, stg, p0 + 32 * blk, q * 32, b);
-                        tma_store_commit();
-                    }
+                for (int u = 0; u < 8; ++u) *reinterpret_cast<uint4 *>(stg + sw128_offset(lane, u)) = make_uint4(0, 0, 0, 0);
+                fence_proxy_async_smem();
+                __syncwarp();
+                if (lane == 0) {
+                    tma_store_3d(tm_out, stg, p0, q * 32, b);
+                    tma_store_commit();
                 }
                 continue;
             }
@@ -638,15 +638,15 @@ __global__ void __launch_bounds__(K1TmCfg::THREADS, 1) k1_project_tm_kernel(cons
                 break;
             phase ^= 1;
             tc_fence_after();
-            // 8-pair steps it = 0 .. 7 (store block it / 4); step it + 1's TMEM loads are issued
-            // before step it's arithmetic
+            // 8-pair steps it = 0 .. 7, each writing 16 bytes of every channel row of the tile's
+            // store block; step it + 1's TMEM loads are issued before step it's arithmetic
             constexpr int NIT = C::TP / 8;
             float g0[8], p0v[8], g1[8], p1v[8];
             tmem_ld8(tbase, g0);
             tmem_ld8(tbase + C::TP, p0v);
             auto step = [&](const int it, float (&gc)[8], float (&pc)[8], float (&gn)[8], float (&pn)[8]) {
-                const int blk = it >> 2, part = it & 3, o = 8 * it;
-                if (part == 0) {
+                const int o = 8 * it;
+                if (it == 0) {          // the store of this team's previous tile has read the block
                     if (lane == 0) tma_store_wait_read<0>();
                     __syncwarp();
                 }
@@ -678,18 +678,18 @@ __global__ void __launch_bounds__(K1TmCfg::THREADS, 1) k1_project_tm_kernel(cons
                         if (it == 0) run = f2_add(run, av);    // the sampled pairs: the tile's first 8
                     }
                 }
-                *reinterpret_cast<uint4 *>(stg + sw64_offset(lane, part)) = make_uint4(outw[0], outw[1], outw[2], outw[3]);
-                if (part == 3) {
+                *reinterpret_cast<uint4 *>(stg + sw128_offset(lane, it)) = make_uint4(outw[0], outw[1], outw[2], outw[3]);
+                if (it == NIT - 1) {
                     fence_proxy_async_smem();
                     __syncwarp();
                     if (lane == 0) {
-                        if (blk == C::TP / 32 - 1) mbar_arrive(&s.sempty[buf]);
-                        tma_store_3d(tm_out, stg, p0 + 32 * blk, q * 32, b);
+                        mbar_arrive(&s.sempty[buf]);
+                        tma_store_3d(tm_out, stg, p0, q * 32, b);
                         tma_store_commit();
                     }
                 }
             };
-#pragma unroll 1
+#pragma unroll
             for (int it = 0; it < NIT; it += 2) {
                 step(it, g0, p0v, g1, p1v);
                 step(it + 1, g1, p1v, g0, p0v);

@@ -459,12 +459,12 @@ static trimul_status_t run_project_bf16(const trimul_layer_t *L, const void *z, 
     {
         uint64_t dims[3] = {NN, (uint64_t)ch, (uint64_t)B};
         uint64_t strides[2] = {NN * 2, (uint64_t)ch * NN * 2};
-        // c_z = 128: each warp of the channel-lane kernel stores a [32 channels][32 pairs] block
-        // through a 64B swizzle; c_z = 384: pair-lane kernel stores [channels][128 pairs] rows
+        // c_z = 128: each warp of the channel-lane kernel stores a [32 channels][64 pairs] block
+        // through a 128B swizzle; c_z = 384: pair-lane kernel stores [channels][128 pairs] rows
         // without swizzle
         const bool cm = k1_row_mode(cz) == 2;
-        uint32_t box[3] = {cm ? 32u : 128u, cm ? 32u : (uint32_t)k1_channels_per_warpgroup(cz), 1};
-        const CUtensorMapSwizzle sw = cm ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_NONE;
+        uint32_t box[3] = {cm ? 64u : 128u, cm ? 32u : (uint32_t)k1_channels_per_warpgroup(cz), 1};
+        const CUtensorMapSwizzle sw = cm ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE;
         TRY(make_map(&p.tm_a, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 3, a, dims, strides, box, sw, "K1 a"));
         TRY(make_map(&p.tm_b, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 3, b, dims, strides, box, sw, "K1 b"));
     }

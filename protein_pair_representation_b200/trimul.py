@@ -313,11 +313,16 @@ class TriMulLayer:
 
     __call__ = forward
 
-    def project(self, z: torch.Tensor, mask: torch.Tensor | None = None, stream=None):
-        """K1 alone: a, b as [B, c_h, N, N] in the intermediate dtype."""
+    def project(self, z: torch.Tensor, mask: torch.Tensor | None = None, stream=None,
+                a: torch.Tensor | None = None, b: torch.Tensor | None = None):
+        """K1 alone: a, b as [B, c_h, N, N] in the intermediate dtype (into `a`, `b` when given)."""
         B, N = z.shape[0], z.shape[1]
-        a = torch.empty((B, self.c_h, N, N), dtype=intermediate_dtype(z.dtype), device=z.device)
-        b = torch.empty_like(a)
+        shape, dt = (B, self.c_h, N, N), intermediate_dtype(z.dtype)
+        for t in (a, b):
+            if t is not None and (tuple(t.shape) != shape or t.dtype != dt or not t.is_contiguous()):
+                raise ValueError(f"a and b must be contiguous {shape} tensors of {dt}")
+        a = torch.empty(shape, dtype=dt, device=z.device) if a is None else a
+        b = torch.empty_like(a) if b is None else b
         zp = _pair(z)
         _check(self._lib.tri_mul_project(ctypes.byref(zp), _mask_ptr(mask, z), self.handle,
                                          a.data_ptr(), b.data_ptr(), _stream_ptr(stream)))
