@@ -507,6 +507,22 @@ def time_steps(wl, steps, first, sync_all, dist=None, dev=None, instrumented=Fal
     return elapsed, kernel_ms
 
 
+def valid_length_pass(tm, wl, steps, sync_all):
+    """The headline steps with the layer told the mask's valid lengths: the library's rule
+    decides whether skipping pays (it does when it leaves out at least 15% of the dense
+    flops); ms per layer and that decision."""
+    lengths = [int(v) for v in wl.inp.lengths]
+    chosen = wl.layer.set_valid_lengths(lengths, wl.inp.N)
+    try:
+        for s in range(3):
+            wl.step(s)
+        el, _ = time_steps(wl, steps, 0, sync_all)
+    finally:
+        wl.layer.set_valid_lengths(None)
+    return {"ms_per_layer": el / (steps * len(wl.dirs)), "skipping_chosen": chosen,
+            "dense_share_left_out": tm.skip_saving(lengths, wl.inp.N, wl.inp.c_z, wl.inp.c_h)}
+
+
 def stage_times(tm, wl, steps, sync_all):
     """Each kernel alone: `steps` back-to-back launches of its stage entry point (K1
     tri_mul_project, K2 tri_mul_contract in both directions in turn, K3 tri_mul_output_gate)
@@ -634,6 +650,8 @@ def run_ours(args):
     # each kernel alone, back to back through its stage entry point
     kernel_ms = stage_times(tm, wl, args.steps, sync_all)
     tm.check_device_status()
+    vl = None if args.skip_masked else valid_length_pass(tm, wl, args.steps, sync_all)
+    tm.check_device_status()
 
     # host-buffer end to end: pinned inputs in, results out, every step
     e2e = None
@@ -684,10 +702,12 @@ def run_ours(args):
                 w_el, _ = time_steps(other, args.steps, 0, sync_all)
                 w_iel, w_kms = time_steps(other, args.steps, args.steps, sync_all, instrumented=True)
                 w_alone = stage_times(tm, other, args.steps, sync_all)
+                w_vl = None if args.skip_masked else valid_length_pass(tm, other, args.steps, sync_all)
                 w_clock_info = w_clocks.stop()
                 tm.check_device_status()
                 n_layers = args.steps * len(other.dirs)
                 workloads[name] = workload_summary(other, w_el / n_layers, w_alone, w_iel / n_layers, peaks, w_kms)
+                workloads[name]["valid_lengths"] = w_vl
                 workloads[name]["clocks"] = w_clock_info
                 del other
                 torch.cuda.empty_cache()
@@ -746,6 +766,7 @@ def run_ours(args):
         "layer_roofline_frac": t_ideal / (layer_ms_single * 1e-3),
         "ms_per_layer_instrumented": instr_elapsed / n_layers,
         "kernels_alone_sum_ms": sum(kernel_ms.values()),
+        "valid_lengths": vl,
         "roofline": roof, "kernels": kernels, "cpu_baseline": cpu, "e2e": e2e, "pair_update": pair,
         "pair_transition": trans, "torch_composition": context, "workloads": workloads,
         "gpu_launches": args.steps * len(dirs) * launches_per_forward,

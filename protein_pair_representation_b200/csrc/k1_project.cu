@@ -75,7 +75,8 @@ struct K1Cfg {
     static constexpr int CHUNK = 128 * 64 * 2;         // one z chunk: 128 pairs x 64 channels
     static constexpr int STG_BYTES = CH_WG * 128 * 2;  // per warpgroup: [channels][128 pairs] bf16
     static constexpr int SNB = 2;                      // stats ring depth
-    static constexpr int FIXED = 1024 + W_BYTES + 2 * STG_BYTES + SNB * 128 * 16 + 1024;
+    static constexpr int CONST_BYTES = CPG * 16;        // folding constants of the group's channels
+    static constexpr int FIXED = 1024 + W_BYTES + 2 * STG_BYTES + SNB * 128 * 16 + CONST_BYTES + 1024;
     static constexpr int S = (232448 - FIXED) / CHUNK > 8 ? 8 : (232448 - FIXED) / CHUNK;
     static constexpr size_t SMEM = FIXED + (size_t)S * CHUNK;
     static constexpr int THREADS = 448;
@@ -103,7 +104,10 @@ __global__ void __launch_bounds__(448, 1) k1_project_kernel(const __grid_constan
     uint8_t *chunks = w_s + C::W_BYTES;                    // S chunks of [128][64] bf16
     uint8_t *staging = chunks + C::S * C::CHUNK;           // 2 x [CH_WG][128] bf16
     float4 *stats = reinterpret_cast<float4 *>(staging + 2 * C::STG_BYTES);  // [SNB][128]
-    K1Smem &s = *reinterpret_cast<K1Smem *>(stats + C::SNB * 128);
+    // the group's folding constants by channel pair k (channels 2k, 2k + 1): [k][0] = gate sums and
+    // shifts {sg0, sg1, hg0, hg1}, [k][1] = projection sums and shifts
+    float4 *cpair = stats + C::SNB * 128;
+    K1Smem &s = *reinterpret_cast<K1Smem *>(cpair + C::CPG);
 
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
@@ -137,6 +141,12 @@ __global__ void __launch_bounds__(448, 1) k1_project_kernel(const __grid_constan
     if (warp == C::MMA_WARP) {
         tmem_alloc(&s.tmem_base, 512);
         tmem_relinquish();
+    }
+    if ((int)threadIdx.x < C::CPG / 2) {
+        const float4 *v = p.vec + operand * C::C_H + ch0 + 2 * threadIdx.x;
+        const float4 v0 = v[0], v1 = v[1];
+        cpair[2 * threadIdx.x] = make_float4(v0.x, v1.x, v0.y, v1.y);
+        cpair[2 * threadIdx.x + 1] = make_float4(v0.z, v1.z, v0.w, v1.w);
     }
     tc_fence_before();
     __syncthreads();
@@ -269,7 +279,7 @@ __global__ void __launch_bounds__(448, 1) k1_project_kernel(const __grid_constan
             if (p.mask && pi < p.NN) m = __uint_as_float((uint32_t)p.mask[(long long)b * p.NN + pi] << 16);
             if (counting) counts.add(p.acc, b, m != 0.f, row < 16, pi % p.N == 0, lane);
             if (!__all_sync(0xffffffffu, mbar_wait(&s.sempty[sbuf], sphase ^ 1, abort_flag, kErrTimeoutEpilogue))) break;
-            stats[sbuf * 128 + row] = make_float4(mean, rstd, m, 0.f);
+            stats[sbuf * 128 + row] = make_float4(-mean, rstd, 0.5f * m, 0.f);   // the form the epilogue uses
             __syncwarp();
             if (lane == 0) mbar_arrive(&s.sfull[sbuf]);
             if (++sbuf == C::SNB) { sbuf = 0; sphase ^= 1; }
@@ -283,7 +293,7 @@ __global__ void __launch_bounds__(448, 1) k1_project_kernel(const __grid_constan
         uint16_t *stg = reinterpret_cast<uint16_t *>(staging + wg * C::STG_BYTES);
         const bool leader = (threadIdx.x & 127) == 0;
         const CUtensorMap *tm_out = operand == 0 ? &p.tm_a : &p.tm_b;
-        const float4 *vec = p.vec + operand * C::C_H + ch0 + wg * C::CH_WG;
+        const float4 *cp = cpair + wg * C::CH_WG;       // this warpgroup's CH_WG / 2 channel pairs
         int abuf = 0;
         uint32_t aphase = 0;
         int sbuf = 0;
@@ -332,7 +342,8 @@ __global__ void __launch_bounds__(448, 1) k1_project_kernel(const __grid_constan
             __syncwarp();
             if (lane == 0) mbar_arrive(&s.sempty[sbuf]);
             if (++sbuf == C::SNB) { sbuf = 0; sphase ^= 1; }
-            const float mean = st.x, rstd = st.y, m = st.z;
+            const float2 nmean2 = make_float2(st.x, st.x), rstd2 = make_float2(st.y, st.y);
+            const float2 hm2 = make_float2(st.z, st.z);
 
             if (!group_all(mbar_wait(&s.tfull[abuf], aphase, abort_flag, kErrTimeoutEpilogue), 1 + wg, 128)) break;
             tc_fence_after();
@@ -343,14 +354,24 @@ __global__ void __launch_bounds__(448, 1) k1_project_kernel(const __grid_constan
                 float v[32];
                 tmem_ld32(tmem_base + abuf * C::NCOL + ((uint32_t)(q * 32) << 16) + (wg * C::BLK_WG + blk) * 32, v);
                 tc_wait_ld();
+                // channels e, e + 1 in packed pairs: the gate as (m/2) tanh(g/2) + m/2 (gate rows
+                // folded with an extra 1/2), times the projection, one f16x2 rounding
 #pragma unroll
-                for (int e = 0; e < 16; ++e) {
-                    const float4 cv = __ldg(&vec[blk * 16 + e]);
-                    const float g = fmaf(rstd, fmaf(-mean, cv.x, v[e]), cv.y);
-                    const float pr = fmaf(rstd, fmaf(-mean, cv.z, v[16 + e]), cv.w);
-                    const float out = sigmoid_tanh(g) * pr * m;
-                    stg[(blk * 16 + e) * 128 + row] = __half_as_ushort(__float2half_rn(out));
-                    if (row < 16) run[blk * 16 + e] += out;   // sampled pairs, unrounded: an estimate needs no more
+                for (int e = 0; e < 16; e += 2) {
+                    const float4 cg = cp[blk * 16 + e], cq = cp[blk * 16 + e + 1];
+                    const float2 gv = f2_fma(rstd2, f2_fma(nmean2, make_float2(cg.x, cg.y), make_float2(v[e], v[e + 1])),
+                                             make_float2(cg.z, cg.w));
+                    const float2 pv = f2_fma(rstd2, f2_fma(nmean2, make_float2(cq.x, cq.y), make_float2(v[16 + e], v[17 + e])),
+                                             make_float2(cq.z, cq.w));
+                    const float2 gm = f2_fma(make_float2(tanh_approx(gv.x), tanh_approx(gv.y)), hm2, hm2);
+                    const float2 av = f2_mul(gm, pv);
+                    const uint32_t h2 = pack_f16x2(av.x, av.y);
+                    stg[(blk * 16 + e) * 128 + row] = (uint16_t)(h2 & 0xFFFFu);
+                    stg[(blk * 16 + e + 1) * 128 + row] = (uint16_t)(h2 >> 16);
+                    if (row < 16) {            // sampled pairs, unrounded: an estimate needs no more
+                        run[blk * 16 + e] += av.x;
+                        run[blk * 16 + e + 1] += av.y;
+                    }
                 }
             }
             tc_fence_before();

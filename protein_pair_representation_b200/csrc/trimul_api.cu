@@ -323,9 +323,9 @@ extern "C" trimul_status_t tri_mul_layer_create(const trimul_weights_desc_t *w, 
                 fa.K = cz;
                 fa.dst = L->k1_w;
                 fa.row_mode = k1_row_mode(cz);
-                // the c_z = 128 kernel evaluates sigmoid(g) as 0.5 + 0.5 tanh(g / 2) and takes
-                // the gate rows pre-scaled by 1/2 (exact in bf16)
-                fa.scale = (fa.row_mode == 2 && kind == 0) ? 0.5f : 1.0f;
+                // both K1 kernels evaluate sigmoid(g) as 0.5 + 0.5 tanh(g / 2) and take the
+                // gate rows pre-scaled by 1/2 (exact in bf16)
+                fa.scale = kind == 0 ? 0.5f : 1.0f;
                 fa.operand = o;
                 fa.kind = kind;
                 fa.ncol = ncol;
