@@ -507,6 +507,27 @@ def time_steps(wl, steps, first, sync_all, dist=None, dev=None, instrumented=Fal
     return elapsed, kernel_ms
 
 
+def bf16_out_pass(tm, wl, steps, sync_all, peaks):
+    """The same steps with `out` in z's dtype (bf16) instead of fp32: ms per layer and K3 alone
+    with 2-byte output, and the layer's roofline fraction at those bytes. (The headline keeps fp32
+    out: a bf16 out alone rounds values near 10x RMS by up to half an ulp, about 0.03 RMS.)"""
+    import torch
+    saved, saved_bytes = wl.outs, wl.out_bytes
+    wl.outs = [torch.empty(wl.z0.shape, dtype=torch.bfloat16, device=wl.z0.device) for _ in wl.dirs]
+    wl.out_bytes = 2
+    try:
+        for s_ in range(3):
+            wl.step(s_)
+        el, _ = time_steps(wl, steps, 0, sync_all)
+        alone = stage_times(tm, wl, steps, sync_all)
+        kernels, _, t_ideal = kernel_record(wl.inp, alone, peaks, 2)
+        layer_ms = el / (steps * len(wl.dirs))
+        return {"ms_per_layer": layer_ms, "layer_roofline_frac": t_ideal / (layer_ms * 1e-3),
+                "k3_output_kernel": kernels["k3_output_kernel"]}
+    finally:
+        wl.outs, wl.out_bytes = saved, saved_bytes
+
+
 def valid_length_pass(tm, wl, steps, sync_all):
     """The headline steps with the layer told the mask's valid lengths: the library's rule
     decides whether skipping pays (it does when it leaves out at least 15% of the dense
@@ -652,6 +673,8 @@ def run_ours(args):
     tm.check_device_status()
     vl = None if args.skip_masked else valid_length_pass(tm, wl, args.steps, sync_all)
     tm.check_device_status()
+    out_bf16 = bf16_out_pass(tm, wl, args.steps, sync_all, measured_peaks()) if args.out_dtype == "f32" else None
+    tm.check_device_status()
 
     # host-buffer end to end: pinned inputs in, results out, every step
     e2e = None
@@ -767,6 +790,7 @@ def run_ours(args):
         "ms_per_layer_instrumented": instr_elapsed / n_layers,
         "kernels_alone_sum_ms": sum(kernel_ms.values()),
         "valid_lengths": vl,
+        "out_bf16": out_bf16,
         "roofline": roof, "kernels": kernels, "cpu_baseline": cpu, "e2e": e2e, "pair_update": pair,
         "pair_transition": trans, "torch_composition": context, "workloads": workloads,
         "gpu_launches": args.steps * len(dirs) * launches_per_forward,
