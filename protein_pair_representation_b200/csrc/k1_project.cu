@@ -413,7 +413,8 @@ __global__ void __launch_bounds__(448, 1) k1_project_kernel(const __grid_constan
 // its epilogue was latency-bound.)
 // A thread of the epilogue owns one channel of one operand for the whole kernel, so that
 // channel's four folding constants stay in registers; the per-pair LayerNorm statistics are
-// read from shared memory (broadcast); consecutive pairs of one channel are consecutive TMEM
+// read from shared memory (broadcast; mask / 2 as bf16, exact, so that one 16-byte load carries
+// a step's eight); consecutive pairs of one channel are consecutive TMEM
 // columns, which pack directly into 16-byte rows of the channel-major output tile.
 // The epilogue's arithmetic is fp32 in packed pairs (f32x2) up to one f16x2 rounding of the
 // result: the gate as (mask/2) tanh(g/2) + mask/2 with one tanh.approx.f32 per output (the gate
@@ -441,7 +442,7 @@ struct K1TmCfg {
     static constexpr int STATS_WARP0 = 16, STATS_WARPS = TP / 32;
     static constexpr int TMA_WARP = 18, MMA_WARP = 19;
     static constexpr int THREADS = 20 * 32;
-    static constexpr int STATS_BYTES = 2 * TP * 12;            // -mean, rstd, mask / 2 (f32)
+    static constexpr int STATS_BYTES = 2 * TP * 10;            // -mean, rstd (f32), mask / 2 (bf16)
     static constexpr int FIXED = 1024 + W_BYTES + STG_TOTAL + STATS_BYTES + 512;
     static constexpr int S = (232448 - FIXED) / TILE > 8 ? 8 : (232448 - FIXED) / TILE;
     static constexpr size_t SMEM = FIXED + (size_t)S * TILE;
@@ -459,8 +460,8 @@ __global__ void __launch_bounds__(K1TmCfg::THREADS, 1) k1_project_tm_kernel(cons
     uint8_t *staging = tiles + C::S * C::TILE;
     float *st_nmean = reinterpret_cast<float *>(staging + C::STG_TOTAL);   // [2][64]
     float *st_rstd = st_nmean + 2 * C::TP;
-    float *st_hmask = st_rstd + 2 * C::TP;
-    K1Smem &s = *reinterpret_cast<K1Smem *>(st_hmask + 2 * C::TP);
+    uint16_t *st_hmask = reinterpret_cast<uint16_t *>(st_rstd + 2 * C::TP);   // mask / 2 in bf16 (exact)
+    K1Smem &s = *reinterpret_cast<K1Smem *>(reinterpret_cast<uint8_t *>(st_hmask) + 2 * C::TP * 2);
 
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
@@ -532,13 +533,13 @@ __global__ void __launch_bounds__(K1TmCfg::THREADS, 1) k1_project_tm_kernel(cons
             bool ok = mbar_wait(&s.wbar, 0, abort_flag, kErrTimeoutMma);
             int stage = 0;
             uint32_t phase = 0;
-            uint32_t aphase[2] = {0, 0};
+            uint32_t aphase = 0;            // bit i: buffer i's phase
             int j = 0;
             TileWalk tw(blockIdx.x, p.tiles_per_batch);
             for (int t = blockIdx.x; ok && t < num_tiles; t += gridDim.x, tw.advance(gridDim.x, p.tiles_per_batch), ++j) {
                 if (SKIP && tile_masked_out<C::TP>(p.ext, tw.b, tw.t * C::TP, p.N, p.NN, p.rowdiv)) continue;
                 const int abuf = j & 1;
-                if (!mbar_wait(&s.tempty[abuf], aphase[abuf] ^ 1, abort_flag, kErrTimeoutMma)) break;
+                if (!mbar_wait(&s.tempty[abuf], ((aphase >> abuf) & 1u) ^ 1u, abort_flag, kErrTimeoutMma)) break;
                 if (!mbar_wait(&s.full[stage], phase, abort_flag, kErrTimeoutMma)) break;
                 tc_fence_after();
                 const uint8_t *zt = tiles + stage * C::TILE;
@@ -554,7 +555,7 @@ __global__ void __launch_bounds__(K1TmCfg::THREADS, 1) k1_project_tm_kernel(cons
                 tc_commit(&s.empty[stage]);
                 if (++stage == C::S) { stage = 0; phase ^= 1; }
                 tc_commit(&s.tfull[abuf]);
-                aphase[abuf] ^= 1;
+                aphase ^= 1u << abuf;
             }
             tc_commit(&s.drain);
             mbar_drain(&s.drain, 0);
@@ -563,7 +564,7 @@ __global__ void __launch_bounds__(K1TmCfg::THREADS, 1) k1_project_tm_kernel(cons
         const int row = (warp - C::STATS_WARP0) * 32 + lane;
         int stage = 0;
         uint32_t phase = 0;
-        uint32_t sphase[2] = {0, 0};
+        uint32_t sphase = 0;                // bit i: statistics buffer i's phase
         int j = -1;
         const bool counting = p.acc != nullptr;
         PairCounts counts;              // the sampled pairs are each tile's first 8
@@ -605,13 +606,13 @@ __global__ void __launch_bounds__(K1TmCfg::THREADS, 1) k1_project_tm_kernel(cons
             const float inv_n = 1.0f / (float)C::CZ;
             const float dm = (s1.x + s1.y) * inv_n;
             const float var = fmaxf((s2.x + s2.y) * inv_n - dm * dm, 0.f);
-            if (!__all_sync(0xffffffffu, mbar_wait(&s.sempty[sbuf], sphase[sbuf] ^ 1, abort_flag, kErrTimeoutEpilogue))) break;
+            if (!__all_sync(0xffffffffu, mbar_wait(&s.sempty[sbuf], ((sphase >> sbuf) & 1u) ^ 1u, abort_flag, kErrTimeoutEpilogue))) break;
             st_nmean[sbuf * C::TP + row] = -(shift + dm);
             st_rstd[sbuf * C::TP + row] = rsqrtf(var + p.eps);
-            st_hmask[sbuf * C::TP + row] = 0.5f * __uint_as_float((uint32_t)mbits << 16);
+            st_hmask[sbuf * C::TP + row] = (uint16_t)(__float_as_uint(0.5f * __uint_as_float((uint32_t)mbits << 16)) >> 16);
             __syncwarp();
             if (lane == 0) mbar_arrive(&s.sfull[sbuf]);
-            sphase[sbuf] ^= 1;
+            sphase ^= 1u << sbuf;
         }
         if (counting && lane == 0) counts.flush(p.acc);
     } else {
@@ -626,7 +627,8 @@ __global__ void __launch_bounds__(K1TmCfg::THREADS, 1) k1_project_tm_kernel(cons
         const float2 cp_sum = make_float2(cv.z, cv.z), cp_shift = make_float2(cv.w, cv.w);
         const int buf = team;
         const uint32_t tbase = tmem_base + buf * 256 + operand * 2 * C::TP + ((uint32_t)(q * 32) << 16);
-        const float *snmean = st_nmean + buf * C::TP, *srstd = st_rstd + buf * C::TP, *shmask = st_hmask + buf * C::TP;
+        const float *snmean = st_nmean + buf * C::TP, *srstd = st_rstd + buf * C::TP;
+        const uint16_t *shmask = st_hmask + buf * C::TP;
         unsigned long long *acc_c = p.acc ? p.acc + operand * C::C_H + c : nullptr;
         int sum_b = -1;
         float2 run = make_float2(0.f, 0.f);
@@ -681,16 +683,17 @@ __global__ void __launch_bounds__(K1TmCfg::THREADS, 1) k1_project_tm_kernel(cons
                     if (lane == 0) mbar_arrive(&s.tempty[buf]);
                 }
                 uint32_t outw[4];
+                const uint4 mk8 = *reinterpret_cast<const uint4 *>(shmask + o);     // the step's 8 mask / 2
 #pragma unroll
                 for (int jj = 0; jj < 8; jj += 4) {
                     const float4 nm = *reinterpret_cast<const float4 *>(snmean + o + jj);
                     const float4 rs = *reinterpret_cast<const float4 *>(srstd + o + jj);
-                    const float4 mk = *reinterpret_cast<const float4 *>(shmask + o + jj);
 #pragma unroll
                     for (int h = 0; h < 2; ++h) {
                         const float2 nm2 = h == 0 ? make_float2(nm.x, nm.y) : make_float2(nm.z, nm.w);
                         const float2 rs2 = h == 0 ? make_float2(rs.x, rs.y) : make_float2(rs.z, rs.w);
-                        const float2 hm2 = h == 0 ? make_float2(mk.x, mk.y) : make_float2(mk.z, mk.w);
+                        const uint32_t mw = jj == 0 ? (h == 0 ? mk8.x : mk8.y) : (h == 0 ? mk8.z : mk8.w);
+                        const float2 hm2 = make_float2(bf16_lo(mw), bf16_hi(mw));
                         const float2 gv = f2_fma(rs2, f2_fma(nm2, cg_sum, make_float2(gc[jj + 2 * h], gc[jj + 2 * h + 1])), cg_shift);
                         const float2 pv = f2_fma(rs2, f2_fma(nm2, cp_sum, make_float2(pc[jj + 2 * h], pc[jj + 2 * h + 1])), cp_shift);
                         const float2 gm = f2_fma(make_float2(tanh_approx(gv.x), tanh_approx(gv.y)), hm2, hm2);
