@@ -118,3 +118,19 @@ def test_pair_update_finds_the_extents_once_and_matches_dense():
     torch.cuda.synchronize()
     tm.check_device_status()
     assert torch.equal(ref, got)
+
+
+def test_pair_update_with_valid_lengths_matches_dense():
+    lengths = [150, 256]
+    inp = ti.generate(2, 256, 128, 128, dtype="bf16", seed=13, mask=("lengths", lengths), biases=True)
+    z, m, w = upload(inp)
+    dense = tm.TriMulLayer(w, eps=inp.eps)
+    vl_out = tm.TriMulLayer(w, eps=inp.eps)
+    vl_in = tm.TriMulLayer(w, eps=inp.eps)
+    assert vl_out.set_valid_lengths(lengths, 256) is (tm.skip_saving(lengths, 256) >= 0.15)
+    vl_in.set_valid_lengths(lengths, 256)
+    ref = tm.pair_update(z, m, dense, dense, out_dtype=torch.float32)
+    got = tm.pair_update(z, m, vl_out, vl_in, out_dtype=torch.float32)
+    torch.cuda.synchronize()
+    tm.check_device_status()
+    assert torch.equal(ref, got)
