@@ -58,7 +58,9 @@ __device__ __forceinline__ int k2_tile_chunks(const K2Args &p, int bc, int m0, i
     const int R = __ldg(p.ext + 2 * b), Cx = __ldg(p.ext + 2 * b + 1);
     if ((p.N & 127) == 0 && (m0 >= R || n0 >= Cx)) return 0;
     const int kend = p.incoming ? R : Cx;
-    const int nk = (kend + k2::BK - 1) / k2::BK;
+    // at least one chunk: a tile the output kernel may still read (N % 128 != 0) is written
+    // even when no k is valid, and there its one chunk sums exact zeros
+    const int nk = kend > 0 ? (kend + k2::BK - 1) / k2::BK : 1;
     return nk < p.k_chunks ? nk : p.k_chunks;
 }
 

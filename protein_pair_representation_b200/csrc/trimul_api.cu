@@ -975,7 +975,8 @@ extern "C" trimul_status_t tri_mul_mask_extents(const void *mask, int64_t B, int
                                                 int32_t *extents, void *stream) {
     if (!mask || !extents) return fail(TRIMUL_ERR_INVALID_ARG, "mask / extents NULL");
     if (dtype != TRIMUL_BF16) return fail(TRIMUL_ERR_UNSUPPORTED_SHAPE, "extents are found for bf16 masks");
-    if (B < 1 || N < 8 || N % 8 || N > 16384) return fail(TRIMUL_ERR_UNSUPPORTED_SHAPE, "N=%lld must be a multiple of 8 in [8, 16384]", (long long)N);
+    if (B < 1 || B > 65535) return fail(TRIMUL_ERR_UNSUPPORTED_SHAPE, "B=%lld outside [1, 65535]", (long long)B);
+    if (N < 8 || N % 8 || N > 16384) return fail(TRIMUL_ERR_UNSUPPORTED_SHAPE, "N=%lld must be a multiple of 8 in [8, 16384]", (long long)N);
     if (!aligned16(mask) || !aligned16(extents)) return fail(TRIMUL_ERR_ALIGNMENT, "mask / extents not 16-byte aligned");
     DeviceInfo d;
     TRY(require_sm100(&d));

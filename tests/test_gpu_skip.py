@@ -134,3 +134,25 @@ def test_pair_update_with_valid_lengths_matches_dense():
     torch.cuda.synchronize()
     tm.check_device_status()
     assert torch.equal(ref, got)
+
+
+@pytest.mark.parametrize("direction", ["outgoing", "incoming"])
+def test_given_extents_with_no_valid_k_leave_no_stale_intermediates(direction):
+    """Extents {100, 0} are a legal bound for an all-zero mask (no nonzero entry anywhere). At
+    N = 136 the output kernel's tiles straddle rows, so it still reads x for rows < 100: the
+    contraction must write those tiles (exact zeros) rather than leave the workspace's old
+    contents, here NaN bit patterns, under masked pairs."""
+    inp = ti.generate(2, 136, 128, 128, dtype="bf16", seed=17, mask=("lengths", [0, 136]), biases=True)
+    z, m, w = upload(inp)
+    dense = tm.TriMulLayer(w, eps=inp.eps)
+    layer = tm.TriMulLayer(w, eps=inp.eps)
+    layer.ensure_workspace(2, 136, torch.bfloat16)
+    layer._ws.fill_(255)                        # every fp16 intermediate reads as NaN
+    ext = torch.tensor([[100, 0], [136, 136]], dtype=torch.int32, device="cuda")
+    got = layer.forward_extents(z, m, ext, direction)
+    ref = dense.forward(z, m, direction)
+    torch.cuda.synchronize()
+    tm.check_device_status()
+    assert torch.isfinite(got).all()
+    assert not torch.any(got[0])
+    assert torch.equal(got, ref)
