@@ -94,17 +94,24 @@ struct K3Args {
 // touches memory the previous kernel may write or read.
 template <typename Kernel, typename Args>
 inline cudaError_t launch_pdl(Kernel kernel, int grid, int block, size_t smem, cudaStream_t stream,
-                              const Args &args) {
+                              const Args &args, int cluster = 1) {
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3((unsigned)grid);
     cfg.blockDim = dim3((unsigned)block);
     cfg.dynamicSmemBytes = smem;
     cfg.stream = stream;
-    cudaLaunchAttribute attr[1];
+    cudaLaunchAttribute attr[2];
     attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
+    if (cluster > 1) {      // clusters of `cluster` consecutive CTAs (grid a multiple of it)
+        attr[1].id = cudaLaunchAttributeClusterDimension;
+        attr[1].val.clusterDim.x = (unsigned)cluster;
+        attr[1].val.clusterDim.y = 1;
+        attr[1].val.clusterDim.z = 1;
+        cfg.numAttrs = 2;
+    }
     return cudaLaunchKernelEx(&cfg, kernel, args);
 }
 
@@ -115,7 +122,7 @@ int k1_ncol(int c_z);
 int k1_channels_per_warpgroup(int c_z);
 cudaError_t k1_launch(int c_z, const K1Args &args, int grid, cudaStream_t stream);
 int k1_row_mode(int c_z);
-int k1_tile_pairs(int c_z);        // pairs per K1 tile (64 at c_z = 128, 128 at c_z = 384)
+int k1_tile_pairs(int c_z);        // pairs per K1 tile (128; at c_z = 128 a CTA pair's, 64 from each CTA)
 
 size_t k2_smem_bytes();
 cudaError_t k2_launch(const K2Args &args, int grid, cudaStream_t stream);

@@ -101,6 +101,86 @@ __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, volati
     }
 }
 
+// ------------------------------------------------------------------ CTA pairs (clusters of two)
+
+__device__ __forceinline__ uint32_t cluster_ctarank() {
+    uint32_t r;
+    asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+    return r;
+}
+
+// The shared::cluster address of the object at `p` (in this CTA's shared memory) in cluster CTA
+// `rank`: the same offset in that CTA's shared memory.
+__device__ __forceinline__ uint32_t mapa_shared(const void *p, uint32_t rank) {
+    uint32_t r;
+    asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(smem_u32(p)), "r"(rank));
+    return r;
+}
+
+// Asynchronous 4-byte store into the shared memory of a cluster CTA (shared::cluster address
+// `addr`) that completes 4 bytes of the transaction count of that CTA's mbarrier at `bar`: a
+// thread waiting on the barrier then sees the data, with no fence on the storing side.
+__device__ __forceinline__ void st_async_u32(uint32_t addr, uint32_t v, uint32_t bar) {
+    asm volatile("st.async.shared::cluster.mbarrier::complete_tx::bytes.u32 [%0], %1, [%2];" ::"r"(addr), "r"(v),
+                 "r"(bar)
+                 : "memory");
+}
+
+// Arrive on the mbarrier at shared::cluster address `addr` (this CTA's or the peer's) with the
+// default semantics (release at CTA scope): enough where the waiter needs no data from this thread
+// (a buffer freed after this thread's loads of it returned, tensor memory read after
+// tcgen05.fence::before_thread_sync), and much cheaper than a cluster-scope release, which waits
+// for the thread's outstanding memory traffic.
+__device__ __forceinline__ void mbar_arrive_remote(uint32_t addr) {
+    asm volatile("mbarrier.arrive.shared::cluster.b64 _, [%0];" ::"r"(addr) : "memory");
+}
+
+// Arrive on the mbarrier at shared::cluster address `addr` (this CTA's or the peer's), releasing
+// this thread's earlier memory operations at cluster scope.
+__device__ __forceinline__ void mbar_arrive_cluster(uint32_t addr) {
+    asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(addr) : "memory");
+}
+
+// (With the suspend-time hint of mbar_try_wait_sleep.)
+__device__ __forceinline__ bool mbar_try_wait_cluster(uint64_t *bar, uint32_t parity, uint32_t hint_ns) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2, %3;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(smem_u32(bar)), "r"(parity), "r"(hint_ns)
+        : "memory");
+    return ok != 0;
+}
+
+// mbar_wait for a barrier that the peer CTA arrives on: acquires at cluster scope, so that what
+// the peer released with its arrival (its stores into this CTA's shared memory, the data it saw
+// land) is visible. Same bound and abort protocol; a waiting thread is suspended like mbar_wait's.
+__device__ __forceinline__ bool mbar_wait_cluster(uint64_t *bar, uint32_t parity, volatile int *abort_flag,
+                                                  unsigned int err_code) {
+    long long start = clock64();
+    uint32_t spins = 0;
+    while (!mbar_try_wait_cluster(bar, parity, 20000u)) {
+        if ((++spins & 15u) == 0) {
+            if (*abort_flag) return false;
+            if (clock64() - start > kWaitLimitCycles) {
+                *abort_flag = 1;
+                atomicOr(&g_device_error, err_code);
+                return false;
+            }
+        }
+    }
+    return true;
+}
+
+// Every thread of both CTAs arrives, then waits for all (release / acquire at cluster scope). Each
+// kernel that uses it calls it from every thread at the same two points (after the barrier
+// initialisation and before the exit), with every role's loop bounded before it.
+__device__ __forceinline__ void cluster_sync_all() {
+    asm volatile("barrier.cluster.arrive.release;\n\tbarrier.cluster.wait.acquire;" ::: "memory");
+}
+
 // Short bounded wait used only on the abort path to let copies in flight land.
 __device__ __forceinline__ void mbar_drain(uint64_t *bar, uint32_t parity) {
     long long start = clock64();
@@ -277,6 +357,22 @@ __device__ __forceinline__ void tmem_dealloc(uint32_t taddr, uint32_t ncols) {
                  : "memory");
 }
 
+// The same for a CTA pair (cta_group::2): one warp of each CTA, with the same warp index and the
+// same destination offset, allocates together; both CTAs get the same column address.
+__device__ __forceinline__ void tmem_alloc_pair(uint32_t *dst_smem, uint32_t ncols) {
+    asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(dst_smem)),
+                 "r"(ncols)
+                 : "memory");
+}
+
+__device__ __forceinline__ void tmem_relinquish_pair() {
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;" ::: "memory");
+}
+
+__device__ __forceinline__ void tmem_dealloc_pair(uint32_t taddr, uint32_t ncols) {
+    asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols) : "memory");
+}
+
 __device__ __forceinline__ void tc_fence_before() {
     asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
 }
@@ -302,6 +398,36 @@ __device__ __forceinline__ void tc_commit(uint64_t *bar) {
         "tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
             smem_u32(bar))
         : "memory");
+}
+
+// CTA-pair MMA, issued by one thread of CTA 0: D (M = 256) = A * B^T with A's rows 0-127 from CTA
+// 0's and rows 128-255 from CTA 1's shared memory, B's first N/2 rows from CTA 0's and the rest
+// from CTA 1's (each at the descriptors' offsets), D's rows 0-127 into CTA 0's TMEM and 128-255 into
+// CTA 1's, both at `tmem_d`.
+__device__ __forceinline__ void tc_mma_bf16_pair(uint32_t tmem_d, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
+                                                 uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::2.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(tmem_d),
+        "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
+        : "memory");
+}
+
+// Arrive once on the mbarrier at this offset in every CTA of `cta_mask` when this thread's
+// earlier CTA-pair MMAs complete.
+__device__ __forceinline__ void tc_commit_pair_mc(uint64_t *bar, uint16_t cta_mask) {
+    asm volatile(
+        "tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64 [%0], %1;" ::"r"(
+            smem_u32(bar)),
+        "h"(cta_mask)
+        : "memory");
+}
+
+// The same, on this CTA's barrier only.
+__device__ __forceinline__ void tc_commit_pair(uint64_t *bar) {
+    asm volatile("tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(smem_u32(bar))
+                 : "memory");
 }
 
 __device__ __forceinline__ void tc_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }

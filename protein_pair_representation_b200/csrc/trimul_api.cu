@@ -439,10 +439,10 @@ static trimul_status_t run_project_bf16(const trimul_layer_t *L, const void *z, 
     const int tp = k1_tile_pairs(cz);
     if (cz == 128) {
         // z [B][NN][128] viewed as {64 channels, NN pairs, 2 halves, B}: one copy brings both
-        // 64-channel halves of a 64-pair tile, laid out [half][pair][64]
+        // 64-channel halves of one CTA's 64 pairs of a tile, laid out [half][pair][64]
         uint64_t dims[4] = {64, NN, 2, (uint64_t)B};
         uint64_t strides[3] = {(uint64_t)cz * 2, 128, NN * cz * 2};
-        uint32_t box[4] = {64, (uint32_t)tp, 2, 1};
+        uint32_t box[4] = {64, 64, 2, 1};
         TRY(make_map(&p.tm_z, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, z, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_128B, "K1 z"));
     } else {
         uint64_t dims[3] = {(uint64_t)cz, NN, (uint64_t)B};
