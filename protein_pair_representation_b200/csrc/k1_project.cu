@@ -415,13 +415,15 @@ __global__ void __launch_bounds__(448, 1) k1_project_kernel(const __grid_constan
 // either epilogue has all 128 pairs' (-mean, rstd, mask / 2).
 // Hand-offs across the pair (every wait bounded):
 //   - CTA 1's MMA warp relays to CTA 0 that CTA 1's weights, and each of its z half-tiles, have
-//     landed (remote mbarrier arrivals, release / acquire at cluster scope, off the epilogue's
-//     path); every TMA copy completes on a barrier of the CTA that issued it;
+//     landed (remote mbarrier arrivals); every TMA copy completes on a barrier of the CTA that
+//     issued it;
 //   - the MMA commits arrive on both CTAs' z-free and accumulator-full barriers (multicast);
 //   - the epilogue warps of both CTAs arrive on CTA 0's accumulator-free barrier and on both
-//     CTAs' statistics-free barriers with CTA-scope release (they hand over no data; a
-//     cluster-scope release waits for the thread's outstanding memory traffic, about a
-//     microsecond per tile here).
+//     CTAs' statistics-free barriers.
+// The remote arrivals release at CTA scope (the default): each signals a completion the waiter
+// needs no data from this thread for (a copy observed to have landed, loads returned, tensor
+// memory read after tcgen05.fence::before_thread_sync); a cluster-scope release waited for the
+// thread's outstanding memory traffic, about a microsecond per arrival here.
 // Two teams of eight epilogue warps take alternate tiles, each team with its own accumulator
 // buffer; warp 4h + q of a team takes pairs [64h, 64h + 64) of its tile and channels
 // [32q, 32q + 32) of the CTA's operand, so that channel's folding constants stay in registers;
@@ -577,7 +579,7 @@ __global__ void __launch_bounds__(K1PairCfg::THREADS, 1) k1_project_pair_kernel(
                 const int abuf = j & 1;
                 if (!mbar_wait(&s.tempty[abuf], ((aphase >> abuf) & 1u) ^ 1u, abort_flag, kErrTimeoutMma)) break;
                 if (!mbar_wait(&s.full[stage], phase, abort_flag, kErrTimeoutMma)) break;
-                if (!mbar_wait_cluster(&s.pfull[stage], phase, abort_flag, kErrTimeoutMma)) break;
+                if (!mbar_wait(&s.pfull[stage], phase, abort_flag, kErrTimeoutMma)) break;
                 tc_fence_after();
                 const uint8_t *zt = tiles + stage * C::TILE;
 #pragma unroll
@@ -608,7 +610,7 @@ __global__ void __launch_bounds__(K1PairCfg::THREADS, 1) k1_project_pair_kernel(
             for (int t = pair; ok && t < num_tiles; t += npairs, tw.advance(npairs, p.tiles_per_batch)) {
                 if (SKIP && tile_masked_out<C::TP>(p.ext, tw.b, (long long)tw.t * C::TP, p.N, p.NN, p.rowdiv)) continue;
                 if (!mbar_wait(&s.full[stage], phase, abort_flag, kErrTimeoutMma)) break;
-                mbar_arrive_cluster(r_pfull + (uint32_t)stage * 8u);
+                mbar_arrive_remote(r_pfull + (uint32_t)stage * 8u);
                 if (++stage == C::S) { stage = 0; phase ^= 1; }
             }
         }

@@ -494,7 +494,7 @@ static trimul_status_t run_contract_tc(const void *a, const void *b, void *x, in
     uint64_t dims[3] = {(uint64_t)N, (uint64_t)N, (uint64_t)BC};
     uint64_t strides[2] = {(uint64_t)N * 2, (uint64_t)N * N * 2};
     if (!incoming) {
-        uint32_t boxa[3] = {64, 128, 1}, boxb[3] = {64, 256, 1};
+        uint32_t boxa[3] = {64, 128, 1}, boxb[3] = {64, 128, 1};   // one CTA's half of a pair tile each
         TRY(make_map(&p.tm_a, dt, 3, a, dims, strides, boxa, CU_TENSOR_MAP_SWIZZLE_128B, "K2 a"));
         TRY(make_map(&p.tm_b, dt, 3, b, dims, strides, boxb, CU_TENSOR_MAP_SWIZZLE_128B, "K2 b"));
     } else {
@@ -514,13 +514,11 @@ static trimul_status_t run_contract_tc(const void *a, const void *b, void *x, in
     p.C = C;
     p.BC = (int)BC;
     p.N = N;
-    p.m_tiles = (N + 127) / 128;
+    p.m_tiles = (N + 255) / 256;        // 256-row tiles of a CTA pair
     p.n_tiles = (N + 255) / 256;
     p.k_chunks = (N + 63) / 64;
     p.incoming = incoming;
-    const long long tiles = (long long)BC * p.m_tiles * p.n_tiles;
-    const int grid = grid_for(d.sms, tiles, 1);
-    TRY_CUDA(k2_launch(p, grid, st), "K2 launch");
+    TRY_CUDA(k2_launch(p, 0, st), "K2 launch");
     return TRIMUL_OK;
 }
 
@@ -921,12 +919,11 @@ extern "C" trimul_status_t tri_mul_shard_finish(const trimul_rows_t *z, const vo
     p.C = L->c_h;
     p.BC = (int)BC;
     p.N = (int)z->N;
-    p.m_tiles = (int)(z->R / 128);
+    p.m_tiles = (int)((z->R + 255) / 256);   // 256-row tiles of a CTA pair
     p.n_tiles = (int)((z->N + 255) / 256);
     p.k_chunks = (int)(z->N / 64);
     p.incoming = incoming;
-    const long long tiles = BC * p.m_tiles * p.n_tiles;
-    TRY_CUDA(k2_shard_launch(sa, grid_for(d.sms, tiles, 1), st), "K2 shard launch");
+    TRY_CUDA(k2_shard_launch(sa, 0, st), "K2 shard launch");
     return run_output_bf16(L, z->data, mask, x, x_scale, out->data, out->dtype == TRIMUL_F32, false, (int)z->B, (int)z->R,
                            (int)z->N, st, nullptr);
 }
