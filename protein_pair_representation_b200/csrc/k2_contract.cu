@@ -20,9 +20,9 @@
 // one CTA took and gave 48 KB each for the same outputs (that bounded it at large N), and L2
 // serves a third fewer bytes.
 //   warp 8      TMA producer (one elected lane)
-//   warp 9      TMEM allocator, and MMA issuer (CTA 0) or relay (CTA 1: tells CTA 0 when each of
-//               its chunks has landed with a remote mbarrier arrival; one with cluster-scope
-//               release took about a microsecond under load, longer than a chunk's MMAs); fp32
+//   warp 9      TMEM allocator, and MMA issuer (CTA 0); each chunk of both CTAs completes on CTA
+//               0's barrier (CTA 1's copies are the pair form, cta_group::2, which may signal the
+//               peer's barrier; CTA 0 expects both halves' bytes); fp32
 //               accumulators in two 256-column TMEM buffers so the epilogue of tile t overlaps the
 //               MMAs of tile t+1; the commits arrive on both CTAs' barriers (multicast)
 //   warps 0-7   epilogue: two warpgroups, each drains 128 of the 256 columns of the CTA's 128
@@ -50,7 +50,7 @@ constexpr int THREADS = 320;
 constexpr int TMEM_COLS = 512;
 
 struct Smem {
-    uint64_t full[STAGES], empty[STAGES], pfull[STAGES];
+    uint64_t full[STAGES], empty[STAGES];
     uint64_t tfull[2], tempty[2];
     uint64_t drain;
     uint32_t tmem_base;
@@ -113,7 +113,6 @@ __global__ void __launch_bounds__(k2::THREADS, 1) k2_contract_kernel(const __gri
         for (int i = 0; i < STAGES; ++i) {
             mbar_init(&s.full[i], 1);
             mbar_init(&s.empty[i], 1);           // the MMA commit
-            mbar_init(&s.pfull[i], 1);           // CTA 1's relay (used in CTA 0)
         }
         for (int i = 0; i < 2; ++i) {
             mbar_init(&s.tfull[i], 1);
@@ -153,7 +152,9 @@ __global__ void __launch_bounds__(k2::THREADS, 1) k2_contract_kernel(const __gri
         if (lane == 0) {
             int stage = 0;
             uint32_t phase = 0;
-            uint32_t filled = 0;  // number of stage fills issued (for the abort drain)
+            uint32_t filled = 0;  // number of stage fills issued (for the drain at the end)
+            // every chunk completes on CTA 0's barrier: CTA 0 expects both CTAs' bytes
+            const uint32_t full0 = mapa_shared(&s.full[0], 0);
             for (int t = pair; t < num_tiles; t += npairs) {
                 const int bc = t / tiles_per_channel;
                 const int r = t - bc * tiles_per_channel;
@@ -166,46 +167,48 @@ __global__ void __launch_bounds__(k2::THREADS, 1) k2_contract_kernel(const __gri
                     if (!mbar_wait(&s.empty[stage], phase ^ 1, abort_flag, kErrTimeoutProducer)) goto producer_abort;
                     uint8_t *sa = stages + stage * STAGE_BYTES;
                     uint8_t *sb = sa + A_BYTES;
-                    mbar_arrive_expect_tx(&s.full[stage], STAGE_BYTES);
+                    if (rank == 0) mbar_arrive_expect_tx(&s.full[stage], 2 * STAGE_BYTES);
+                    const uint32_t fb = full0 + (uint32_t)stage * 8u;
                     const int k0 = kc * BK;
                     if constexpr (SHARD) {
                         if (!p.incoming) {
-                            tma_load_3d(sa, &p.tm_a, &s.full[stage], k0, mr, bc);
+                            tma_load_3d_pair(sa, &p.tm_a, fb, k0, mr, bc);
                             const int g = shard_of(pa, nr);     // 128 b rows lie in one shard
-                            tma_load_3d(sb, &pa.tm_sb[g], &s.full[stage], k0, nr - pa.row0[g], bc);
+                            tma_load_3d_pair(sb, &pa.tm_sb[g], fb, k0, nr - pa.row0[g], bc);
                         } else {
                             const int g = shard_of(pa, k0);     // a 64-row k chunk lies in one shard
                             const int kl = k0 - pa.row0[g];
 #pragma unroll
                             for (int h = 0; h < BM / 64; ++h)
-                                tma_load_3d(sa + h * 8192, &pa.tm_sa[g], &s.full[stage], pa.i0 + mr + 64 * h, kl, bc);
+                                tma_load_3d_pair(sa + h * 8192, &pa.tm_sa[g], fb, pa.i0 + mr + 64 * h, kl, bc);
 #pragma unroll
                             for (int h = 0; h < HN / 64; ++h)
-                                tma_load_3d(sb + h * 8192, &pa.tm_sb[g], &s.full[stage], nr + 64 * h, kl, bc);
+                                tma_load_3d_pair(sb + h * 8192, &pa.tm_sb[g], fb, nr + 64 * h, kl, bc);
                         }
                     } else if (!p.incoming) {
-                        tma_load_3d(sa, &p.tm_a, &s.full[stage], k0, mr, bc);
-                        tma_load_3d(sb, &p.tm_b, &s.full[stage], k0, nr, bc);
+                        tma_load_3d_pair(sa, &p.tm_a, fb, k0, mr, bc);
+                        tma_load_3d_pair(sb, &p.tm_b, fb, k0, nr, bc);
                     } else {
 #pragma unroll
                         for (int h = 0; h < BM / 64; ++h)
-                            tma_load_3d(sa + h * 8192, &p.tm_a, &s.full[stage], mr + 64 * h, k0, bc);
+                            tma_load_3d_pair(sa + h * 8192, &p.tm_a, fb, mr + 64 * h, k0, bc);
 #pragma unroll
                         for (int h = 0; h < HN / 64; ++h)
-                            tma_load_3d(sb + h * 8192, &p.tm_b, &s.full[stage], nr + 64 * h, k0, bc);
+                            tma_load_3d_pair(sb + h * 8192, &p.tm_b, fb, nr + 64 * h, k0, bc);
                     }
                     ++filled;
                     if (++stage == STAGES) { stage = 0; phase ^= 1; }
                 }
             }
-            goto producer_done;
         producer_abort:
-            // let the copies already issued land before the CTA exits
+            // (also the normal end) let the copies already issued land before the CTA exits: CTA 0
+            // through their barrier (both CTAs' bytes), CTA 1 through the MMA commits that free its
+            // stages once they have been read
             for (uint32_t i = 0; i < (filled < (uint32_t)STAGES ? filled : (uint32_t)STAGES); ++i) {
                 uint32_t f = filled - 1 - i;
-                mbar_drain(&s.full[f % STAGES], (f / STAGES) & 1);
+                if (rank == 0) mbar_drain(&s.full[f % STAGES], (f / STAGES) & 1);
+                else mbar_drain(&s.empty[f % STAGES], (f / STAGES) & 1);
             }
-        producer_done:;
         }
     } else if (warp == MMA_WARP) {
         if (lane == 0 && rank == 0) {
@@ -224,8 +227,7 @@ __global__ void __launch_bounds__(k2::THREADS, 1) k2_contract_kernel(const __gri
                 const uint32_t d_tmem = tmem_base + abuf * BN;
                 bool ok = true;
                 for (int kc = 0; kc < nk; ++kc) {
-                    if (!mbar_wait(&s.full[stage], phase, abort_flag, kErrTimeoutMma) ||
-                        !mbar_wait(&s.pfull[stage], phase, abort_flag, kErrTimeoutMma)) {
+                    if (!mbar_wait(&s.full[stage], phase, abort_flag, kErrTimeoutMma)) {
                         ok = false;
                         break;
                     }
@@ -254,22 +256,6 @@ __global__ void __launch_bounds__(k2::THREADS, 1) k2_contract_kernel(const __gri
             // all MMAs issued by this thread are complete once this arrives
             tc_commit_pair(&s.drain);
             mbar_drain(&s.drain, 0);
-        } else if (lane == 0) {
-            // CTA 1: tell CTA 0 when each of this CTA's chunks has landed
-            const uint32_t r_pfull = mapa_shared(&s.pfull[0], 0);
-            int stage = 0;
-            uint32_t phase = 0;
-            bool ok = true;
-            for (int t = pair; ok && t < num_tiles; t += npairs) {
-                const int bc = t / tiles_per_channel;
-                const int r = t - bc * tiles_per_channel;
-                const int nk = k2_tile_chunks(p, bc, (r / p.n_tiles) * PM, (r % p.n_tiles) * BN);
-                for (int kc = 0; kc < nk; ++kc) {
-                    if (!mbar_wait(&s.full[stage], phase, abort_flag, kErrTimeoutMma)) { ok = false; break; }
-                    mbar_arrive_remote(r_pfull + (uint32_t)stage * 8u);
-                    if (++stage == STAGES) { stage = 0; phase ^= 1; }
-                }
-            }
         }
     } else {
         // epilogue warpgroups
